@@ -1,0 +1,311 @@
+"""fp64 CPU oracle for ExTernD greedy sequential ternary ALS.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path imports, links or runs
+this module: only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg
+of ``bench.py`` do.  It shares no code with the CUDA library.
+
+Source: "ExTernD: Expanded-Rank Ternary Decomposition" (academ.us HTML of
+arXiv 2607.13511), cited below by section and display equation:
+
+* §2.1 display equation: A ~ B diag(D) C with B in {-1,0,1}^{m x k},
+  C in {-1,0,1}^{k x n}, D in R^k; energy E = 1 - ||A - Ahat||_F^2 / ||A||_F^2.
+* §2.2 display equation: T_tau(u)_i = sign(u_i) * 1[|u_i| > tau * (1/m) sum_j |u_j|],
+  keeping the single largest entry when the result would be all-zero; and the
+  optimal ternary projection (sort |u|, keep the prefix s* maximizing
+  (1/sqrt(s)) sum_{i<=s} |u|_(i)).
+* §2.3 steps 1-3: R <- A; for each component: 15 alternating fits
+  v <- T_tau(R^T u), u <- T_tau(R v); scale d = u^T R v / (||u||^2 ||v||^2);
+  deflate R <- R - d u v^T; store B[:, i] = u, C[i, :] = v^T.
+* §2.6 Eq. (1): bpw_eff = mu (m + n) / max(m, n) * (2 - sparsity).
+
+Everything is plain numpy in float64, written in the pages' order.  Readings
+where the pages are silent (each one is listed with its reason in the design
+notes of the repository):
+
+* start vector: the pages start the alternation from some u without saying
+  which; here u^(0) = T_tau(z) with z ~ N(0, 1)^m drawn per component from the
+  counter-based generator Philox4x32-10 (Salmon et al., "Parallel random
+  numbers: as easy as 1, 2, 3", SC'11) keyed by the seed, followed by the
+  Box-Muller transform (cosine branch).
+* "15 iterations" = 15 (V-step, U-step) pairs; the scale uses the final u and
+  the v of the same pair.
+* the mean inside T_tau runs over the vector's own length (n for the V-step,
+  m for the U-step); the comparison is strict.
+* all-zero fallback: the lowest index among the entries of largest magnitude
+  keeps its sign; an identically zero vector yields +1 at index 0.
+* k = round-half-away-from-zero(mu * min(m, n)).
+* if u^T R v = 0 the component gets d = 0 and R is unchanged.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+
+# ----------------------------------------------------------------------------
+# Inner rank (§2.1: k = mu * min(m, n))
+# ----------------------------------------------------------------------------
+
+
+def rank(m: int, n: int, mu: float) -> int:
+    """k = mu * min(m, n) rounded half away from zero; -1 if that is below 1."""
+    if m < 1 or n < 1 or not math.isfinite(mu):
+        return -1
+    x = mu * min(m, n)
+    k = int(math.floor(abs(x) + 0.5)) * (1 if x >= 0 else -1)
+    return k if k >= 1 else -1
+
+
+# ----------------------------------------------------------------------------
+# Start vectors: Philox4x32-10 + Box-Muller (reading of §2.3, which is silent)
+# ----------------------------------------------------------------------------
+
+_MASK32 = np.uint64(0xFFFFFFFF)
+_PHILOX_M0 = np.uint64(0xD2511F53)
+_PHILOX_M1 = np.uint64(0xCD9E8D57)
+_PHILOX_W0 = np.uint64(0x9E3779B9)
+_PHILOX_W1 = np.uint64(0xBB67AE85)
+INIT_STREAM = 1            # third counter word for start vectors
+TWO_PI = 6.283185307179586  # nearest double to 2*pi
+
+
+def philox4x32_10(c0, c1, c2, c3, k0, k1):
+    """Philox4x32 with 10 rounds, as defined by Salmon et al. (SC'11).
+
+    Each round multiplies counter words 0 and 2 by the two Philox multipliers,
+    splits the 64-bit products into high and low halves and mixes them with the
+    other two words and the key; the key is bumped by the Weyl constants before
+    every round but the first.  Inputs are integer arrays holding 32-bit values.
+    """
+    c0, c1, c2, c3 = (np.asarray(c, dtype=np.uint64) & _MASK32 for c in (c0, c1, c2, c3))
+    k0 = np.asarray(k0, dtype=np.uint64) & _MASK32
+    k1 = np.asarray(k1, dtype=np.uint64) & _MASK32
+    for r in range(10):
+        if r > 0:
+            k0 = (k0 + _PHILOX_W0) & _MASK32
+            k1 = (k1 + _PHILOX_W1) & _MASK32
+        p0 = _PHILOX_M0 * c0
+        p1 = _PHILOX_M1 * c2
+        hi0, lo0 = p0 >> np.uint64(32), p0 & _MASK32
+        hi1, lo1 = p1 >> np.uint64(32), p1 & _MASK32
+        c0, c1, c2, c3 = (hi1 ^ c1 ^ k0), lo1, (hi0 ^ c3 ^ k1), lo0
+    return c0, c1, c2, c3
+
+
+def _uniform53(hi, lo):
+    """(hi:lo) 64-bit word -> double in (0, 1): top 53 bits, offset by half a step."""
+    w = (hi << np.uint64(32)) | lo
+    return ((w >> np.uint64(11)).astype(np.float64) + 0.5) * (2.0 ** -53)
+
+
+def start_normals(seed: int, comp: int, m: int) -> np.ndarray:
+    """z_j ~ N(0, 1), j < m, for component ``comp``: counter (j, comp, 1, 0), key = seed."""
+    j = np.arange(m, dtype=np.uint64)
+    x0, x1, x2, x3 = philox4x32_10(j, np.uint64(comp), np.uint64(INIT_STREAM), np.uint64(0),
+                                   np.uint64(seed & 0xFFFFFFFF), np.uint64(seed >> 32))
+    u1 = _uniform53(x1, x0)
+    u2 = _uniform53(x3, x2)
+    return np.sqrt(-2.0 * np.log(u1)) * np.cos(TWO_PI * u2)
+
+
+# ----------------------------------------------------------------------------
+# §2.2 ternarization operator and optimal ternary projection
+# ----------------------------------------------------------------------------
+
+
+def ternarize(x: np.ndarray, tau: float):
+    """T_tau(x) of §2.2.  Returns (trits int8, threshold, fallback_used)."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    thr = tau * a.sum() / x.shape[0]
+    out = np.where(a > thr, np.where(x < 0, -1, 1), 0).astype(np.int8)
+    fallback = False
+    if not out.any():
+        fallback = True
+        j = int(np.argmax(a))              # first index among the largest magnitudes
+        out[j] = -1 if x[j] < 0 else 1     # x == 0 everywhere -> +1 at index 0
+    return out, thr, fallback
+
+
+def relative_margin(x: np.ndarray, thr: float) -> float:
+    """min_c | |x_c| - thr | / thr : how close the vector came to a threshold tie."""
+    if thr <= 0:
+        return math.inf
+    return float(np.min(np.abs(np.abs(np.asarray(x, dtype=np.float64)) - thr)) / thr)
+
+
+def optimal_ternary_projection(u: np.ndarray):
+    """argmin_{t, alpha} ||u - alpha t||_2 over ternary t (§2.2 closed form).
+
+    Sort |u| descending, keep the prefix length s* that maximizes
+    (1/sqrt(s)) * sum_{i<=s} |u|_(i); t = sign(u) on that prefix, alpha = mean of
+    the kept magnitudes.  Returns (t int8, alpha, s*).
+    """
+    u = np.asarray(u, dtype=np.float64)
+    order = np.argsort(-np.abs(u), kind="stable")
+    csum = np.cumsum(np.abs(u)[order])
+    s_range = np.arange(1, u.shape[0] + 1, dtype=np.float64)
+    score = csum / np.sqrt(s_range)
+    s_star = int(np.argmax(score)) + 1
+    t = np.zeros(u.shape[0], dtype=np.int8)
+    keep = order[:s_star]
+    t[keep] = np.where(u[keep] < 0, -1, 1)
+    alpha = csum[s_star - 1] / s_star
+    return t, alpha, s_star
+
+
+# ----------------------------------------------------------------------------
+# §2.3 greedy sequential ALS
+# ----------------------------------------------------------------------------
+
+
+def ls_scale(R: np.ndarray, u: np.ndarray, v: np.ndarray) -> float:
+    """§2.3 step 2: d = u^T R v / (||u||^2 ||v||^2); 0 when u^T R v = 0."""
+    u = np.asarray(u, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    p = float(u @ (R @ v))
+    if p == 0.0:
+        return 0.0
+    return p / (float(u @ u) * float(v @ v))
+
+
+def half_step(R: np.ndarray, trits_in: np.ndarray, tau: float, transpose: bool):
+    """One half of §2.3 step 1 on a given residual.
+
+    transpose=True : x = R^T u, v = T_tau(x)   (V-step, input length m, output n)
+    transpose=False: y = R v,   u = T_tau(y)   (U-step, input length n, output m)
+    Returns (pre-threshold vector, threshold, output trits, fallback_used).
+    """
+    R = np.asarray(R, dtype=np.float64)
+    w = np.asarray(trits_in, dtype=np.float64)
+    pre = R.T @ w if transpose else R @ w
+    out, thr, fb = ternarize(pre, tau)
+    return pre, thr, out, fb
+
+
+@dataclass
+class ComponentFit:
+    u: np.ndarray          # int8, m
+    v: np.ndarray          # int8, n
+    d: float
+    p: float               # u^T R v
+    decrease: float        # ||R||^2 - ||R - d u v^T||^2 = p^2 / (nnz u * nnz v)
+    min_margin: float      # closest approach of any half-step to a threshold tie
+    u_first: np.ndarray    # start trits
+
+
+def fit_component(R: np.ndarray, u0: np.ndarray, tau: float, iters: int) -> ComponentFit:
+    """§2.3 steps 1-2 for one component, from start trits u0, on residual R (fp64)."""
+    u = np.asarray(u0, dtype=np.int8)
+    v = None
+    y = None
+    margin = math.inf
+    for _ in range(iters):
+        x = R.T @ u.astype(np.float64)               # V-step: x = R^T u
+        v, tv, _ = ternarize(x, tau)
+        margin = min(margin, relative_margin(x, tv))
+        y = R @ v.astype(np.float64)                 # U-step: y = R v
+        u, tu, _ = ternarize(y, tau)
+        margin = min(margin, relative_margin(y, tu))
+    p = float(u.astype(np.float64) @ y)              # u^T R v with the final pair
+    nu = int(np.count_nonzero(u))
+    nv = int(np.count_nonzero(v))
+    d = 0.0 if p == 0.0 else p / (nu * nv)
+    return ComponentFit(u=u, v=v, d=d, p=p, decrease=(p * p) / (nu * nv), min_margin=margin,
+                        u_first=np.asarray(u0, dtype=np.int8))
+
+
+@dataclass
+class Factorization:
+    B: np.ndarray              # m x k int8
+    C: np.ndarray              # k x n int8
+    D: np.ndarray              # k float64
+    energy: np.ndarray         # k float64, incremental: 1 - ||R_i||^2 / ||A||^2
+    energy_final: float        # explicit 1 - ||A - Ahat||^2 / ||A||^2 at the end
+    norm_a2: float
+    margins: np.ndarray        # per component min relative threshold margin
+    safeguard_hits: int        # components whose decrease fell below max_rc R_rc^2
+    residual_norms: np.ndarray = field(default=None)  # ||R_i||^2 explicit, per component
+
+    @property
+    def k(self) -> int:
+        return self.D.shape[0]
+
+    def zero_fraction(self, upto: int | None = None) -> float:
+        kk = self.k if upto is None else upto
+        zb = np.count_nonzero(self.B[:, :kk] == 0)
+        zc = np.count_nonzero(self.C[:kk, :] == 0)
+        return (zb + zc) / ((self.B.shape[0] + self.C.shape[1]) * kk)
+
+
+def greedy_als(A: np.ndarray, k: int, tau: float, iters: int = 15, seed: int = 0,
+               track_residual: bool = False) -> Factorization:
+    """§2.3: greedy sequential ALS with deflation, in fp64."""
+    R = np.array(A, dtype=np.float64, copy=True)       # R <- A
+    m, n = R.shape
+    norm_a2 = float(np.sum(R * R))
+    if norm_a2 == 0.0:
+        raise ValueError("||A||_F = 0: energy is undefined")
+    B = np.zeros((m, k), dtype=np.int8)
+    C = np.zeros((k, n), dtype=np.int8)
+    D = np.zeros(k, dtype=np.float64)
+    energy = np.zeros(k, dtype=np.float64)
+    margins = np.zeros(k, dtype=np.float64)
+    res = np.zeros(k, dtype=np.float64) if track_residual else None
+    r2 = norm_a2
+    hits = 0
+    for i in range(k):
+        u0, _, _ = ternarize(start_normals(seed, i, m), tau)
+        fit = fit_component(R, u0, tau, iters)
+        # Appendix 7 reading: the single-entry component (one residual entry of
+        # largest magnitude) decreases ||R||^2 by max R_rc^2; count components
+        # where ALS did worse (the pages say this never happens in practice).
+        if fit.decrease < float(np.max(R * R)):
+            hits += 1
+        if fit.d != 0.0:
+            R -= fit.d * np.outer(fit.u.astype(np.float64), fit.v.astype(np.float64))
+        r2 -= fit.decrease
+        B[:, i] = fit.u
+        C[i, :] = fit.v
+        D[i] = fit.d
+        energy[i] = 1.0 - r2 / norm_a2
+        margins[i] = fit.min_margin
+        if track_residual:
+            res[i] = float(np.sum(R * R))
+    e_final = 1.0 - float(np.sum(R * R)) / norm_a2
+    return Factorization(B=B, C=C, D=D, energy=energy, energy_final=e_final, norm_a2=norm_a2,
+                         margins=margins, safeguard_hits=hits, residual_norms=res)
+
+
+def residual_after(A: np.ndarray, B: np.ndarray, D: np.ndarray, C: np.ndarray, upto: int) -> np.ndarray:
+    """R_i = A - sum_{j < upto} d_j b_j c_j^T in fp64 (teacher forcing from given factors)."""
+    Bf = np.asarray(B[:, :upto], dtype=np.float64)
+    Cf = np.asarray(C[:upto, :], dtype=np.float64)
+    return np.asarray(A, dtype=np.float64) - (Bf * np.asarray(D[:upto], dtype=np.float64)) @ Cf
+
+
+# ----------------------------------------------------------------------------
+# §2.1 reconstruction / energy, §2.6 Eq. (1)
+# ----------------------------------------------------------------------------
+
+
+def reconstruct(B: np.ndarray, D: np.ndarray, C: np.ndarray) -> np.ndarray:
+    """Ahat = B diag(D) C in fp64."""
+    return (np.asarray(B, dtype=np.float64) * np.asarray(D, dtype=np.float64)) @ np.asarray(C, dtype=np.float64)
+
+
+def energy(A: np.ndarray, Ahat: np.ndarray) -> float:
+    A = np.asarray(A, dtype=np.float64)
+    diff = A - np.asarray(Ahat, dtype=np.float64)
+    return 1.0 - float(np.sum(diff * diff)) / float(np.sum(A * A))
+
+
+def bpw_eff(mu: float, m: int, n: int, sparsity: float) -> float:
+    """§2.6 Eq. (1): mask+sign packing bits per original weight."""
+    return mu * (m + n) / max(m, n) * (2.0 - sparsity)
+
+
+def gaussian_zero_fraction(tau: float) -> float:
+    """P(|z| <= tau * E|z|) for z ~ N(0,1): 2 Phi(tau sqrt(2/pi)) - 1 = erf(tau / sqrt(pi))."""
+    return math.erf(tau / math.sqrt(math.pi))
