@@ -1,0 +1,172 @@
+/*
+ * externd.h -- C ABI of the B200 (sm_100a) library for ExTernD greedy
+ * sequential ternary ALS.
+ *
+ * Method: "ExTernD: Expanded-Rank Ternary Decomposition" (arXiv 2607.13511),
+ *   §2.1  A ~ Ahat = B diag(D) C, B in {-1,0,1}^{m x k}, C in {-1,0,1}^{k x n},
+ *         k = mu * min(m, n); energy E = 1 - ||A - Ahat||_F^2 / ||A||_F^2.
+ *   §2.2  T_tau(x)_i = sign(x_i) * 1[|x_i| > tau * mean_j |x_j|], keeping the
+ *         single largest entry when the result would be all-zero.
+ *   §2.3  R <- A; per component: 15 x {v <- T_tau(R^T u), u <- T_tau(R v)},
+ *         d = u^T R v / (||u||^2 ||v||^2), R <- R - d u v^T.
+ *
+ * Readings where the pages are silent (start vector, tie-breaks, k rounding)
+ * are fixed below and documented with the library.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Matrices are fp32, row-major, leading dimension = number of columns.
+ * - Pointers may be device memory or host memory (pageable or pinned); the
+ *   library detects which with cudaPointerGetAttributes.  Host buffers are
+ *   staged through device memory on `stream` (copies inside the call).
+ *   Device buffers of B/C rows must be 16-byte aligned.
+ * - `stream` is a cudaStream_t (NULL = legacy default stream) of the current
+ *   device.  Every call is stream-ordered and SYNCHRONOUS: it returns after
+ *   the work finished, because the return code carries the device status.
+ * - The library keeps no pointer after return.  Workspace (a copy of the
+ *   residual in two layouts, exchange buffers, start trits) is allocated
+ *   stream-ordered inside the call and released before it returns.
+ * - Ternary outputs are packed 2 bits per trit: 00 = 0, 01 = +1, 11 = -1
+ *   (10 is never written).  Trit j of a row sits in byte j/4, bits 2*(j%4).
+ *   A row of `len` trits occupies externd_trit_bytes(len) bytes (ceil(len/4)
+ *   rounded up to 16); padding trits are 0.
+ * - Start vector of component i (0-based): u0 = T_tau(z), z_j ~ N(0,1) for
+ *   j < m from Philox4x32-10 (Salmon et al., SC'11) with counter
+ *   (j, i, 1, 0) and key (seed & 0xffffffff, seed >> 32); two 53-bit uniforms
+ *   u1 = words (1:0), u2 = words (3:2), each ((w >> 11) + 0.5) * 2^-53;
+ *   z = sqrt(-2 ln u1) * cos(2 pi u2).
+ * - "15 iterations" = 15 (V-step, U-step) pairs; d uses the final u and the v
+ *   of the same pair.  T_tau's mean runs over the vector's own length.  The
+ *   all-zero fallback keeps the lowest index among the largest magnitudes;
+ *   an identically zero vector becomes +1 at index 0.  If u^T R v = 0 the
+ *   component is stored with d = 0 and R is unchanged.
+ */
+#ifndef EXTERND_H
+#define EXTERND_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    EXTERND_OK = 0,
+    EXTERND_EINVAL = -1,      /* null pointer, m or n < 1, non-finite mu/tau, tau < 0, iters < 1, k < 1, misaligned rows */
+    EXTERND_EZERO = -2,       /* ||A||_F = 0: the energy of §2.1 is undefined */
+    EXTERND_ENONFINITE = -3,  /* A (or R) holds NaN or Inf */
+    EXTERND_ENOMEM = -4,      /* workspace allocation failed */
+    EXTERND_ECUDA = -5,       /* a CUDA runtime call failed */
+    EXTERND_ELAUNCH = -6,     /* the cooperative ALS grid cannot be co-resident */
+    EXTERND_ETIMEOUT = -7,    /* a device-side wait gave up (limit per wait, default 2 s) */
+    EXTERND_ELIMIT = -8       /* shape beyond this build's limits (m + n too large for on-chip lists) */
+} externd_status;
+
+/* k = mu * min(m, n) rounded half away from zero (§2.1); -1 if m < 1, n < 1,
+ * mu is not finite, or the result is < 1. */
+int64_t externd_rank(int64_t m, int64_t n, double mu);
+
+/* Bytes of one packed trit row of length `len`: ceil(len/4) rounded up to 16.
+ * 0 for len < 1. */
+size_t externd_trit_bytes(int64_t len);
+
+/* Factor one matrix by greedy sequential ALS (§2.3).
+ *   A          [in]  m x n fp32 row-major; not modified.
+ *   mu, tau          inner-rank multiplier (k = externd_rank(m, n, mu)) and
+ *                    T_tau scale (finite, >= 0).
+ *   iters            alternating fits per component (the pages use 15), >= 1.
+ *   seed             start-vector seed (see conventions).
+ *   B_out      [out] k rows x externd_trit_bytes(m) bytes: row i = column i of B.
+ *   D_out      [out] k fp32 scales d_i.
+ *   C_out      [out] k rows x externd_trit_bytes(n) bytes: row i = row i of C.
+ *   energy_out [out] nullable; k doubles, E after component i, accumulated
+ *                    in fp64 from the exact decrease p_i^2 / (nnz(u_i) nnz(v_i)).
+ * Returns EXTERND_OK or a negative externd_status. */
+int externd_factor(const float* A, int64_t m, int64_t n, double mu, double tau, int iters,
+                   uint64_t seed, uint8_t* B_out, float* D_out, uint8_t* C_out,
+                   double* energy_out, void* stream);
+
+/* Factor `count` independent matrices in one cooperative launch; the SMs are
+ * split into groups and each group factors its matrices one after another.
+ * Every array argument has `count` entries (host arrays of pointers/values);
+ * energy_out may be NULL or hold NULL entries.  status_out[b] receives the
+ * status of matrix b; the return value is EXTERND_OK if all succeeded, else
+ * the first failing status (argument errors are reported before any work). */
+int externd_factor_batched(int count, const float* const* A, const int64_t* m, const int64_t* n,
+                           const double* mu, const double* tau, int iters, const uint64_t* seed,
+                           uint8_t* const* B_out, float* const* D_out, uint8_t* const* C_out,
+                           double* const* energy_out, int* status_out, void* stream);
+
+/* Ahat = B diag(D) C (§2.1) with fp64 accumulation, written as fp32 m x n
+ * row-major.  B, C packed as produced by externd_factor. */
+int externd_reconstruct(const uint8_t* B, const float* D, const uint8_t* C, int64_t m, int64_t n,
+                        int64_t k, float* A_hat_out, void* stream);
+
+/* Human-readable message for a status code (static storage). */
+const char* externd_strerror(int status);
+
+/* Test hook: ONE half-step of §2.3 step 1 on a caller-given residual, run by
+ * the same kernel code as externd_factor.
+ *   R          [in]  m x n fp32 row-major.
+ *   transpose        1: V-step x = R^T u (in_trits has m trits, outputs n);
+ *                    0: U-step y = R v   (in_trits has n trits, outputs m).
+ *   in_trits   [in]  packed trits (externd_trit_bytes(len_in) bytes).
+ *   tau              T_tau scale.
+ *   pre_out    [out] fp64 pre-threshold vector (len_out).
+ *   thresh_out [out] one double: tau * mean |pre|.
+ *   out_trits  [out] packed T_tau(pre) (externd_trit_bytes(len_out) bytes). */
+int externd_debug_halfstep(const float* R, int64_t m, int64_t n, int transpose,
+                           const uint8_t* in_trits, double tau, double* pre_out,
+                           double* thresh_out, uint8_t* out_trits, void* stream);
+
+/* Test hook: the packed start trits u0_i = T_tau(z_i) of components
+ * i = 0..k-1 for a matrix with m rows (see conventions), as used by
+ * externd_factor.  out: k rows x externd_trit_bytes(m) bytes. */
+int externd_debug_start_trits(int64_t m, int64_t k, double tau, uint64_t seed, uint8_t* out,
+                              void* stream);
+
+/* Knobs and extra outputs for externd_factor_ex.  Zero-initialise and set
+ * only what is needed. */
+typedef struct {
+    int grid;              /* CTAs per matrix; 0 = automatic */
+    int pending;           /* deflations held as rank-1 vector corrections before being folded into R; 0 = automatic */
+    double wait_limit_s;   /* limit of each device-side wait, seconds; 0 = 2.0 */
+    int fault_skip_cta;    /* test hook, used only if fault_inject != 0: this CTA never signals */
+    int fault_inject;
+    double* d64_out;       /* nullable: k fp64 scales */
+} externd_options;
+
+/* externd_factor with options (opt may be NULL). */
+int externd_factor_ex(const float* A, int64_t m, int64_t n, double mu, double tau, int iters,
+                      uint64_t seed, uint8_t* B_out, float* D_out, uint8_t* C_out,
+                      double* energy_out, void* stream, const externd_options* opt);
+
+/* Figures of the last call made by this host thread. */
+typedef struct {
+    double als_ms;             /* device time of the cooperative ALS kernel (CUDA events) */
+    double setup_ms;           /* residual layout copy + ||A||^2 */
+    double init_ms;            /* start-vector generation */
+    double total_ms;           /* all device work of the call, staging copies included */
+    double alg_bytes;          /* algorithmic bytes of the ALS kernel, summed over matrices */
+    double residual_energy;    /* 1 - ||R_k||^2 / ||A||^2 from the final fp32 residual (matrix 0) */
+    int64_t components;        /* components fitted, summed over matrices */
+    int64_t half_steps;        /* V- and U-steps executed, summed over matrices */
+    int64_t fallbacks;         /* T_tau all-zero fallbacks taken */
+    int launches;              /* kernels launched by the call */
+    int grid;                  /* CTAs of the ALS launch */
+    int group;                 /* CTAs per matrix */
+    int block;                 /* threads per CTA */
+    int vec_v, vec_u;          /* vector width of the two residual layouts */
+    int pending;               /* lazy-deflation depth used */
+    size_t smem_bytes;         /* dynamic shared memory per CTA */
+    size_t workspace_bytes;
+} externd_stats;
+
+int externd_last_stats(externd_stats* out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXTERND_H */

@@ -1,0 +1,263 @@
+"""Python binding of the ExTernD C ABI (include/externd.h).
+
+Argument marshalling only: tensors are turned into pointers, every step of the
+factorization runs in the CUDA library.  PyTorch provides device memory and
+streams.  Inputs may live on the GPU (device pointers) or on the host (the
+library stages them through device memory inside the call).
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass, field
+from typing import Optional, Sequence
+
+import numpy as np
+import torch
+
+from . import _lib
+
+
+class ExterndError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {strerror(status)} (status {status})")
+
+
+STATUS = {
+    "OK": 0, "EINVAL": -1, "EZERO": -2, "ENONFINITE": -3, "ENOMEM": -4,
+    "ECUDA": -5, "ELAUNCH": -6, "ETIMEOUT": -7, "ELIMIT": -8,
+}
+
+
+def strerror(status: int) -> str:
+    return _lib.load().externd_strerror(int(status)).decode()
+
+
+def rank(m: int, n: int, mu: float) -> int:
+    return int(_lib.load().externd_rank(int(m), int(n), float(mu)))
+
+
+def trit_bytes(length: int) -> int:
+    return int(_lib.load().externd_trit_bytes(int(length)))
+
+
+def last_stats() -> dict:
+    st = _lib.Stats()
+    _lib.load().externd_last_stats(ctypes.byref(st))
+    return st.as_dict()
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise ExterndError(rc, what)
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, torch.Tensor):
+        return t.data_ptr()
+    if isinstance(t, np.ndarray):
+        return t.ctypes.data
+    raise TypeError(type(t))
+
+
+def _stream(stream, device) -> int:
+    if stream is not None:
+        return int(getattr(stream, "cuda_stream", stream))
+    if device is not None and device.type == "cuda":
+        return torch.cuda.current_stream(device).cuda_stream
+    if torch.cuda.is_available():
+        return torch.cuda.current_stream().cuda_stream
+    return 0
+
+
+def _as_matrix(A) -> torch.Tensor:
+    if isinstance(A, np.ndarray):
+        A = torch.from_numpy(np.ascontiguousarray(A, dtype=np.float32))
+    if not isinstance(A, torch.Tensor) or A.dim() != 2:
+        raise ValueError("A must be a 2-D float32 tensor or array")
+    if A.dtype != torch.float32:
+        raise ValueError("A must be float32")
+    return A.contiguous()
+
+
+def _empty(shape, dtype, like: torch.Tensor) -> torch.Tensor:
+    if like.is_cuda:
+        return torch.empty(shape, dtype=dtype, device=like.device)
+    return torch.empty(shape, dtype=dtype, pin_memory=like.is_pinned())
+
+
+class _on_device:
+    def __init__(self, t: torch.Tensor):
+        self.ctx = torch.cuda.device(t.device) if t.is_cuda else None
+
+    def __enter__(self):
+        if self.ctx:
+            self.ctx.__enter__()
+
+    def __exit__(self, *a):
+        if self.ctx:
+            self.ctx.__exit__(*a)
+
+
+@dataclass
+class Factors:
+    """B diag(D) C with packed ternary rows (2 bits per trit)."""
+    B: torch.Tensor                 # uint8 [k, trit_bytes(m)]  row i = column i of B
+    D: torch.Tensor                 # float32 [k]
+    C: torch.Tensor                 # uint8 [k, trit_bytes(n)]  row i = row i of C
+    energy: Optional[torch.Tensor]  # float64 [k]
+    m: int
+    n: int
+    k: int
+    mu: float
+    tau: float
+    d64: Optional[torch.Tensor] = None
+    stats: dict = field(default_factory=dict)
+
+    def trits(self):
+        """Unpacked (B as m x k int8, C as k x n int8) on the host."""
+        Bu = unpack_trits(self.B.cpu().numpy(), self.m).T.copy()
+        Cu = unpack_trits(self.C.cpu().numpy(), self.n)
+        return Bu, Cu
+
+
+def factor(A, mu: float, tau: float, iters: int = 15, seed: int = 0, *, grid: int = 0, pending: int = 0,
+           wait_limit_s: float = 0.0, fault_skip_cta: Optional[int] = None, want_d64: bool = False,
+           want_energy: bool = True, stream=None) -> Factors:
+    """Factor one matrix (externd_factor_ex).  Outputs are allocated where A lives."""
+    A = _as_matrix(A)
+    m, n = A.shape
+    k = rank(m, n, mu)
+    if k < 1:
+        raise ExterndError(STATUS["EINVAL"], "externd_rank")
+    B = _empty((k, trit_bytes(m)), torch.uint8, A)
+    C = _empty((k, trit_bytes(n)), torch.uint8, A)
+    D = _empty((k,), torch.float32, A)
+    E = _empty((k,), torch.float64, A) if want_energy else None
+    d64 = _empty((k,), torch.float64, A) if want_d64 else None
+    opt = _lib.Options()
+    opt.grid = int(grid)
+    opt.pending = int(pending)
+    opt.wait_limit_s = float(wait_limit_s)
+    opt.fault_inject = 1 if fault_skip_cta is not None else 0
+    opt.fault_skip_cta = int(fault_skip_cta) if fault_skip_cta is not None else -1
+    opt.d64_out = _ptr(d64)
+    with _on_device(A):
+        rc = _lib.load().externd_factor_ex(_ptr(A), m, n, float(mu), float(tau), int(iters), int(seed),
+                                           _ptr(B), _ptr(D), _ptr(C), _ptr(E),
+                                           _stream(stream, A.device), ctypes.byref(opt))
+    _check(rc, "externd_factor")
+    return Factors(B=B, D=D, C=C, energy=E, m=m, n=n, k=k, mu=float(mu), tau=float(tau), d64=d64,
+                   stats=last_stats())
+
+
+def factor_batched(As: Sequence, mus: Sequence[float], taus: Sequence[float], iters: int = 15,
+                   seeds: Optional[Sequence[int]] = None, *, stream=None):
+    """Factor independent matrices in one launch (externd_factor_batched).
+
+    Returns (list of Factors, list of per-matrix status codes)."""
+    mats = [_as_matrix(a) for a in As]
+    cnt = len(mats)
+    if seeds is None:
+        seeds = list(range(cnt))
+    outs = []
+    for A, mu, tau in zip(mats, mus, taus):
+        m, n = A.shape
+        k = rank(m, n, mu)
+        if k < 1:
+            raise ExterndError(STATUS["EINVAL"], "externd_rank")
+        outs.append((_empty((k, trit_bytes(m)), torch.uint8, A), _empty((k,), torch.float32, A),
+                     _empty((k, trit_bytes(n)), torch.uint8, A), _empty((k,), torch.float64, A), k))
+    P = ctypes.c_void_p * cnt
+    a_ptrs = P(*[_ptr(a) for a in mats])
+    b_ptrs = P(*[_ptr(o[0]) for o in outs])
+    d_ptrs = P(*[_ptr(o[1]) for o in outs])
+    c_ptrs = P(*[_ptr(o[2]) for o in outs])
+    e_ptrs = P(*[_ptr(o[3]) for o in outs])
+    ms = (ctypes.c_int64 * cnt)(*[a.shape[0] for a in mats])
+    ns = (ctypes.c_int64 * cnt)(*[a.shape[1] for a in mats])
+    mu_a = (ctypes.c_double * cnt)(*[float(x) for x in mus])
+    tau_a = (ctypes.c_double * cnt)(*[float(x) for x in taus])
+    seed_a = (ctypes.c_uint64 * cnt)(*[int(s) for s in seeds])
+    st = (ctypes.c_int * cnt)()
+    with _on_device(mats[0]):
+        rc = _lib.load().externd_factor_batched(cnt, a_ptrs, ms, ns, mu_a, tau_a, int(iters), seed_a,
+                                                b_ptrs, d_ptrs, c_ptrs, e_ptrs, st,
+                                                _stream(stream, mats[0].device))
+    stats = last_stats()
+    res = []
+    for A, mu, tau, o in zip(mats, mus, taus, outs):
+        res.append(Factors(B=o[0], D=o[1], C=o[2], energy=o[3], m=A.shape[0], n=A.shape[1], k=o[4],
+                           mu=float(mu), tau=float(tau), stats=stats))
+    statuses = list(st)
+    if rc != 0 and all(s == 0 for s in statuses):
+        _check(rc, "externd_factor_batched")
+    return res, statuses
+
+
+def reconstruct(B: torch.Tensor, D: torch.Tensor, C: torch.Tensor, m: int, n: int, *, stream=None) -> torch.Tensor:
+    """Ahat = B diag(D) C as an m x n float32 tensor on B's device."""
+    k = D.shape[0]
+    out = _empty((m, n), torch.float32, B)
+    with _on_device(B):
+        rc = _lib.load().externd_reconstruct(_ptr(B), _ptr(D), _ptr(C), int(m), int(n), int(k), _ptr(out),
+                                             _stream(stream, B.device))
+    _check(rc, "externd_reconstruct")
+    return out
+
+
+def debug_halfstep(R, trits_in: torch.Tensor, tau: float, transpose: bool, *, stream=None):
+    """One V-step (transpose=True: x = R^T u) or U-step (y = R v) through the ALS kernel.
+
+    Returns (pre-threshold fp64 vector, threshold, packed output trits)."""
+    R = _as_matrix(R)
+    m, n = R.shape
+    lout = n if transpose else m
+    pre = _empty((lout,), torch.float64, R)
+    thr = _empty((1,), torch.float64, R)
+    out = _empty((trit_bytes(lout),), torch.uint8, R)
+    with _on_device(R):
+        rc = _lib.load().externd_debug_halfstep(_ptr(R), m, n, 1 if transpose else 0, _ptr(trits_in), float(tau),
+                                                _ptr(pre), _ptr(thr), _ptr(out), _stream(stream, R.device))
+    _check(rc, "externd_debug_halfstep")
+    return pre, float(thr[0].item()), out
+
+
+def debug_start_trits(m: int, k: int, tau: float, seed: int, device="cuda", *, stream=None) -> torch.Tensor:
+    """Packed start trits of components 0..k-1 (k x trit_bytes(m)), generated on the GPU."""
+    out = torch.empty((k, trit_bytes(m)), dtype=torch.uint8, device=device)
+    with _on_device(out):
+        rc = _lib.load().externd_debug_start_trits(int(m), int(k), float(tau), int(seed), _ptr(out),
+                                                   _stream(stream, out.device))
+    _check(rc, "externd_debug_start_trits")
+    return out
+
+
+# ---------------------------------------------------------------------------
+# host codecs of the packed 2-bit format: 00 = 0, 01 = +1, 11 = -1
+# ---------------------------------------------------------------------------
+
+def unpack_trits(packed: np.ndarray, length: int) -> np.ndarray:
+    """uint8 rows (..., nbytes) -> int8 (..., length)."""
+    p = np.asarray(packed, dtype=np.uint8)
+    shifts = np.array([0, 2, 4, 6], dtype=np.uint8)
+    codes = (p[..., :, None] >> shifts) & 3
+    codes = codes.reshape(*p.shape[:-1], p.shape[-1] * 4)[..., :length]
+    out = np.zeros(codes.shape, dtype=np.int8)
+    out[codes == 1] = 1
+    out[codes == 3] = -1
+    return out
+
+
+def pack_trits(t: np.ndarray) -> np.ndarray:
+    """int8 (..., length) in {-1, 0, 1} -> uint8 (..., trit_bytes(length))."""
+    t = np.asarray(t, dtype=np.int8)
+    length = t.shape[-1]
+    nb = trit_bytes(length)
+    codes = np.zeros((*t.shape[:-1], nb * 4), dtype=np.uint8)
+    codes[..., :length][t == 1] = 1
+    codes[..., :length][t == -1] = 3
+    codes = codes.reshape(*t.shape[:-1], nb, 4)
+    return (codes[..., 0] | (codes[..., 1] << 2) | (codes[..., 2] << 4) | (codes[..., 3] << 6)).astype(np.uint8)

@@ -1,0 +1,299 @@
+// Device code of the ExTernD greedy sequential ALS library (sm_100a).
+//
+// Method: "ExTernD: Expanded-Rank Ternary Decomposition" (arXiv 2607.13511)
+// §2.2 (T_tau) and §2.3 (greedy sequential ALS: alternating ternary fits,
+// closed-form scale, rank-1 deflation).
+//
+// Design (B200):
+//  * One persistent cooperative launch runs every component of a matrix.  A
+//    matrix is served by a group of G CTAs (one per SM, 512 threads each).
+//  * The residual R is kept twice in HBM, each copy cut into one private block
+//    per CTA so that both half-steps read only what they need and no CTA ever
+//    reads another CTA's residual:
+//      V-layout: CTA q owns a stripe of columns [c0, c1) of R, stored as an
+//                m x pitch row-major block.  V-step x = R^T u reads only the
+//                rows r with u_r != 0 and produces x over its own columns.
+//      U-layout: CTA q owns a stripe of rows [r0, r1) of R, stored as an
+//                n x pitch block (column c of R restricted to the stripe is
+//                contiguous).  U-step y = R v reads only the columns with
+//                v_c != 0 and produces y over its own rows.
+//    So each half-step needs no cross-CTA reduction of vectors, only the
+//    scalar sum of |x| for the threshold: every CTA publishes its slice of the
+//    output and its partial sum, meets the others at one counter, then reads
+//    the whole vector back and thresholds it itself (all CTAs derive the
+//    identical trit vector because they use the same data in the same order).
+//  * Deflation is lazy: the last L components (d_j, u_j, v_j) are held as
+//    bit masks in shared memory and applied as rank-1 corrections to each
+//    GEMV output (x -= sum_j d_j (u_j . u) v_j); every L components each CTA
+//    folds them into its own two blocks in one pass (fp64 sum, one fp32
+//    rounding per entry).
+//  * All accumulation is fp64 (each fp32 residual entry is added exactly), so
+//    threshold decisions are taken on fp64 values like the fp64 oracle.
+//  * Every device-side wait is bounded by %globaltimer; a wait that runs out
+//    raises a status word and the kernel returns.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace externd {
+
+constexpr int NT = 512;               // threads per CTA of the ALS kernel
+constexpr int NWARP = NT / 32;
+constexpr int MAX_PENDING = 32;       // lazy deflation depth cap
+constexpr unsigned FULL = 0xffffffffu;
+
+// Status codes written by kernels (mirror externd_status).
+constexpr int ST_OK = 0;
+constexpr int ST_EZERO = -2;
+constexpr int ST_ENONFINITE = -3;
+constexpr int ST_ETIMEOUT = -7;
+constexpr int ST_RUNNING = 1;         // set by the host before launch
+
+// Balanced split of `len` indices into G stripes made of `vec`-wide units.
+struct Part {
+    int64_t len;
+    int64_t units;    // ceil(len / vec)
+    int vec;
+    int G;
+    __host__ __device__ int64_t ustart(int q) const { return ((int64_t)q * units) / G; }
+    __host__ __device__ int64_t start(int q) const { int64_t s = ustart(q) * vec; return s < len ? s : len; }
+    __host__ __device__ int64_t end(int q) const { int64_t e = ustart(q + 1) * vec; return e < len ? e : len; }
+    __host__ __device__ int pitch(int q) const { return (int)((ustart(q + 1) - ustart(q)) * vec); }
+    // stripe holding index i: the largest q with ustart(q) <= i / vec
+    __host__ __device__ int owner(int64_t i) const {
+        int64_t u = i / vec;
+        return (int)(((u + 1) * (int64_t)G - 1) / units);
+    }
+    // element offset of stripe q's block when the other dimension has `other` entries
+    __host__ __device__ int64_t block_offset(int q, int64_t other) const { return other * vec * ustart(q); }
+    __host__ __device__ int64_t total(int64_t other) const { return other * vec * units; }
+};
+
+struct Slot {                 // one CTA's published scalars for one half-step
+    double S;                 // sum |out| over its stripe
+    double M;                 // max |out| over its stripe (-1 if empty)
+    long long J;              // lowest index attaining M
+    long long pad;
+};
+
+struct GroupSync {            // one per CTA group, 128 B apart
+    unsigned arrive;
+    int abort;
+    unsigned pad[30];
+};
+
+struct DevStats {
+    unsigned long long sum_nu;      // rows read by V-steps
+    unsigned long long sum_nv;      // columns read by U-steps
+    unsigned long long sum_nunv;    // sum nnz(u_i) nnz(v_i)
+    unsigned long long half_steps;
+    unsigned long long fallbacks;
+    double residual2;               // ||R_k||^2 from the final fp32 residual
+    double norm_a2;
+    double pad;
+};
+
+enum Mode { MODE_FACTOR = 0, MODE_HALF_V = 1, MODE_HALF_U = 2 };
+
+struct Prob {
+    const float* A;
+    int64_t m, n, k;
+    double tau;
+    int iters;
+    int mode;
+    uint64_t seed;
+    uint8_t* B;               // k rows of b_bytes
+    float* D;
+    uint8_t* C;               // k rows of c_bytes
+    double* energy;           // nullable
+    double* d64;              // nullable
+    int64_t b_bytes, c_bytes;
+    float* Rv;                // V-layout blocks
+    float* Ru;                // U-layout blocks
+    double* xbuf;             // n, published V-step outputs
+    double* ybuf;             // m, published U-step outputs
+    const uint32_t* start;    // start trits (k rows of start_words) or debug input (1 row)
+    int64_t start_words;
+    double* norm_part;        // per setup-tile partial sums of A^2
+    int64_t n_norm_part;
+    unsigned* nonfinite;
+    int* status;
+    DevStats* stats;
+    double* pre_out;          // debug half-step outputs
+    double* thr_out;
+    uint8_t* trit_out;
+    Part pv;                  // column stripes (len n)
+    Part pu;                  // row stripes (len m)
+};
+
+struct KCfg {
+    const Prob* probs;
+    int nprob;
+    int Gg;                   // CTAs per group
+    int NG;                   // groups
+    GroupSync* gsync;         // NG
+    Slot* slots;              // NG x 2 x Gg
+    int Lcap;                 // lazy deflation depth
+    int m_max, n_max;         // for shared-memory carving
+    uint64_t limit_ns;
+    int fault_skip;           // CTA rank (within group) that never arrives; -1 = off
+};
+
+// ---------------------------------------------------------------------------
+// small helpers
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint64_t gtimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ int ld_relaxed_s32(const int* p) {
+    int v;
+    asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// bits 0,2,4,...,30 of x -> bits 0..15
+__host__ __device__ __forceinline__ uint32_t compact_even(uint32_t x) {
+    x &= 0x55555555u;
+    x = (x | (x >> 1)) & 0x33333333u;
+    x = (x | (x >> 2)) & 0x0F0F0F0Fu;
+    x = (x | (x >> 4)) & 0x00FF00FFu;
+    x = (x | (x >> 8)) & 0x0000FFFFu;
+    return x;
+}
+
+// bits 0..15 of x -> bits 0,2,...,30
+__host__ __device__ __forceinline__ uint32_t spread_even(uint32_t x) {
+    x &= 0x0000FFFFu;
+    x = (x | (x << 8)) & 0x00FF00FFu;
+    x = (x | (x << 4)) & 0x0F0F0F0Fu;
+    x = (x | (x << 2)) & 0x33333333u;
+    x = (x | (x << 1)) & 0x55555555u;
+    return x;
+}
+
+__device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
+__device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
+
+// Block-wide fp64 sum with a fixed combination order (same inputs -> same bits).
+__device__ __forceinline__ double block_sum(double v, double* sh) {
+    #pragma unroll
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
+    if (lane_id() == 0) sh[warp_id()] = v;
+    __syncthreads();
+    if (warp_id() == 0) {
+        double w = lane_id() < NWARP ? sh[lane_id()] : 0.0;
+        #pragma unroll
+        for (int o = 16; o; o >>= 1) w += __shfl_xor_sync(FULL, w, o);
+        if (lane_id() == 0) sh[NWARP] = w;
+    }
+    __syncthreads();
+    double r = sh[NWARP];
+    __syncthreads();
+    return r;
+}
+
+// max |.| with the lowest index on ties
+__device__ __forceinline__ void maxloc_merge(double& m, long long& j, double m2, long long j2) {
+    if (m2 > m || (m2 == m && j2 < j)) { m = m2; j = j2; }
+}
+
+__device__ __forceinline__ void block_maxloc(double& m, long long& j, double* shm, long long* shj) {
+    #pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        double m2 = __shfl_xor_sync(FULL, m, o);
+        long long j2 = __shfl_xor_sync(FULL, j, o);
+        maxloc_merge(m, j, m2, j2);
+    }
+    if (lane_id() == 0) { shm[warp_id()] = m; shj[warp_id()] = j; }
+    __syncthreads();
+    if (warp_id() == 0) {
+        double mm = lane_id() < NWARP ? shm[lane_id()] : -1.0;
+        long long jj = lane_id() < NWARP ? shj[lane_id()] : (long long)0x7fffffffffffffffLL;
+        #pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            double m2 = __shfl_xor_sync(FULL, mm, o);
+            long long j2 = __shfl_xor_sync(FULL, jj, o);
+            maxloc_merge(mm, jj, m2, j2);
+        }
+        if (lane_id() == 0) { shm[NWARP] = mm; shj[NWARP] = jj; }
+    }
+    __syncthreads();
+    m = shm[NWARP];
+    j = shj[NWARP];
+    __syncthreads();
+}
+
+// Exclusive scan of a[0..W) in place; returns the total.  sh: NWARP+1 ints.
+__device__ int block_exclusive_scan(int* a, int W, int* sh) {
+    const int per = (W + NT - 1) / NT;
+    const int b = threadIdx.x * per;
+    const int e = min(W, b + per);
+    int s = 0;
+    for (int i = b; i < e; ++i) s += a[i];
+    int incl = s;
+    #pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int t = __shfl_up_sync(FULL, incl, o);
+        if (lane_id() >= o) incl += t;
+    }
+    if (lane_id() == 31) sh[warp_id()] = incl;
+    __syncthreads();
+    if (warp_id() == 0) {
+        int v = lane_id() < NWARP ? sh[lane_id()] : 0;
+        int inc = v;
+        #pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int t = __shfl_up_sync(FULL, inc, o);
+            if (lane_id() >= o) inc += t;
+        }
+        if (lane_id() < NWARP) sh[lane_id()] = inc - v;
+        if (lane_id() == NWARP - 1) sh[NWARP] = inc;
+    }
+    __syncthreads();
+    int run = sh[warp_id()] + incl - s;
+    for (int i = b; i < e; ++i) { int c = a[i]; a[i] = run; run += c; }
+    const int total = sh[NWARP];
+    __syncthreads();
+    return total;
+}
+
+// ---------------------------------------------------------------------------
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11) and Box-Muller start normals
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void philox4x32_10(uint32_t c[4], uint32_t k0, uint32_t k1) {
+    #pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        if (r > 0) { k0 += 0x9E3779B9u; k1 += 0xBB67AE85u; }
+        const uint32_t hi0 = __umulhi(0xD2511F53u, c[0]);
+        const uint32_t lo0 = 0xD2511F53u * c[0];
+        const uint32_t hi1 = __umulhi(0xCD9E8D57u, c[2]);
+        const uint32_t lo1 = 0xCD9E8D57u * c[2];
+        const uint32_t n0 = hi1 ^ c[1] ^ k0;
+        const uint32_t n2 = hi0 ^ c[3] ^ k1;
+        c[0] = n0; c[1] = lo1; c[2] = n2; c[3] = lo0;
+    }
+}
+
+__device__ __forceinline__ double start_normal(uint64_t seed, uint32_t comp, uint32_t j) {
+    uint32_t c[4] = {j, comp, 1u, 0u};
+    philox4x32_10(c, (uint32_t)(seed & 0xffffffffu), (uint32_t)(seed >> 32));
+    const uint64_t w1 = ((uint64_t)c[1] << 32) | c[0];
+    const uint64_t w2 = ((uint64_t)c[3] << 32) | c[2];
+    const double u1 = ((double)(w1 >> 11) + 0.5) * 0x1.0p-53;
+    const double u2 = ((double)(w2 >> 11) + 0.5) * 0x1.0p-53;
+    return sqrt(-2.0 * log(u1)) * cos(6.283185307179586 * u2);
+}
+
+}  // namespace externd

@@ -1,0 +1,86 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every
+symbol declared in include/externd.h, and its pure host functions and argument
+validation behave as documented."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import ternary_rank_weight_b200 as ext
+from ternary_rank_weight_b200 import _lib
+from oracle import externd_oracle as ora
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    src = open(os.path.join(ROOT, "include", "externd.h")).read()
+    return sorted(set(re.findall(r"\b(externd_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = _lib.load()
+    declared = _declared_symbols()
+    assert declared, "no declarations found"
+    for name in declared:
+        assert hasattr(L, name), name
+    assert set(declared) == set(_lib.EXPORTS)
+
+
+def test_rank_matches_oracle_rounding():
+    for m, n, mu in [(256, 256, 2.0), (2560, 6912, 3.0), (1536, 1536, 2.5), (4096, 4096, 3.5),
+                     (3, 5, 0.5), (3, 5, 0.1), (7, 9, 1.2345), (1, 1, 1.0), (0, 5, 1.0), (5, 5, float("nan"))]:
+        assert ext.rank(m, n, mu) == ora.rank(m, n, mu), (m, n, mu)
+
+
+def test_trit_bytes():
+    assert ext.trit_bytes(0) == 0
+    assert ext.trit_bytes(1) == 16
+    assert ext.trit_bytes(64) == 16
+    assert ext.trit_bytes(65) == 32
+    assert ext.trit_bytes(2560) == 640
+    assert ext.trit_bytes(6912) == 1728
+
+
+def test_trit_codec_round_trip_and_layout():
+    rng = np.random.default_rng(0)
+    for length in (1, 3, 4, 5, 63, 64, 65, 1000):
+        t = rng.integers(-1, 2, size=(3, length)).astype(np.int8)
+        p = ext.pack_trits(t)
+        assert p.shape == (3, ext.trit_bytes(length))
+        assert np.array_equal(ext.unpack_trits(p, length), t)
+    # trit j in byte j/4, bits 2*(j%4); 01 = +1, 11 = -1
+    p = ext.pack_trits(np.array([[1, 0, -1, 1, -1]], dtype=np.int8))
+    assert p[0, 0] == 0b01_11_00_01 and p[0, 1] == 0b11
+    assert np.all(p[0, 2:] == 0)
+
+
+def test_status_strings():
+    for s in range(-8, 1):
+        assert ext.strerror(s) and ext.strerror(s) != "unknown status"
+
+
+def test_argument_validation_before_any_device_work():
+    L = _lib.load()
+    buf = (ctypes.c_uint8 * 64)()
+    A = (ctypes.c_float * 4)(1, 2, 3, 4)
+    args_ok = dict(A=ctypes.addressof(A), m=2, n=2, mu=1.0, tau=0.7, iters=15)
+    def call(**kw):
+        a = dict(args_ok, **kw)
+        return L.externd_factor(a["A"], a["m"], a["n"], a["mu"], a["tau"], a["iters"], 0,
+                                ctypes.addressof(buf), ctypes.addressof(buf), ctypes.addressof(buf), None, None)
+    einval = ext.STATUS["EINVAL"]
+    assert call(A=None) == einval
+    assert call(m=0) == einval
+    assert call(n=-3) == einval
+    assert call(iters=0) == einval
+    assert call(tau=-0.1) == einval
+    assert call(tau=float("inf")) == einval
+    assert call(mu=float("nan")) == einval
+    assert call(mu=0.1) == einval            # k rounds to 0
+    assert L.externd_reconstruct(None, None, None, 1, 1, 1, None, None) == einval
+    assert L.externd_debug_halfstep(None, 1, 1, 1, None, 0.7, None, None, None, None) == einval
+    assert L.externd_factor_batched(0, None, None, None, None, None, 15, None, None, None, None, None, None,
+                                    None) == einval

@@ -1,0 +1,271 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Tolerances (from the factorization's arithmetic and the fixed acceptance bar):
+* trits: bit-exact, except entries whose pre-threshold magnitude lies within
+  1e-5 relative of the threshold (a threshold tie: both sides decide in fp64,
+  but sum in different orders and the GPU residual is fp32-rounded);
+* pre-threshold vectors on a shared residual: 1e-12 relative to sum |terms|
+  (fp64 accumulation of exactly-representable fp32 terms);
+* scale d_i: 1e-4 relative; energy E: 2e-3 absolute; zero fraction: 0.5
+  percentage points.  Trajectories may diverge after a tie; divergences are
+  counted and must be explained by a near-tie on the oracle side.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import ternary_rank_weight_b200 as ext
+from oracle import externd_oracle as ora
+from ternary_rank_weight_b200.workloads import WORKLOADS, iid_matrix, llm_matrix
+
+pytestmark = pytest.mark.gpu
+
+TIE = 1e-5
+
+
+def _trits_equal_modulo_ties(got, want, pre, thr):
+    bad = np.nonzero(got != want)[0]
+    if bad.size == 0:
+        return True, 0
+    near = np.abs(np.abs(pre[bad]) - thr) <= TIE * max(thr, 1e-300)
+    return bool(np.all(near)), int(bad.size)
+
+
+# ---------------------------------------------------------------------------
+# start vectors
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("m,k,tau,seed", [(1, 3, 0.7, 0), (5, 4, 2.0, 1), (256, 16, 0.7, 0),
+                                          (1000, 8, 1.0, 7), (4096, 4, 0.7, (1 << 40) + 3)])
+def test_start_trits_match_oracle(m, k, tau, seed):
+    got = ext.unpack_trits(ext.debug_start_trits(m, k, tau, seed).cpu().numpy(), m)
+    for i in range(k):
+        z = ora.start_normals(seed, i, m)
+        want, thr, _ = ora.ternarize(z, tau)
+        ok, nbad = _trits_equal_modulo_ties(got[i], want, z, thr)
+        assert ok, (i, nbad)
+
+
+# ---------------------------------------------------------------------------
+# one half-step on a shared residual
+# ---------------------------------------------------------------------------
+
+HALF_SHAPES = [(1, 1), (1, 9), (9, 1), (7, 5), (33, 65), (300, 517), (1024, 2048), (2560, 6912)]
+
+
+@pytest.mark.parametrize("m,n", HALF_SHAPES)
+@pytest.mark.parametrize("transpose", [True, False])
+def test_halfstep_matches_oracle(m, n, transpose):
+    rng = np.random.default_rng(m * 131 + n)
+    R = (rng.standard_normal((m, n)) * 0.02).astype(np.float32)
+    Rg = torch.from_numpy(R).cuda()
+    lin = m if transpose else n
+    for tau in (0.0, 0.7, 1.0, 2.0, 50.0):
+        t_in = rng.integers(-1, 2, size=lin).astype(np.int8)
+        packed = torch.from_numpy(ext.pack_trits(t_in)).cuda()
+        pre, thr, out = ext.debug_halfstep(Rg, packed, tau, transpose)
+        pre = pre.cpu().numpy()
+        got = ext.unpack_trits(out.cpu().numpy(), n if transpose else m)
+        want_pre, want_thr, want, _ = ora.half_step(R, t_in, tau, transpose)
+        scale = (np.abs(R).T @ np.abs(t_in) if transpose else np.abs(R) @ np.abs(t_in)) + 1e-300
+        assert np.all(np.abs(pre - want_pre) <= 1e-12 * scale + 1e-300)
+        assert thr == pytest.approx(want_thr, rel=1e-12, abs=1e-300)
+        ok, nbad = _trits_equal_modulo_ties(got, want, want_pre, want_thr)
+        assert ok, (tau, nbad)
+
+
+def test_halfstep_zero_input_and_zero_residual_take_the_fallback():
+    R = np.zeros((6, 10), dtype=np.float32)
+    for transpose in (True, False):
+        lin = 6 if transpose else 10
+        packed = torch.from_numpy(ext.pack_trits(np.zeros(lin, dtype=np.int8))).cuda()
+        pre, thr, out = ext.debug_halfstep(torch.from_numpy(R).cuda(), packed, 0.7, transpose)
+        got = ext.unpack_trits(out.cpu().numpy(), 10 if transpose else 6)
+        assert thr == 0.0 and np.all(pre.cpu().numpy() == 0)
+        assert got[0] == 1 and np.count_nonzero(got) == 1     # x == 0 -> +1 at index 0
+
+
+# ---------------------------------------------------------------------------
+# whole factorizations
+# ---------------------------------------------------------------------------
+
+def _run_pair(A, mu, tau, seed, iters=15, **kw):
+    f = ext.factor(torch.from_numpy(A).cuda(), mu, tau, iters=iters, seed=seed, want_d64=True, **kw)
+    Bg, Cg = f.trits()
+    ref = ora.greedy_als(A, k=f.k, tau=tau, iters=iters, seed=seed)
+    return f, Bg, Cg, ref
+
+
+def _first_divergence(Bg, Cg, ref):
+    k = ref.k
+    for i in range(k):
+        if not (np.array_equal(Bg[:, i], ref.B[:, i]) and np.array_equal(Cg[i], ref.C[i])):
+            return i
+    return k
+
+
+def _zero_fraction(B, C):
+    return (np.count_nonzero(B == 0) + np.count_nonzero(C == 0)) / (B.size + C.size)
+
+
+def _check_end_to_end(f, Bg, Cg, ref):
+    e = f.energy.cpu().numpy()
+    assert np.all(np.diff(e) >= -1e-12), "energy must not decrease"
+    assert np.max(np.abs(e - ref.energy)) < 2e-3
+    assert abs(_zero_fraction(Bg, Cg) - ref.zero_fraction()) < 0.005
+    div = _first_divergence(Bg, Cg, ref)
+    d64 = f.d64.cpu().numpy()
+    if div > 0:
+        assert np.allclose(d64[:div], ref.D[:div], rtol=1e-4, atol=0)
+    if div < ref.k:
+        # a divergence must start at a near-tie on the oracle's trajectory
+        assert ref.margins[div] < 1e-3, (div, ref.margins[div])
+    # the incremental energy matches the explicit residual of the fp32 factorization
+    assert f.stats["residual_energy"] == pytest.approx(e[-1], abs=1e-5)
+    return div
+
+
+@pytest.mark.parametrize("grid,pending", [(0, 0), (1, 1), (3, 4), (8, 32)])
+def test_small_iid_workload_matches_oracle(grid, pending):
+    w = WORKLOADS["iid_256x256_mu2_tau0.7"]
+    A = w.matrix(0)
+    f, Bg, Cg, ref = _run_pair(A, w.mu[0], w.tau[0], w.seeds[0], grid=grid, pending=pending)
+    assert f.k == 512
+    div = _check_end_to_end(f, Bg, Cg, ref)
+    assert div >= 16, div
+
+
+@pytest.mark.parametrize("m,n,mu,tau", [(1, 1, 1.0, 0.7), (1, 7, 1.0, 0.7), (7, 1, 2.0, 1.0), (7, 5, 3.0, 0.7),
+                                        (33, 65, 1.5, 1.0), (65, 33, 1.5, 2.0), (129, 250, 1.0, 0.7)])
+def test_ragged_shapes_match_oracle(m, n, mu, tau):
+    A = llm_matrix(m, n, seed=m + n, outliers=min(2, n))
+    f, Bg, Cg, ref = _run_pair(A, mu, tau, seed=3, grid=min(3, m, n))
+    _check_end_to_end(f, Bg, Cg, ref)
+
+
+def test_rank_one_ternary_matrix_is_recovered_exactly():
+    rng = np.random.default_rng(1)
+    u = rng.choice([-1, 0, 1], size=40, p=[0.35, 0.3, 0.35]).astype(np.float64)
+    v = rng.choice([-1, 0, 1], size=24, p=[0.35, 0.3, 0.35]).astype(np.float64)
+    A = (0.125 * np.outer(u, v)).astype(np.float32)
+    seed = next(s for s in range(50)
+                if ora.ternarize(ora.start_normals(s, 0, 40), 0.7)[0].astype(np.float64) @ u != 0)
+    f = ext.factor(torch.from_numpy(A).cuda(), 1.0 / 24, 0.7, seed=seed, want_d64=True)
+    Bg, Cg = f.trits()
+    assert np.array_equal(f.d64[0].item() * np.outer(Bg[:, 0], Cg[0]), 0.125 * np.outer(u, v))
+    assert f.energy[0].item() == pytest.approx(1.0, abs=1e-12)
+
+
+def test_teacher_forced_components_match_oracle():
+    """Oracle rebuilds R_i from the GPU's own factors and refits component i."""
+    A = llm_matrix(192, 320, seed=11)
+    f = ext.factor(torch.from_numpy(A).cuda(), 2.0, 1.0, seed=4, want_d64=True, grid=5, pending=7)
+    Bg, Cg = f.trits()
+    d64 = f.d64.cpu().numpy()
+    mism = 0
+    checked = 0
+    for i in list(range(0, 24)) + list(range(100, 384, 37)):
+        R = ora.residual_after(A, Bg, d64, Cg, i)
+        u0, _, _ = ora.ternarize(ora.start_normals(4, i, 192), 1.0)
+        fit = ora.fit_component(R, u0, 1.0, 15)
+        checked += 1
+        if np.array_equal(fit.u, Bg[:, i]) and np.array_equal(fit.v, Cg[i]):
+            assert d64[i] == pytest.approx(fit.d, rel=1e-4)
+        else:
+            mism += 1
+            assert fit.min_margin < 1e-3, (i, fit.min_margin)
+    assert mism <= max(1, checked // 10)
+
+
+def test_reconstruct_matches_oracle_and_energy():
+    A = llm_matrix(300, 200, seed=2)
+    f = ext.factor(torch.from_numpy(A).cuda(), 1.5, 0.7, seed=1)
+    Ah = ext.reconstruct(f.B, f.D, f.C, f.m, f.n).cpu().numpy()
+    Bg, Cg = f.trits()
+    want = ora.reconstruct(Bg, f.D.cpu().numpy().astype(np.float64), Cg)
+    assert np.allclose(Ah, want, rtol=1e-6, atol=1e-7 * np.abs(want).max())
+    e_explicit = ora.energy(A, Ah)
+    assert e_explicit == pytest.approx(f.energy[-1].item(), abs=1e-4)
+
+
+def test_host_buffers_give_the_same_result_as_device_buffers():
+    A = llm_matrix(160, 96, seed=8)
+    fd = ext.factor(torch.from_numpy(A).cuda(), 1.0, 0.7, seed=2)
+    fh = ext.factor(torch.from_numpy(A).pin_memory(), 1.0, 0.7, seed=2)
+    assert fh.B.device.type == "cpu"
+    assert torch.equal(fd.B.cpu(), fh.B) and torch.equal(fd.C.cpu(), fh.C) and torch.equal(fd.D.cpu(), fh.D)
+    fp = ext.factor(A, 1.0, 0.7, seed=2)                 # pageable numpy input
+    assert torch.equal(fd.B.cpu(), fp.B)
+
+
+def test_batched_equals_single_calls_with_the_same_group_size():
+    mats = [llm_matrix(200, 150, seed=20), iid_matrix(96, 300, seed=21), llm_matrix(250, 250, seed=22),
+            llm_matrix(64, 80, seed=23)]
+    mus = [1.5, 1.0, 2.0, 2.5]
+    taus = [0.7, 1.0, 2.0, 0.7]
+    seeds = [5, 6, 7, 8]
+    res, st = ext.factor_batched([torch.from_numpy(a).cuda() for a in mats], mus, taus, seeds=seeds)
+    assert st == [0, 0, 0, 0]
+    G = res[0].stats["group"]
+    for A, mu, tau, sd, r in zip(mats, mus, taus, seeds, res):
+        f = ext.factor(torch.from_numpy(A).cuda(), mu, tau, seed=sd, grid=G)
+        assert torch.equal(f.B, r.B) and torch.equal(f.C, r.C) and torch.equal(f.D, r.D)
+        assert torch.equal(f.energy, r.energy)
+
+
+def test_errors_zero_and_nonfinite():
+    with pytest.raises(ext.ExterndError) as e:
+        ext.factor(torch.zeros(8, 8, device="cuda"), 1.0, 0.7)
+    assert e.value.status == ext.STATUS["EZERO"]
+    A = torch.randn(8, 8, device="cuda")
+    A[3, 4] = float("nan")
+    with pytest.raises(ext.ExterndError) as e:
+        ext.factor(A, 1.0, 0.7)
+    assert e.value.status == ext.STATUS["ENONFINITE"]
+    A[3, 4] = float("inf")
+    with pytest.raises(ext.ExterndError) as e:
+        ext.factor(A, 1.0, 0.7)
+    assert e.value.status == ext.STATUS["ENONFINITE"]
+
+
+def test_bounded_wait_reports_timeout_and_context_stays_usable():
+    """A CTA that never signals (host-set test flag): the others' waits run out."""
+    A = torch.from_numpy(llm_matrix(256, 256, seed=3)).cuda()
+    with pytest.raises(ext.ExterndError) as e:
+        ext.factor(A, 1.0, 0.7, grid=4, fault_skip_cta=2, wait_limit_s=0.2)
+    assert e.value.status == ext.STATUS["ETIMEOUT"]
+    f = ext.factor(A, 1.0, 0.7, grid=4)
+    assert f.energy[-1].item() > 0.5
+
+
+# ---------------------------------------------------------------------------
+# full size: the headline workload in the launch configuration the bench times
+# ---------------------------------------------------------------------------
+
+def test_headline_workload_full_size_sampled_parity():
+    w = WORKLOADS["mlp_2560x6912_bf16_mu3_tau1.0"]
+    A = w.matrix(0)
+    f = ext.factor(torch.from_numpy(A).cuda(), w.mu[0], w.tau[0], seed=w.seeds[0], want_d64=True)
+    assert f.k == 7680
+    e = f.energy.cpu().numpy()
+    assert np.all(np.diff(e) >= -1e-12)
+    assert f.stats["residual_energy"] == pytest.approx(e[-1], abs=1e-4)
+    assert 0.5 < e[-1] < 1.0
+    Bg, Cg = f.trits()
+    zf = _zero_fraction(Bg, Cg)
+    assert abs(zf - ora.gaussian_zero_fraction(1.0)) < 0.05
+    d64 = f.d64.cpu().numpy()
+    mism = 0
+    samples = [0, 1, 2, 57, 1000, 4097, 7679]
+    for i in samples:
+        R = ora.residual_after(A, Bg, d64, Cg, i)
+        u0, _, _ = ora.ternarize(ora.start_normals(w.seeds[0], i, 2560), w.tau[0])
+        fit = ora.fit_component(R, u0, w.tau[0], 15)
+        if np.array_equal(fit.u, Bg[:, i]) and np.array_equal(fit.v, Cg[i]):
+            assert d64[i] == pytest.approx(fit.d, rel=1e-4)
+        else:
+            mism += 1
+            assert fit.min_margin < 1e-3, (i, fit.min_margin)
+    assert mism <= 2
