@@ -1,0 +1,362 @@
+"""Benchmark: ternary components fitted per second by greedy sequential ALS.
+
+Default workload: one 2560 x 6912 MLP-shaped matrix (LLM-like synthetic weights
+rounded to bf16, held as fp32), mu = 3 (k = 7680 components), tau = 1.0,
+15 alternating fits per component.  A "step" factors the whole matrix.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
+                    [--workload NAME | --all]
+
+N > 1 is launched by torch.distributed.run: each rank factors its own matrix
+(seed + rank), no data-path collective (weak scaling); the barrier and the
+max-over-ranks time use NCCL.  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle (test infrastructure) on the host
+cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "ternary components fitted/s at 2560×6912 μ=3; achieved GB/s vs HBM peak"
+UNIT = "components/s"
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+L2_BYTES = 126 * 1024 * 1024
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def _kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("externd.cu", "externd_kernels.cuh"):
+        with open(os.path.join(ROOT, "ternary_rank_weight_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def _ncu_traffic(workload: str):
+    """DRAM bytes per ALS launch from the committed ncu summary, if it was taken on this kernel source."""
+    path = os.path.join(ROOT, "profiles", "als_kernel_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    if rec.get("source_sha256") != _kernel_source_hash():
+        return None
+    per = rec.get("dram_bytes_per_launch_scaled", {}).get(workload)
+    return float(per) if per is not None else None
+
+
+class ClockSampler:
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={CLOCK_FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        try:
+            for line in open(self.path):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    sm.append(float(f[1]))
+                    mx.append(float(f[2]))
+                except ValueError:
+                    continue
+                for nm, val in zip(names, f[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(nm)
+        except Exception:
+            pass
+        finally:
+            try:
+                os.unlink(self.path)
+            except Exception:
+                pass
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def _workload_arrays(name: str, rank: int, mu=None):
+    import dataclasses
+    from ternary_rank_weight_b200.workloads import WORKLOADS
+    w = WORKLOADS[name]
+    if mu is not None:
+        w = dataclasses.replace(w, mu=tuple(mu for _ in w.mu))
+    mats = []
+    for b in range(w.count):
+        if rank == 0:
+            mats.append(w.matrix(b))
+        else:  # weak scaling: each rank its own matrices, same shapes and recipe
+            wr = dataclasses.replace(w, seeds=tuple(s + 1000 * rank for s in w.seeds))
+            mats.append(wr.matrix(b))
+    return w, mats
+
+
+def _config(w, extra=None):
+    shapes = sorted(set(w.shapes))
+    cfg = {"workload": w.name, "matrices": w.count,
+           "shape": list(shapes[0]) if len(shapes) == 1 else [list(s) for s in shapes],
+           "mu": w.mu[0] if len(set(w.mu)) == 1 else list(w.mu),
+           "tau": w.tau[0] if len(set(w.tau)) == 1 else list(w.tau),
+           "iters": w.iters, "recipe": w.recipe + ("+bf16" if w.bf16 else ""),
+           "l2": "inputs larger than L2 (A + two residual copies exceed 126 MB); no flush"}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+
+def _oracle_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def time_oracle(w, mats, budget_s: float = 15.0):
+    """Time the fp64 oracle on a bounded prefix of components of matrix 0 of the workload."""
+    from oracle import externd_oracle as ora
+    A = mats[0]
+    m, n = A.shape
+    k_full = ora.rank(m, n, w.mu[0])
+    # calibrate with 2 components, then size the sample to the budget
+    t0 = time.perf_counter()
+    ora.greedy_als(A, k=2, tau=w.tau[0], iters=w.iters, seed=w.seeds[0])
+    per = (time.perf_counter() - t0) / 2
+    kk = int(max(2, min(k_full, budget_s / max(per, 1e-6))))
+    t0 = time.perf_counter()
+    ora.greedy_als(A, k=kk, tau=w.tau[0], iters=w.iters, seed=w.seeds[0])
+    dt = time.perf_counter() - t0
+    return {"value": kk / dt, "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
+            "sample": f"first {kk} of {k_full} components of matrix 0 ({m}x{n}, mu={w.mu[0]}, tau={w.tau[0]}), "
+                      f"{dt:.1f} s, numpy fp64"}
+
+
+def run_reference(args):
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    w, mats = _workload_arrays(args.workload, 0, args.mu)
+    for _ in range(args.warmup):
+        pass   # the oracle has nothing to warm up beyond the calibration inside time_oracle
+    vals = []
+    last = None
+    t_all = time.perf_counter()
+    for _ in range(args.steps):
+        last = time_oracle(w, mats, budget_s=args.ref_budget)
+        vals.append(last["value"])
+    wall = time.perf_counter() - t_all
+    value = statistics.mean(vals)
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": wall * 1000 / max(args.steps, 1), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": _config(w), "cpu_baseline": dict(last, value=value),
+           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# CUDA path
+# ---------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import ternary_rank_weight_b200 as ext
+
+    ws, rank, local = _dist()
+    if ws > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    w, mats = _workload_arrays(args.workload, rank, args.mu)
+    As = [torch.from_numpy(a).to(dev) for a in mats]
+    host_As = [torch.from_numpy(a).pin_memory() for a in mats]
+    k_total = sum(ext.rank(a.shape[0], a.shape[1], mu) for a, mu in zip(mats, w.mu))
+    stream = torch.cuda.current_stream(dev)
+
+    def step(inputs):
+        if w.count == 1:
+            f = ext.factor(inputs[0], w.mu[0], w.tau[0], iters=w.iters, seed=w.seeds[0] + 1000 * rank,
+                           grid=args.grid, pending=args.pending)
+            return [f], f.stats
+        res, st = ext.factor_batched(inputs, w.mu, w.tau, iters=w.iters,
+                                     seeds=[s + 1000 * rank for s in w.seeds])
+        assert all(s == 0 for s in st), st
+        return res, res[0].stats
+
+    def barrier():
+        if ws > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x: float) -> float:
+        if ws == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step(As)
+
+    # ---- device-resident inputs
+    als_ms, alg_bytes, launches = [], [], 0
+    barrier()
+    with ClockSampler(dev.index) as clk:
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            res, st = step(As)
+            als_ms.append(st["als_ms"])
+            alg_bytes.append(st["alg_bytes"])
+            launches += st["launches"]
+        ev1.record(stream)
+        barrier()
+    t_ms = max_over_ranks(ev0.elapsed_time(ev1))
+    clocks = clk.summary()
+    value = ws * k_total * args.steps / (t_ms / 1000.0)
+
+    # ---- end to end through the public API with pinned host buffers
+    step(host_As)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    h2d = d2h = 0
+    for _ in range(args.steps):
+        res, _ = step(host_As)
+        h2d = sum(a.numel() * 4 for a in host_As)
+        d2h = sum(r.B.numel() + r.C.numel() + r.D.numel() * 4 + (r.energy.numel() * 8 if r.energy is not None else 0)
+                  for r in res)
+    e1.record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_value = ws * k_total * args.steps / (e2e_ms / 1000.0)
+
+    peak, peak_kind = _peaks()
+    mean_als = statistics.mean(als_ms)
+    mean_bytes = statistics.mean(alg_bytes)
+    achieved = mean_bytes / (mean_als / 1000.0) / 1e9
+    traffic = _ncu_traffic(w.name)
+    energy_final = float(res[0].energy[-1].item()) if res[0].energy is not None else None
+    out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": t_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f32 residual, f64 accumulation", "data": "synthetic",
+           "config": _config(w, {"k": k_total, "grid": st["grid"], "group": st["group"], "block": st["block"],
+                                 "pending": st["pending"], "vec": [st["vec_v"], st["vec_u"]],
+                                 "parallelism": f"replicas x{ws} (independent matrices per rank)"}),
+           "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                        "frac": achieved / peak, "traffic": traffic,
+                        "kernel": "externd::als_kernel", "peak_kind": f"{peak_kind} copy bandwidth",
+                        "alg_bytes_per_launch": mean_bytes, "kernel_ms": mean_als},
+           "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+           "gpu_launches": launches,
+           "clocks": clocks,
+           "energy": energy_final,
+           "components_per_step": ws * k_total,
+           "wall_s_per_matrix": (t_ms / 1000.0) / args.steps / w.count}
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = time_oracle(w, mats, budget_s=args.ref_budget)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if ws > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main():
+    from ternary_rank_weight_b200.workloads import HEADLINE, WORKLOADS
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(WORKLOADS))
+    ap.add_argument("--all", action="store_true", help="one line per workload (reporting, not the driver's line)")
+    ap.add_argument("--grid", type=int, default=0)
+    ap.add_argument("--pending", type=int, default=0)
+    ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of oracle work per sample")
+    ap.add_argument("--mu", type=float, default=None, help="override mu (short runs for profiling)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.ref_budget = min(args.ref_budget, 150.0 / max(args.steps, 1))
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.all:
+        for name in WORKLOADS:
+            args.workload = name
+            run_ours(args)
+        return 0
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
