@@ -137,25 +137,58 @@ __global__ void __launch_bounds__(NTI) init_kernel(const Prob* __restrict__ prob
 // ALS kernel pieces
 // ---------------------------------------------------------------------------
 
-struct Smem {
-    double* red;     // NT*4
-    double* sc;      // 64
-    double* pd;      // Lc
-    double* coef;    // Lc
-    long long* scj;  // 64
-    int* sci;        // 64
-    uint32_t *nzU, *sgU, *nzV, *sgV;
-    uint32_t *pnzU, *psgU, *pnzV, *psgV;
-    int* ulist;
-    int* vlist;
-    int* wcnt;
+// Shared-memory carve of the ALS kernel (host and device use the same layout).
+struct SmemLayout {
+    size_t red, pd, coef, scal, wS, wM, wp, gS, gM, wJ, gJ, wc, dotp, sflag, nzU, sgU, nzV, sgV, pnzU, psgU, pnzV,
+        psgV, cnzV, csgV, cnzU, csgU, ulist, vlist, total;
+    __host__ __device__ SmemLayout(int64_t m_max, int64_t n_max, int Lc, int pv_max, int pu_max) {
+        const size_t Wm = (size_t)((m_max + 31) / 32), Wn = (size_t)((n_max + 31) / 32);
+        size_t o = 0;
+        red = o;  o += 8 * (size_t)NT * 4;
+        pd = o;   o += 8 * (size_t)Lc;
+        coef = o; o += 8 * (size_t)Lc;
+        scal = o; o += 8 * 16;
+        wS = o;   o += 8 * NWARP;
+        wM = o;   o += 8 * NWARP;
+        wp = o;   o += 8 * NWARP;
+        gS = o;   o += 8 * NWARP;
+        gM = o;   o += 8 * NWARP;
+        wJ = o;   o += 8 * NWARP;
+        gJ = o;   o += 8 * NWARP;
+        wc = o;   o += 4 * NWARP;
+        dotp = o; o += 4 * NWARP * MAX_PENDING;
+        sflag = o; o += 16;
+        nzU = o;  o += 4 * Wm;
+        sgU = o;  o += 4 * Wm;
+        nzV = o;  o += 4 * Wn;
+        sgV = o;  o += 4 * Wn;
+        pnzU = o; o += 4 * Wm * Lc;
+        psgU = o; o += 4 * Wm * Lc;
+        pnzV = o; o += 4 * Wn * Lc;
+        psgV = o; o += 4 * Wn * Lc;
+        cnzV = o; o += 4 * (size_t)pv_max;
+        csgV = o; o += 4 * (size_t)pv_max;
+        cnzU = o; o += 4 * (size_t)pu_max;
+        csgU = o; o += 4 * (size_t)pu_max;
+        ulist = o; o += 4 * (size_t)m_max;
+        vlist = o; o += 4 * (size_t)n_max;
+        total = (o + 15) & ~(size_t)15;
+    }
 };
 
-struct OutAcc {
-    double S;
-    double M;
-    long long J;
+struct Smem {
+    double *red, *pd, *coef, *scal, *wS, *wM, *wp, *gS, *gM;
+    long long *wJ, *gJ;
+    int *wc, *dotp, *sflag;
+    uint32_t *nzU, *sgU, *nzV, *sgV;         // current u, v
+    uint32_t *pnzU, *psgU, *pnzV, *psgV;     // pending components (full length, stride W)
+    uint32_t *cnzV, *csgV, *cnzU, *csgU;     // pending trits at this CTA's outputs, bit l = component l
+    int *ulist, *vlist;                      // compacted supports (index | sign << 31)
 };
+
+__device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 
 template <int VEC>
 __device__ __forceinline__ void load_vec(const float* p, float* v) {
@@ -170,44 +203,46 @@ __device__ __forceinline__ void load_vec(const float* p, float* v) {
     }
 }
 
-// sum_l coef_l * t_l(i) over the pending components, t_l from bit masks
-__device__ __forceinline__ double corr_at(int64_t i, int L, const double* coef, const uint32_t* pnz,
-                                          const uint32_t* psg, int W) {
-    double c = 0.0;
-    const int w = (int)(i >> 5);
-    const uint32_t b = 1u << (i & 31);
-    for (int l = 0; l < L; ++l) {
-        if (pnz[l * W + w] & b) c += (psg[l * W + w] & b) ? -coef[l] : coef[l];
-    }
-    return c;
-}
-
-struct CorrArgs {
-    int L;
+// Lazy-deflation correction at one of this CTA's outputs: sum_l coef_l t_l(c),
+// t_l from the per-output pending bit masks, in increasing l.
+struct HalfCorr {
     const double* coef;
-    const uint32_t* pnz;
-    const uint32_t* psg;
-    int W;
+    const uint32_t* cnz;
+    const uint32_t* csg;
 };
 
-__device__ __forceinline__ void emit_out(double v, int64_t gi, double* gout, const CorrArgs& ca, OutAcc& a) {
-    if (ca.L > 0) v -= corr_at(gi, ca.L, ca.coef, ca.pnz, ca.psg, ca.W);
-    gout[gi] = v;
+__device__ __forceinline__ double corr_local(int c, const HalfCorr& hc) {
+    uint32_t bits = hc.cnz[c];
+    const uint32_t sgn = hc.csg[c];
+    double v = 0.0;
+    while (bits) {
+        const int l = __ffs(bits) - 1;
+        bits &= bits - 1u;
+        v += ((sgn >> l) & 1u) ? -hc.coef[l] : hc.coef[l];
+    }
+    return v;
+}
+
+__device__ __forceinline__ void emit_out(double v, int c, int64_t out0, double* gout, const HalfCorr& hc, double& S,
+                                         double& M, long long& J) {
+    v -= corr_local(c, hc);
+    gout[out0 + c] = v;
     const double av = fabs(v);
-    a.S += av;
-    if (av > a.M) { a.M = av; a.J = gi; }
+    S += av;
+    if (av > M) { M = av; J = out0 + c; }
 }
 
 // One half-step GEMV over this CTA's private block: out[c] = sum_{e in list} s_e blk[r_e][c]
-// for the block's `valid` columns, written to gout[out0 + c] after the lazy
-// deflation corrections.  fp64 accumulation, fixed summation order.
+// for the block's `valid` columns, minus the lazy-deflation correction, written to
+// gout[out0 + c].  fp64 accumulation of exact fp32 terms, fixed summation order.
 template <int VEC>
-__device__ void stripe_gemv(const float* __restrict__ blk, int pitch, int valid, int64_t out0,
-                            const int* __restrict__ list, int nlist, double* red, double* gout,
-                            const CorrArgs& ca, OutAcc& a) {
-    a.S = 0.0; a.M = -1.0; a.J = LLONG_MAX;
+__device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, int64_t out0,
+                          const int* __restrict__ list, int nlist, double* red, double* gout, const HalfCorr& hc,
+                          double& S, double& M, long long& J) {
+    S = 0.0; M = -1.0; J = LLONG_MAX;
     const int nvec = pitch / VEC;
     if (nvec <= 0) return;
+    constexpr int U = (VEC == 4) ? 8 : 16;
     if (nvec <= NT) {
         const int lanes = NT / nvec;
         const int j = threadIdx.x % nvec;
@@ -218,26 +253,28 @@ __device__ void stripe_gemv(const float* __restrict__ blk, int pitch, int valid,
             for (int e = 0; e < VEC; ++e) acc[e] = 0.0;
             const float* base = blk + j * VEC;
             int idx = g;
-            for (; idx + 7 * lanes < nlist; idx += 8 * lanes) {
-                int ent[8];
-                float v[8][VEC];
+            for (; idx + (U - 1) * lanes < nlist; idx += U * lanes) {
+                int ent[U];
+                float v[U][VEC];
                 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
+                for (int u = 0; u < U; ++u) {
                     ent[u] = list[idx + u * lanes];
                     load_vec<VEC>(base + (int64_t)(ent[u] & 0x7fffffff) * pitch, v[u]);
                 }
                 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
+                for (int u = 0; u < U; ++u) {
+                    const unsigned sm = (unsigned)ent[u] & 0x80000000u;
                     #pragma unroll
-                    for (int e = 0; e < VEC; ++e) acc[e] += (ent[u] < 0) ? -(double)v[u][e] : (double)v[u][e];
+                    for (int e = 0; e < VEC; ++e) acc[e] += (double)__uint_as_float(__float_as_uint(v[u][e]) ^ sm);
                 }
             }
             for (; idx < nlist; idx += lanes) {
                 const int ent = list[idx];
                 float v[VEC];
                 load_vec<VEC>(base + (int64_t)(ent & 0x7fffffff) * pitch, v);
+                const unsigned sm = (unsigned)ent & 0x80000000u;
                 #pragma unroll
-                for (int e = 0; e < VEC; ++e) acc[e] += (ent < 0) ? -(double)v[e] : (double)v[e];
+                for (int e = 0; e < VEC; ++e) acc[e] += (double)__uint_as_float(__float_as_uint(v[e]) ^ sm);
             }
             #pragma unroll
             for (int e = 0; e < VEC; ++e) red[g * pitch + j * VEC + e] = acc[e];
@@ -253,9 +290,8 @@ __device__ void stripe_gemv(const float* __restrict__ blk, int pitch, int valid,
             if (c < pitch)
                 for (int gg = s; gg < lanes; gg += tpc) v += red[gg * pitch + c];
             for (int o = tpc >> 1; o; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
-            if (s == 0 && c < valid) emit_out(v, out0 + c, gout, ca, a);
+            if (s == 0 && c < valid) emit_out(v, c, out0, gout, hc, S, M, J);
         }
-        __syncthreads();
     } else {
         for (int j = threadIdx.x; j < nvec; j += NT) {
             double acc[VEC];
@@ -263,31 +299,33 @@ __device__ void stripe_gemv(const float* __restrict__ blk, int pitch, int valid,
             for (int e = 0; e < VEC; ++e) acc[e] = 0.0;
             const float* base = blk + j * VEC;
             int idx = 0;
-            for (; idx + 7 < nlist; idx += 8) {
-                int ent[8];
-                float v[8][VEC];
+            for (; idx + U - 1 < nlist; idx += U) {
+                int ent[U];
+                float v[U][VEC];
                 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
+                for (int u = 0; u < U; ++u) {
                     ent[u] = list[idx + u];
                     load_vec<VEC>(base + (int64_t)(ent[u] & 0x7fffffff) * pitch, v[u]);
                 }
                 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
+                for (int u = 0; u < U; ++u) {
+                    const unsigned sm = (unsigned)ent[u] & 0x80000000u;
                     #pragma unroll
-                    for (int e = 0; e < VEC; ++e) acc[e] += (ent[u] < 0) ? -(double)v[u][e] : (double)v[u][e];
+                    for (int e = 0; e < VEC; ++e) acc[e] += (double)__uint_as_float(__float_as_uint(v[u][e]) ^ sm);
                 }
             }
             for (; idx < nlist; ++idx) {
                 const int ent = list[idx];
                 float v[VEC];
                 load_vec<VEC>(base + (int64_t)(ent & 0x7fffffff) * pitch, v);
+                const unsigned sm = (unsigned)ent & 0x80000000u;
                 #pragma unroll
-                for (int e = 0; e < VEC; ++e) acc[e] += (ent < 0) ? -(double)v[e] : (double)v[e];
+                for (int e = 0; e < VEC; ++e) acc[e] += (double)__uint_as_float(__float_as_uint(v[e]) ^ sm);
             }
             #pragma unroll
             for (int e = 0; e < VEC; ++e) {
                 const int c = j * VEC + e;
-                if (c < valid) emit_out(acc[e], out0 + c, gout, ca, a);
+                if (c < valid) emit_out(acc[e], c, out0, gout, hc, S, M, J);
             }
         }
     }
@@ -295,18 +333,18 @@ __device__ void stripe_gemv(const float* __restrict__ blk, int pitch, int valid,
 
 __device__ __forceinline__ void gemv_dispatch(int vec, const float* blk, int pitch, int valid, int64_t out0,
                                               const int* list, int nlist, double* red, double* gout,
-                                              const CorrArgs& ca, OutAcc& a) {
-    if (vec == 4) stripe_gemv<4>(blk, pitch, valid, out0, list, nlist, red, gout, ca, a);
-    else if (vec == 2) stripe_gemv<2>(blk, pitch, valid, out0, list, nlist, red, gout, ca, a);
-    else stripe_gemv<1>(blk, pitch, valid, out0, list, nlist, red, gout, ca, a);
+                                              const HalfCorr& hc, double& S, double& M, long long& J) {
+    if (vec == 4) gemv_emit<4>(blk, pitch, valid, out0, list, nlist, red, gout, hc, S, M, J);
+    else if (vec == 2) gemv_emit<2>(blk, pitch, valid, out0, list, nlist, red, gout, hc, S, M, J);
+    else gemv_emit<1>(blk, pitch, valid, out0, list, nlist, red, gout, hc, S, M, J);
 }
 
 // Fold the L pending components into this CTA's block:
-// blk[r][c] -= sum_l d_l * tR_l(r) * tC_l(col0 + c), fp64 sum, one fp32 rounding.
+// blk[r][c] -= sum_l d_l * tR_l(r) * tC_l(col0 + c), fp64 sum in increasing l, one fp32 rounding.
 template <int VEC>
-__device__ void flush_block(float* blk, int pitch, int64_t rows, int64_t col0, int valid, int L, const double* pd,
-                            const uint32_t* pnzR, const uint32_t* psgR, int WR,
-                            const uint32_t* pnzC, const uint32_t* psgC, int WC) {
+__device__ void flush_block(float* blk, int pitch, int64_t rows, int valid, int L, const double* pd,
+                            const uint32_t* pnzR, const uint32_t* psgR, int WR, const uint32_t* cnz,
+                            const uint32_t* csg) {
     const int nvec = pitch / VEC;
     if (nvec <= 0 || L <= 0) return;
     const int64_t total = rows * nvec;
@@ -315,100 +353,76 @@ __device__ void flush_block(float* blk, int pitch, int64_t rows, int64_t col0, i
         const int j = (int)(t - r * nvec);
         const int wr = (int)(r >> 5);
         const uint32_t br = 1u << (r & 31);
-        double cr[VEC];
-        #pragma unroll
-        for (int e = 0; e < VEC; ++e) cr[e] = 0.0;
-        bool any = false;
+        uint32_t rnz = 0, rsg = 0;
         for (int l = 0; l < L; ++l) {
-            if (pnzR[l * WR + wr] & br) {
-                const double dl = (psgR[l * WR + wr] & br) ? -pd[l] : pd[l];
-                #pragma unroll
-                for (int e = 0; e < VEC; ++e) {
-                    const int64_t c = col0 + j * VEC + e;
-                    const int wc = (int)(c >> 5);
-                    const uint32_t bc = 1u << (c & 31);
-                    if (pnzC[l * WC + wc] & bc) {
-                        cr[e] += (psgC[l * WC + wc] & bc) ? -dl : dl;
-                        any = true;
-                    }
-                }
-            }
+            rnz |= ((pnzR[l * WR + wr] & br) ? 1u : 0u) << l;
+            rsg |= ((psgR[l * WR + wr] & br) ? 1u : 0u) << l;
         }
-        if (any) {
-            float* p = blk + r * pitch + j * VEC;
-            #pragma unroll
-            for (int e = 0; e < VEC; ++e) {
-                if (j * VEC + e < valid && cr[e] != 0.0) p[e] = (float)((double)__ldcg(p + e) - cr[e]);
+        if (!rnz) continue;
+        float* p = blk + r * pitch + j * VEC;
+        #pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+            const int c = j * VEC + e;
+            if (c >= valid) continue;
+            uint32_t bits = rnz & cnz[c];
+            if (!bits) continue;
+            const uint32_t neg = rsg ^ csg[c];
+            double corr = 0.0;
+            while (bits) {
+                const int l = __ffs(bits) - 1;
+                bits &= bits - 1u;
+                corr += ((neg >> l) & 1u) ? -pd[l] : pd[l];
             }
+            p[e] = (float)((double)__ldcg(p + e) - corr);
         }
     }
 }
 
-__device__ __forceinline__ void flush_dispatch(int vec, float* blk, int pitch, int64_t rows, int64_t col0, int valid,
-                                               int L, const double* pd, const uint32_t* pnzR, const uint32_t* psgR,
-                                               int WR, const uint32_t* pnzC, const uint32_t* psgC, int WC) {
-    if (vec == 4) flush_block<4>(blk, pitch, rows, col0, valid, L, pd, pnzR, psgR, WR, pnzC, psgC, WC);
-    else if (vec == 2) flush_block<2>(blk, pitch, rows, col0, valid, L, pd, pnzR, psgR, WR, pnzC, psgC, WC);
-    else flush_block<1>(blk, pitch, rows, col0, valid, L, pd, pnzR, psgR, WR, pnzC, psgC, WC);
-}
-
-// Threshold a published vector (every CTA reads all of it), write masks and
-// the compacted list of its support; returns nnz.  p_out (nullable) gets
-// sum_{|x|>thr} |x| in a fixed order.
-__device__ int build_from_vector(const double* gvec, int64_t len, double thr, uint32_t* nz, uint32_t* sg,
-                                 int* list, int* wcnt, int* shi, double* shd, double* p_out) {
-    const int W = (int)((len + 31) >> 5);
-    double ps = 0.0;
-    for (int w = warp_id(); w < W; w += NWARP) {
-        const int64_t i = ((int64_t)w << 5) + lane_id();
-        const bool in = i < len;
-        const double x = in ? __ldcg(gvec + i) : 0.0;
-        const bool z = in && (fabs(x) > thr);
-        const bool ng = z && (x < 0.0);
-        const unsigned bz = __ballot_sync(FULL, z);
-        const unsigned bs = __ballot_sync(FULL, ng);
-        if (lane_id() == 0) { nz[w] = bz; sg[w] = bs; wcnt[w] = __popc(bz); }
-        if (z) ps += fabs(x);
-    }
-    __syncthreads();
-    const int total = block_exclusive_scan(wcnt, W, shi);
-    for (int w = warp_id(); w < W; w += NWARP) {
-        const unsigned bz = nz[w];
-        if ((bz >> lane_id()) & 1u) {
-            const int pos = wcnt[w] + __popc(bz & ((1u << lane_id()) - 1u));
-            list[pos] = (int)(((unsigned)w << 5) + lane_id()) | (int)(((sg[w] >> lane_id()) & 1u) << 31);
-        }
-    }
-    double p = 0.0;
-    if (p_out) p = block_sum(ps, shd);
-    __syncthreads();
-    if (p_out) *p_out = p;
-    return total;
+__device__ __forceinline__ void flush_dispatch(int vec, float* blk, int pitch, int64_t rows, int valid, int L,
+                                               const double* pd, const uint32_t* pnzR, const uint32_t* psgR, int WR,
+                                               const uint32_t* cnz, const uint32_t* csg) {
+    if (vec == 4) flush_block<4>(blk, pitch, rows, valid, L, pd, pnzR, psgR, WR, cnz, csg);
+    else if (vec == 2) flush_block<2>(blk, pitch, rows, valid, L, pd, pnzR, psgR, WR, cnz, csg);
+    else flush_block<1>(blk, pitch, rows, valid, L, pd, pnzR, psgR, WR, cnz, csg);
 }
 
 // Start trits (2-bit packed words) -> masks and list; returns nnz.
 __device__ int build_from_trits(const uint32_t* words, int64_t nwords, int64_t len, uint32_t* nz, uint32_t* sg,
-                                int* list, int* wcnt, int* shi) {
+                                int* list, const Smem& s) {
     const int W = (int)((len + 31) >> 5);
-    for (int w = threadIdx.x; w < W; w += NT) {
+    const int wpw = (W + NWARP - 1) / NWARP;
+    const int w0 = min(W, warp_id() * wpw), w1 = min(W, w0 + wpw);
+    int cnt = 0;
+    for (int w = w0 + lane_id(); w < w1; w += 32) {
         const int64_t a = 2 * (int64_t)w, b = a + 1;
         const uint32_t lo = a < nwords ? __ldcg(words + a) : 0u;
         const uint32_t hi = b < nwords ? __ldcg(words + b) : 0u;
         uint32_t z = compact_even(lo) | (compact_even(hi) << 16);
-        uint32_t s = compact_even(lo >> 1) | (compact_even(hi >> 1) << 16);
+        uint32_t sb = compact_even(lo >> 1) | (compact_even(hi >> 1) << 16);
         const int64_t rem = len - ((int64_t)w << 5);
         if (rem < 32) z &= (1u << rem) - 1u;
-        s &= z;
-        nz[w] = z; sg[w] = s; wcnt[w] = __popc(z);
+        sb &= z;
+        nz[w] = z;
+        sg[w] = sb;
+        cnt += __popc(z);
     }
+    #pragma unroll
+    for (int o = 16; o; o >>= 1) cnt += __shfl_xor_sync(FULL, cnt, o);
+    if (lane_id() == 0) s.wc[warp_id()] = cnt;
     __syncthreads();
-    const int total = block_exclusive_scan(wcnt, W, shi);
-    for (int w = warp_id(); w < W; w += NWARP) {
-        const unsigned bz = nz[w];
-        if ((bz >> lane_id()) & 1u) {
-            const int pos = wcnt[w] + __popc(bz & ((1u << lane_id()) - 1u));
-            list[pos] = (int)(((unsigned)w << 5) + lane_id()) | (int)(((sg[w] >> lane_id()) & 1u) << 31);
-        }
+    int off = 0, total = 0;
+    for (int w = 0; w < NWARP; ++w) {
+        const int c = s.wc[w];
+        off += (w < warp_id()) ? c : 0;
+        total += c;
+    }
+    int run = off;
+    for (int w = w0; w < w1; ++w) {
+        const uint32_t bz = nz[w];
+        if ((bz >> lane_id()) & 1u)
+            list[run + __popc(bz & ((1u << lane_id()) - 1u))] =
+                (int)(((unsigned)w << 5) + lane_id()) | (int)(((sg[w] >> lane_id()) & 1u) << 31);
+        run += __popc(bz);
     }
     __syncthreads();
     return total;
@@ -443,20 +457,37 @@ __device__ void pack_row(const uint32_t* nz, const uint32_t* sg, int W, uint32_t
     }
 }
 
-// Arrive at the group counter and wait until every CTA of the group arrived.
-// Bounded by limit_ns; on expiry raises the group abort flag and the status.
-__device__ bool group_barrier(GroupSync* gs, unsigned& target, int Gg, uint64_t limit_ns, bool skip_arrive,
-                              int* status, int* sflag) {
-    __threadfence();
+// Publish this CTA's (sum |out|, max |out|, argmax) and arrive at the group counter,
+// then wait until every CTA of the group arrived.  Arrival is a release by one
+// thread after a CTA barrier, the wait an acquire by the same thread followed by a
+// CTA barrier, so the slice of the output vector each CTA stored before arriving
+// is visible to all CTAs after the wait.  Bounded by limit_ns; on expiry the group
+// abort flag and the status word are raised.
+__device__ bool publish_and_wait(Slot* slot, double S, double M, long long J, const Smem& s, GroupSync* gs,
+                                 unsigned& target, int Gg, uint64_t limit_ns, bool skip_arrive, int* status) {
+    #pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        S += __shfl_xor_sync(FULL, S, o);
+        const double m2 = __shfl_xor_sync(FULL, M, o);
+        const long long j2 = __shfl_xor_sync(FULL, J, o);
+        maxloc_merge(M, J, m2, j2);
+    }
+    if (lane_id() == 0) { s.wS[warp_id()] = S; s.wM[warp_id()] = M; s.wJ[warp_id()] = J; }
     __syncthreads();
     if (threadIdx.x == 0) {
+        double S2 = 0.0, M2 = -1.0;
+        long long J2 = LLONG_MAX;
+        for (int w = 0; w < NWARP; ++w) { S2 += s.wS[w]; maxloc_merge(M2, J2, s.wM[w], s.wJ[w]); }
+        slot->S = S2;
+        slot->M = M2;
+        slot->J = J2;
         target += (unsigned)Gg;
-        if (!skip_arrive) atomicAdd(&gs->arrive, 1u);
+        if (!skip_arrive) red_release_add(&gs->arrive, 1u);
         int ok = 1;
         const uint64_t t0 = gtimer();
         unsigned spins = 0;
         while ((int)(ld_acquire_u32(&gs->arrive) - target) < 0) {
-            if ((++spins & 31u) == 0u) {
+            if ((++spins & 15u) == 0u) {
                 if (ld_relaxed_s32(&gs->abort)) { ok = 0; break; }
                 if (gtimer() - t0 > limit_ns) {
                     atomicExch(&gs->abort, 1);
@@ -466,58 +497,150 @@ __device__ bool group_barrier(GroupSync* gs, unsigned& target, int Gg, uint64_t 
                 }
             }
         }
-        __threadfence();
-        *sflag = ok;
+        *s.sflag = ok;
     }
     __syncthreads();
-    const bool ok = *sflag != 0;
-    __syncthreads();
-    return ok;
+    return *s.sflag != 0;
 }
 
-// Sum of the group's published S (fixed order) and the global max |.| / lowest index.
-__device__ void gather_slots(const Slot* sl, int Gg, double* sc, long long* scj) {
-    if (warp_id() == 0) {
-        double S = 0.0, M = -1.0;
-        long long J = LLONG_MAX;
-        for (int t = lane_id(); t < Gg; t += 32) {
-            S += __ldcg(&sl[t].S);
-            maxloc_merge(M, J, __ldcg(&sl[t].M), __ldcg(&sl[t].J));
+// After publish_and_wait: sum of the group's published S in a fixed order.
+__device__ double gather_sum(const Slot* sl, int Gg, const Smem& s) {
+    double S = ((int)threadIdx.x < Gg) ? __ldcg(&sl[threadIdx.x].S) : 0.0;
+    #pragma unroll
+    for (int o = 16; o; o >>= 1) S += __shfl_xor_sync(FULL, S, o);
+    if (lane_id() == 0) s.gS[warp_id()] = S;
+    __syncthreads();
+    double t = 0.0;
+    for (int w = 0; w < NWARP; ++w) t += s.gS[w];
+    __syncthreads();
+    return t;
+}
+
+// After publish_and_wait: read the group's slots and the whole published vector,
+// threshold it (T_tau of §2.2 with the all-zero fallback), write its masks and
+// compacted support list, the coefficients d_l (t_l . t) of the pending
+// components for the next half-step, and p = sum over the support of |x| into
+// s.scal[0].  Every CTA of the group derives identical results (same data, same
+// order).  Returns nnz.
+__device__ int gather_threshold(const Slot* sl, int Gg, const double* gvec, int64_t len, double tau, uint32_t* nz,
+                                uint32_t* sg, int* list, const Smem& s, int L, const uint32_t* pnz,
+                                const uint32_t* psg, double& thr_out) {
+    const int lane = lane_id(), warp = warp_id();
+    const int W = (int)((len + 31) >> 5);
+    const int wpw = (W + NWARP - 1) / NWARP;
+    const int w0 = min(W, warp * wpw), w1 = min(W, w0 + wpw);
+    double S = 0.0, M = -1.0;
+    long long J = LLONG_MAX;
+    if ((int)threadIdx.x < Gg) {
+        S = __ldcg(&sl[threadIdx.x].S);
+        M = __ldcg(&sl[threadIdx.x].M);
+        J = __ldcg(&sl[threadIdx.x].J);
+    }
+    constexpr int CH = 16;
+    double xv[CH];
+    #pragma unroll
+    for (int i = 0; i < CH; ++i) {
+        const int w = w0 + i;
+        const int64_t idx = ((int64_t)w << 5) + lane;
+        xv[i] = (w < w1 && idx < len) ? __ldcg(gvec + idx) : 0.0;
+    }
+    #pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        S += __shfl_xor_sync(FULL, S, o);
+        const double m2 = __shfl_xor_sync(FULL, M, o);
+        const long long j2 = __shfl_xor_sync(FULL, J, o);
+        maxloc_merge(M, J, m2, j2);
+    }
+    if (lane == 0) { s.gS[warp] = S; s.gM[warp] = M; s.gJ[warp] = J; }
+    __syncthreads();
+    double St = 0.0, Mt = -1.0;
+    long long Jt = LLONG_MAX;
+    for (int w = 0; w < NWARP; ++w) { St += s.gS[w]; maxloc_merge(Mt, Jt, s.gM[w], s.gJ[w]); }
+    const double thr = tau * St / (double)len;
+    thr_out = thr;
+
+    int cnt = 0, dot = 0;
+    double ps = 0.0;
+    for (int base = w0; base < w1; base += CH) {
+        if (base != w0) {
+            #pragma unroll
+            for (int i = 0; i < CH; ++i) {
+                const int w = base + i;
+                const int64_t idx = ((int64_t)w << 5) + lane;
+                xv[i] = (w < w1 && idx < len) ? __ldcg(gvec + idx) : 0.0;
+            }
         }
         #pragma unroll
-        for (int o = 16; o; o >>= 1) {
-            S += __shfl_xor_sync(FULL, S, o);
-            const double m2 = __shfl_xor_sync(FULL, M, o);
-            const long long j2 = __shfl_xor_sync(FULL, J, o);
-            maxloc_merge(M, J, m2, j2);
+        for (int i = 0; i < CH; ++i) {
+            const int w = base + i;
+            if (w < w1) {
+                const int64_t idx = ((int64_t)w << 5) + lane;
+                const bool z = (idx < len) && (fabs(xv[i]) > thr);
+                const bool ng = z && (xv[i] < 0.0);
+                const unsigned bz = __ballot_sync(FULL, z);
+                const unsigned bs = __ballot_sync(FULL, ng);
+                if (lane == 0) { nz[w] = bz; sg[w] = bs; }
+                cnt += __popc(bz);
+                if (z) ps += fabs(xv[i]);
+                if (lane < L) {
+                    const uint32_t both = pnz[lane * W + w] & bz;
+                    const uint32_t diff = psg[lane * W + w] ^ bs;
+                    dot += __popc(both & ~diff) - __popc(both & diff);
+                }
+            }
         }
-        if (lane_id() == 0) { sc[0] = S; sc[1] = M; scj[40] = J; }
     }
+    #pragma unroll
+    for (int o = 16; o; o >>= 1) ps += __shfl_xor_sync(FULL, ps, o);
+    if (lane == 0) { s.wc[warp] = cnt; s.wp[warp] = ps; }
+    if (lane < L) s.dotp[warp * MAX_PENDING + lane] = dot;
     __syncthreads();
-}
-
-// All-zero fallback of T_tau: keep the lowest index among the largest magnitudes.
-__device__ int apply_fallback(const double* gvec, int64_t len, long long J, uint32_t* nz, uint32_t* sg, int* list,
-                              double* p_out) {
-    if (J < 0 || J >= len) J = 0;   // only reachable with non-finite data, which the setup rejects
-    if (threadIdx.x == 0) {
-        const double x = __ldcg(gvec + J);
+    int off = 0, total = 0;
+    double p = 0.0;
+    for (int w = 0; w < NWARP; ++w) {
+        const int c = s.wc[w];
+        off += (w < warp) ? c : 0;
+        total += c;
+        p += s.wp[w];
+    }
+    if (total > 0) {
+        if ((int)threadIdx.x < L) {
+            int d = 0;
+            for (int w = 0; w < NWARP; ++w) d += s.dotp[w * MAX_PENDING + threadIdx.x];
+            s.coef[threadIdx.x] = s.pd[threadIdx.x] * (double)d;
+        }
+        int run = off;
+        for (int w = w0; w < w1; ++w) {
+            const uint32_t bz = nz[w];
+            if ((bz >> lane) & 1u)
+                list[run + __popc(bz & ((1u << lane) - 1u))] =
+                    (int)(((unsigned)w << 5) + lane) | (int)(((sg[w] >> lane) & 1u) << 31);
+            run += __popc(bz);
+        }
+        if (threadIdx.x == 0) { s.scal[0] = p; s.scal[1] = 0.0; }
+    } else {
+        // all-zero fallback: keep the lowest index among the largest magnitudes
+        const long long Jc = (Jt >= 0 && Jt < len) ? Jt : 0;   // out of range only with non-finite data
+        const double x = __ldcg(gvec + Jc);
         const bool neg = x < 0.0;
-        nz[J >> 5] |= 1u << (J & 31);
-        if (neg) sg[J >> 5] |= 1u << (J & 31);
-        list[0] = (int)J | (neg ? (int)0x80000000 : 0);
-        if (p_out) *p_out = fabs(x);
+        const int wj = (int)(Jc >> 5);
+        const uint32_t bj = 1u << (Jc & 31);
+        if ((int)threadIdx.x < L) {
+            int t = (pnz[threadIdx.x * W + wj] & bj) ? 1 : 0;
+            if (t && ((psg[threadIdx.x * W + wj] & bj) != 0u) != neg) t = -1;
+            s.coef[threadIdx.x] = s.pd[threadIdx.x] * (double)t;
+        }
+        if (threadIdx.x == 0) {
+            nz[wj] |= bj;
+            if (neg) sg[wj] |= bj;
+            list[0] = (int)Jc | (neg ? (int)0x80000000 : 0);
+            s.scal[0] = fabs(x);
+            s.scal[1] = 1.0;
+        }
+        total = 1;
     }
     __syncthreads();
-    return 1;
-}
-
-__device__ __forceinline__ void publish_slot(Slot* sl, const OutAcc& a, double* sc, long long* scj) {
-    double S = block_sum(a.S, sc + 8);
-    double M = a.M;
-    long long J = a.J;
-    block_maxloc(M, J, sc + 32, scj);
-    if (threadIdx.x == 0) { sl->S = S; sl->M = M; sl->J = J; }
+    return total;
 }
 
 // Factor (or run one debug half-step of) one matrix with this CTA group.
@@ -549,42 +672,44 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
     if (mode == MODE_FACTOR) {
         double ps = 0.0;
         for (int64_t t = tid; t < P.n_norm_part; t += NT) ps += __ldcg(P.norm_part + t);
-        N0 = block_sum(ps, s.sc + 8);
+        N0 = block_sum(ps, s.red);
         if (!(N0 > 0.0)) {
             if (lead && tid == 0) atomicExch(P.status, ST_EZERO);
             return true;
         }
     }
+    for (int c = tid; c < pitchV; c += NT) { s.cnzV[c] = 0u; s.csgV[c] = 0u; }
+    for (int c = tid; c < pitchU; c += NT) { s.cnzU[c] = 0u; s.csgU[c] = 0u; }
+    __syncthreads();
 
     double RN2 = N0;
     int L = 0;
     unsigned long long sum_nu = 0, sum_nv = 0, sum_nunv = 0, hs = 0, fb = 0;
     const int64_t kk = (mode == MODE_FACTOR) ? P.k : 1;
     int nU = 0, nV = 0;
-    double p = 0.0;
-    OutAcc a;
+    double p = 0.0, S, M, thr;
+    long long J;
+    const HalfCorr hcV{s.coef, s.cnzV, s.csgV};
+    const HalfCorr hcU{s.coef, s.cnzU, s.csgU};
 
     for (int64_t i = 0; i < kk; ++i) {
         if (mode != MODE_HALF_U) {
-            nU = build_from_trits(P.start + i * P.start_words, P.start_words, m, s.nzU, s.sgU, s.ulist, s.wcnt, s.sci);
+            nU = build_from_trits(P.start + i * P.start_words, P.start_words, m, s.nzU, s.sgU, s.ulist, s);
             if (L > 0) pending_coef(L, Wm, s.pnzU, s.psgU, s.nzU, s.sgU, s.pd, s.coef);
         } else {
-            nV = build_from_trits(P.start, P.start_words, n, s.nzV, s.sgV, s.vlist, s.wcnt, s.sci);
+            nV = build_from_trits(P.start, P.start_words, n, s.nzV, s.sgV, s.vlist, s);
         }
         for (int it = 0; it < P.iters; ++it) {
             if (mode != MODE_HALF_U) {
                 // ---- V-step: x = R^T u on this CTA's columns (§2.3 step 1, first half)
-                const CorrArgs ca{L, s.coef, s.pnzV, s.psgV, Wn};
-                gemv_dispatch(P.pv.vec, blkV, pitchV, validV, c0, s.ulist, nU, s.red, P.xbuf, ca, a);
-                publish_slot(slots + par * Gg + q, a, s.sc, s.scj);
-                if (!group_barrier(gs, target, Gg, cfg.limit_ns, skip, P.status, s.sci + 20)) return false;
-                gather_slots(slots + par * Gg, Gg, s.sc, s.scj);
+                gemv_dispatch(P.pv.vec, blkV, pitchV, validV, c0, s.ulist, nU, s.red, P.xbuf, hcV, S, M, J);
+                if (!publish_and_wait(slots + par * Gg + q, S, M, J, s, gs, target, Gg, cfg.limit_ns, skip, P.status))
+                    return false;
+                const int nv2 = gather_threshold(slots + par * Gg, Gg, P.xbuf, n, P.tau, s.nzV, s.sgV, s.vlist, s, L,
+                                                 s.pnzV, s.psgV, thr);
                 par ^= 1;
-                const double thr = P.tau * s.sc[0] / (double)n;
-                const long long J = s.scj[40];
-                __syncthreads();
-                nV = build_from_vector(P.xbuf, n, thr, s.nzV, s.sgV, s.vlist, s.wcnt, s.sci, s.sc + 8, nullptr);
-                if (nV == 0) { nV = apply_fallback(P.xbuf, n, J, s.nzV, s.sgV, s.vlist, nullptr); ++fb; }
+                fb += (s.scal[1] != 0.0) ? 1 : 0;
+                nV = nv2;
                 sum_nu += (unsigned long long)nU;
                 ++hs;
                 if (mode == MODE_HALF_V) {
@@ -597,25 +722,16 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
                     }
                     return true;
                 }
-                if (L > 0) pending_coef(L, Wn, s.pnzV, s.psgV, s.nzV, s.sgV, s.pd, s.coef);
             }
             // ---- U-step: y = R v on this CTA's rows (§2.3 step 1, second half)
-            const CorrArgs cu{L, s.coef, s.pnzU, s.psgU, Wm};
-            gemv_dispatch(P.pu.vec, blkU, pitchU, validU, r0, s.vlist, nV, s.red, P.ybuf, cu, a);
-            publish_slot(slots + par * Gg + q, a, s.sc, s.scj);
-            if (!group_barrier(gs, target, Gg, cfg.limit_ns, skip, P.status, s.sci + 20)) return false;
-            gather_slots(slots + par * Gg, Gg, s.sc, s.scj);
+            gemv_dispatch(P.pu.vec, blkU, pitchU, validU, r0, s.vlist, nV, s.red, P.ybuf, hcU, S, M, J);
+            if (!publish_and_wait(slots + par * Gg + q, S, M, J, s, gs, target, Gg, cfg.limit_ns, skip, P.status))
+                return false;
+            nU = gather_threshold(slots + par * Gg, Gg, P.ybuf, m, P.tau, s.nzU, s.sgU, s.ulist, s, L, s.pnzU,
+                                  s.psgU, thr);
             par ^= 1;
-            const double thr = P.tau * s.sc[0] / (double)m;
-            const long long J = s.scj[40];
-            __syncthreads();
-            nU = build_from_vector(P.ybuf, m, thr, s.nzU, s.sgU, s.ulist, s.wcnt, s.sci, s.sc + 8, &p);
-            if (nU == 0) {
-                nU = apply_fallback(P.ybuf, m, J, s.nzU, s.sgU, s.ulist, s.sc + 4);
-                p = s.sc[4];
-                ++fb;
-            }
-            __syncthreads();
+            p = s.scal[0];
+            fb += (s.scal[1] != 0.0) ? 1 : 0;
             sum_nv += (unsigned long long)nV;
             ++hs;
             if (mode == MODE_HALF_U) {
@@ -628,9 +744,8 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
                 }
                 return true;
             }
-            if (L > 0) pending_coef(L, Wm, s.pnzU, s.psgU, s.nzU, s.sgU, s.pd, s.coef);
         }
-        // ---- scale (§2.3 step 2): d = u^T R v / (nnz(u) nnz(v)), p = u^T y
+        // ---- scale (§2.3 step 2): d = u^T R v / (nnz(u) nnz(v)), with u^T R v = u^T y = p
         const double d = (p == 0.0) ? 0.0 : p / ((double)nU * (double)nV);
         RN2 -= p * d;
         sum_nunv += (unsigned long long)nU * (unsigned long long)nV;
@@ -647,11 +762,30 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
         if (tid == 0) s.pd[L] = d;
         for (int w = tid; w < Wm; w += NT) { s.pnzU[L * Wm + w] = s.nzU[w]; s.psgU[L * Wm + w] = s.sgU[w]; }
         for (int w = tid; w < Wn; w += NT) { s.pnzV[L * Wn + w] = s.nzV[w]; s.psgV[L * Wn + w] = s.sgV[w]; }
+        for (int c = tid; c < validV; c += NT) {
+            const int64_t gc = c0 + c;
+            const uint32_t b = 1u << (gc & 31);
+            if (s.nzV[gc >> 5] & b) {
+                s.cnzV[c] |= 1u << L;
+                if (s.sgV[gc >> 5] & b) s.csgV[c] |= 1u << L;
+            }
+        }
+        for (int r = tid; r < validU; r += NT) {
+            const int64_t gr = r0 + r;
+            const uint32_t b = 1u << (gr & 31);
+            if (s.nzU[gr >> 5] & b) {
+                s.cnzU[r] |= 1u << L;
+                if (s.sgU[gr >> 5] & b) s.csgU[r] |= 1u << L;
+            }
+        }
         ++L;
         __syncthreads();
         if (L == cfg.Lcap || i == kk - 1) {
-            flush_dispatch(P.pv.vec, blkV, pitchV, m, c0, validV, L, s.pd, s.pnzU, s.psgU, Wm, s.pnzV, s.psgV, Wn);
-            flush_dispatch(P.pu.vec, blkU, pitchU, n, r0, validU, L, s.pd, s.pnzV, s.psgV, Wn, s.pnzU, s.psgU, Wm);
+            flush_dispatch(P.pv.vec, blkV, pitchV, m, validV, L, s.pd, s.pnzU, s.psgU, Wm, s.cnzV, s.csgV);
+            flush_dispatch(P.pu.vec, blkU, pitchU, n, validU, L, s.pd, s.pnzV, s.psgV, Wn, s.cnzU, s.csgU);
+            __syncthreads();
+            for (int c = tid; c < pitchV; c += NT) { s.cnzV[c] = 0u; s.csgV[c] = 0u; }
+            for (int c = tid; c < pitchU; c += NT) { s.cnzU[c] = 0u; s.csgU[c] = 0u; }
             L = 0;
             __syncthreads();
         }
@@ -668,10 +802,9 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
             rs += v * v;
         }
     }
-    OutAcc ra{rs, 0.0, 0};
-    publish_slot(slots + par * Gg + q, ra, s.sc, s.scj);
-    if (!group_barrier(gs, target, Gg, cfg.limit_ns, skip, P.status, s.sci + 20)) return false;
-    gather_slots(slots + par * Gg, Gg, s.sc, s.scj);
+    if (!publish_and_wait(slots + par * Gg + q, rs, 0.0, 0, s, gs, target, Gg, cfg.limit_ns, skip, P.status))
+        return false;
+    const double R2 = gather_sum(slots + par * Gg, Gg, s);
     par ^= 1;
     if (lead && tid == 0) {
         P.stats->sum_nu = sum_nu;
@@ -679,7 +812,7 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
         P.stats->sum_nunv = sum_nunv;
         P.stats->half_steps = hs;
         P.stats->fallbacks = fb;
-        P.stats->residual2 = s.sc[0];
+        P.stats->residual2 = R2;
         P.stats->norm_a2 = N0;
         __threadfence();
         atomicExch(P.status, ST_OK);
@@ -693,25 +826,36 @@ __global__ void __launch_bounds__(NT, 1) als_kernel(const KCfg cfg) {
     const int grp = blockIdx.x / cfg.Gg;
     const int q = blockIdx.x - grp * cfg.Gg;
     const int Lc = cfg.Lcap > 0 ? cfg.Lcap : 1;
-    const int Wm = (cfg.m_max + 31) >> 5, Wn = (cfg.n_max + 31) >> 5;
+    const SmemLayout lay(cfg.m_max, cfg.n_max, Lc, cfg.pv_max, cfg.pu_max);
     Smem s;
-    s.red = reinterpret_cast<double*>(smem_raw);
-    s.sc = s.red + NT * 4;
-    s.pd = s.sc + 64;
-    s.coef = s.pd + Lc;
-    s.scj = reinterpret_cast<long long*>(s.coef + Lc);
-    s.sci = reinterpret_cast<int*>(s.scj + 64);
-    s.nzU = reinterpret_cast<uint32_t*>(s.sci + 64);
-    s.sgU = s.nzU + Wm;
-    s.nzV = s.sgU + Wm;
-    s.sgV = s.nzV + Wn;
-    s.pnzU = s.sgV + Wn;
-    s.psgU = s.pnzU + (size_t)Lc * Wm;
-    s.pnzV = s.psgU + (size_t)Lc * Wm;
-    s.psgV = s.pnzV + (size_t)Lc * Wn;
-    s.ulist = reinterpret_cast<int*>(s.psgV + (size_t)Lc * Wn);
-    s.vlist = s.ulist + cfg.m_max;
-    s.wcnt = s.vlist + cfg.n_max;
+    s.red = reinterpret_cast<double*>(smem_raw + lay.red);
+    s.pd = reinterpret_cast<double*>(smem_raw + lay.pd);
+    s.coef = reinterpret_cast<double*>(smem_raw + lay.coef);
+    s.scal = reinterpret_cast<double*>(smem_raw + lay.scal);
+    s.wS = reinterpret_cast<double*>(smem_raw + lay.wS);
+    s.wM = reinterpret_cast<double*>(smem_raw + lay.wM);
+    s.wp = reinterpret_cast<double*>(smem_raw + lay.wp);
+    s.gS = reinterpret_cast<double*>(smem_raw + lay.gS);
+    s.gM = reinterpret_cast<double*>(smem_raw + lay.gM);
+    s.wJ = reinterpret_cast<long long*>(smem_raw + lay.wJ);
+    s.gJ = reinterpret_cast<long long*>(smem_raw + lay.gJ);
+    s.wc = reinterpret_cast<int*>(smem_raw + lay.wc);
+    s.dotp = reinterpret_cast<int*>(smem_raw + lay.dotp);
+    s.sflag = reinterpret_cast<int*>(smem_raw + lay.sflag);
+    s.nzU = reinterpret_cast<uint32_t*>(smem_raw + lay.nzU);
+    s.sgU = reinterpret_cast<uint32_t*>(smem_raw + lay.sgU);
+    s.nzV = reinterpret_cast<uint32_t*>(smem_raw + lay.nzV);
+    s.sgV = reinterpret_cast<uint32_t*>(smem_raw + lay.sgV);
+    s.pnzU = reinterpret_cast<uint32_t*>(smem_raw + lay.pnzU);
+    s.psgU = reinterpret_cast<uint32_t*>(smem_raw + lay.psgU);
+    s.pnzV = reinterpret_cast<uint32_t*>(smem_raw + lay.pnzV);
+    s.psgV = reinterpret_cast<uint32_t*>(smem_raw + lay.psgV);
+    s.cnzV = reinterpret_cast<uint32_t*>(smem_raw + lay.cnzV);
+    s.csgV = reinterpret_cast<uint32_t*>(smem_raw + lay.csgV);
+    s.cnzU = reinterpret_cast<uint32_t*>(smem_raw + lay.cnzU);
+    s.csgU = reinterpret_cast<uint32_t*>(smem_raw + lay.csgU);
+    s.ulist = reinterpret_cast<int*>(smem_raw + lay.ulist);
+    s.vlist = reinterpret_cast<int*>(smem_raw + lay.vlist);
 
     GroupSync* gs = cfg.gsync + grp;
     Slot* slots = cfg.slots + (size_t)grp * 2 * cfg.Gg;
@@ -870,20 +1014,8 @@ Part make_part(int64_t len, int G, int vec) {
     return p;
 }
 
-size_t als_smem_bytes(int64_t m_max, int64_t n_max, int L) {
-    const int64_t Wm = (m_max + 31) / 32, Wn = (n_max + 31) / 32;
-    const int64_t Lc = L > 0 ? L : 1;
-    size_t b = 0;
-    b += 8 * (size_t)NT * 4;          // red
-    b += 8 * 64;                      // sc
-    b += 8 * 2 * (size_t)Lc;          // pd, coef
-    b += 8 * 64;                      // scj
-    b += 4 * 64;                      // sci
-    b += 4 * (size_t)(2 * Wm + 2 * Wn);
-    b += 4 * (size_t)(2 * Lc * Wm + 2 * Lc * Wn);
-    b += 4 * (size_t)(m_max + n_max);
-    b += 4 * (size_t)(Wm > Wn ? Wm : Wn);
-    return round_up(b, 16);
+size_t als_smem_bytes(int64_t m_max, int64_t n_max, int L, int pv_max, int pu_max) {
+    return SmemLayout(m_max, n_max, L > 0 ? L : 1, pv_max, pu_max).total;
 }
 
 struct ProbIn {
@@ -966,10 +1098,21 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
     if (Gg < 1) Gg = 1;
 
     // ---- lazy deflation depth from the shared-memory budget
+    if (Gg > NT) Gg = NT;   // one slot per thread when the group's slots are gathered
+    std::vector<int> vecv(np), vecu(np);
+    int pv_max = 1, pu_max = 1;
+    for (int b = 0; b < np; ++b) {
+        vecv[b] = choose_vec(in[b].n, Gg);
+        vecu[b] = choose_vec(in[b].m, Gg);
+        const int64_t uv = (in[b].n + vecv[b] - 1) / vecv[b], uu = (in[b].m + vecu[b] - 1) / vecu[b];
+        const int pv = (int)(((uv + Gg - 1) / Gg) * vecv[b]), pu = (int)(((uu + Gg - 1) / Gg) * vecu[b]);
+        pv_max = pv > pv_max ? pv : pv_max;
+        pu_max = pu > pu_max ? pu : pu_max;
+    }
     int Lcap = MAX_PENDING;
-    while (Lcap > 1 && als_smem_bytes(m_max, n_max, Lcap) > di.smem_optin) --Lcap;
+    while (Lcap > 1 && als_smem_bytes(m_max, n_max, Lcap, pv_max, pu_max) > di.smem_optin) --Lcap;
     if (opt.pending > 0 && opt.pending < Lcap) Lcap = opt.pending;
-    const size_t smem = als_smem_bytes(m_max, n_max, Lcap);
+    const size_t smem = als_smem_bytes(m_max, n_max, Lcap, pv_max, pu_max);
     if (smem > di.smem_optin) return EXTERND_ELIMIT;
 
     int nb = 0;
@@ -1000,7 +1143,7 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
     const size_t zero_from = ws;
     for (int b = 0; b < np; ++b) {
         const ProbIn& I = in[b];
-        const int vv = choose_vec(I.n, Gg), vu = choose_vec(I.m, Gg);
+        const int vv = vecv[b], vu = vecu[b];
         Prob& P = probs[b];
         memset(&P, 0, sizeof(P));
         P.m = I.m; P.n = I.n; P.k = I.k; P.tau = I.tau; P.iters = I.iters; P.mode = I.mode; P.seed = I.seed;
@@ -1130,6 +1273,8 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
             cfg.Lcap = Lcap;
             cfg.m_max = (int)m_max;
             cfg.n_max = (int)n_max;
+            cfg.pv_max = pv_max;
+            cfg.pu_max = pu_max;
             const double lim = opt.wait_limit_s > 0 ? opt.wait_limit_s : 2.0;
             cfg.limit_ns = (uint64_t)(lim * 1e9);
             cfg.fault_skip = opt.fault_skip;

@@ -136,6 +136,7 @@ struct KCfg {
     Slot* slots;              // NG x 2 x Gg
     int Lcap;                 // lazy deflation depth
     int m_max, n_max;         // for shared-memory carving
+    int pv_max, pu_max;       // largest stripe pitch of the two layouts
     uint64_t limit_ns;
     int fault_skip;           // CTA rank (within group) that never arrives; -1 = off
 };
