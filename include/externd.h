@@ -161,6 +161,8 @@ typedef struct {
     int pending;               /* lazy-deflation depth used */
     size_t smem_bytes;         /* dynamic shared memory per CTA */
     size_t workspace_bytes;
+    int64_t phase_cycles[4];   /* SM cycles spent by CTA 0 of matrix 0 in: GEMV, publish + wait,
+                                  gather + threshold, per-component work (start vector, output, deflation) */
 } externd_stats;
 
 int externd_last_stats(externd_stats* out);

@@ -57,10 +57,13 @@ class Stats(ctypes.Structure):
         ("pending", ctypes.c_int),
         ("smem_bytes", ctypes.c_size_t),
         ("workspace_bytes", ctypes.c_size_t),
+        ("phase_cycles", ctypes.c_int64 * 4),
     ]
 
     def as_dict(self):
-        return {name: getattr(self, name) for name, _ in self._fields_}
+        d = {name: getattr(self, name) for name, _ in self._fields_}
+        d["phase_cycles"] = list(self.phase_cycles)
+        return d
 
 
 _lib = None

@@ -242,7 +242,7 @@ __device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, i
     S = 0.0; M = -1.0; J = LLONG_MAX;
     const int nvec = pitch / VEC;
     if (nvec <= 0) return;
-    constexpr int U = (VEC == 4) ? 8 : 16;
+    constexpr int U = (VEC == 4) ? 16 : (VEC == 2 ? 24 : 32);
     if (nvec <= NT) {
         const int lanes = NT / nvec;
         const int j = threadIdx.x % nvec;
@@ -252,14 +252,20 @@ __device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, i
             #pragma unroll
             for (int e = 0; e < VEC; ++e) acc[e] = 0.0;
             const float* base = blk + j * VEC;
-            int idx = g;
-            for (; idx + (U - 1) * lanes < nlist; idx += U * lanes) {
+            // every batch issues all of its loads before using any (predicated tail)
+            for (int idx = g; idx < nlist; idx += U * lanes) {
                 int ent[U];
                 float v[U][VEC];
                 #pragma unroll
                 for (int u = 0; u < U; ++u) {
-                    ent[u] = list[idx + u * lanes];
-                    load_vec<VEC>(base + (int64_t)(ent[u] & 0x7fffffff) * pitch, v[u]);
+                    const int ii = idx + u * lanes;
+                    ent[u] = ii < nlist ? list[ii] : 0;
+                    if (ii < nlist) {
+                        load_vec<VEC>(base + (int64_t)(ent[u] & 0x7fffffff) * pitch, v[u]);
+                    } else {
+                        #pragma unroll
+                        for (int e = 0; e < VEC; ++e) v[u][e] = 0.f;
+                    }
                 }
                 #pragma unroll
                 for (int u = 0; u < U; ++u) {
@@ -267,14 +273,6 @@ __device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, i
                     #pragma unroll
                     for (int e = 0; e < VEC; ++e) acc[e] += (double)__uint_as_float(__float_as_uint(v[u][e]) ^ sm);
                 }
-            }
-            for (; idx < nlist; idx += lanes) {
-                const int ent = list[idx];
-                float v[VEC];
-                load_vec<VEC>(base + (int64_t)(ent & 0x7fffffff) * pitch, v);
-                const unsigned sm = (unsigned)ent & 0x80000000u;
-                #pragma unroll
-                for (int e = 0; e < VEC; ++e) acc[e] += (double)__uint_as_float(__float_as_uint(v[e]) ^ sm);
             }
             #pragma unroll
             for (int e = 0; e < VEC; ++e) red[g * pitch + j * VEC + e] = acc[e];
@@ -298,14 +296,19 @@ __device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, i
             #pragma unroll
             for (int e = 0; e < VEC; ++e) acc[e] = 0.0;
             const float* base = blk + j * VEC;
-            int idx = 0;
-            for (; idx + U - 1 < nlist; idx += U) {
+            for (int idx = 0; idx < nlist; idx += U) {
                 int ent[U];
                 float v[U][VEC];
                 #pragma unroll
                 for (int u = 0; u < U; ++u) {
-                    ent[u] = list[idx + u];
-                    load_vec<VEC>(base + (int64_t)(ent[u] & 0x7fffffff) * pitch, v[u]);
+                    const int ii = idx + u;
+                    ent[u] = ii < nlist ? list[ii] : 0;
+                    if (ii < nlist) {
+                        load_vec<VEC>(base + (int64_t)(ent[u] & 0x7fffffff) * pitch, v[u]);
+                    } else {
+                        #pragma unroll
+                        for (int e = 0; e < VEC; ++e) v[u][e] = 0.f;
+                    }
                 }
                 #pragma unroll
                 for (int u = 0; u < U; ++u) {
@@ -313,14 +316,6 @@ __device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, i
                     #pragma unroll
                     for (int e = 0; e < VEC; ++e) acc[e] += (double)__uint_as_float(__float_as_uint(v[u][e]) ^ sm);
                 }
-            }
-            for (; idx < nlist; ++idx) {
-                const int ent = list[idx];
-                float v[VEC];
-                load_vec<VEC>(base + (int64_t)(ent & 0x7fffffff) * pitch, v);
-                const unsigned sm = (unsigned)ent & 0x80000000u;
-                #pragma unroll
-                for (int e = 0; e < VEC; ++e) acc[e] += (double)__uint_as_float(__float_as_uint(v[e]) ^ sm);
             }
             #pragma unroll
             for (int e = 0; e < VEC; ++e) {
@@ -691,6 +686,16 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
     long long J;
     const HalfCorr hcV{s.coef, s.cnzV, s.csgV};
     const HalfCorr hcU{s.coef, s.cnzU, s.csgU};
+    // phase clock of thread 0 of CTA 0 (diagnostics; a few clock reads per half-step)
+    const bool tim = lead && tid == 0;
+    unsigned long long ph[4] = {0, 0, 0, 0};
+    long long t_prev = clock64();
+#define EXTERND_PHASE(k)                                   \
+    if (tim) {                                             \
+        const long long t_ = clock64();                    \
+        ph[k] += (unsigned long long)(t_ - t_prev);        \
+        t_prev = t_;                                       \
+    }
 
     for (int64_t i = 0; i < kk; ++i) {
         if (mode != MODE_HALF_U) {
@@ -702,11 +707,15 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
         for (int it = 0; it < P.iters; ++it) {
             if (mode != MODE_HALF_U) {
                 // ---- V-step: x = R^T u on this CTA's columns (§2.3 step 1, first half)
+                EXTERND_PHASE(3);
                 gemv_dispatch(P.pv.vec, blkV, pitchV, validV, c0, s.ulist, nU, s.red, P.xbuf, hcV, S, M, J);
+                EXTERND_PHASE(0);
                 if (!publish_and_wait(slots + par * Gg + q, S, M, J, s, gs, target, Gg, cfg.limit_ns, skip, P.status))
                     return false;
+                EXTERND_PHASE(1);
                 const int nv2 = gather_threshold(slots + par * Gg, Gg, P.xbuf, n, P.tau, s.nzV, s.sgV, s.vlist, s, L,
                                                  s.pnzV, s.psgV, thr);
+                EXTERND_PHASE(2);
                 par ^= 1;
                 fb += (s.scal[1] != 0.0) ? 1 : 0;
                 nV = nv2;
@@ -724,11 +733,15 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
                 }
             }
             // ---- U-step: y = R v on this CTA's rows (§2.3 step 1, second half)
+            EXTERND_PHASE(3);
             gemv_dispatch(P.pu.vec, blkU, pitchU, validU, r0, s.vlist, nV, s.red, P.ybuf, hcU, S, M, J);
+            EXTERND_PHASE(0);
             if (!publish_and_wait(slots + par * Gg + q, S, M, J, s, gs, target, Gg, cfg.limit_ns, skip, P.status))
                 return false;
+            EXTERND_PHASE(1);
             nU = gather_threshold(slots + par * Gg, Gg, P.ybuf, m, P.tau, s.nzU, s.sgU, s.ulist, s, L, s.pnzU,
                                   s.psgU, thr);
+            EXTERND_PHASE(2);
             par ^= 1;
             p = s.scal[0];
             fb += (s.scal[1] != 0.0) ? 1 : 0;
@@ -814,11 +827,14 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
         P.stats->fallbacks = fb;
         P.stats->residual2 = R2;
         P.stats->norm_a2 = N0;
+        EXTERND_PHASE(3);
+        for (int k2 = 0; k2 < 4; ++k2) P.stats->phase[k2] = ph[k2];
         __threadfence();
         atomicExch(P.status, ST_OK);
     }
     __syncthreads();
     return true;
+#undef EXTERND_PHASE
 }
 
 __global__ void __launch_bounds__(NT, 1) als_kernel(const KCfg cfg) {
@@ -1340,7 +1356,10 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
             st.components += in[b].k;
             st.half_steps += (int64_t)d.half_steps;
             st.fallbacks += (int64_t)d.fallbacks;
-            if (b == 0) st.residual_energy = d.norm_a2 > 0 ? 1.0 - d.residual2 / d.norm_a2 : 0.0;
+            if (b == 0) {
+                st.residual_energy = d.norm_a2 > 0 ? 1.0 - d.residual2 / d.norm_a2 : 0.0;
+                for (int k2 = 0; k2 < 4; ++k2) st.phase_cycles[k2] = (int64_t)d.phase[k2];
+            }
         }
     }
     rc = EXTERND_OK;

@@ -92,6 +92,7 @@ struct DevStats {
     double residual2;               // ||R_k||^2 from the final fp32 residual
     double norm_a2;
     double pad;
+    unsigned long long phase[4];    // SM cycles of CTA 0: GEMV, publish+wait, gather+threshold, per-component work
 };
 
 enum Mode { MODE_FACTOR = 0, MODE_HALF_V = 1, MODE_HALF_U = 2 };
