@@ -161,8 +161,9 @@ typedef struct {
     int pending;               /* lazy-deflation depth used */
     size_t smem_bytes;         /* dynamic shared memory per CTA */
     size_t workspace_bytes;
-    int64_t phase_cycles[4];   /* SM cycles spent by CTA 0 of matrix 0 in: GEMV, publish + wait,
-                                  gather + threshold, per-component work (start vector, output, deflation) */
+    int64_t phase_cycles[11];  /* [10]: exchanged words found not yet visible by CTA 0; [0..9]: SM cycles of CTA 0 of matrix 0 (diagnostics): GEMV loads, GEMV reduce +
+                                  emit, publish, wait, partials + first loads, threshold, compaction,
+                                  start vector, output + pending push, deflation fold */
 } externd_stats;
 
 int externd_last_stats(externd_stats* out);

@@ -57,7 +57,7 @@ class Stats(ctypes.Structure):
         ("pending", ctypes.c_int),
         ("smem_bytes", ctypes.c_size_t),
         ("workspace_bytes", ctypes.c_size_t),
-        ("phase_cycles", ctypes.c_int64 * 4),
+        ("phase_cycles", ctypes.c_int64 * 11),
     ]
 
     def as_dict(self):

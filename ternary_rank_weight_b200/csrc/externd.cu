@@ -139,12 +139,12 @@ __global__ void __launch_bounds__(NTI) init_kernel(const Prob* __restrict__ prob
 
 // Shared-memory carve of the ALS kernel (host and device use the same layout).
 struct SmemLayout {
-    size_t red, pd, coef, scal, wS, wM, wp, gS, gM, wJ, gJ, wc, dotp, sflag, nzU, sgU, nzV, sgV, pnzU, psgU, pnzV,
-        psgV, cnzV, csgV, cnzU, csgU, ulist, vlist, total;
+    size_t red, pd, coef, scal, wS, wM, wp, gS, gM, wJ, gJ, wc, dotp, sflag, clk, nzU, sgU, nzV, sgV, pnzU, psgU, pnzV,
+        psgV, cnzV, csgV, cnzU, csgU, ulist, vlist, corr, total;
     __host__ __device__ SmemLayout(int64_t m_max, int64_t n_max, int Lc, int pv_max, int pu_max) {
         const size_t Wm = (size_t)((m_max + 31) / 32), Wn = (size_t)((n_max + 31) / 32);
         size_t o = 0;
-        red = o;  o += 8 * (size_t)NT * 4;
+        red = o;  o += 8 * (size_t)NT * 5;   // lanes * (pitch + 1) <= NT * (VEC + 1)
         pd = o;   o += 8 * (size_t)Lc;
         coef = o; o += 8 * (size_t)Lc;
         scal = o; o += 8 * 16;
@@ -158,6 +158,7 @@ struct SmemLayout {
         wc = o;   o += 4 * NWARP;
         dotp = o; o += 4 * NWARP * MAX_PENDING;
         sflag = o; o += 16;
+        clk = o;  o += 8 * 12;
         nzU = o;  o += 4 * Wm;
         sgU = o;  o += 4 * Wm;
         nzV = o;  o += 4 * Wn;
@@ -172,19 +173,43 @@ struct SmemLayout {
         csgU = o; o += 4 * (size_t)pu_max;
         ulist = o; o += 4 * (size_t)m_max;
         vlist = o; o += 4 * (size_t)n_max;
+        o = (o + 7) & ~(size_t)7;
+        corr = o; o += 8 * (size_t)(pv_max > pu_max ? pv_max : pu_max);
         total = (o + 15) & ~(size_t)15;
     }
 };
 
 struct Smem {
-    double *red, *pd, *coef, *scal, *wS, *wM, *wp, *gS, *gM;
+    double *red, *pd, *coef, *scal, *wS, *wM, *wp, *gS, *gM;   // red: NT*5
     long long *wJ, *gJ;
     int *wc, *dotp, *sflag;
+    unsigned long long* clk;                 // [0..9] phase cycles, [11] last stamp (thread 0 of CTA 0)
     uint32_t *nzU, *sgU, *nzV, *sgV;         // current u, v
     uint32_t *pnzU, *psgU, *pnzV, *psgV;     // pending components (full length, stride W)
     uint32_t *cnzV, *csgV, *cnzU, *csgU;     // pending trits at this CTA's outputs, bit l = component l
-    int *ulist, *vlist;                      // compacted supports (index | sign << 31)
+    int *ulist, *vlist;                      // compacted supports: element offset (index * block pitch) | sign << 31
+    double* corr;                            // lazy-deflation correction per output of this CTA
 };
+
+// Phase clock (diagnostics): thread 0 of the first CTA adds the cycles since its
+// previous stamp to phase k.  A clock read and two shared-memory accesses.
+__device__ __forceinline__ void phase_mark(unsigned long long* clk, int k) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        const unsigned long long t = (unsigned long long)clock64();
+        clk[k] += t - clk[11];
+        clk[11] = t;
+    }
+}
+__device__ __forceinline__ void phase_mark(const Smem& s, int k) { phase_mark(s.clk, k); }
+
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// fp64 value with its 8 low mantissa bits replaced by a half-step tag (see the exchange below)
+__device__ __forceinline__ unsigned long long tag_value(double v, unsigned tag) {
+    return ((unsigned long long)__double_as_longlong(v) & ~0xFFull) | (unsigned long long)tag;
+}
 
 __device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
@@ -209,27 +234,61 @@ struct HalfCorr {
     const double* coef;
     const uint32_t* cnz;
     const uint32_t* csg;
+    double* corr;     // out: correction per output of this CTA (filled by the GEMV)
+    int L;
 };
 
-__device__ __forceinline__ double corr_local(int c, const HalfCorr& hc) {
-    uint32_t bits = hc.cnz[c];
-    const uint32_t sgn = hc.csg[c];
-    double v = 0.0;
-    while (bits) {
-        const int l = __ffs(bits) - 1;
-        bits &= bits - 1u;
-        v += ((sgn >> l) & 1u) ? -hc.coef[l] : hc.coef[l];
+// corr[c] = sum_l coef_l t_l(c) for this CTA's outputs: warp w takes outputs w, w+NWARP, ...;
+// lane l contributes component l, summed by a fixed butterfly.
+__device__ __forceinline__ void corrections(int valid, const HalfCorr& hc) {
+    if (hc.L <= 0) return;
+    const int lane = lane_id();
+    const double cl = lane < hc.L ? hc.coef[lane] : 0.0;
+    for (int c = warp_id(); c < valid; c += NWARP) {
+        const uint32_t z = hc.cnz[c], g = hc.csg[c];
+        double t = ((z >> lane) & 1u) ? (((g >> lane) & 1u) ? -cl : cl) : 0.0;
+        #pragma unroll
+        for (int o = 16; o; o >>= 1) t += __shfl_xor_sync(FULL, t, o);
+        if (lane == 0) hc.corr[c] = t;
     }
-    return v;
 }
 
-__device__ __forceinline__ void emit_out(double v, int c, int64_t out0, double* gout, const HalfCorr& hc, double& S,
-                                         double& M, long long& J) {
-    v -= corr_local(c, hc);
-    gout[out0 + c] = v;
-    const double av = fabs(v);
-    S += av;
-    if (av > M) { M = av; J = out0 + c; }
+// Publish one output word and fold its (published, 44-bit) value into this thread's
+// partial |.| sum and max.
+__device__ __forceinline__ void emit_tagged(double v, int64_t gi, unsigned long long* gout, unsigned tag, bool skip,
+                                            double& S) {
+    const unsigned long long w = tag_value(v, tag);
+    if (!skip) st_relaxed_u64(gout + gi, w);
+    S += fabs(__longlong_as_double((long long)(w & ~0xFFull)));
+}
+
+// acc += sum_u s_u v_u for one batch of loaded rows (s_u = sign bit of the list entry).
+// Default: every fp32 term is converted and added in fp64 (exact terms, fp64 sum).
+// EXTERND_PRESUM4: groups of 4 signed terms are first summed in fp32 (pairwise),
+// then converted and added in fp64.
+template <int VEC, int U>
+__device__ __forceinline__ void accumulate_batch(double* acc, const int* ent, float (*v)[VEC]) {
+#ifdef EXTERND_PRESUM4
+    static_assert(U % 4 == 0, "batch must be a multiple of 4");
+    #pragma unroll
+    for (int u = 0; u < U; u += 4) {
+        #pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+            const float a0 = __uint_as_float(__float_as_uint(v[u][e]) ^ ((unsigned)ent[u] & 0x80000000u));
+            const float a1 = __uint_as_float(__float_as_uint(v[u + 1][e]) ^ ((unsigned)ent[u + 1] & 0x80000000u));
+            const float a2 = __uint_as_float(__float_as_uint(v[u + 2][e]) ^ ((unsigned)ent[u + 2] & 0x80000000u));
+            const float a3 = __uint_as_float(__float_as_uint(v[u + 3][e]) ^ ((unsigned)ent[u + 3] & 0x80000000u));
+            acc[e] += (double)((a0 + a1) + (a2 + a3));
+        }
+    }
+#else
+    #pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const unsigned sm = (unsigned)ent[u] & 0x80000000u;
+        #pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[e] += (double)__uint_as_float(__float_as_uint(v[u][e]) ^ sm);
+    }
+#endif
 }
 
 // One half-step GEMV over this CTA's private block: out[c] = sum_{e in list} s_e blk[r_e][c]
@@ -237,16 +296,18 @@ __device__ __forceinline__ void emit_out(double v, int c, int64_t out0, double* 
 // gout[out0 + c].  fp64 accumulation of exact fp32 terms, fixed summation order.
 template <int VEC>
 __device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, int64_t out0,
-                          const int* __restrict__ list, int nlist, double* red, double* gout, const HalfCorr& hc,
-                          double& S, double& M, long long& J) {
-    S = 0.0; M = -1.0; J = LLONG_MAX;
+                          const int* __restrict__ list, int nlist, double* red, unsigned long long* gout,
+                          const HalfCorr& hc, unsigned tag, bool skip, double& S, unsigned long long* clk) {
+    S = 0.0;
     const int nvec = pitch / VEC;
     if (nvec <= 0) return;
-    constexpr int U = (VEC == 4) ? 16 : (VEC == 2 ? 24 : 32);
+    corrections(valid, hc);   // read after the CTA barrier below (or in the same thread)
+    constexpr int U = (NT >= 1024) ? ((VEC == 4) ? 8 : (VEC == 2 ? 12 : 16)) : ((VEC == 4) ? 16 : (VEC == 2 ? 24 : 32));
     if (nvec <= NT) {
         const int lanes = NT / nvec;
         const int j = threadIdx.x % nvec;
         const int g = threadIdx.x / nvec;
+        const int rs = pitch | 1;   // odd row stride (in doubles): the column sums below are bank-conflict free
         if (g < lanes) {
             double acc[VEC];
             #pragma unroll
@@ -261,23 +322,19 @@ __device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, i
                     const int ii = idx + u * lanes;
                     ent[u] = ii < nlist ? list[ii] : 0;
                     if (ii < nlist) {
-                        load_vec<VEC>(base + (int64_t)(ent[u] & 0x7fffffff) * pitch, v[u]);
+                        load_vec<VEC>(base + (ent[u] & 0x7fffffff), v[u]);
                     } else {
                         #pragma unroll
                         for (int e = 0; e < VEC; ++e) v[u][e] = 0.f;
                     }
                 }
-                #pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const unsigned sm = (unsigned)ent[u] & 0x80000000u;
-                    #pragma unroll
-                    for (int e = 0; e < VEC; ++e) acc[e] += (double)__uint_as_float(__float_as_uint(v[u][e]) ^ sm);
-                }
+                accumulate_batch<VEC, U>(acc, ent, v);
             }
             #pragma unroll
-            for (int e = 0; e < VEC; ++e) red[g * pitch + j * VEC + e] = acc[e];
+            for (int e = 0; e < VEC; ++e) red[g * rs + j * VEC + e] = acc[e];
         }
         __syncthreads();
+        phase_mark(clk, 0);
         int tpc = 1;
         while (tpc < 32 && tpc * 2 * pitch <= NT) tpc *= 2;
         const int cpr = NT / tpc;
@@ -286,11 +343,12 @@ __device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, i
             const int s = (int)threadIdx.x % tpc;
             double v = 0.0;
             if (c < pitch)
-                for (int gg = s; gg < lanes; gg += tpc) v += red[gg * pitch + c];
+                for (int gg = s; gg < lanes; gg += tpc) v += red[gg * rs + c];
             for (int o = tpc >> 1; o; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
-            if (s == 0 && c < valid) emit_out(v, c, out0, gout, hc, S, M, J);
+            if (s == 0 && c < valid) emit_tagged(hc.L > 0 ? v - hc.corr[c] : v, out0 + c, gout, tag, skip, S);
         }
     } else {
+        __syncthreads();   // corrections
         for (int j = threadIdx.x; j < nvec; j += NT) {
             double acc[VEC];
             #pragma unroll
@@ -304,86 +362,108 @@ __device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, i
                     const int ii = idx + u;
                     ent[u] = ii < nlist ? list[ii] : 0;
                     if (ii < nlist) {
-                        load_vec<VEC>(base + (int64_t)(ent[u] & 0x7fffffff) * pitch, v[u]);
+                        load_vec<VEC>(base + (ent[u] & 0x7fffffff), v[u]);
                     } else {
                         #pragma unroll
                         for (int e = 0; e < VEC; ++e) v[u][e] = 0.f;
                     }
                 }
-                #pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const unsigned sm = (unsigned)ent[u] & 0x80000000u;
-                    #pragma unroll
-                    for (int e = 0; e < VEC; ++e) acc[e] += (double)__uint_as_float(__float_as_uint(v[u][e]) ^ sm);
-                }
+                accumulate_batch<VEC, U>(acc, ent, v);
             }
             #pragma unroll
             for (int e = 0; e < VEC; ++e) {
                 const int c = j * VEC + e;
-                if (c < valid) emit_out(acc[e], c, out0, gout, hc, S, M, J);
+                if (c < valid) emit_tagged(hc.L > 0 ? acc[e] - hc.corr[c] : acc[e], out0 + c, gout, tag, skip, S);
             }
         }
     }
 }
 
 __device__ __forceinline__ void gemv_dispatch(int vec, const float* blk, int pitch, int valid, int64_t out0,
-                                              const int* list, int nlist, double* red, double* gout,
-                                              const HalfCorr& hc, double& S, double& M, long long& J) {
-    if (vec == 4) gemv_emit<4>(blk, pitch, valid, out0, list, nlist, red, gout, hc, S, M, J);
-    else if (vec == 2) gemv_emit<2>(blk, pitch, valid, out0, list, nlist, red, gout, hc, S, M, J);
-    else gemv_emit<1>(blk, pitch, valid, out0, list, nlist, red, gout, hc, S, M, J);
+                                              const int* list, int nlist, double* red, unsigned long long* gout,
+                                              const HalfCorr& hc, unsigned tag, bool skip, double& S,
+                                              unsigned long long* clk) {
+    if (vec == 4) gemv_emit<4>(blk, pitch, valid, out0, list, nlist, red, gout, hc, tag, skip, S, clk);
+    else if (vec == 2) gemv_emit<2>(blk, pitch, valid, out0, list, nlist, red, gout, hc, tag, skip, S, clk);
+    else gemv_emit<1>(blk, pitch, valid, out0, list, nlist, red, gout, hc, tag, skip, S, clk);
 }
 
 // Fold the L pending components into this CTA's block:
-// blk[r][c] -= sum_l d_l * tR_l(r) * tC_l(col0 + c), fp64 sum in increasing l, one fp32 rounding.
+// blk[r][c] -= sum_l d_l * tR_l(r) * tC_l(c), fp64 sum in increasing l, one fp32 rounding.
+// A warp takes 32 block rows at a time: the word-major pending masks of those rows
+// (lane l holds component l's 32 row bits) are bit-transposed with ballots so that
+// lane b holds row b's mask over the components; tC_l(c) comes from the
+// per-output masks cnz/csg.  scratch: 64 words per warp.
 template <int VEC>
-__device__ void flush_block(float* blk, int pitch, int64_t rows, int valid, int L, const double* pd,
-                            const uint32_t* pnzR, const uint32_t* psgR, int WR, const uint32_t* cnz,
-                            const uint32_t* csg) {
+__device__ void flush_block(float* blk, int pitch, int64_t rows, int valid, int L, int Ls, const double* pd,
+                            const uint32_t* pnzR, const uint32_t* psgR, const uint32_t* cnz, const uint32_t* csg,
+                            uint32_t* scratch) {
     const int nvec = pitch / VEC;
     if (nvec <= 0 || L <= 0) return;
-    const int64_t total = rows * nvec;
-    for (int64_t t = threadIdx.x; t < total; t += NT) {
-        const int64_t r = t / nvec;
-        const int j = (int)(t - r * nvec);
-        const int wr = (int)(r >> 5);
-        const uint32_t br = 1u << (r & 31);
-        uint32_t rnz = 0, rsg = 0;
-        for (int l = 0; l < L; ++l) {
-            rnz |= ((pnzR[l * WR + wr] & br) ? 1u : 0u) << l;
-            rsg |= ((psgR[l * WR + wr] & br) ? 1u : 0u) << l;
-        }
-        if (!rnz) continue;
-        float* p = blk + r * pitch + j * VEC;
+    const int lane = lane_id();
+    uint32_t* my = scratch + warp_id() * 64;
+    const int64_t WR = (rows + 31) >> 5;
+    for (int64_t wr = warp_id(); wr < WR; wr += NWARP) {
+        const uint32_t pz = lane < L ? pnzR[wr * Ls + lane] : 0u;
+        const uint32_t ps = lane < L ? psgR[wr * Ls + lane] : 0u;
+        uint32_t rz = 0u, rsg = 0u;
         #pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-            const int c = j * VEC + e;
-            if (c >= valid) continue;
-            uint32_t bits = rnz & cnz[c];
-            if (!bits) continue;
-            const uint32_t neg = rsg ^ csg[c];
-            double corr = 0.0;
-            while (bits) {
-                const int l = __ffs(bits) - 1;
-                bits &= bits - 1u;
-                corr += ((neg >> l) & 1u) ? -pd[l] : pd[l];
-            }
-            p[e] = (float)((double)__ldcg(p + e) - corr);
+        for (int b = 0; b < 32; ++b) {
+            const uint32_t z = __ballot_sync(FULL, (pz >> b) & 1u);
+            const uint32_t g = __ballot_sync(FULL, (ps >> b) & 1u);
+            if (lane == b) { rz = z; rsg = g; }
         }
+        my[lane] = rz;
+        my[32 + lane] = rsg;
+        __syncwarp();
+        const int nrows = (int)min((int64_t)32, rows - (wr << 5));
+        const int pairs = nrows * nvec;
+        for (int t = lane; t < pairs; t += 32) {
+            const int b = t / nvec;
+            const int j = t - b * nvec;
+            const uint32_t rnz = my[b];
+            if (!rnz) continue;
+            const uint32_t rsn = my[32 + b];
+            float* p = blk + ((wr << 5) + b) * pitch + j * VEC;
+            float v[VEC];
+            load_vec<VEC>(p, v);
+            bool changed = false;
+            #pragma unroll
+            for (int e = 0; e < VEC; ++e) {
+                const int c = j * VEC + e;
+                if (c >= valid) continue;
+                uint32_t bits = rnz & cnz[c];
+                if (!bits) continue;
+                const uint32_t neg = rsn ^ csg[c];
+                double corr = 0.0;
+                while (bits) {
+                    const int l = __ffs(bits) - 1;
+                    bits &= bits - 1u;
+                    corr += ((neg >> l) & 1u) ? -pd[l] : pd[l];
+                }
+                v[e] = (float)((double)v[e] - corr);
+                changed = true;
+            }
+            if (changed) {
+                #pragma unroll
+                for (int e = 0; e < VEC; ++e) p[e] = v[e];
+            }
+        }
+        __syncwarp();
     }
 }
 
-__device__ __forceinline__ void flush_dispatch(int vec, float* blk, int pitch, int64_t rows, int valid, int L,
-                                               const double* pd, const uint32_t* pnzR, const uint32_t* psgR, int WR,
-                                               const uint32_t* cnz, const uint32_t* csg) {
-    if (vec == 4) flush_block<4>(blk, pitch, rows, valid, L, pd, pnzR, psgR, WR, cnz, csg);
-    else if (vec == 2) flush_block<2>(blk, pitch, rows, valid, L, pd, pnzR, psgR, WR, cnz, csg);
-    else flush_block<1>(blk, pitch, rows, valid, L, pd, pnzR, psgR, WR, cnz, csg);
+__device__ __forceinline__ void flush_dispatch(int vec, float* blk, int pitch, int64_t rows, int valid, int L, int Ls,
+                                               const double* pd, const uint32_t* pnzR, const uint32_t* psgR,
+                                               const uint32_t* cnz, const uint32_t* csg, uint32_t* scratch) {
+    if (vec == 4) flush_block<4>(blk, pitch, rows, valid, L, Ls, pd, pnzR, psgR, cnz, csg, scratch);
+    else if (vec == 2) flush_block<2>(blk, pitch, rows, valid, L, Ls, pd, pnzR, psgR, cnz, csg, scratch);
+    else flush_block<1>(blk, pitch, rows, valid, L, Ls, pd, pnzR, psgR, cnz, csg, scratch);
 }
 
 // Start trits (2-bit packed words) -> masks and list; returns nnz.
 __device__ int build_from_trits(const uint32_t* words, int64_t nwords, int64_t len, uint32_t* nz, uint32_t* sg,
-                                int* list, const Smem& s) {
+                                int* list, int rowpitch, const Smem& s) {
     const int W = (int)((len + 31) >> 5);
     const int wpw = (W + NWARP - 1) / NWARP;
     const int w0 = min(W, warp_id() * wpw), w1 = min(W, w0 + wpw);
@@ -416,7 +496,7 @@ __device__ int build_from_trits(const uint32_t* words, int64_t nwords, int64_t l
         const uint32_t bz = nz[w];
         if ((bz >> lane_id()) & 1u)
             list[run + __popc(bz & ((1u << lane_id()) - 1u))] =
-                (int)(((unsigned)w << 5) + lane_id()) | (int)(((sg[w] >> lane_id()) & 1u) << 31);
+                (int)((((unsigned)w << 5) + lane_id()) * (unsigned)rowpitch) | (int)(((sg[w] >> lane_id()) & 1u) << 31);
         run += __popc(bz);
     }
     __syncthreads();
@@ -424,13 +504,13 @@ __device__ int build_from_trits(const uint32_t* words, int64_t nwords, int64_t l
 }
 
 // coef_l = d_l * (t_l . t) for every pending component (integer dot product of trit masks)
-__device__ void pending_coef(int L, int W, const uint32_t* pnz, const uint32_t* psg, const uint32_t* nz,
+__device__ void pending_coef(int L, int Ls, int W, const uint32_t* pnz, const uint32_t* psg, const uint32_t* nz,
                              const uint32_t* sg, const double* pd, double* coef) {
     for (int l = warp_id(); l < L; l += NWARP) {
         int acc = 0;
         for (int w = lane_id(); w < W; w += 32) {
-            const uint32_t both = pnz[l * W + w] & nz[w];
-            const uint32_t diff = psg[l * W + w] ^ sg[w];
+            const uint32_t both = pnz[w * Ls + l] & nz[w];
+            const uint32_t diff = psg[w * Ls + l] ^ sg[w];
             acc += __popc(both & ~diff) - __popc(both & diff);
         }
         #pragma unroll
@@ -452,108 +532,153 @@ __device__ void pack_row(const uint32_t* nz, const uint32_t* sg, int W, uint32_t
     }
 }
 
-// Publish this CTA's (sum |out|, max |out|, argmax) and arrive at the group counter,
-// then wait until every CTA of the group arrived.  Arrival is a release by one
-// thread after a CTA barrier, the wait an acquire by the same thread followed by a
-// CTA barrier, so the slice of the output vector each CTA stored before arriving
-// is visible to all CTAs after the wait.  Bounded by limit_ns; on expiry the group
-// abort flag and the status word are raised.
-__device__ bool publish_and_wait(Slot* slot, double S, double M, long long J, const Smem& s, GroupSync* gs,
-                                 unsigned& target, int Gg, uint64_t limit_ns, bool skip_arrive, int* status) {
-    #pragma unroll
-    for (int o = 16; o; o >>= 1) {
-        S += __shfl_xor_sync(FULL, S, o);
-        const double m2 = __shfl_xor_sync(FULL, M, o);
-        const long long j2 = __shfl_xor_sync(FULL, J, o);
-        maxloc_merge(M, J, m2, j2);
+// ---------------------------------------------------------------------------
+// Exchange of the half-step outputs between the CTAs of a group.
+//
+// Each output value is published as one 8-byte word: the fp64 value with its 8
+// low mantissa bits replaced by a tag that names the half-step (1..255).  An
+// 8-byte relaxed store/load at gpu scope is single-copy atomic, so a reader that
+// sees the expected tag sees the value of that half-step, with no flag, fence or
+// counter.  The value keeps 44 mantissa bits (relative change < 2^-44); every CTA
+// reads the same words, so all of them derive the same threshold and trits.  A
+// buffer is rewritten only two half-steps later, after every CTA has read it, so a
+// stale word always carries the tag of two half-steps before.
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ double untag(unsigned long long b) { return __longlong_as_double((long long)(b & ~0xFFull)); }
+
+// half-step counter -> tag in 1..255 (0 is the zero-initialised buffer)
+__device__ __forceinline__ unsigned gen_tag(unsigned gen) { return (gen % 255u) + 1u; }
+
+// Bounded spin until *p carries `tag`; returns the word, or sets ok = 0 on timeout/abort.
+__device__ __forceinline__ unsigned long long wait_tagged(const unsigned long long* p, unsigned tag, GroupSync* gs,
+                                                          uint64_t limit_ns, int* status, int& ok,
+                                                          unsigned long long* stale_ctr = nullptr) {
+    unsigned long long b = ld_relaxed_u64(p);
+    if ((unsigned)(b & 0xFFull) == tag) return b;
+    if (stale_ctr && blockIdx.x == 0) atomicAdd(stale_ctr, 1ull);
+    const uint64_t t0 = gtimer();
+    unsigned spins = 0;
+    while (true) {
+        b = ld_relaxed_u64(p);
+        if ((unsigned)(b & 0xFFull) == tag) return b;
+        if ((++spins & 15u) == 0u) {
+            if (ld_relaxed_s32(&gs->abort)) { ok = 0; return 0ull; }
+            if (gtimer() - t0 > limit_ns) {
+                atomicExch(&gs->abort, 1);
+                atomicCAS(status, ST_RUNNING, ST_ETIMEOUT);
+                ok = 0;
+                return 0ull;
+            }
+        }
     }
-    if (lane_id() == 0) { s.wS[warp_id()] = S; s.wM[warp_id()] = M; s.wJ[warp_id()] = J; }
+}
+
+__device__ __forceinline__ void red_relaxed_add(unsigned* p, unsigned v) {
+    asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Publish this CTA's partial sum |out| of the half-step as a tagged word
+// partials[q] and count its arrival on counter q % NCTR; wait until every CTA of
+// the group has arrived (NCTR threads poll one counter each, bounded), read all
+// partials (tag-checked), read the whole output vector (tag-checked, re-polling any
+// word not yet visible), threshold it (T_tau of §2.2 with the all-zero fallback),
+// write its masks and compacted support list, the coefficients d_l (t_l . t) of the
+// pending components for the next half-step, and p = sum over the support of |x|
+// into s.scal[0] (s.scal[1] = 1 if the fallback was taken).  Sums are combined in
+// one fixed order, so every CTA of the group derives identical results.  Arrival
+// needs no fence: the tags validate every word that is read.
+// Returns nnz; ok = false if a wait ran out.
+__device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, unsigned tag, unsigned& arrivals,
+                                  bool skip, double S, const unsigned long long* gvec, int64_t len, double tau,
+                                  uint32_t* nz, uint32_t* sg, int* list, int rowpitch, const Smem& s, int L, int Ls,
+                                  const uint32_t* pnz, const uint32_t* psg, double& thr_out, GroupSync* gs,
+                                  uint64_t limit_ns, int* status, bool& ok_out) {
+    const int lane = lane_id(), warp = warp_id();
+    // ---- this CTA's partial (fixed butterfly + fixed cross-warp combine)
+    #pragma unroll
+    for (int o = 16; o; o >>= 1) S += __shfl_xor_sync(FULL, S, o);
+    if (lane == 0) s.wS[warp] = S;
     __syncthreads();
-    if (threadIdx.x == 0) {
-        double S2 = 0.0, M2 = -1.0;
-        long long J2 = LLONG_MAX;
-        for (int w = 0; w < NWARP; ++w) { S2 += s.wS[w]; maxloc_merge(M2, J2, s.wM[w], s.wJ[w]); }
-        slot->S = S2;
-        slot->M = M2;
-        slot->J = J2;
-        target += (unsigned)Gg;
-        if (!skip_arrive) red_release_add(&gs->arrive, 1u);
-        int ok = 1;
-        const uint64_t t0 = gtimer();
-        unsigned spins = 0;
-        while ((int)(ld_acquire_u32(&gs->arrive) - target) < 0) {
-            if ((++spins & 15u) == 0u) {
-                if (ld_relaxed_s32(&gs->abort)) { ok = 0; break; }
-                if (gtimer() - t0 > limit_ns) {
-                    atomicExch(&gs->abort, 1);
-                    atomicCAS(status, ST_RUNNING, ST_ETIMEOUT);
-                    ok = 0;
-                    break;
+    if (warp == 0) {
+        double S2 = lane < NWARP ? s.wS[lane] : 0.0;
+        #pragma unroll
+        for (int o = 16; o; o >>= 1) S2 += __shfl_xor_sync(FULL, S2, o);
+        if (lane == 0 && !skip) {
+            st_relaxed_u64(partials + q, tag_value(S2, tag));
+#ifdef EXTERND_RELEASE_ARRIVE
+            red_release_add(&gs->ctr[q % NCTR][0], 1u);
+#else
+            red_relaxed_add(&gs->ctr[q % NCTR][0], 1u);
+#endif
+        }
+    }
+    ++arrivals;
+    phase_mark(s, 2);
+    // ---- wait for all arrivals, then everyone's partials
+    int ok = 1;
+    if ((int)threadIdx.x < NCTR && (int)threadIdx.x < Gg) {
+        const int c = threadIdx.x;
+        const unsigned want = arrivals * (unsigned)((Gg - c + NCTR - 1) / NCTR);
+        const unsigned* ctr = &gs->ctr[c][0];
+        if ((int)(ld_relaxed_u32(ctr) - want) < 0) {
+            const uint64_t t0 = gtimer();
+            unsigned spins = 0;
+            while ((int)(ld_relaxed_u32(ctr) - want) < 0) {
+                if ((++spins & 15u) == 0u) {
+                    if (ld_relaxed_s32(&gs->abort)) { ok = 0; break; }
+                    if (gtimer() - t0 > limit_ns) {
+                        atomicExch(&gs->abort, 1);
+                        atomicCAS(status, ST_RUNNING, ST_ETIMEOUT);
+                        ok = 0;
+                        break;
+                    }
                 }
             }
         }
-        *s.sflag = ok;
     }
-    __syncthreads();
-    return *s.sflag != 0;
-}
-
-// After publish_and_wait: sum of the group's published S in a fixed order.
-__device__ double gather_sum(const Slot* sl, int Gg, const Smem& s) {
-    double S = ((int)threadIdx.x < Gg) ? __ldcg(&sl[threadIdx.x].S) : 0.0;
-    #pragma unroll
-    for (int o = 16; o; o >>= 1) S += __shfl_xor_sync(FULL, S, o);
-    if (lane_id() == 0) s.gS[warp_id()] = S;
-    __syncthreads();
-    double t = 0.0;
-    for (int w = 0; w < NWARP; ++w) t += s.gS[w];
-    __syncthreads();
-    return t;
-}
-
-// After publish_and_wait: read the group's slots and the whole published vector,
-// threshold it (T_tau of §2.2 with the all-zero fallback), write its masks and
-// compacted support list, the coefficients d_l (t_l . t) of the pending
-// components for the next half-step, and p = sum over the support of |x| into
-// s.scal[0].  Every CTA of the group derives identical results (same data, same
-// order).  Returns nnz.
-__device__ int gather_threshold(const Slot* sl, int Gg, const double* gvec, int64_t len, double tau, uint32_t* nz,
-                                uint32_t* sg, int* list, const Smem& s, int L, const uint32_t* pnz,
-                                const uint32_t* psg, double& thr_out) {
-    const int lane = lane_id(), warp = warp_id();
+    ok = __syncthreads_and(ok);
+    phase_mark(s, 3);
+    if (!ok) { ok_out = false; return 0; }
+    // the first chunk of this warp's words is loaded together with the partials
     const int W = (int)((len + 31) >> 5);
     const int wpw = (W + NWARP - 1) / NWARP;
     const int w0 = min(W, warp * wpw), w1 = min(W, w0 + wpw);
-    double S = 0.0, M = -1.0;
-    long long J = LLONG_MAX;
-    if ((int)threadIdx.x < Gg) {
-        S = __ldcg(&sl[threadIdx.x].S);
-        M = __ldcg(&sl[threadIdx.x].M);
-        J = __ldcg(&sl[threadIdx.x].J);
-    }
-    constexpr int CH = 16;
-    double xv[CH];
+    constexpr int CH = (NT >= 1024) ? 8 : 16;
+    unsigned long long wb[CH];
     #pragma unroll
     for (int i = 0; i < CH; ++i) {
         const int w = w0 + i;
         const int64_t idx = ((int64_t)w << 5) + lane;
-        xv[i] = (w < w1 && idx < len) ? __ldcg(gvec + idx) : 0.0;
+        wb[i] = (w < w1 && idx < len) ? ld_relaxed_u64(gvec + idx) : (unsigned long long)tag;
     }
+    double Sq = 0.0;
+    if ((int)threadIdx.x < Gg) Sq = untag(wait_tagged(partials + threadIdx.x, tag, gs, limit_ns, status, ok));
     #pragma unroll
-    for (int o = 16; o; o >>= 1) {
-        S += __shfl_xor_sync(FULL, S, o);
-        const double m2 = __shfl_xor_sync(FULL, M, o);
-        const long long j2 = __shfl_xor_sync(FULL, J, o);
-        maxloc_merge(M, J, m2, j2);
-    }
-    if (lane == 0) { s.gS[warp] = S; s.gM[warp] = M; s.gJ[warp] = J; }
-    __syncthreads();
-    double St = 0.0, Mt = -1.0;
-    long long Jt = LLONG_MAX;
-    for (int w = 0; w < NWARP; ++w) { St += s.gS[w]; maxloc_merge(Mt, Jt, s.gM[w], s.gJ[w]); }
+    for (int o = 16; o; o >>= 1) Sq += __shfl_xor_sync(FULL, Sq, o);
+    if (lane == 0) s.gS[warp] = Sq;
+    ok = __syncthreads_and(ok);
+    phase_mark(s, 4);
+    if (!ok) { ok_out = false; return 0; }
+    double St = lane < NWARP ? s.gS[lane] : 0.0;
+    #pragma unroll
+    for (int o = 16; o; o >>= 1) St += __shfl_xor_sync(FULL, St, o);
     const double thr = tau * St / (double)len;
     thr_out = thr;
 
+    // ---- one pass over the vector: threshold, masks, counts, pending dots
     int cnt = 0, dot = 0;
     double ps = 0.0;
     for (int base = w0; base < w1; base += CH) {
@@ -562,24 +687,30 @@ __device__ int gather_threshold(const Slot* sl, int Gg, const double* gvec, int6
             for (int i = 0; i < CH; ++i) {
                 const int w = base + i;
                 const int64_t idx = ((int64_t)w << 5) + lane;
-                xv[i] = (w < w1 && idx < len) ? __ldcg(gvec + idx) : 0.0;
+                wb[i] = (w < w1 && idx < len) ? ld_relaxed_u64(gvec + idx) : (unsigned long long)tag;
             }
+        }
+        #pragma unroll
+        for (int i = 0; i < CH; ++i) {
+            if ((unsigned)(wb[i] & 0xFFull) != tag)
+                wb[i] = wait_tagged(gvec + ((int64_t)(base + i) << 5) + lane, tag, gs, limit_ns, status, ok, s.clk + 10);
         }
         #pragma unroll
         for (int i = 0; i < CH; ++i) {
             const int w = base + i;
             if (w < w1) {
                 const int64_t idx = ((int64_t)w << 5) + lane;
-                const bool z = (idx < len) && (fabs(xv[i]) > thr);
-                const bool ng = z && (xv[i] < 0.0);
+                const double x = untag(wb[i]);
+                const bool z = (idx < len) && (fabs(x) > thr);
+                const bool ng = z && (x < 0.0);
                 const unsigned bz = __ballot_sync(FULL, z);
                 const unsigned bs = __ballot_sync(FULL, ng);
                 if (lane == 0) { nz[w] = bz; sg[w] = bs; }
                 cnt += __popc(bz);
-                if (z) ps += fabs(xv[i]);
+                if (z) ps += fabs(x);
                 if (lane < L) {
-                    const uint32_t both = pnz[lane * W + w] & bz;
-                    const uint32_t diff = psg[lane * W + w] ^ bs;
+                    const uint32_t both = pnz[w * Ls + lane] & bz;
+                    const uint32_t diff = psg[w * Ls + lane] ^ bs;
                     dot += __popc(both & ~diff) - __popc(both & diff);
                 }
             }
@@ -589,15 +720,21 @@ __device__ int gather_threshold(const Slot* sl, int Gg, const double* gvec, int6
     for (int o = 16; o; o >>= 1) ps += __shfl_xor_sync(FULL, ps, o);
     if (lane == 0) { s.wc[warp] = cnt; s.wp[warp] = ps; }
     if (lane < L) s.dotp[warp * MAX_PENDING + lane] = dot;
-    __syncthreads();
-    int off = 0, total = 0;
-    double p = 0.0;
-    for (int w = 0; w < NWARP; ++w) {
-        const int c = s.wc[w];
-        off += (w < warp) ? c : 0;
-        total += c;
-        p += s.wp[w];
+    ok = __syncthreads_and(ok);
+    phase_mark(s, 5);
+    if (!ok) { ok_out = false; return 0; }
+    int cw = lane < NWARP ? s.wc[lane] : 0;
+    double p = lane < NWARP ? s.wp[lane] : 0.0;
+    int incl = cw;
+    #pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(FULL, incl, o);
+        if (lane >= o) incl += t;
     }
+    const int off = __shfl_sync(FULL, incl - cw, warp);
+    const int total = __shfl_sync(FULL, incl, 31);
+    #pragma unroll
+    for (int o = 16; o; o >>= 1) p += __shfl_xor_sync(FULL, p, o);
     if (total > 0) {
         if ((int)threadIdx.x < L) {
             int d = 0;
@@ -609,39 +746,62 @@ __device__ int gather_threshold(const Slot* sl, int Gg, const double* gvec, int6
             const uint32_t bz = nz[w];
             if ((bz >> lane) & 1u)
                 list[run + __popc(bz & ((1u << lane) - 1u))] =
-                    (int)(((unsigned)w << 5) + lane) | (int)(((sg[w] >> lane) & 1u) << 31);
+                    (int)((((unsigned)w << 5) + lane) * (unsigned)rowpitch) | (int)(((sg[w] >> lane) & 1u) << 31);
             run += __popc(bz);
         }
         if (threadIdx.x == 0) { s.scal[0] = p; s.scal[1] = 0.0; }
     } else {
         // all-zero fallback: keep the lowest index among the largest magnitudes
+        // (every CTA scans the same vector in the same order)
+        double Mx = -1.0;
+        long long Jx = LLONG_MAX;
+        for (int64_t i = threadIdx.x; i < len; i += NT) {
+            const double a = fabs(untag(ld_relaxed_u64(gvec + i)));
+            if (a > Mx) { Mx = a; Jx = i; }
+        }
+        long long Jt = Jx;
+        block_maxloc(Mx, Jt, s.red, reinterpret_cast<long long*>(s.red + 64));   // red is free here
         const long long Jc = (Jt >= 0 && Jt < len) ? Jt : 0;   // out of range only with non-finite data
-        const double x = __ldcg(gvec + Jc);
+        const double x = untag(ld_relaxed_u64(gvec + Jc));
         const bool neg = x < 0.0;
         const int wj = (int)(Jc >> 5);
         const uint32_t bj = 1u << (Jc & 31);
         if ((int)threadIdx.x < L) {
-            int t = (pnz[threadIdx.x * W + wj] & bj) ? 1 : 0;
-            if (t && ((psg[threadIdx.x * W + wj] & bj) != 0u) != neg) t = -1;
+            int t = (pnz[wj * Ls + threadIdx.x] & bj) ? 1 : 0;
+            if (t && ((psg[wj * Ls + threadIdx.x] & bj) != 0u) != neg) t = -1;
             s.coef[threadIdx.x] = s.pd[threadIdx.x] * (double)t;
         }
         if (threadIdx.x == 0) {
             nz[wj] |= bj;
             if (neg) sg[wj] |= bj;
-            list[0] = (int)Jc | (neg ? (int)0x80000000 : 0);
+            list[0] = (int)((unsigned)Jc * (unsigned)rowpitch) | (neg ? (int)0x80000000 : 0);
             s.scal[0] = fabs(x);
             s.scal[1] = 1.0;
         }
-        total = 1;
     }
     __syncthreads();
-    return total;
+    phase_mark(s, 6);
+    ok_out = true;
+    return total > 0 ? total : 1;
+}
+
+// Sum of one fp64 value per CTA of the group (fixed order), exchanged as tagged words.
+__device__ bool exchange_sum(unsigned long long* sums, int q, int Gg, double v, const Smem& s, GroupSync* gs,
+                             uint64_t limit_ns, int* status, bool skip, double& out) {
+    const double t = block_sum(v, s.red);
+    if (threadIdx.x == 0 && !skip) st_relaxed_u64(sums + q, tag_value(t, 1u));
+    int ok = 1;
+    double x = 0.0;
+    if ((int)threadIdx.x < Gg) x = untag(wait_tagged(sums + threadIdx.x, 1u, gs, limit_ns, status, ok));
+    ok = __syncthreads_and(ok);
+    if (!ok) return false;
+    out = block_sum(x, s.red);
+    return true;
 }
 
 // Factor (or run one debug half-step of) one matrix with this CTA group.
 // Returns false if the group aborted.
-__device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s, GroupSync* gs, Slot* slots,
-                            unsigned& target, int& par) {
+__device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s, GroupSync* gs, unsigned& arrivals) {
     const int64_t m = P.m, n = P.n;
     const int Wm = (int)((m + 31) >> 5), Wn = (int)((n + 31) >> 5);
     const int mode = P.mode;
@@ -649,6 +809,7 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
     const int tid = threadIdx.x;
     const bool lead = (q == 0);
     const bool skip = (cfg.fault_skip == q);
+    const int Ls = cfg.Lcap > 0 ? cfg.Lcap : 1;   // stride of the word-major pending masks
 
     float* blkV = P.Rv + P.pv.block_offset(q, m);
     const int pitchV = P.pv.pitch(q);
@@ -682,48 +843,44 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
     unsigned long long sum_nu = 0, sum_nv = 0, sum_nunv = 0, hs = 0, fb = 0;
     const int64_t kk = (mode == MODE_FACTOR) ? P.k : 1;
     int nU = 0, nV = 0;
-    double p = 0.0, S, M, thr;
-    long long J;
-    const HalfCorr hcV{s.coef, s.cnzV, s.csgV};
-    const HalfCorr hcU{s.coef, s.cnzU, s.csgU};
-    // phase clock of thread 0 of CTA 0 (diagnostics; a few clock reads per half-step)
-    const bool tim = lead && tid == 0;
-    unsigned long long ph[4] = {0, 0, 0, 0};
-    long long t_prev = clock64();
-#define EXTERND_PHASE(k)                                   \
-    if (tim) {                                             \
-        const long long t_ = clock64();                    \
-        ph[k] += (unsigned long long)(t_ - t_prev);        \
-        t_prev = t_;                                       \
+    double p = 0.0, thr;
+    unsigned gen = 0;   // half-step counter of this matrix (tags of the exchanged words)
+    HalfCorr hcV{s.coef, s.cnzV, s.csgV, s.corr, 0};
+    HalfCorr hcU{s.coef, s.cnzU, s.csgU, s.corr, 0};
+    if (blockIdx.x == 0 && tid == 0) {
+        for (int k2 = 0; k2 < 11; ++k2) s.clk[k2] = 0ull;
+        s.clk[11] = (unsigned long long)clock64();
     }
 
     for (int64_t i = 0; i < kk; ++i) {
         if (mode != MODE_HALF_U) {
-            nU = build_from_trits(P.start + i * P.start_words, P.start_words, m, s.nzU, s.sgU, s.ulist, s);
-            if (L > 0) pending_coef(L, Wm, s.pnzU, s.psgU, s.nzU, s.sgU, s.pd, s.coef);
+            nU = build_from_trits(P.start + i * P.start_words, P.start_words, m, s.nzU, s.sgU, s.ulist, pitchV, s);
+            if (L > 0) pending_coef(L, Ls, Wm, s.pnzU, s.psgU, s.nzU, s.sgU, s.pd, s.coef);
         } else {
-            nV = build_from_trits(P.start, P.start_words, n, s.nzV, s.sgV, s.vlist, s);
+            nV = build_from_trits(P.start, P.start_words, n, s.nzV, s.sgV, s.vlist, pitchU, s);
         }
+        phase_mark(s, 7);
         for (int it = 0; it < P.iters; ++it) {
             if (mode != MODE_HALF_U) {
                 // ---- V-step: x = R^T u on this CTA's columns (§2.3 step 1, first half)
-                EXTERND_PHASE(3);
-                gemv_dispatch(P.pv.vec, blkV, pitchV, validV, c0, s.ulist, nU, s.red, P.xbuf, hcV, S, M, J);
-                EXTERND_PHASE(0);
-                if (!publish_and_wait(slots + par * Gg + q, S, M, J, s, gs, target, Gg, cfg.limit_ns, skip, P.status))
-                    return false;
-                EXTERND_PHASE(1);
-                const int nv2 = gather_threshold(slots + par * Gg, Gg, P.xbuf, n, P.tau, s.nzV, s.sgV, s.vlist, s, L,
-                                                 s.pnzV, s.psgV, thr);
-                EXTERND_PHASE(2);
-                par ^= 1;
+                phase_mark(s, 6);
+                const unsigned tg = gen_tag(++gen);
+                double S;
+                hcV.L = L;
+                gemv_dispatch(P.pv.vec, blkV, pitchV, validV, c0, s.ulist, nU, s.red, P.xbuf, hcV, tg, skip, S, s.clk);
+                phase_mark(s, 1);
+                bool ok = true;
+                const int nv2 = exchange_threshold(P.partV, q, Gg, tg, arrivals, skip, S, P.xbuf, n, P.tau, s.nzV,
+                                                   s.sgV, s.vlist, pitchU, s, L, Ls, s.pnzV, s.psgV, thr, gs, cfg.limit_ns,
+                                                   P.status, ok);
+                if (!ok) return false;
                 fb += (s.scal[1] != 0.0) ? 1 : 0;
                 nV = nv2;
                 sum_nu += (unsigned long long)nU;
                 ++hs;
                 if (mode == MODE_HALF_V) {
                     if (lead) {
-                        for (int64_t t = tid; t < n; t += NT) P.pre_out[t] = __ldcg(P.xbuf + t);
+                        for (int64_t t = tid; t < n; t += NT) P.pre_out[t] = untag(ld_relaxed_u64(P.xbuf + t));
                         if (tid == 0) *P.thr_out = thr;
                         pack_row(s.nzV, s.sgV, Wn, reinterpret_cast<uint32_t*>(P.trit_out), P.c_bytes / 4);
                         __syncthreads();
@@ -733,23 +890,23 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
                 }
             }
             // ---- U-step: y = R v on this CTA's rows (§2.3 step 1, second half)
-            EXTERND_PHASE(3);
-            gemv_dispatch(P.pu.vec, blkU, pitchU, validU, r0, s.vlist, nV, s.red, P.ybuf, hcU, S, M, J);
-            EXTERND_PHASE(0);
-            if (!publish_and_wait(slots + par * Gg + q, S, M, J, s, gs, target, Gg, cfg.limit_ns, skip, P.status))
-                return false;
-            EXTERND_PHASE(1);
-            nU = gather_threshold(slots + par * Gg, Gg, P.ybuf, m, P.tau, s.nzU, s.sgU, s.ulist, s, L, s.pnzU,
-                                  s.psgU, thr);
-            EXTERND_PHASE(2);
-            par ^= 1;
+            phase_mark(s, 6);
+            const unsigned tg = gen_tag(++gen);
+            double S;
+            hcU.L = L;
+            gemv_dispatch(P.pu.vec, blkU, pitchU, validU, r0, s.vlist, nV, s.red, P.ybuf, hcU, tg, skip, S, s.clk);
+            phase_mark(s, 1);
+            bool ok = true;
+            nU = exchange_threshold(P.partU, q, Gg, tg, arrivals, skip, S, P.ybuf, m, P.tau, s.nzU, s.sgU, s.ulist,
+                                    pitchV, s, L, Ls, s.pnzU, s.psgU, thr, gs, cfg.limit_ns, P.status, ok);
+            if (!ok) return false;
             p = s.scal[0];
             fb += (s.scal[1] != 0.0) ? 1 : 0;
             sum_nv += (unsigned long long)nV;
             ++hs;
             if (mode == MODE_HALF_U) {
                 if (lead) {
-                    for (int64_t t = tid; t < m; t += NT) P.pre_out[t] = __ldcg(P.ybuf + t);
+                    for (int64_t t = tid; t < m; t += NT) P.pre_out[t] = untag(ld_relaxed_u64(P.ybuf + t));
                     if (tid == 0) *P.thr_out = thr;
                     pack_row(s.nzU, s.sgU, Wm, reinterpret_cast<uint32_t*>(P.trit_out), P.b_bytes / 4);
                     __syncthreads();
@@ -773,8 +930,8 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
         }
         // ---- deflation (§2.3 step 3), held lazily as a pending rank-1 term
         if (tid == 0) s.pd[L] = d;
-        for (int w = tid; w < Wm; w += NT) { s.pnzU[L * Wm + w] = s.nzU[w]; s.psgU[L * Wm + w] = s.sgU[w]; }
-        for (int w = tid; w < Wn; w += NT) { s.pnzV[L * Wn + w] = s.nzV[w]; s.psgV[L * Wn + w] = s.sgV[w]; }
+        for (int w = tid; w < Wm; w += NT) { s.pnzU[w * Ls + L] = s.nzU[w]; s.psgU[w * Ls + L] = s.sgU[w]; }
+        for (int w = tid; w < Wn; w += NT) { s.pnzV[w * Ls + L] = s.nzV[w]; s.psgV[w * Ls + L] = s.sgV[w]; }
         for (int c = tid; c < validV; c += NT) {
             const int64_t gc = c0 + c;
             const uint32_t b = 1u << (gc & 31);
@@ -793,15 +950,18 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
         }
         ++L;
         __syncthreads();
+        phase_mark(s, 8);
         if (L == cfg.Lcap || i == kk - 1) {
-            flush_dispatch(P.pv.vec, blkV, pitchV, m, validV, L, s.pd, s.pnzU, s.psgU, Wm, s.cnzV, s.csgV);
-            flush_dispatch(P.pu.vec, blkU, pitchU, n, validU, L, s.pd, s.pnzV, s.psgV, Wn, s.cnzU, s.csgU);
+            uint32_t* scratch = reinterpret_cast<uint32_t*>(s.red);
+            flush_dispatch(P.pv.vec, blkV, pitchV, m, validV, L, Ls, s.pd, s.pnzU, s.psgU, s.cnzV, s.csgV, scratch);
+            flush_dispatch(P.pu.vec, blkU, pitchU, n, validU, L, Ls, s.pd, s.pnzV, s.psgV, s.cnzU, s.csgU, scratch);
             __syncthreads();
             for (int c = tid; c < pitchV; c += NT) { s.cnzV[c] = 0u; s.csgV[c] = 0u; }
             for (int c = tid; c < pitchU; c += NT) { s.cnzU[c] = 0u; s.csgU[c] = 0u; }
             L = 0;
             __syncthreads();
         }
+        phase_mark(s, 9);
     }
 
     // ---- explicit ||R_k||^2 from the folded fp32 residual (V-layout covers all of R)
@@ -815,10 +975,8 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
             rs += v * v;
         }
     }
-    if (!publish_and_wait(slots + par * Gg + q, rs, 0.0, 0, s, gs, target, Gg, cfg.limit_ns, skip, P.status))
-        return false;
-    const double R2 = gather_sum(slots + par * Gg, Gg, s);
-    par ^= 1;
+    double R2 = 0.0;
+    if (!exchange_sum(P.sums, q, Gg, rs, s, gs, cfg.limit_ns, P.status, skip, R2)) return false;
     if (lead && tid == 0) {
         P.stats->sum_nu = sum_nu;
         P.stats->sum_nv = sum_nv;
@@ -827,14 +985,13 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
         P.stats->fallbacks = fb;
         P.stats->residual2 = R2;
         P.stats->norm_a2 = N0;
-        EXTERND_PHASE(3);
-        for (int k2 = 0; k2 < 4; ++k2) P.stats->phase[k2] = ph[k2];
+        phase_mark(s, 7);
+        for (int k2 = 0; k2 < 11; ++k2) P.stats->phase[k2] = s.clk[k2];
         __threadfence();
         atomicExch(P.status, ST_OK);
     }
     __syncthreads();
     return true;
-#undef EXTERND_PHASE
 }
 
 __global__ void __launch_bounds__(NT, 1) als_kernel(const KCfg cfg) {
@@ -858,6 +1015,7 @@ __global__ void __launch_bounds__(NT, 1) als_kernel(const KCfg cfg) {
     s.wc = reinterpret_cast<int*>(smem_raw + lay.wc);
     s.dotp = reinterpret_cast<int*>(smem_raw + lay.dotp);
     s.sflag = reinterpret_cast<int*>(smem_raw + lay.sflag);
+    s.clk = reinterpret_cast<unsigned long long*>(smem_raw + lay.clk);
     s.nzU = reinterpret_cast<uint32_t*>(smem_raw + lay.nzU);
     s.sgU = reinterpret_cast<uint32_t*>(smem_raw + lay.sgU);
     s.nzV = reinterpret_cast<uint32_t*>(smem_raw + lay.nzV);
@@ -872,13 +1030,12 @@ __global__ void __launch_bounds__(NT, 1) als_kernel(const KCfg cfg) {
     s.csgU = reinterpret_cast<uint32_t*>(smem_raw + lay.csgU);
     s.ulist = reinterpret_cast<int*>(smem_raw + lay.ulist);
     s.vlist = reinterpret_cast<int*>(smem_raw + lay.vlist);
+    s.corr = reinterpret_cast<double*>(smem_raw + lay.corr);
 
     GroupSync* gs = cfg.gsync + grp;
-    Slot* slots = cfg.slots + (size_t)grp * 2 * cfg.Gg;
-    unsigned target = 0;
-    int par = 0;
+    unsigned arrivals = 0;   // exchanges this CTA took part in (counter targets)
     for (int pi = grp; pi < cfg.nprob; pi += cfg.NG) {
-        if (!run_problem(cfg.probs[pi], q, cfg, s, gs, slots, target, par)) return;
+        if (!run_problem(cfg.probs[pi], q, cfg, s, gs, arrivals)) return;
     }
 }
 
@@ -1114,7 +1271,7 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
     if (Gg < 1) Gg = 1;
 
     // ---- lazy deflation depth from the shared-memory budget
-    if (Gg > NT) Gg = NT;   // one slot per thread when the group's slots are gathered
+    if (Gg > NT) Gg = NT;   // one thread per CTA of the group polls its stripe
     std::vector<int> vecv(np), vecu(np);
     int pv_max = 1, pu_max = 1;
     for (int b = 0; b < np; ++b) {
@@ -1125,6 +1282,8 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
         pv_max = pv > pv_max ? pv : pv_max;
         pu_max = pu > pu_max ? pu : pu_max;
     }
+    for (int b = 0; b < np; ++b)
+        if ((double)in[b].m * pv_max >= 2147483647.0 || (double)in[b].n * pu_max >= 2147483647.0) return EXTERND_ELIMIT;
     int Lcap = MAX_PENDING;
     while (Lcap > 1 && als_smem_bytes(m_max, n_max, Lcap, pv_max, pu_max) > di.smem_optin) --Lcap;
     if (opt.pending > 0 && opt.pending < Lcap) Lcap = opt.pending;
@@ -1140,13 +1299,11 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
 
     // ---- plan the workspace
     std::vector<Prob> probs(np);
-    std::vector<size_t> off_rv(np), off_ru(np), off_x(np), off_y(np), off_start(np), off_norm(np), off_A(np),
+    std::vector<size_t> off_rv(np), off_ru(np), off_x(np), off_y(np), off_sums(np), off_start(np), off_norm(np), off_A(np),
         off_B(np), off_C(np), off_D(np), off_E(np), off_d64(np), off_pre(np), off_thr(np), off_tro(np);
     size_t ctl = 0;
     const size_t off_gsync = ctl;
     ctl += round_up(sizeof(GroupSync) * NG, 256);
-    const size_t off_slots = ctl;
-    ctl += round_up(sizeof(Slot) * 2 * (size_t)Gg * NG, 256);
     const size_t off_status = ctl;
     ctl += round_up(sizeof(int) * np, 256);
     const size_t off_nonfin = ctl;
@@ -1171,13 +1328,15 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
         P.n_norm_part = ((I.m + 31) / 32) * ((I.n + 31) / 32);
         off_rv[b] = ws; ws += round_up(sizeof(float) * (size_t)P.pv.total(I.m), 256);
         off_ru[b] = ws; ws += round_up(sizeof(float) * (size_t)P.pu.total(I.n), 256);
+        // exchange buffers: zero = "no half-step yet" (tags are 1..255)
+        off_x[b] = ws; ws += round_up(sizeof(unsigned long long) * (size_t)I.n, 256);
+        off_y[b] = ws; ws += round_up(sizeof(unsigned long long) * (size_t)I.m, 256);
+        off_sums[b] = ws; ws += round_up(sizeof(unsigned long long) * (size_t)Gg * 3, 256);
     }
     const size_t zero_to = ws;
     for (int b = 0; b < np; ++b) {
         const ProbIn& I = in[b];
         Prob& P = probs[b];
-        off_x[b] = ws; ws += round_up(sizeof(double) * (size_t)I.n, 256);
-        off_y[b] = ws; ws += round_up(sizeof(double) * (size_t)I.m, 256);
         const int64_t srows = (I.mode == MODE_FACTOR) ? I.k : 1;
         off_start[b] = ws; ws += round_up(sizeof(uint32_t) * (size_t)(P.start_words * srows), 256);
         off_norm[b] = ws; ws += round_up(sizeof(double) * (size_t)P.n_norm_part, 256);
@@ -1220,8 +1379,11 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
         P.A = off_A[b] == SIZE_MAX ? I.A : reinterpret_cast<const float*>(dws + off_A[b]);
         P.Rv = reinterpret_cast<float*>(dws + off_rv[b]);
         P.Ru = reinterpret_cast<float*>(dws + off_ru[b]);
-        P.xbuf = reinterpret_cast<double*>(dws + off_x[b]);
-        P.ybuf = reinterpret_cast<double*>(dws + off_y[b]);
+        P.xbuf = reinterpret_cast<unsigned long long*>(dws + off_x[b]);
+        P.ybuf = reinterpret_cast<unsigned long long*>(dws + off_y[b]);
+        P.sums = reinterpret_cast<unsigned long long*>(dws + off_sums[b]);
+        P.partV = P.sums + Gg;
+        P.partU = P.sums + 2 * Gg;
         P.start = reinterpret_cast<uint32_t*>(dws + off_start[b]);
         P.norm_part = reinterpret_cast<double*>(dws + off_norm[b]);
         P.nonfinite = reinterpret_cast<unsigned*>(dws + off_nonfin) + b;
@@ -1285,7 +1447,6 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
             cfg.Gg = Gg;
             cfg.NG = NG;
             cfg.gsync = reinterpret_cast<GroupSync*>(dws + off_gsync);
-            cfg.slots = reinterpret_cast<Slot*>(dws + off_slots);
             cfg.Lcap = Lcap;
             cfg.m_max = (int)m_max;
             cfg.n_max = (int)n_max;
@@ -1358,7 +1519,7 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
             st.fallbacks += (int64_t)d.fallbacks;
             if (b == 0) {
                 st.residual_energy = d.norm_a2 > 0 ? 1.0 - d.residual2 / d.norm_a2 : 0.0;
-                for (int k2 = 0; k2 < 4; ++k2) st.phase_cycles[k2] = (int64_t)d.phase[k2];
+                for (int k2 = 0; k2 < 11; ++k2) st.phase_cycles[k2] = (int64_t)d.phase[k2];
             }
         }
     }

@@ -6,7 +6,7 @@
 //
 // Design (B200):
 //  * One persistent cooperative launch runs every component of a matrix.  A
-//    matrix is served by a group of G CTAs (one per SM, 512 threads each).
+//    matrix is served by a group of G CTAs (one per SM, 1024 threads each).
 //  * The residual R is kept twice in HBM, each copy cut into one private block
 //    per CTA so that both half-steps read only what they need and no CTA ever
 //    reads another CTA's residual:
@@ -38,7 +38,10 @@
 
 namespace externd {
 
-constexpr int NT = 512;               // threads per CTA of the ALS kernel
+#ifndef EXTERND_NT
+#define EXTERND_NT 1024
+#endif
+constexpr int NT = EXTERND_NT;        // threads per CTA of the ALS kernel
 constexpr int NWARP = NT / 32;
 constexpr int MAX_PENDING = 32;       // lazy deflation depth cap
 constexpr unsigned FULL = 0xffffffffu;
@@ -70,17 +73,12 @@ struct Part {
     __host__ __device__ int64_t total(int64_t other) const { return other * vec * units; }
 };
 
-struct Slot {                 // one CTA's published scalars for one half-step
-    double S;                 // sum |out| over its stripe
-    double M;                 // max |out| over its stripe (-1 if empty)
-    long long J;              // lowest index attaining M
-    long long pad;
-};
+constexpr int NCTR = 8;       // arrival counters per group (spread over L2 lines)
 
-struct GroupSync {            // one per CTA group, 128 B apart
-    unsigned arrive;
-    int abort;
-    unsigned pad[30];
+struct GroupSync {            // one per CTA group
+    int abort;                // raised by the first wait of the group that runs out
+    int pad[63];
+    unsigned ctr[NCTR][64];   // counter c (one per 256 B) counts arrivals of the CTAs q with q % NCTR == c
 };
 
 struct DevStats {
@@ -92,7 +90,7 @@ struct DevStats {
     double residual2;               // ||R_k||^2 from the final fp32 residual
     double norm_a2;
     double pad;
-    unsigned long long phase[4];    // SM cycles of CTA 0: GEMV, publish+wait, gather+threshold, per-component work
+    unsigned long long phase[11];   // SM cycles of CTA 0 per phase (see run_problem); [10] stale words seen
 };
 
 enum Mode { MODE_FACTOR = 0, MODE_HALF_V = 1, MODE_HALF_U = 2 };
@@ -112,8 +110,11 @@ struct Prob {
     int64_t b_bytes, c_bytes;
     float* Rv;                // V-layout blocks
     float* Ru;                // U-layout blocks
-    double* xbuf;             // n, published V-step outputs
-    double* ybuf;             // m, published U-step outputs
+    unsigned long long* xbuf; // n, published V-step outputs (tagged fp64 words, zero-initialised)
+    unsigned long long* ybuf; // m, published U-step outputs (tagged fp64 words, zero-initialised)
+    unsigned long long* sums; // G, per-CTA partial sums of the final residual (tagged, zero-initialised)
+    unsigned long long* partV;// G, per-CTA sum |out| of the V-step (tagged, zero-initialised)
+    unsigned long long* partU;// G, same for the U-step
     const uint32_t* start;    // start trits (k rows of start_words) or debug input (1 row)
     int64_t start_words;
     double* norm_part;        // per setup-tile partial sums of A^2
@@ -134,7 +135,6 @@ struct KCfg {
     int Gg;                   // CTAs per group
     int NG;                   // groups
     GroupSync* gsync;         // NG
-    Slot* slots;              // NG x 2 x Gg
     int Lcap;                 // lazy deflation depth
     int m_max, n_max;         // for shared-memory carving
     int pv_max, pu_max;       // largest stripe pitch of the two layouts
