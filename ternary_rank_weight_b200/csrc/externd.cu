@@ -262,33 +262,23 @@ __device__ __forceinline__ void emit_tagged(double v, int64_t gi, unsigned long 
     S += fabs(__longlong_as_double((long long)(w & ~0xFFull)));
 }
 
-// acc += sum_u s_u v_u for one batch of loaded rows (s_u = sign bit of the list entry).
-// Default: every fp32 term is converted and added in fp64 (exact terms, fp64 sum).
-// EXTERND_PRESUM4: groups of 4 signed terms are first summed in fp32 (pairwise),
-// then converted and added in fp64.
+// acc += sum_u s_u v_u for one batch of loaded rows (s_u = +1/-1 from the sign bit
+// of the list entry).  The batch is summed in fp32 with one fused multiply-add per
+// term (|error| <= (U-1) 2^-24 sum|terms|), then converted and added to the fp64
+// accumulator: this keeps the GEMV at ~2 instructions per element.
 template <int VEC, int U>
 __device__ __forceinline__ void accumulate_batch(double* acc, const int* ent, float (*v)[VEC]) {
-#ifdef EXTERND_PRESUM4
-    static_assert(U % 4 == 0, "batch must be a multiple of 4");
+    float b[VEC];
     #pragma unroll
-    for (int u = 0; u < U; u += 4) {
-        #pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-            const float a0 = __uint_as_float(__float_as_uint(v[u][e]) ^ ((unsigned)ent[u] & 0x80000000u));
-            const float a1 = __uint_as_float(__float_as_uint(v[u + 1][e]) ^ ((unsigned)ent[u + 1] & 0x80000000u));
-            const float a2 = __uint_as_float(__float_as_uint(v[u + 2][e]) ^ ((unsigned)ent[u + 2] & 0x80000000u));
-            const float a3 = __uint_as_float(__float_as_uint(v[u + 3][e]) ^ ((unsigned)ent[u + 3] & 0x80000000u));
-            acc[e] += (double)((a0 + a1) + (a2 + a3));
-        }
-    }
-#else
+    for (int e = 0; e < VEC; ++e) b[e] = 0.f;
     #pragma unroll
     for (int u = 0; u < U; ++u) {
-        const unsigned sm = (unsigned)ent[u] & 0x80000000u;
+        const float sgn = ent[u] < 0 ? -1.f : 1.f;   // inactive slots hold v = 0
         #pragma unroll
-        for (int e = 0; e < VEC; ++e) acc[e] += (double)__uint_as_float(__float_as_uint(v[u][e]) ^ sm);
+        for (int e = 0; e < VEC; ++e) b[e] = fmaf(sgn, v[u][e], b[e]);
     }
-#endif
+    #pragma unroll
+    for (int e = 0; e < VEC; ++e) acc[e] += (double)b[e];
 }
 
 // One half-step GEMV over this CTA's private block: out[c] = sum_{e in list} s_e blk[r_e][c]
@@ -1163,17 +1153,17 @@ int64_t rank_of(int64_t m, int64_t n, double mu) {
 
 size_t trit_bytes(int64_t len) { return len < 1 ? 0 : round_up((size_t)((len + 3) / 4), 16); }
 
-// Largest vector width whose stripe imbalance stays within 6 %, else the least imbalanced.
+// Vector width of a stripe layout: minimise the largest stripe's GEMV cost,
+// (units per stripe) * width * (instructions per element at that width).
 int choose_vec(int64_t len, int G) {
-    const double ideal = (double)len / G;
-    int best = 1;
-    double best_imb = 1e30;
+    int best = 4;
+    double best_cost = 1e300;
     for (int vec : {4, 2, 1}) {
+        const double per_elem = vec == 4 ? 2.25 : (vec == 2 ? 3.5 : 6.0);
         const int64_t units = (len + vec - 1) / vec;
         const int64_t maxu = (units + G - 1) / G;
-        const double imb = (double)(maxu * vec) / (ideal > 0 ? ideal : 1.0);
-        if (imb <= 1.06) return vec;
-        if (imb < best_imb - 1e-12) { best_imb = imb; best = vec; }
+        const double cost = (double)(maxu * vec) * per_elem;
+        if (cost < best_cost * (1.0 - 1e-9)) { best_cost = cost; best = vec; }
     }
     return best;
 }

@@ -4,8 +4,11 @@ Tolerances (from the factorization's arithmetic and the fixed acceptance bar):
 * trits: bit-exact, except entries whose pre-threshold magnitude lies within
   1e-5 relative of the threshold (a threshold tie: both sides decide in fp64,
   but sum in different orders and the GPU residual is fp32-rounded);
-* pre-threshold vectors on a shared residual: 1e-12 relative to sum |terms|
-  (fp64 accumulation of exactly-representable fp32 terms);
+* pre-threshold vectors on a shared residual: 1e-6 relative to sum |terms|.
+  The kernel sums batches of at most 16 signed fp32 terms in fp32 (fused
+  multiply-add, |error| <= 15 * 2^-24 * sum |terms| = 8.9e-7 sum |terms|), adds
+  the batch sums in fp64, and publishes values rounded to 44 mantissa bits
+  (2^-44 relative);
 * scale d_i: 1e-4 relative; energy E: 2e-3 absolute; zero fraction: 0.5
   percentage points.  Trajectories may diverge after a tie; divergences are
   counted and must be explained by a near-tie on the oracle side.
@@ -70,8 +73,9 @@ def test_halfstep_matches_oracle(m, n, transpose):
         got = ext.unpack_trits(out.cpu().numpy(), n if transpose else m)
         want_pre, want_thr, want, _ = ora.half_step(R, t_in, tau, transpose)
         scale = (np.abs(R).T @ np.abs(t_in) if transpose else np.abs(R) @ np.abs(t_in)) + 1e-300
-        assert np.all(np.abs(pre - want_pre) <= 1e-12 * scale + 1e-300)
-        assert thr == pytest.approx(want_thr, rel=1e-12, abs=1e-300)
+        assert np.all(np.abs(pre - want_pre) <= 1e-6 * scale + 1e-300)
+        lout = pre.shape[0]
+        assert abs(thr - want_thr) <= tau / lout * 1e-6 * scale.sum() + 1e-15 * want_thr
         ok, nbad = _trits_equal_modulo_ties(got, want, want_pre, want_thr)
         assert ok, (tau, nbad)
 
