@@ -87,6 +87,35 @@ int externd_factor(const float* A, int64_t m, int64_t n, double mu, double tau, 
                    uint64_t seed, uint8_t* B_out, float* D_out, uint8_t* C_out,
                    double* energy_out, void* stream);
 
+/* Allocation-free variant of externd_factor.  The pages have no counterpart:
+ * this entry point exists for callers that cannot allocate device memory while
+ * it runs -- for example an inference or conversion service whose memory pool
+ * has already reserved the GPU's memory, or a caller that must not take the
+ * implicit device synchronisation an allocation can cause.
+ *
+ * It runs the same kernels as externd_factor, but its scratch (the two residual
+ * layouts, exchange buffers, start trits, control words) lives in one static
+ * device array of EXTERND_NOALLOC_SCRATCH_BYTES that every GPU loading this
+ * library holds until the process exits.  It calls no cudaMalloc / cudaFree and
+ * no allocating library routine.
+ *   - A, B_out, D_out, C_out, energy_out must be DEVICE pointers (EXTERND_EINVAL
+ *     otherwise: host buffers would need staging memory).
+ *   - A matrix whose scratch would exceed EXTERND_NOALLOC_SCRATCH_BYTES is
+ *     rejected with EXTERND_ELIMIT (about 8 m n + k ceil(m/4) bytes; e.g.
+ *     1024 x 1024 at mu = 2 needs ~8.6 MiB).
+ *   - The first call on a device looks up the array's device address; make that
+ *     first call before any stream capture.
+ *   - All calls share the one array and it keeps the previous call's contents
+ *     (each call clears what must start at zero).  Calls that overlap on the GPU
+ *     (e.g. on two streams, or from two host threads) race and corrupt each
+ *     other: serialise them.
+ *   - externd_last_stats is not updated by this call (it records no events).
+ * Arguments and results are those of externd_factor. */
+#define EXTERND_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+int externd_factor_noalloc(const float* A, int64_t m, int64_t n, double mu, double tau, int iters,
+                           uint64_t seed, uint8_t* B_out, float* D_out, uint8_t* C_out,
+                           double* energy_out, void* stream);
+
 /* Factor `count` independent matrices in one cooperative launch; the SMs are
  * split into groups and each group factors its matrices one after another.
  * Every array argument has `count` entries (host arrays of pointers/values);

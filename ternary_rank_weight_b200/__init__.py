@@ -4,11 +4,11 @@ The factorization runs in the CUDA library ``libexternd.so`` (C ABI in
 include/externd.h); this package is its Python binding plus the seeded
 synthetic workload generators.
 """
-from .api import (ExterndError, Factors, STATUS, debug_halfstep, debug_start_trits, factor,  # noqa: F401
-                  factor_batched, last_stats, pack_trits, rank, reconstruct, strerror, trit_bytes,
+from .api import (ExterndError, Factors, NOALLOC_SCRATCH_BYTES, STATUS, debug_halfstep, debug_start_trits,  # noqa: F401
+                  factor, factor_batched, factor_noalloc, last_stats, pack_trits, rank, reconstruct, strerror, trit_bytes,
                   unpack_trits)
 
 __all__ = [
-    "ExterndError", "Factors", "STATUS", "debug_halfstep", "debug_start_trits", "factor", "factor_batched",
+    "ExterndError", "Factors", "NOALLOC_SCRATCH_BYTES", "STATUS", "factor_noalloc", "debug_halfstep", "debug_start_trits", "factor", "factor_batched",
     "last_stats", "pack_trits", "rank", "reconstruct", "strerror", "trit_bytes", "unpack_trits",
 ]

@@ -153,6 +153,39 @@ def factor(A, mu: float, tau: float, iters: int = 15, seed: int = 0, *, grid: in
                    stats=last_stats())
 
 
+def factor_noalloc(A: torch.Tensor, mu: float, tau: float, iters: int = 15, seed: int = 0, *, out=None,
+                   stream=None) -> Factors:
+    """externd_factor_noalloc: the same factorization with no device allocation inside the call.
+
+    For callers that cannot allocate device memory while the factorization runs
+    (e.g. a service whose pool already reserved the GPU).  The library's scratch is
+    a fixed static device array (``NOALLOC_SCRATCH_BYTES``); larger shapes are
+    rejected (ELIMIT).  A and the outputs must live on the GPU; pass preallocated
+    outputs as ``out=(B, D, C, energy)`` to keep this call allocation-free on the
+    Python side too.  Calls share the scratch and must not overlap on the GPU."""
+    if not (isinstance(A, torch.Tensor) and A.is_cuda and A.dtype == torch.float32 and A.dim() == 2):
+        raise ValueError("A must be a 2-D float32 CUDA tensor")
+    A = A.contiguous()
+    m, n = A.shape
+    k = rank(m, n, mu)
+    if k < 1:
+        raise ExterndError(STATUS["EINVAL"], "externd_rank")
+    if out is None:
+        out = (torch.empty((k, trit_bytes(m)), dtype=torch.uint8, device=A.device),
+               torch.empty((k,), dtype=torch.float32, device=A.device),
+               torch.empty((k, trit_bytes(n)), dtype=torch.uint8, device=A.device),
+               torch.empty((k,), dtype=torch.float64, device=A.device))
+    B, D, C, E = out
+    with _on_device(A):
+        rc = _lib.load().externd_factor_noalloc(_ptr(A), m, n, float(mu), float(tau), int(iters), int(seed),
+                                                _ptr(B), _ptr(D), _ptr(C), _ptr(E), _stream(stream, A.device))
+    _check(rc, "externd_factor_noalloc")
+    return Factors(B=B, D=D, C=C, energy=E, m=m, n=n, k=k, mu=float(mu), tau=float(tau))
+
+
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
+
+
 def factor_batched(As: Sequence, mus: Sequence[float], taus: Sequence[float], iters: int = 15,
                    seeds: Optional[Sequence[int]] = None, *, stream=None):
     """Factor independent matrices in one launch (externd_factor_batched).

@@ -1029,6 +1029,14 @@ __global__ void __launch_bounds__(NT, 1) als_kernel(const KCfg cfg) {
     }
 }
 
+// Writes one problem descriptor and its running status into a caller-fixed workspace.
+__global__ void init_control_kernel(const Prob p, Prob* dst, int* status) {
+    if (threadIdx.x == 0) {
+        *dst = p;
+        *status = ST_RUNNING;
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Reconstruction Ahat = B diag(D) C (§2.1), fp64 accumulation
 // ---------------------------------------------------------------------------
@@ -1226,7 +1234,14 @@ struct Buf {  // device staging for a possibly-host pointer
 
 // Runs setup + init + ALS for `np` problems.  All pointers in `in` may be
 // host or device.  statuses[np] receives per-problem status.
-int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* statuses) {
+// Caller-fixed workspace (no allocation, no host-side copies, no events).
+struct FixedWs {
+    unsigned char* base = nullptr;
+    size_t cap = 0;
+};
+
+int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* statuses,
+        const FixedWs* fixed = nullptr) {
     int rc = EXTERND_OK;
     DevInfo di;
     if ((rc = dev_info(di)) != EXTERND_OK) return rc;
@@ -1350,6 +1365,14 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
         }
     }
 
+    if (fixed) {
+        for (int b = 0; b < np; ++b)
+            if (off_A[b] != SIZE_MAX || off_B[b] != SIZE_MAX || off_C[b] != SIZE_MAX || off_D[b] != SIZE_MAX ||
+                off_E[b] != SIZE_MAX || off_d64[b] != SIZE_MAX || off_pre[b] != SIZE_MAX || off_thr[b] != SIZE_MAX ||
+                off_tro[b] != SIZE_MAX)
+                return EXTERND_EINVAL;   // host buffers would need staging memory
+        if (ws > fixed->cap) return EXTERND_ELIMIT;
+    }
     unsigned char* dws = nullptr;
     cudaEvent_t ev[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
     std::vector<unsigned char> hctl(ctl, 0);
@@ -1358,9 +1381,13 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
     int launches = 0;
     float ms_setup = 0, ms_init = 0, ms_als = 0, ms_total = 0;
 
-    for (int i = 0; i < 5; ++i) CK(cudaEventCreate(&ev[i]));
-    CK(cudaMallocAsync((void**)&dws, ws, stream));
-    CK(cudaEventRecord(ev[0], stream));
+    if (fixed) {
+        dws = fixed->base;
+    } else {
+        for (int i = 0; i < 5; ++i) CK(cudaEventCreate(&ev[i]));
+        CK(cudaMallocAsync((void**)&dws, ws, stream));
+    }
+    if (ev[0]) CK(cudaEventRecord(ev[0], stream));
 
     // ---- fill problem descriptors and the control region
     for (int b = 0; b < np; ++b) {
@@ -1393,7 +1420,17 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
         reinterpret_cast<int*>(hctl.data() + off_status)[b] = ST_RUNNING;
     }
     memcpy(hctl.data() + off_probs, probs.data(), sizeof(Prob) * np);
-    CK(cudaMemcpyAsync(dws, hctl.data(), ctl, cudaMemcpyHostToDevice, stream));
+    if (fixed) {
+        // control region: zeros, then the descriptors and statuses written by a kernel
+        CK(cudaMemsetAsync(dws, 0, ctl, stream));
+        for (int b = 0; b < np; ++b) {
+            init_control_kernel<<<1, 32, 0, stream>>>(probs[b], reinterpret_cast<Prob*>(dws + off_probs) + b,
+                                                      reinterpret_cast<int*>(dws + off_status) + b);
+            CK(cudaGetLastError());
+        }
+    } else {
+        CK(cudaMemcpyAsync(dws, hctl.data(), ctl, cudaMemcpyHostToDevice, stream));
+    }
     if (zero_to > zero_from) CK(cudaMemsetAsync(dws + zero_from, 0, zero_to - zero_from, stream));
     for (int b = 0; b < np; ++b) {
         const ProbIn& I = in[b];
@@ -1420,7 +1457,7 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
             CK(cudaGetLastError());
             ++launches;
         }
-        CK(cudaEventRecord(ev[1], stream));
+        if (ev[1]) CK(cudaEventRecord(ev[1], stream));
         bool any_factor = false;
         for (int b = 0; b < np; ++b) any_factor |= (in[b].mode == MODE_FACTOR);
         if (any_factor) {
@@ -1429,7 +1466,7 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
             CK(cudaGetLastError());
             ++launches;
         }
-        CK(cudaEventRecord(ev[2], stream));
+        if (ev[2]) CK(cudaEventRecord(ev[2], stream));
         if (!opt.init_only) {
             KCfg cfg;
             cfg.probs = dprobs;
@@ -1449,7 +1486,7 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
             CK(cudaLaunchCooperativeKernel((void*)als_kernel, dim3((unsigned)(NG * Gg)), dim3(NT), args, smem, stream));
             ++launches;
         }
-        CK(cudaEventRecord(ev[3], stream));
+        if (ev[3]) CK(cudaEventRecord(ev[3], stream));
     }
 
     // ---- results back to host-side buffers
@@ -1475,13 +1512,15 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
     }
     CK(cudaMemcpyAsync(hstatus.data(), dws + off_status, sizeof(int) * np, cudaMemcpyDeviceToHost, stream));
     CK(cudaMemcpyAsync(hstats.data(), dws + off_stats, sizeof(DevStats) * np, cudaMemcpyDeviceToHost, stream));
-    CK(cudaEventRecord(ev[4], stream));
+    if (ev[4]) CK(cudaEventRecord(ev[4], stream));
     CK(cudaStreamSynchronize(stream));
 
-    cudaEventElapsedTime(&ms_setup, ev[0], ev[1]);
-    cudaEventElapsedTime(&ms_init, ev[1], ev[2]);
-    cudaEventElapsedTime(&ms_als, ev[2], ev[3]);
-    cudaEventElapsedTime(&ms_total, ev[0], ev[4]);
+    if (ev[0]) {
+        cudaEventElapsedTime(&ms_setup, ev[0], ev[1]);
+        cudaEventElapsedTime(&ms_init, ev[1], ev[2]);
+        cudaEventElapsedTime(&ms_als, ev[2], ev[3]);
+        cudaEventElapsedTime(&ms_total, ev[0], ev[4]);
+    }
     st.setup_ms = ms_setup;
     st.init_ms = ms_init;
     st.als_ms = ms_als;
@@ -1518,7 +1557,7 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
         if (statuses[b] != ST_OK) { rc = statuses[b]; break; }
 
 done:
-    if (dws) { cudaFreeAsync(dws, stream); cudaStreamSynchronize(stream); }
+    if (dws && !fixed) { cudaFreeAsync(dws, stream); cudaStreamSynchronize(stream); }
     for (int i = 0; i < 5; ++i)
         if (ev[i]) cudaEventDestroy(ev[i]);
     cudaGetLastError();
@@ -1540,6 +1579,37 @@ int validate_factor(const float* A, int64_t m, int64_t n, double mu, double tau,
     if (m > INT_MAX / 2 || n > INT_MAX / 2 || k > INT_MAX) return EXTERND_ELIMIT;
     if (check_rows_aligned(B) || check_rows_aligned(C)) return EXTERND_EINVAL;
     *k_out = k;
+    return EXTERND_OK;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// Scratch memory of externd_factor_noalloc: one file-scope device array,
+// EXTERND_NOALLOC_SCRATCH_BYTES on every device that loads this library, kept
+// until the process exits.  Host code may not use the array's name as a device
+// address: the address is looked up once per device with cudaGetSymbolAddress.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[EXTERND_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+std::mutex g_noalloc_mu;
+unsigned char* g_noalloc_base[64] = {};
+
+// Device address of the scratch array on the current device (set up on first use).
+int noalloc_scratch(unsigned char** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return EXTERND_ECUDA; }
+    if (dev < 0 || dev >= 64) return EXTERND_ECUDA;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_base[dev]) {
+        void* ptr = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess || ptr == nullptr) { cudaGetLastError(); return EXTERND_ECUDA; }
+        g_noalloc_base[dev] = static_cast<unsigned char*>(ptr);
+    }
+    *out = g_noalloc_base[dev];
     return EXTERND_OK;
 }
 
@@ -1590,6 +1660,24 @@ int externd_factor_ex(const float* A, int64_t m, int64_t n, double mu, double ta
 int externd_factor(const float* A, int64_t m, int64_t n, double mu, double tau, int iters, uint64_t seed,
                    uint8_t* B_out, float* D_out, uint8_t* C_out, double* energy_out, void* stream) {
     return externd_factor_ex(A, m, n, mu, tau, iters, seed, B_out, D_out, C_out, energy_out, stream, nullptr);
+}
+
+int externd_factor_noalloc(const float* A, int64_t m, int64_t n, double mu, double tau, int iters, uint64_t seed,
+                           uint8_t* B_out, float* D_out, uint8_t* C_out, double* energy_out, void* stream) {
+    int64_t k = 0;
+    int rc = validate_factor(A, m, n, mu, tau, iters, B_out, D_out, C_out, &k);
+    if (rc != EXTERND_OK) return rc;
+    unsigned char* base = nullptr;
+    if ((rc = noalloc_scratch(&base)) != EXTERND_OK) return rc;
+    ProbIn I = {};
+    I.A = A; I.m = m; I.n = n; I.k = k; I.tau = tau; I.iters = iters; I.seed = seed;
+    I.B = B_out; I.D = D_out; I.C = C_out; I.energy = energy_out; I.mode = MODE_FACTOR;
+    RunOpts ro;
+    FixedWs fw;
+    fw.base = base;
+    fw.cap = EXTERND_NOALLOC_SCRATCH_BYTES;
+    int st = 0;
+    return run(&I, 1, ro, reinterpret_cast<cudaStream_t>(stream), &st, &fw);
 }
 
 int externd_factor_batched(int count, const float* const* A, const int64_t* m, const int64_t* n, const double* mu,
