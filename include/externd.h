@@ -177,7 +177,12 @@ typedef struct {
     double setup_ms;           /* residual layout copy + ||A||^2 */
     double init_ms;            /* start-vector generation */
     double total_ms;           /* all device work of the call, staging copies included */
-    double alg_bytes;          /* algorithmic bytes of the ALS kernel, summed over matrices */
+    double alg_bytes;          /* algorithmic bytes of the ALS kernel, summed over matrices: per component
+                                  4 (n sum_t nnz(u_t) + m sum_t nnz(v_t)) + 8 nnz(u) nnz(v), t over the
+                                  half-steps, i.e. what a direct evaluation of every GEMV touches */
+    double read_bytes;         /* residual bytes this kernel reads: its GEMVs run over the trits that
+                                  changed since the previous half-step of the same kind (4 (n rows +
+                                  m columns) per half-step), plus the same deflation term */
     double residual_energy;    /* 1 - ||R_k||^2 / ||A||^2 from the final fp32 residual (matrix 0) */
     int64_t components;        /* components fitted, summed over matrices */
     int64_t half_steps;        /* V- and U-steps executed, summed over matrices */

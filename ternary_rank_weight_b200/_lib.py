@@ -45,6 +45,7 @@ class Stats(ctypes.Structure):
         ("init_ms", ctypes.c_double),
         ("total_ms", ctypes.c_double),
         ("alg_bytes", ctypes.c_double),
+        ("read_bytes", ctypes.c_double),
         ("residual_energy", ctypes.c_double),
         ("components", ctypes.c_int64),
         ("half_steps", ctypes.c_int64),

@@ -139,14 +139,18 @@ __global__ void __launch_bounds__(NTI) init_kernel(const Prob* __restrict__ prob
 
 // Shared-memory carve of the ALS kernel (host and device use the same layout).
 struct SmemLayout {
-    size_t red, pd, coef, scal, wS, wM, wp, gS, gM, wJ, gJ, wc, dotp, sflag, clk, nzU, sgU, nzV, sgV, pnzU, psgU, pnzV,
-        psgV, cnzV, csgV, cnzU, csgU, ulist, vlist, corr, total;
+    size_t red, pd, coef, coefV, dotU, dotV, scal, wS, wM, wp, gS, gM, wJ, gJ, wc, dotp, sflag, clk, nzU, sgU, nzV, sgV, pnzU, psgU, pnzV,
+        psgV, cnzV, csgV, cnzU, csgU, ulist, vlist, wd, onzU, osgU, onzV, osgV, gV, gU, corr, total;
     __host__ __device__ SmemLayout(int64_t m_max, int64_t n_max, int Lc, int pv_max, int pu_max) {
         const size_t Wm = (size_t)((m_max + 31) / 32), Wn = (size_t)((n_max + 31) / 32);
         size_t o = 0;
         red = o;  o += 8 * (size_t)NT * 5;   // lanes * (pitch + 1) <= NT * (VEC + 1)
         pd = o;   o += 8 * (size_t)Lc;
         coef = o; o += 8 * (size_t)Lc;
+        coefV = o; o += 8 * (size_t)Lc;
+        dotU = o; o += 4 * (size_t)Lc;
+        dotV = o; o += 4 * (size_t)Lc;
+        o = (o + 7) & ~(size_t)7;
         scal = o; o += 8 * 16;
         wS = o;   o += 8 * NWARP;
         wM = o;   o += 8 * NWARP;
@@ -173,21 +177,33 @@ struct SmemLayout {
         csgU = o; o += 4 * (size_t)pu_max;
         ulist = o; o += 4 * (size_t)m_max;
         vlist = o; o += 4 * (size_t)n_max;
+        wd = o;   o += 4 * NWARP;
+        onzU = o; o += 4 * Wm;
+        osgU = o; o += 4 * Wm;
+        onzV = o; o += 4 * Wn;
+        osgV = o; o += 4 * Wn;
         o = (o + 7) & ~(size_t)7;
+        gV = o;   o += 8 * (size_t)pv_max;
+        gU = o;   o += 8 * (size_t)pu_max;
         corr = o; o += 8 * (size_t)(pv_max > pu_max ? pv_max : pu_max);
         total = (o + 15) & ~(size_t)15;
     }
 };
 
 struct Smem {
-    double *red, *pd, *coef, *scal, *wS, *wM, *wp, *gS, *gM;   // red: NT*5
+    double *red, *pd, *scal, *wS, *wM, *wp, *gS, *gM;          // red: NT*5
+    double *coef, *coefV;                    // d_l (t_l . u) and d_l (t_l . v) for the pending components
+    int *dotU, *dotV;                        // the integer dot products t_l . u and t_l . v
     long long *wJ, *gJ;
     int *wc, *dotp, *sflag;
     unsigned long long* clk;                 // [0..9] phase cycles, [11] last stamp (thread 0 of CTA 0)
     uint32_t *nzU, *sgU, *nzV, *sgV;         // current u, v
     uint32_t *pnzU, *psgU, *pnzV, *psgV;     // pending components (full length, stride W)
     uint32_t *cnzV, *csgV, *cnzU, *csgU;     // pending trits at this CTA's outputs, bit l = component l
-    int *ulist, *vlist;                      // compacted supports: element offset (index * block pitch) | sign << 31
+    int *ulist, *vlist;                      // compacted trit changes: element offset (index * block pitch) | sign << 31 | (|delta| == 2) << 30
+    int* wd;                                 // per-warp count of changed trits
+    uint32_t *onzU, *osgU, *onzV, *osgV;     // masks of the previous u and v of this component
+    double *gV, *gU;                         // running GEMV sums R^T u, R v of this CTA's outputs (before lazy-deflation correction)
     double* corr;                            // lazy-deflation correction per output of this CTA
 };
 
@@ -211,10 +227,6 @@ __device__ __forceinline__ unsigned long long tag_value(double v, unsigned tag) 
     return ((unsigned long long)__double_as_longlong(v) & ~0xFFull) | (unsigned long long)tag;
 }
 
-__device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
-    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
 template <int VEC>
 __device__ __forceinline__ void load_vec(const float* p, float* v) {
     if constexpr (VEC == 4) {
@@ -235,21 +247,24 @@ struct HalfCorr {
     const uint32_t* cnz;
     const uint32_t* csg;
     double* corr;     // out: correction per output of this CTA (filled by the GEMV)
+    double* g;        // running sum of the GEMV over this component's trit changes, per output
     int L;
 };
 
-// corr[c] = sum_l coef_l t_l(c) for this CTA's outputs: warp w takes outputs w, w+NWARP, ...;
-// lane l contributes component l, summed by a fixed butterfly.
+// corr[c] = sum_l coef_l t_l(c) for this CTA's outputs: one thread per output, the
+// pending components that touch it added in increasing l.
 __device__ __forceinline__ void corrections(int valid, const HalfCorr& hc) {
     if (hc.L <= 0) return;
-    const int lane = lane_id();
-    const double cl = lane < hc.L ? hc.coef[lane] : 0.0;
-    for (int c = warp_id(); c < valid; c += NWARP) {
-        const uint32_t z = hc.cnz[c], g = hc.csg[c];
-        double t = ((z >> lane) & 1u) ? (((g >> lane) & 1u) ? -cl : cl) : 0.0;
-        #pragma unroll
-        for (int o = 16; o; o >>= 1) t += __shfl_xor_sync(FULL, t, o);
-        if (lane == 0) hc.corr[c] = t;
+    for (int c = threadIdx.x; c < valid; c += NT) {
+        uint32_t z = hc.cnz[c];
+        const uint32_t g = hc.csg[c];
+        double t = 0.0;
+        while (z) {
+            const int l = __ffs(z) - 1;
+            z &= z - 1u;
+            t += ((g >> l) & 1u) ? -hc.coef[l] : hc.coef[l];
+        }
+        hc.corr[c] = t;
     }
 }
 
@@ -273,7 +288,9 @@ __device__ __forceinline__ void accumulate_batch(double* acc, const int* ent, fl
     for (int e = 0; e < VEC; ++e) b[e] = 0.f;
     #pragma unroll
     for (int u = 0; u < U; ++u) {
-        const float sgn = ent[u] < 0 ? -1.f : 1.f;   // inactive slots hold v = 0
+        // coefficient of the entry: -1/+1 from bit 31, doubled by bit 30 (a trit that
+        // flipped sign); inactive slots hold v = 0
+        const float sgn = (ent[u] < 0 ? -1.f : 1.f) * ((ent[u] & 0x40000000) ? 2.f : 1.f);
         #pragma unroll
         for (int e = 0; e < VEC; ++e) b[e] = fmaf(sgn, v[u][e], b[e]);
     }
@@ -281,9 +298,40 @@ __device__ __forceinline__ void accumulate_batch(double* acc, const int* ent, fl
     for (int e = 0; e < VEC; ++e) acc[e] += (double)b[e];
 }
 
-// One half-step GEMV over this CTA's private block: out[c] = sum_{e in list} s_e blk[r_e][c]
-// for the block's `valid` columns, minus the lazy-deflation correction, written to
-// gout[out0 + c].  fp64 accumulation of exact fp32 terms, fixed summation order.
+// Rows per batch of the GEMV: enough loads in flight per thread within the register budget.
+template <int VEC>
+__host__ __device__ constexpr int GEMV_U() {
+    return (NT >= 1024) ? ((VEC == 4) ? 8 : (VEC == 2 ? 12 : 16)) : ((VEC == 4) ? 16 : (VEC == 2 ? 24 : 32));
+}
+
+// acc += sum over the list entries g, g + lanes, g + 2 lanes, ... of this thread's VEC
+// columns, U entries per batch (every batch issues all its loads before using any).
+template <int VEC, int U>
+__device__ __forceinline__ void gemv_rows(double* acc, const float* base, const int* __restrict__ list, int nlist,
+                                          int g, int lanes) {
+    for (int idx = g; idx < nlist; idx += U * lanes) {
+        int ent[U];
+        float v[U][VEC];
+        #pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int ii = idx + u * lanes;
+            ent[u] = ii < nlist ? list[ii] : 0;
+            if (ii < nlist) {
+                load_vec<VEC>(base + (ent[u] & 0x3fffffff), v[u]);
+            } else {
+                #pragma unroll
+                for (int e = 0; e < VEC; ++e) v[u][e] = 0.f;
+            }
+        }
+        accumulate_batch<VEC, U>(acc, ent, v);
+    }
+}
+
+// One half-step GEMV over this CTA's private block.  The list holds the trits that
+// changed since the previous half-step of the same kind in this component (all of
+// them in the first one, where g starts at 0), so g[c] += sum_{e in list} s_e blk[r_e][c]
+// keeps g = R^T t (or R t) for the current input trits t; out[c] = g[c] minus the
+// lazy-deflation correction is written to gout[out0 + c].  fp64 accumulation of exact fp32 terms, fixed summation order.
 template <int VEC>
 __device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, int64_t out0,
                           const int* __restrict__ list, int nlist, double* red, unsigned long long* gout,
@@ -292,34 +340,24 @@ __device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, i
     const int nvec = pitch / VEC;
     if (nvec <= 0) return;
     corrections(valid, hc);   // read after the CTA barrier below (or in the same thread)
-    constexpr int U = (NT >= 1024) ? ((VEC == 4) ? 8 : (VEC == 2 ? 12 : 16)) : ((VEC == 4) ? 16 : (VEC == 2 ? 24 : 32));
     if (nvec <= NT) {
         const int lanes = NT / nvec;
+        const int act = min(lanes, nlist);   // row groups that get at least one entry
         const int j = threadIdx.x % nvec;
         const int g = threadIdx.x / nvec;
         const int rs = pitch | 1;   // odd row stride (in doubles): the column sums below are bank-conflict free
-        if (g < lanes) {
+        if (g < act) {
             double acc[VEC];
             #pragma unroll
             for (int e = 0; e < VEC; ++e) acc[e] = 0.0;
             const float* base = blk + j * VEC;
-            // every batch issues all of its loads before using any (predicated tail)
-            for (int idx = g; idx < nlist; idx += U * lanes) {
-                int ent[U];
-                float v[U][VEC];
-                #pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const int ii = idx + u * lanes;
-                    ent[u] = ii < nlist ? list[ii] : 0;
-                    if (ii < nlist) {
-                        load_vec<VEC>(base + (ent[u] & 0x7fffffff), v[u]);
-                    } else {
-                        #pragma unroll
-                        for (int e = 0; e < VEC; ++e) v[u][e] = 0.f;
-                    }
-                }
-                accumulate_batch<VEC, U>(acc, ent, v);
-            }
+            // batch width from the longest group (uniform over the CTA): short change
+            // lists issue few predicated slots
+            const int per = (nlist + lanes - 1) / lanes;
+            if (per <= 1) gemv_rows<VEC, 1>(acc, base, list, nlist, g, lanes);
+            else if (per <= 2) gemv_rows<VEC, 2>(acc, base, list, nlist, g, lanes);
+            else if (per <= 4) gemv_rows<VEC, 4>(acc, base, list, nlist, g, lanes);
+            else gemv_rows<VEC, GEMV_U<VEC>()>(acc, base, list, nlist, g, lanes);
             #pragma unroll
             for (int e = 0; e < VEC; ++e) red[g * rs + j * VEC + e] = acc[e];
         }
@@ -333,11 +371,16 @@ __device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, i
             const int s = (int)threadIdx.x % tpc;
             double v = 0.0;
             if (c < pitch)
-                for (int gg = s; gg < lanes; gg += tpc) v += red[gg * rs + c];
+                for (int gg = s; gg < act; gg += tpc) v += red[gg * rs + c];
             for (int o = tpc >> 1; o; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
-            if (s == 0 && c < valid) emit_tagged(hc.L > 0 ? v - hc.corr[c] : v, out0 + c, gout, tag, skip, S);
+            if (s == 0 && c < valid) {
+                const double gc = hc.g[c] + v;
+                hc.g[c] = gc;
+                emit_tagged(hc.L > 0 ? gc - hc.corr[c] : gc, out0 + c, gout, tag, skip, S);
+            }
         }
     } else {
+        constexpr int U = GEMV_U<VEC>();
         __syncthreads();   // corrections
         for (int j = threadIdx.x; j < nvec; j += NT) {
             double acc[VEC];
@@ -352,7 +395,7 @@ __device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, i
                     const int ii = idx + u;
                     ent[u] = ii < nlist ? list[ii] : 0;
                     if (ii < nlist) {
-                        load_vec<VEC>(base + (ent[u] & 0x7fffffff), v[u]);
+                        load_vec<VEC>(base + (ent[u] & 0x3fffffff), v[u]);
                     } else {
                         #pragma unroll
                         for (int e = 0; e < VEC; ++e) v[u][e] = 0.f;
@@ -363,7 +406,11 @@ __device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, i
             #pragma unroll
             for (int e = 0; e < VEC; ++e) {
                 const int c = j * VEC + e;
-                if (c < valid) emit_tagged(hc.L > 0 ? acc[e] - hc.corr[c] : acc[e], out0 + c, gout, tag, skip, S);
+                if (c < valid) {
+                    const double gc = hc.g[c] + acc[e];
+                    hc.g[c] = gc;
+                    emit_tagged(hc.L > 0 ? gc - hc.corr[c] : gc, out0 + c, gout, tag, skip, S);
+                }
             }
         }
     }
@@ -493,9 +540,10 @@ __device__ int build_from_trits(const uint32_t* words, int64_t nwords, int64_t l
     return total;
 }
 
-// coef_l = d_l * (t_l . t) for every pending component (integer dot product of trit masks)
+// dot_l = t_l . t and coef_l = d_l dot_l for every pending component (integer dot
+// product of trit masks)
 __device__ void pending_coef(int L, int Ls, int W, const uint32_t* pnz, const uint32_t* psg, const uint32_t* nz,
-                             const uint32_t* sg, const double* pd, double* coef) {
+                             const uint32_t* sg, const double* pd, int* dots, double* coef) {
     for (int l = warp_id(); l < L; l += NWARP) {
         int acc = 0;
         for (int w = lane_id(); w < W; w += 32) {
@@ -505,7 +553,7 @@ __device__ void pending_coef(int L, int Ls, int W, const uint32_t* pnz, const ui
         }
         #pragma unroll
         for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(FULL, acc, o);
-        if (lane_id() == 0) coef[l] = pd[l] * (double)acc;
+        if (lane_id() == 0) { dots[l] = acc; coef[l] = pd[l] * (double)acc; }
     }
     __syncthreads();
 }
@@ -534,6 +582,54 @@ __device__ void pack_row(const uint32_t* nz, const uint32_t* sg, int W, uint32_t
 // buffer is rewritten only two half-steps later, after every CTA has read it, so a
 // stale word always carries the tag of two half-steps before.
 // ---------------------------------------------------------------------------
+
+// Positions where the trit vector changed from (oz, os) to (bz, bs) (nonzero mask,
+// negative mask), the sign of the change new - old, and whether it is +-2 (a flip).
+__device__ __forceinline__ uint32_t delta_mask(uint32_t oz, uint32_t os, uint32_t bz, uint32_t bs, uint32_t& neg,
+                                               uint32_t& two) {
+    two = oz & bz & (os ^ bs);
+    neg = (bz & bs) | (~bz & oz & ~os);
+    return (oz ^ bz) | two;
+}
+
+// List entry of one changed trit: element offset | negative << 31 | (|change| == 2) << 30.
+__device__ __forceinline__ int delta_entry(unsigned idx, int rowpitch, uint32_t neg, uint32_t two, int bit) {
+    return (int)(idx * (unsigned)rowpitch) | (int)(((neg >> bit) & 1u) << 31) | (int)(((two >> bit) & 1u) << 30);
+}
+
+// Block-wide: compacted list of the changes (onz, osg) -> (nz, sg) over W mask words,
+// in index order.  Returns the count.
+__device__ int build_delta_list(int W, const uint32_t* onz, const uint32_t* osg, const uint32_t* nz,
+                                const uint32_t* sg, int* list, int rowpitch, const Smem& s) {
+    const int lane = lane_id(), warp = warp_id();
+    const int wpw = (W + NWARP - 1) / NWARP;
+    const int w0 = min(W, warp * wpw), w1 = min(W, w0 + wpw);
+    int cnt = 0;
+    for (int w = w0 + lane; w < w1; w += 32) {
+        uint32_t ng, tw;
+        cnt += __popc(delta_mask(onz[w], osg[w], nz[w], sg[w], ng, tw));
+    }
+    #pragma unroll
+    for (int o = 16; o; o >>= 1) cnt += __shfl_xor_sync(FULL, cnt, o);
+    if (lane == 0) s.wd[warp] = cnt;
+    __syncthreads();
+    int off = 0, total = 0;
+    for (int w = 0; w < NWARP; ++w) {
+        const int c = s.wd[w];
+        off += (w < warp) ? c : 0;
+        total += c;
+    }
+    int run = off;
+    for (int w = w0; w < w1; ++w) {
+        uint32_t ng, tw;
+        const uint32_t ch = delta_mask(onz[w], osg[w], nz[w], sg[w], ng, tw);
+        if ((ch >> lane) & 1u)
+            list[run + __popc(ch & ((1u << lane) - 1u))] = delta_entry(((unsigned)w << 5) + lane, rowpitch, ng, tw, lane);
+        run += __popc(ch);
+    }
+    __syncthreads();
+    return total;
+}
 
 __device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
     unsigned long long v;
@@ -593,8 +689,9 @@ __device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned* p) {
 // Returns nnz; ok = false if a wait ran out.
 __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, unsigned tag, unsigned& arrivals,
                                   bool skip, double S, const unsigned long long* gvec, int64_t len, double tau,
-                                  uint32_t* nz, uint32_t* sg, int* list, int rowpitch, const Smem& s, int L, int Ls,
-                                  const uint32_t* pnz, const uint32_t* psg, double& thr_out, GroupSync* gs,
+                                  uint32_t* nz, uint32_t* sg, uint32_t* onz, uint32_t* osg, int* list, int rowpitch,
+                                  const Smem& s, int L, int Ls, const uint32_t* pnz, const uint32_t* psg, int* dots,
+                                  double* coef, bool want_p, double& thr_out, int& ndelta, GroupSync* gs,
                                   uint64_t limit_ns, int* status, bool& ok_out) {
     const int lane = lane_id(), warp = warp_id();
     // ---- this CTA's partial (fixed butterfly + fixed cross-warp combine)
@@ -608,16 +705,13 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
         for (int o = 16; o; o >>= 1) S2 += __shfl_xor_sync(FULL, S2, o);
         if (lane == 0 && !skip) {
             st_relaxed_u64(partials + q, tag_value(S2, tag));
-#ifdef EXTERND_RELEASE_ARRIVE
-            red_release_add(&gs->ctr[q % NCTR][0], 1u);
-#else
             red_relaxed_add(&gs->ctr[q % NCTR][0], 1u);
-#endif
         }
     }
     ++arrivals;
     phase_mark(s, 2);
-    // ---- wait for all arrivals, then everyone's partials
+    // ---- wait for all arrivals (NCTR threads poll one counter each, bounded), then
+    //      everyone's partials
     int ok = 1;
     if ((int)threadIdx.x < NCTR && (int)threadIdx.x < Gg) {
         const int c = threadIdx.x;
@@ -668,77 +762,123 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
     const double thr = tau * St / (double)len;
     thr_out = thr;
 
-    // ---- one pass over the vector: threshold, masks, counts, pending dots
-    int cnt = 0, dot = 0;
+    // ---- one pass over the vector: threshold, masks, counts, pending dots.  The warp
+    //      takes its words in groups of up to 32: first every ballot (registers only),
+    //      then lane i handles word base + i (old masks, changes, stores) in parallel.
+    int cnt = 0, dcnt = 0, dot = 0;
     double ps = 0.0;
-    for (int base = w0; base < w1; base += CH) {
-        if (base != w0) {
+    for (int base = w0; base < w1; base += 32) {
+        const int K = min(32, w1 - base);
+        uint32_t my_bz = 0u, my_bs = 0u;
+        for (int c0 = 0; c0 < K; c0 += CH) {
+            if (base != w0 || c0 != 0) {
+                #pragma unroll
+                for (int i = 0; i < CH; ++i) {
+                    const int w = base + c0 + i;
+                    const int64_t idx = ((int64_t)w << 5) + lane;
+                    wb[i] = (c0 + i < K && idx < len) ? ld_relaxed_u64(gvec + idx) : (unsigned long long)tag;
+                }
+            }
             #pragma unroll
             for (int i = 0; i < CH; ++i) {
-                const int w = base + i;
-                const int64_t idx = ((int64_t)w << 5) + lane;
-                wb[i] = (w < w1 && idx < len) ? ld_relaxed_u64(gvec + idx) : (unsigned long long)tag;
+                if ((unsigned)(wb[i] & 0xFFull) != tag)
+                    wb[i] = wait_tagged(gvec + ((int64_t)(base + c0 + i) << 5) + lane, tag, gs, limit_ns, status, ok,
+                                        s.clk + 10);
             }
-        }
-        #pragma unroll
-        for (int i = 0; i < CH; ++i) {
-            if ((unsigned)(wb[i] & 0xFFull) != tag)
-                wb[i] = wait_tagged(gvec + ((int64_t)(base + i) << 5) + lane, tag, gs, limit_ns, status, ok, s.clk + 10);
-        }
-        #pragma unroll
-        for (int i = 0; i < CH; ++i) {
-            const int w = base + i;
-            if (w < w1) {
-                const int64_t idx = ((int64_t)w << 5) + lane;
-                const double x = untag(wb[i]);
-                const bool z = (idx < len) && (fabs(x) > thr);
-                const bool ng = z && (x < 0.0);
-                const unsigned bz = __ballot_sync(FULL, z);
-                const unsigned bs = __ballot_sync(FULL, ng);
-                if (lane == 0) { nz[w] = bz; sg[w] = bs; }
-                cnt += __popc(bz);
-                if (z) ps += fabs(x);
-                if (lane < L) {
-                    const uint32_t both = pnz[w * Ls + lane] & bz;
-                    const uint32_t diff = psg[w * Ls + lane] ^ bs;
-                    dot += __popc(both & ~diff) - __popc(both & diff);
+            #pragma unroll
+            for (int i = 0; i < CH; ++i) {
+                if (c0 + i < K) {
+                    const double x = untag(wb[i]);           // padding words untag to 0
+                    const bool z = fabs(x) > thr;
+                    const unsigned bz = __ballot_sync(FULL, z);
+                    const unsigned bs = __ballot_sync(FULL, z && (x < 0.0));
+                    if (lane == c0 + i) { my_bz = bz; my_bs = bs; }
+                    if (want_p && z) ps += fabs(x);
                 }
             }
         }
+        const int w = base + lane;
+        uint32_t oz = 0u, os = 0u, ch = 0u, dn, dt;
+        if (lane < K) {
+            oz = nz[w];
+            os = sg[w];
+            ch = delta_mask(oz, os, my_bz, my_bs, dn, dt);
+        }
+        __syncwarp();
+        if (lane < K) { nz[w] = my_bz; sg[w] = my_bs; onz[w] = oz; osg[w] = os; }
+        cnt += __popc(my_bz);
+        dcnt += __popc(ch);
+        // change of t_l . t over the words that changed (lane l = pending component l)
+        unsigned chw = __ballot_sync(FULL, ch != 0u);
+        while (chw) {
+            const int i = __ffs(chw) - 1;
+            chw &= chw - 1u;
+            const uint32_t zi = __shfl_sync(FULL, my_bz, i), si = __shfl_sync(FULL, my_bs, i);
+            const uint32_t ozi = __shfl_sync(FULL, oz, i), osi = __shfl_sync(FULL, os, i);
+            const uint32_t chi = __shfl_sync(FULL, ch, i);
+            if (lane < L) {
+                const uint32_t pz = pnz[(base + i) * Ls + lane], pg = psg[(base + i) * Ls + lane];
+                const uint32_t zn = pz & zi & chi, zo = pz & ozi & chi;
+                const uint32_t sn = pg ^ si, so = pg ^ osi;
+                dot += (__popc(zn & ~sn) - __popc(zn & sn)) - (__popc(zo & ~so) - __popc(zo & so));
+            }
+        }
     }
+    cnt = __reduce_add_sync(FULL, cnt);
+    dcnt = __reduce_add_sync(FULL, dcnt);
     #pragma unroll
     for (int o = 16; o; o >>= 1) ps += __shfl_xor_sync(FULL, ps, o);
-    if (lane == 0) { s.wc[warp] = cnt; s.wp[warp] = ps; }
+    if (lane == 0) { s.wc[warp] = cnt; s.wd[warp] = dcnt; s.wp[warp] = ps; }
     if (lane < L) s.dotp[warp * MAX_PENDING + lane] = dot;
     ok = __syncthreads_and(ok);
     phase_mark(s, 5);
     if (!ok) { ok_out = false; return 0; }
     int cw = lane < NWARP ? s.wc[lane] : 0;
+    const int dw = lane < NWARP ? s.wd[lane] : 0;
     double p = lane < NWARP ? s.wp[lane] : 0.0;
-    int incl = cw;
+    int incl = dw;
     #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const int t = __shfl_up_sync(FULL, incl, o);
         if (lane >= o) incl += t;
+        cw += __shfl_xor_sync(FULL, cw, o);
     }
-    const int off = __shfl_sync(FULL, incl - cw, warp);
-    const int total = __shfl_sync(FULL, incl, 31);
+    const int off = __shfl_sync(FULL, incl - dw, warp);
+    const int dtotal = __shfl_sync(FULL, incl, 31);
+    const int total = cw;
     #pragma unroll
     for (int o = 16; o; o >>= 1) p += __shfl_xor_sync(FULL, p, o);
     if (total > 0) {
-        if ((int)threadIdx.x < L) {
-            int d = 0;
-            for (int w = 0; w < NWARP; ++w) d += s.dotp[w * MAX_PENDING + threadIdx.x];
-            s.coef[threadIdx.x] = s.pd[threadIdx.x] * (double)d;
+        for (int l = warp; l < L; l += NWARP) {
+            int d = lane < NWARP ? s.dotp[lane * MAX_PENDING + l] : 0;
+            #pragma unroll
+            for (int o = 16; o; o >>= 1) d += __shfl_xor_sync(FULL, d, o);
+            if (lane == 0) {
+                d += dots[l];
+                dots[l] = d;
+                coef[l] = s.pd[l] * (double)d;
+            }
         }
         int run = off;
-        for (int w = w0; w < w1; ++w) {
-            const uint32_t bz = nz[w];
-            if ((bz >> lane) & 1u)
-                list[run + __popc(bz & ((1u << lane) - 1u))] =
-                    (int)((((unsigned)w << 5) + lane) * (unsigned)rowpitch) | (int)(((sg[w] >> lane) & 1u) << 31);
-            run += __popc(bz);
+        for (int base = w0; base < w1; base += 32) {
+            const int w = base + lane;
+            uint32_t ch = 0u, ng = 0u, tw = 0u;
+            if (w < w1) ch = delta_mask(onz[w], osg[w], nz[w], sg[w], ng, tw);
+            const int c = __popc(ch);
+            int incl = c;
+            #pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(FULL, incl, o);
+                if (lane >= o) incl += t;
+            }
+            int at = run + incl - c;
+            for (uint32_t mk = ch; mk; mk &= mk - 1u) {
+                const int b = __ffs(mk) - 1;
+                list[at++] = delta_entry(((unsigned)w << 5) + b, rowpitch, ng, tw, b);
+            }
+            run += __shfl_sync(FULL, incl, 31);
         }
+        ndelta = dtotal;
         if (threadIdx.x == 0) { s.scal[0] = p; s.scal[1] = 0.0; }
     } else {
         // all-zero fallback: keep the lowest index among the largest magnitudes
@@ -756,18 +896,15 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
         const bool neg = x < 0.0;
         const int wj = (int)(Jc >> 5);
         const uint32_t bj = 1u << (Jc & 31);
-        if ((int)threadIdx.x < L) {
-            int t = (pnz[wj * Ls + threadIdx.x] & bj) ? 1 : 0;
-            if (t && ((psg[wj * Ls + threadIdx.x] & bj) != 0u) != neg) t = -1;
-            s.coef[threadIdx.x] = s.pd[threadIdx.x] * (double)t;
-        }
         if (threadIdx.x == 0) {
             nz[wj] |= bj;
             if (neg) sg[wj] |= bj;
-            list[0] = (int)((unsigned)Jc * (unsigned)rowpitch) | (neg ? (int)0x80000000 : 0);
             s.scal[0] = fabs(x);
             s.scal[1] = 1.0;
         }
+        __syncthreads();
+        ndelta = build_delta_list((int)((len + 31) >> 5), onz, osg, nz, sg, list, rowpitch, s);
+        if (L > 0) pending_coef(L, Ls, (int)((len + 31) >> 5), pnz, psg, nz, sg, s.pd, dots, coef);
     }
     __syncthreads();
     phase_mark(s, 6);
@@ -830,24 +967,33 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
 
     double RN2 = N0;
     int L = 0;
-    unsigned long long sum_nu = 0, sum_nv = 0, sum_nunv = 0, hs = 0, fb = 0;
+    unsigned long long sum_nu = 0, sum_nv = 0, sum_du = 0, sum_dv = 0, sum_nunv = 0, hs = 0, fb = 0;
     const int64_t kk = (mode == MODE_FACTOR) ? P.k : 1;
-    int nU = 0, nV = 0;
+    int nU = 0, nV = 0, dU = 0, dV = 0;   // support sizes and list lengths (trit changes)
     double p = 0.0, thr;
     unsigned gen = 0;   // half-step counter of this matrix (tags of the exchanged words)
-    HalfCorr hcV{s.coef, s.cnzV, s.csgV, s.corr, 0};
-    HalfCorr hcU{s.coef, s.cnzU, s.csgU, s.corr, 0};
+    HalfCorr hcV{s.coef, s.cnzV, s.csgV, s.corr, s.gV, 0};
+    HalfCorr hcU{s.coefV, s.cnzU, s.csgU, s.corr, s.gU, 0};
     if (blockIdx.x == 0 && tid == 0) {
         for (int k2 = 0; k2 < 11; ++k2) s.clk[k2] = 0ull;
         s.clk[11] = (unsigned long long)clock64();
     }
 
     for (int64_t i = 0; i < kk; ++i) {
+        // a new component: the GEMV sums restart from zero and the previous trits
+        // of the output vectors are zero, so the first lists hold whole supports
+        for (int c = tid; c < pitchV; c += NT) s.gV[c] = 0.0;
+        for (int c = tid; c < pitchU; c += NT) s.gU[c] = 0.0;
         if (mode != MODE_HALF_U) {
+            for (int w = tid; w < Wn; w += NT) { s.nzV[w] = 0u; s.sgV[w] = 0u; }
             nU = build_from_trits(P.start + i * P.start_words, P.start_words, m, s.nzU, s.sgU, s.ulist, pitchV, s);
-            if (L > 0) pending_coef(L, Ls, Wm, s.pnzU, s.psgU, s.nzU, s.sgU, s.pd, s.coef);
+            dU = nU;
+            if (L > 0) pending_coef(L, Ls, Wm, s.pnzU, s.psgU, s.nzU, s.sgU, s.pd, s.dotU, s.coef);
+            for (int l = tid; l < L; l += NT) { s.dotV[l] = 0; s.coefV[l] = 0.0; }
         } else {
+            for (int w = tid; w < Wm; w += NT) { s.nzU[w] = 0u; s.sgU[w] = 0u; }
             nV = build_from_trits(P.start, P.start_words, n, s.nzV, s.sgV, s.vlist, pitchU, s);
+            dV = nV;
         }
         phase_mark(s, 7);
         for (int it = 0; it < P.iters; ++it) {
@@ -857,16 +1003,17 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
                 const unsigned tg = gen_tag(++gen);
                 double S;
                 hcV.L = L;
-                gemv_dispatch(P.pv.vec, blkV, pitchV, validV, c0, s.ulist, nU, s.red, P.xbuf, hcV, tg, skip, S, s.clk);
+                gemv_dispatch(P.pv.vec, blkV, pitchV, validV, c0, s.ulist, dU, s.red, P.xbuf, hcV, tg, skip, S, s.clk);
                 phase_mark(s, 1);
                 bool ok = true;
                 const int nv2 = exchange_threshold(P.partV, q, Gg, tg, arrivals, skip, S, P.xbuf, n, P.tau, s.nzV,
-                                                   s.sgV, s.vlist, pitchU, s, L, Ls, s.pnzV, s.psgV, thr, gs, cfg.limit_ns,
-                                                   P.status, ok);
+                                                   s.sgV, s.onzV, s.osgV, s.vlist, pitchU, s, L, Ls, s.pnzV, s.psgV,
+                                                   s.dotV, s.coefV, false, thr, dV, gs, cfg.limit_ns, P.status, ok);
                 if (!ok) return false;
                 fb += (s.scal[1] != 0.0) ? 1 : 0;
-                nV = nv2;
                 sum_nu += (unsigned long long)nU;
+                sum_du += (unsigned long long)dU;
+                nV = nv2;
                 ++hs;
                 if (mode == MODE_HALF_V) {
                     if (lead) {
@@ -884,15 +1031,17 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
             const unsigned tg = gen_tag(++gen);
             double S;
             hcU.L = L;
-            gemv_dispatch(P.pu.vec, blkU, pitchU, validU, r0, s.vlist, nV, s.red, P.ybuf, hcU, tg, skip, S, s.clk);
+            gemv_dispatch(P.pu.vec, blkU, pitchU, validU, r0, s.vlist, dV, s.red, P.ybuf, hcU, tg, skip, S, s.clk);
             phase_mark(s, 1);
             bool ok = true;
-            nU = exchange_threshold(P.partU, q, Gg, tg, arrivals, skip, S, P.ybuf, m, P.tau, s.nzU, s.sgU, s.ulist,
-                                    pitchV, s, L, Ls, s.pnzU, s.psgU, thr, gs, cfg.limit_ns, P.status, ok);
+            sum_nv += (unsigned long long)nV;
+            sum_dv += (unsigned long long)dV;
+            nU = exchange_threshold(P.partU, q, Gg, tg, arrivals, skip, S, P.ybuf, m, P.tau, s.nzU, s.sgU, s.onzU,
+                                    s.osgU, s.ulist, pitchV, s, L, Ls, s.pnzU, s.psgU, s.dotU, s.coef, true, thr, dU,
+                                    gs, cfg.limit_ns, P.status, ok);
             if (!ok) return false;
             p = s.scal[0];
             fb += (s.scal[1] != 0.0) ? 1 : 0;
-            sum_nv += (unsigned long long)nV;
             ++hs;
             if (mode == MODE_HALF_U) {
                 if (lead) {
@@ -970,6 +1119,8 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
     if (lead && tid == 0) {
         P.stats->sum_nu = sum_nu;
         P.stats->sum_nv = sum_nv;
+        P.stats->sum_du = sum_du;
+        P.stats->sum_dv = sum_dv;
         P.stats->sum_nunv = sum_nunv;
         P.stats->half_steps = hs;
         P.stats->fallbacks = fb;
@@ -994,6 +1145,9 @@ __global__ void __launch_bounds__(NT, 1) als_kernel(const KCfg cfg) {
     s.red = reinterpret_cast<double*>(smem_raw + lay.red);
     s.pd = reinterpret_cast<double*>(smem_raw + lay.pd);
     s.coef = reinterpret_cast<double*>(smem_raw + lay.coef);
+    s.coefV = reinterpret_cast<double*>(smem_raw + lay.coefV);
+    s.dotU = reinterpret_cast<int*>(smem_raw + lay.dotU);
+    s.dotV = reinterpret_cast<int*>(smem_raw + lay.dotV);
     s.scal = reinterpret_cast<double*>(smem_raw + lay.scal);
     s.wS = reinterpret_cast<double*>(smem_raw + lay.wS);
     s.wM = reinterpret_cast<double*>(smem_raw + lay.wM);
@@ -1020,6 +1174,13 @@ __global__ void __launch_bounds__(NT, 1) als_kernel(const KCfg cfg) {
     s.csgU = reinterpret_cast<uint32_t*>(smem_raw + lay.csgU);
     s.ulist = reinterpret_cast<int*>(smem_raw + lay.ulist);
     s.vlist = reinterpret_cast<int*>(smem_raw + lay.vlist);
+    s.wd = reinterpret_cast<int*>(smem_raw + lay.wd);
+    s.onzU = reinterpret_cast<uint32_t*>(smem_raw + lay.onzU);
+    s.osgU = reinterpret_cast<uint32_t*>(smem_raw + lay.osgU);
+    s.onzV = reinterpret_cast<uint32_t*>(smem_raw + lay.onzV);
+    s.osgV = reinterpret_cast<uint32_t*>(smem_raw + lay.osgV);
+    s.gV = reinterpret_cast<double*>(smem_raw + lay.gV);
+    s.gU = reinterpret_cast<double*>(smem_raw + lay.gU);
     s.corr = reinterpret_cast<double*>(smem_raw + lay.corr);
 
     GroupSync* gs = cfg.gsync + grp;
@@ -1288,7 +1449,7 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
         pu_max = pu > pu_max ? pu : pu_max;
     }
     for (int b = 0; b < np; ++b)
-        if ((double)in[b].m * pv_max >= 2147483647.0 || (double)in[b].n * pu_max >= 2147483647.0) return EXTERND_ELIMIT;
+        if ((double)in[b].m * pv_max >= 1073741824.0 || (double)in[b].n * pu_max >= 1073741824.0) return EXTERND_ELIMIT;
     int Lcap = MAX_PENDING;
     while (Lcap > 1 && als_smem_bytes(m_max, n_max, Lcap, pv_max, pu_max) > di.smem_optin) --Lcap;
     if (opt.pending > 0 && opt.pending < Lcap) Lcap = opt.pending;
@@ -1543,6 +1704,8 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
             const DevStats& d = hstats[b];
             st.alg_bytes += 4.0 * ((double)in[b].n * (double)d.sum_nu + (double)in[b].m * (double)d.sum_nv) +
                             8.0 * (double)d.sum_nunv;
+            st.read_bytes += 4.0 * ((double)in[b].n * (double)d.sum_du + (double)in[b].m * (double)d.sum_dv) +
+                             8.0 * (double)d.sum_nunv;
             st.components += in[b].k;
             st.half_steps += (int64_t)d.half_steps;
             st.fallbacks += (int64_t)d.fallbacks;

@@ -22,13 +22,22 @@
 //    output and its partial sum, meets the others at one counter, then reads
 //    the whole vector back and thresholds it itself (all CTAs derive the
 //    identical trit vector because they use the same data in the same order).
+//  * Incremental GEMVs: within a component R is fixed, so each CTA keeps the
+//    running sums g = R^T u (its columns) and R v (its rows) in shared memory
+//    and each half-step reads only the rows (columns) whose trit changed since
+//    the previous half-step of the same kind: g += R^T (u_new - u_old), with
+//    coefficients +-1 or +-2.  The first half-steps of a component start from
+//    g = 0 and the whole support.  After the first few fits only a few percent
+//    of the trits change per fit, so most half-steps read a small part of R.
 //  * Deflation is lazy: the last L components (d_j, u_j, v_j) are held as
 //    bit masks in shared memory and applied as rank-1 corrections to each
-//    GEMV output (x -= sum_j d_j (u_j . u) v_j); every L components each CTA
-//    folds them into its own two blocks in one pass (fp64 sum, one fp32
-//    rounding per entry).
-//  * All accumulation is fp64 (each fp32 residual entry is added exactly), so
-//    threshold decisions are taken on fp64 values like the fp64 oracle.
+//    GEMV output (x -= sum_j d_j (u_j . u) v_j, the integer dot products kept
+//    up to date from the changed trits); every L components each CTA folds
+//    them into its own two blocks in one pass (fp64 sum, one fp32 rounding
+//    per entry).
+//  * Accumulation: batches of at most 16 signed fp32 residual entries are
+//    summed in fp32 with fused multiply-adds, batch sums are added in fp64,
+//    and the threshold decisions are taken on fp64 values like the oracle.
 //  * Every device-side wait is bounded by %globaltimer; a wait that runs out
 //    raises a status word and the kernel returns.
 #pragma once
@@ -82,8 +91,10 @@ struct GroupSync {            // one per CTA group
 };
 
 struct DevStats {
-    unsigned long long sum_nu;      // rows read by V-steps
-    unsigned long long sum_nv;      // columns read by U-steps
+    unsigned long long sum_nu;      // sum of nnz(u) over V-steps (rows a direct evaluation reads)
+    unsigned long long sum_nv;      // sum of nnz(v) over U-steps
+    unsigned long long sum_du;      // rows read by V-steps (trit changes of u)
+    unsigned long long sum_dv;      // columns read by U-steps (trit changes of v)
     unsigned long long sum_nunv;    // sum nnz(u_i) nnz(v_i)
     unsigned long long half_steps;
     unsigned long long fallbacks;
