@@ -126,26 +126,21 @@ class ClockSampler:
 
 
 def _dist():
-    ws = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    return ws, rank, local
+    from ternary_rank_weight_b200.dist import rank_info
+    r = rank_info()
+    return r.world, r.rank, r.local
 
 
 def _workload_arrays(name: str, rank: int, mu=None):
+    """This rank's workload (weak scaling: same shapes and recipe, seeds offset by rank) and matrices."""
     import dataclasses
+    from ternary_rank_weight_b200.dist import rank_workload
     from ternary_rank_weight_b200.workloads import WORKLOADS
     w = WORKLOADS[name]
     if mu is not None:
         w = dataclasses.replace(w, mu=tuple(mu for _ in w.mu))
-    mats = []
-    for b in range(w.count):
-        if rank == 0:
-            mats.append(w.matrix(b))
-        else:  # weak scaling: each rank its own matrices, same shapes and recipe
-            wr = dataclasses.replace(w, seeds=tuple(s + 1000 * rank for s in w.seeds))
-            mats.append(wr.matrix(b))
-    return w, mats
+    w = rank_workload(w, rank)
+    return w, w.matrices()
 
 
 def _config(w, extra=None):
@@ -240,27 +235,22 @@ def run_ours(args):
     k_total = sum(ext.rank(a.shape[0], a.shape[1], mu) for a, mu in zip(mats, w.mu))
     stream = torch.cuda.current_stream(dev)
 
+    from ternary_rank_weight_b200 import dist
+
     def step(inputs):
         if w.count == 1:
-            f = ext.factor(inputs[0], w.mu[0], w.tau[0], iters=w.iters, seed=w.seeds[0] + 1000 * rank,
+            f = ext.factor(inputs[0], w.mu[0], w.tau[0], iters=w.iters, seed=w.seeds[0],
                            grid=args.grid, pending=args.pending)
             return [f], f.stats
-        res, st = ext.factor_batched(inputs, w.mu, w.tau, iters=w.iters,
-                                     seeds=[s + 1000 * rank for s in w.seeds])
+        res, st = ext.factor_batched(inputs, w.mu, w.tau, iters=w.iters, seeds=list(w.seeds))
         assert all(s == 0 for s in st), st
         return res, res[0].stats
 
     def barrier():
-        if ws > 1:
-            torch.distributed.barrier()
-        torch.cuda.synchronize()
+        dist.barrier(dev)
 
     def max_over_ranks(x: float) -> float:
-        if ws == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
+        return dist.max_over_ranks(x, dev)
 
     for _ in range(args.warmup):
         step(As)
@@ -282,7 +272,7 @@ def run_ours(args):
         barrier()
     t_ms = max_over_ranks(ev0.elapsed_time(ev1))
     clocks = clk.summary()
-    value = ws * k_total * args.steps / (t_ms / 1000.0)
+    value = dist.throughput(dist.sum_over_ranks(k_total * args.steps, dev), t_ms)
 
     # ---- end to end through the public API with pinned host buffers
     step(host_As)
@@ -299,7 +289,7 @@ def run_ours(args):
     e1.record(stream)
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-    e2e_value = ws * k_total * args.steps / (e2e_ms / 1000.0)
+    e2e_value = dist.throughput(dist.sum_over_ranks(k_total * args.steps, dev), e2e_ms)
 
     peak, peak_kind = _peaks()
     mean_als = statistics.mean(als_ms)
