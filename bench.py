@@ -297,6 +297,13 @@ def run_ours(args):
     achieved = mean_bytes / (mean_als / 1000.0) / 1e9
     traffic = _ncu_traffic(w.name)
     energy_final = float(res[0].energy[-1].item()) if res[0].energy is not None else None
+    energy_curve = None
+    if w.mu_sweep and res[0].energy is not None:
+        # the start vector of component i depends only on (seed, i), so the first k
+        # components of the largest-mu run are the run at smaller mu (prefix property)
+        e = res[0].energy.cpu()
+        m0, n0 = w.shapes[0]
+        energy_curve = {str(mu): float(e[ext.rank(m0, n0, mu) - 1].item()) for mu in w.mu_sweep}
     out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": t_ms / args.steps, "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
@@ -314,6 +321,7 @@ def run_ours(args):
            "gpu_launches": launches,
            "clocks": clocks,
            "energy": energy_final,
+           "energy_vs_mu": energy_curve,
            "components_per_step": ws * k_total,
            "wall_s_per_matrix": (t_ms / 1000.0) / args.steps / w.count}
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
