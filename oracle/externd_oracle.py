@@ -16,7 +16,9 @@ arXiv 2607.13511), cited below by section and display equation:
 * §2.3 steps 1-3: R <- A; for each component: 15 alternating fits
   v <- T_tau(R^T u), u <- T_tau(R v); scale d = u^T R v / (||u||^2 ||v||^2);
   deflate R <- R - d u v^T; store B[:, i] = u, C[i, :] = v^T.
-* §2.6 Eq. (1): bpw_eff = mu (m + n) / max(m, n) * (2 - sparsity).
+* §2.6 Cost model: inference computes y = B (diag(D) (C x)); mask+sign packing
+  stores one zero/nonzero mask bit per element plus one sign bit per nonzero,
+  and Eq. (1): bpw_eff = mu (m + n) / max(m, n) * (2 - sparsity).
 
 Everything is plain numpy in float64, written in the pages' order.  Readings
 where the pages are silent (each one is listed with its reason in the design
@@ -309,3 +311,50 @@ def bpw_eff(mu: float, m: int, n: int, sparsity: float) -> float:
 def gaussian_zero_fraction(tau: float) -> float:
     """P(|z| <= tau * E|z|) for z ~ N(0,1): 2 Phi(tau sqrt(2/pi)) - 1 = erf(tau / sqrt(pi))."""
     return math.erf(tau / math.sqrt(math.pi))
+
+
+# ----------------------------------------------------------------------------
+# §2.6 inference with the factors and mask+sign storage
+# ----------------------------------------------------------------------------
+
+
+def factored_matvec(B: np.ndarray, D: np.ndarray, C: np.ndarray, X: np.ndarray) -> np.ndarray:
+    """§2.6: y = B (diag(D) (C x)) for each column x of X, in fp64, in the pages' order.
+
+    B: m x k trits, D: k scales, C: k x n trits, X: n x batch.  Returns m x batch.
+    """
+    z = np.asarray(C, dtype=np.float64) @ np.asarray(X, dtype=np.float64)     # C x: k ternary sums each
+    z = np.asarray(D, dtype=np.float64)[:, None] * z                           # diag(D): k multiplies
+    return np.asarray(B, dtype=np.float64) @ z                                 # B (.): m ternary sums each
+
+
+def ternary_op_count(B: np.ndarray, C: np.ndarray) -> int:
+    """Add/subtract operations of y = B(diag(D)(Cx)) counted as the nonzero trits touched."""
+    return int(np.count_nonzero(B)) + int(np.count_nonzero(C))
+
+
+def mask_sign_pack(t: np.ndarray):
+    """§2.6 mask+sign packing of one trit row: a 1-bit zero/nonzero mask per element and
+    one sign bit per nonzero element (1 = negative), both least-significant bit first.
+
+    Returns (mask bytes, sign bytes, number of nonzeros)."""
+    t = np.asarray(t, dtype=np.int8)
+    nz = t != 0
+    mask = np.packbits(nz.astype(np.uint8), bitorder="little")
+    signs = np.packbits((t[nz] < 0).astype(np.uint8), bitorder="little")
+    return mask, signs, int(nz.sum())
+
+
+def mask_sign_unpack(mask: np.ndarray, signs: np.ndarray, length: int) -> np.ndarray:
+    nz = np.unpackbits(np.asarray(mask, dtype=np.uint8), bitorder="little")[:length].astype(bool)
+    cnt = int(nz.sum())
+    neg = np.unpackbits(np.asarray(signs, dtype=np.uint8), bitorder="little")[:cnt].astype(bool)
+    t = np.zeros(length, dtype=np.int8)
+    vals = np.where(neg, -1, 1).astype(np.int8)
+    t[nz] = vals
+    return t
+
+
+def mask_sign_bits(B: np.ndarray, C: np.ndarray) -> int:
+    """Storage of the factors in mask+sign form: one mask bit per element, one sign bit per nonzero."""
+    return int(B.size + C.size + np.count_nonzero(B) + np.count_nonzero(C))

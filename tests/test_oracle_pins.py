@@ -296,3 +296,52 @@ def test_rank_rounding_and_bpw_eq1():
 def test_zero_matrix_rejected():
     with pytest.raises(ValueError):
         ora.greedy_als(np.zeros((4, 4), dtype=np.float32), k=2, tau=0.7)
+
+
+# --------------------------------------------------------------------------
+# §2.6 inference y = B(diag(D)(Cx)) and mask+sign storage
+# --------------------------------------------------------------------------
+
+def test_factored_matvec_hand_example():
+    B = np.array([[1, 0], [-1, 1], [0, -1]], dtype=np.int8)      # m=3, k=2
+    D = np.array([0.5, 2.0])
+    C = np.array([[1, -1, 0, 1], [0, 1, 1, 0]], dtype=np.int8)   # k=2, n=4
+    x = np.array([[1.0], [2.0], [3.0], [4.0]])
+    # C x = [1 - 2 + 4, 2 + 3] = [3, 5]; D * = [1.5, 10]; B . = [1.5, -1.5 + 10, -10]
+    y = ora.factored_matvec(B, D, C, x)
+    assert y[:, 0].tolist() == [1.5, 8.5, -10.0]
+    assert ora.ternary_op_count(B, C) == 4 + 5
+
+
+def test_factored_matvec_equals_reconstruction_times_x():
+    A = np.random.default_rng(31).standard_normal((40, 56)).astype(np.float32) * 0.02
+    f = ora.greedy_als(A, k=ora.rank(40, 56, 1.5), tau=1.0, seed=4)
+    X = np.random.default_rng(32).standard_normal((56, 3))
+    y = ora.factored_matvec(f.B, f.D, f.C, X)
+    want = ora.reconstruct(f.B, f.D, f.C) @ X
+    assert np.allclose(y, want, rtol=1e-12, atol=1e-14)
+    # the pages' count: at most k (m + n) ternary add/subtracts (zeros cost nothing here)
+    k = f.k
+    assert ora.ternary_op_count(f.B, f.C) <= k * (40 + 56)
+    assert ora.ternary_op_count(f.B, f.C) == round(k * (40 + 56) * (1.0 - f.zero_fraction()))
+
+
+def test_mask_sign_pack_hand_example_and_round_trip():
+    mask, signs, nnz = ora.mask_sign_pack(np.array([1, 0, -1, 1, 0], dtype=np.int8))
+    assert nnz == 3 and mask.tolist() == [0b01101] and signs.tolist() == [0b010]
+    rng = np.random.default_rng(9)
+    for length in (1, 7, 8, 9, 64, 1000):
+        t = rng.choice([-1, 0, 1], size=length, p=[0.3, 0.4, 0.3]).astype(np.int8)
+        m_, s_, c_ = ora.mask_sign_pack(t)
+        assert len(m_) == (length + 7) // 8 and len(s_) == (c_ + 7) // 8
+        assert np.array_equal(ora.mask_sign_unpack(m_, s_, length), t)
+
+
+def test_mask_sign_storage_matches_eq1():
+    """Bits of the mask+sign form divided by m n equal Eq. (1) with the factors' own sparsity."""
+    for m, n, mu, tau in ((48, 80, 2.0, 1.0), (64, 32, 1.5, 0.7)):
+        A = np.random.default_rng(m + n).standard_normal((m, n)).astype(np.float32)
+        k = ora.rank(m, n, mu)
+        f = ora.greedy_als(A, k=k, tau=tau, seed=1)
+        bits = ora.mask_sign_bits(f.B, f.C)
+        assert bits / (m * n) == pytest.approx(ora.bpw_eff(mu, m, n, f.zero_fraction()), rel=1e-12)
