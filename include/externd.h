@@ -132,6 +132,46 @@ int externd_factor_batched(int count, const float* const* A, const int64_t* m, c
 int externd_reconstruct(const uint8_t* B, const float* D, const uint8_t* C, int64_t m, int64_t n,
                         int64_t k, float* A_hat_out, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Inference with the factors (§2.6 Cost model: y = B (diag(D) (C x)), k (m + n)
+ * ternary add/subtracts plus k multiplies) and mask+sign storage (§2.6 Eq. 1).
+ * All pointers are DEVICE pointers (EXTERND_EINVAL otherwise); trit rows are
+ * in the 2-bit format above.
+ * ------------------------------------------------------------------------- */
+
+/* Transpose a matrix of trits: T has `rows` rows of `len` trits (row stride
+ * externd_trit_bytes(len)); Tt_out receives `len` rows of `rows` trits (row stride
+ * externd_trit_bytes(rows)), Tt[j][r] = T[r][j].  Used once per factorization to
+ * lay B out for inference: externd_transpose_trits(B_out, k, m, Bt) gives Bt with
+ * row r = B[r, 0..k).  Synchronous; returns EXTERND_OK or a negative status. */
+int externd_transpose_trits(const uint8_t* T, int64_t rows, int64_t len, uint8_t* Tt_out, void* stream);
+
+/* Y[b] = B diag(D) C X[b] for b < batch (§2.6).
+ *   Bt      [in]  m rows x externd_trit_bytes(k): B transposed (externd_transpose_trits).
+ *   D       [in]  k fp32 scales.
+ *   C       [in]  k rows x externd_trit_bytes(n), as returned by externd_factor.
+ *   X       [in]  batch x n fp32, row-major (one input vector per row).
+ *   Y       [out] batch x m fp32, row-major.
+ *   z_work  [tmp] k x min(batch, 8) fp32 scratch owned by the caller (C x per vector).
+ * fp32 arithmetic; stream-ordered and asynchronous (no allocation, no host sync). */
+int externd_matvec(const uint8_t* Bt, const float* D, const uint8_t* C, int64_t m, int64_t n, int64_t k,
+                   const float* X, int64_t batch, float* Y, float* z_work, void* stream);
+
+/* Mask+sign storage of trit rows (§2.6): one zero/nonzero bit per element and
+ * one sign bit (1 = negative) per nonzero element.
+ *   T                [in]  rows x externd_trit_bytes(len) 2-bit trits.
+ *   mask_out         [out] rows x ceil(len / 8) bytes; bit j % 8 of byte j / 8 of
+ *                          row r is T[r][j] != 0.
+ *   sign_out         [out] one bit stream of sign_words 32-bit words: the signs of
+ *                          row r's nonzeros, in order, start at bit
+ *                          sign_offsets_out[r] (bit b = bit b % 32 of word b / 32).
+ *   sign_offsets_out [out] rows + 1 int64; the last entry is the total number of
+ *                          nonzeros.  EXTERND_ELIMIT if they need more than
+ *                          sign_words words.
+ * Synchronous (allocates a small stream-ordered buffer). */
+int externd_pack_mask_sign(const uint8_t* T, int64_t rows, int64_t len, uint8_t* mask_out, uint32_t* sign_out,
+                           int64_t sign_words, int64_t* sign_offsets_out, void* stream);
+
 /* Human-readable message for a status code (static storage). */
 const char* externd_strerror(int status);
 

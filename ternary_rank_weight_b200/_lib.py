@@ -24,6 +24,9 @@ EXPORTS = (
     "externd_debug_halfstep",
     "externd_debug_start_trits",
     "externd_last_stats",
+    "externd_transpose_trits",
+    "externd_matvec",
+    "externd_pack_mask_sign",
 )
 
 
@@ -106,5 +109,11 @@ def load():
     L.externd_debug_start_trits.restype = c_int
     L.externd_last_stats.argtypes = [ctypes.POINTER(Stats)]
     L.externd_last_stats.restype = c_int
+    L.externd_transpose_trits.argtypes = [vp, i64, i64, vp, vp]
+    L.externd_transpose_trits.restype = c_int
+    L.externd_matvec.argtypes = [vp, vp, vp, i64, i64, i64, vp, i64, vp, vp, vp]
+    L.externd_matvec.restype = c_int
+    L.externd_pack_mask_sign.argtypes = [vp, i64, i64, vp, vp, i64, vp, vp]
+    L.externd_pack_mask_sign.restype = c_int
     _lib = L
     return L

@@ -294,3 +294,55 @@ def pack_trits(t: np.ndarray) -> np.ndarray:
     codes[..., :length][t == -1] = 3
     codes = codes.reshape(*t.shape[:-1], nb, 4)
     return (codes[..., 0] | (codes[..., 1] << 2) | (codes[..., 2] << 4) | (codes[..., 3] << 6)).astype(np.uint8)
+
+
+# ---------------------------------------------------------------------------
+# inference with the factors and mask+sign storage (§2.6)
+# ---------------------------------------------------------------------------
+
+def transpose_trits(T: torch.Tensor, rows: int, length: int, *, stream=None) -> torch.Tensor:
+    """(rows x length) packed trits -> (length x rows) packed trits, on T's device."""
+    out = torch.empty((length, trit_bytes(rows)), dtype=torch.uint8, device=T.device)
+    with _on_device(T):
+        rc = _lib.load().externd_transpose_trits(_ptr(T), int(rows), int(length), _ptr(out), _stream(stream, T.device))
+    _check(rc, "externd_transpose_trits")
+    return out
+
+
+def inference_layout(f: "Factors") -> torch.Tensor:
+    """B laid out for inference: m rows x trit_bytes(k), row r = B[r, 0..k)."""
+    return transpose_trits(f.B, f.k, f.m)
+
+
+def matvec(Bt: torch.Tensor, D: torch.Tensor, C: torch.Tensor, m: int, n: int, X: torch.Tensor, *,
+           out: Optional[torch.Tensor] = None, z_work: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Y = B diag(D) C X for X of shape (batch, n) or (n,), fp32 on the GPU (externd_matvec)."""
+    k = D.shape[0]
+    squeeze = X.dim() == 1
+    X2 = X.reshape(1, -1) if squeeze else X
+    if X2.dtype != torch.float32 or not X2.is_cuda:
+        raise ValueError("X must be a float32 CUDA tensor")
+    X2 = X2.contiguous()
+    batch = X2.shape[0]
+    Y = out if out is not None else torch.empty((batch, m), dtype=torch.float32, device=X2.device)
+    Z = z_work if z_work is not None else torch.empty((min(batch, 8), k), dtype=torch.float32, device=X2.device)
+    with _on_device(X2):
+        rc = _lib.load().externd_matvec(_ptr(Bt), _ptr(D), _ptr(C), int(m), int(n), int(k), _ptr(X2), int(batch),
+                                        _ptr(Y), _ptr(Z), _stream(stream, X2.device))
+    _check(rc, "externd_matvec")
+    return Y.reshape(-1) if squeeze else Y
+
+
+def pack_mask_sign(T: torch.Tensor, rows: int, length: int, *, stream=None):
+    """Mask+sign storage of packed trit rows: (mask bytes rows x ceil(length/8),
+    sign bit stream as int32 words, bit offsets per row (rows + 1))."""
+    mask = torch.empty((rows, (length + 7) // 8), dtype=torch.uint8, device=T.device)
+    words = max(1, (rows * length + 31) // 32)
+    signs = torch.empty((words,), dtype=torch.int32, device=T.device)
+    offs = torch.empty((rows + 1,), dtype=torch.int64, device=T.device)
+    with _on_device(T):
+        rc = _lib.load().externd_pack_mask_sign(_ptr(T), int(rows), int(length), _ptr(mask), _ptr(signs), int(words),
+                                                _ptr(offs), _stream(stream, T.device))
+    _check(rc, "externd_pack_mask_sign")
+    total = int(offs[-1].item())
+    return mask, signs[: (total + 31) // 32], offs

@@ -11,7 +11,7 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SOURCES = [os.path.join(HERE, "csrc", "externd.cu")]
+SOURCES = [os.path.join(HERE, "csrc", "externd.cu"), os.path.join(HERE, "csrc", "infer.cu")]
 DEPS = SOURCES + [os.path.join(HERE, "csrc", "externd_kernels.cuh"), os.path.join(ROOT, "include", "externd.h")]
 OUT = os.path.join(HERE, "libexternd.so")
 

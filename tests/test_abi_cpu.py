@@ -84,3 +84,18 @@ def test_argument_validation_before_any_device_work():
     assert L.externd_debug_halfstep(None, 1, 1, 1, None, 0.7, None, None, None, None) == einval
     assert L.externd_factor_batched(0, None, None, None, None, None, 15, None, None, None, None, None, None,
                                     None) == einval
+
+
+def test_inference_entry_points_reject_bad_arguments_before_device_work():
+    L = _lib.load()
+    einval = ext.STATUS["EINVAL"]
+    host = (ctypes.c_uint8 * 64)()
+    p = ctypes.addressof(host)
+    assert L.externd_transpose_trits(None, 1, 1, p, None) == einval
+    assert L.externd_transpose_trits(p, 0, 1, p, None) == einval
+    assert L.externd_transpose_trits(p, 4, 4, p, None) == einval          # host memory is refused
+    assert L.externd_matvec(None, p, p, 1, 1, 1, p, 1, p, p, None) == einval
+    assert L.externd_matvec(p, p, p, 1, 1, 1, p, 0, p, p, None) == einval   # batch < 1
+    assert L.externd_matvec(p, p, p, 2, 2, 2, p, 1, p, p, None) == einval   # host memory is refused
+    assert L.externd_pack_mask_sign(p, 1, 1, p, p, 0, p, None) == einval    # no room for signs
+    assert L.externd_pack_mask_sign(None, 1, 1, p, p, 1, p, None) == einval
