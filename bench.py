@@ -334,6 +334,82 @@ def run_ours(args):
     return 0
 
 
+# ---------------------------------------------------------------------------
+# Inference with the factors (§2.6): y = B diag(D) C x on the headline's factors
+# ---------------------------------------------------------------------------
+
+def run_matvec(args):
+    """Time externd_matvec on the factors of the workload's matrix 0 (factorization untimed).
+
+    Between timed calls a 256 MiB buffer is overwritten (L2 is 126 MB), so every call
+    streams the packed factors from HBM; each call is timed alone with CUDA events."""
+    import torch
+    import ternary_rank_weight_b200 as ext
+    from ternary_rank_weight_b200 import dist
+
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w, mats = _workload_arrays(args.workload, rank, args.mu)
+    f = ext.factor(torch.from_numpy(mats[0]).to(dev), w.mu[0], w.tau[0], iters=w.iters, seed=w.seeds[0])
+    Bt = ext.inference_layout(f)
+    batch = args.batch
+    X = torch.randn((batch, f.n), device=dev, dtype=torch.float32, generator=torch.Generator(device=dev).manual_seed(7))
+    Y = torch.empty((batch, f.m), device=dev, dtype=torch.float32)
+    Z = torch.empty((min(batch, 8), f.k), device=dev, dtype=torch.float32)
+    # 1 GiB overwritten before every call: longer on the device (~160 us) than the host
+    # needs to enqueue the next call, so the events bracket device work only
+    flush = torch.empty(1024 * 1024 * 1024 // 4, device=dev, dtype=torch.float32)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        ext.matvec(Bt, f.D, f.C, f.m, f.n, X, out=Y, z_work=Z)
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(dev.index) as clk:
+        for e0, e1 in ev:
+            flush.fill_(1.0)
+            e0.record(stream)
+            ext.matvec(Bt, f.D, f.C, f.m, f.n, X, out=Y, z_work=Z)
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+    times = [e0.elapsed_time(e1) for e0, e1 in ev]
+    dist.barrier(dev)
+    t_ms = dist.max_over_ranks(statistics.median(times), dev)
+    factor_bytes = Bt.numel() + f.C.numel() + 4 * f.k
+    vec_bytes = 4 * batch * (f.n + f.m) + 2 * 4 * min(batch, 8) * f.k * ((batch + 7) // 8)
+    alg = factor_bytes + vec_bytes
+    peak, peak_kind = _peaks()
+    achieved = alg / (t_ms / 1000.0) / 1e9
+    # the dense fp16 weight the factors replace, for context: m n 2 bytes at the same peak
+    dense_us = 2.0 * f.m * f.n / (peak * 1e9) * 1e6
+    out = {"op": "matvec", "metric": "factored ternary matvec y = B diag(D) C x (2-bit trits)",
+           "value": 1000.0 / t_ms * dist.sum_over_ranks(1, dev), "unit": "matvec/s", "n_gpus": ws,
+           "steps": args.steps, "warmup": args.warmup, "us_per_call": t_ms * 1000.0, "higher_is_better": True,
+           "dtype": "f32", "data": "synthetic",
+           "config": {"workload": w.name, "m": f.m, "n": f.n, "k": f.k, "batch": batch,
+                      "l2": "1 GiB buffer overwritten before every timed call"},
+           "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                        "bytes_per_call": alg, "factor_bytes": factor_bytes, "peak_kind": f"{peak_kind} copy bandwidth"},
+           "dense_fp16_floor_us": dense_us, "gpu_launches_per_call": 2 * ((batch + 7) // 8),
+           "clocks": clk.summary()}
+    if rank == 0 and not args.no_cpu_baseline:
+        from oracle import externd_oracle as ora
+        Bh, Ch = f.trits()
+        Dh = f.D.cpu().numpy().astype(np.float64)
+        Xh = X.cpu().numpy().astype(np.float64).T
+        t0 = time.perf_counter()
+        reps = 0
+        while time.perf_counter() - t0 < 5.0:
+            ora.factored_matvec(Bh, Dh, Ch, Xh)
+            reps += 1
+        dt = (time.perf_counter() - t0) / reps
+        out["cpu_baseline"] = {"value": 1.0 / dt, "unit": "matvec/s", "cores": _oracle_threads(), "kind": "oracle",
+                               "sample": f"{reps} calls of numpy fp64 B (D (C X)) on dense int8 trits, batch {batch}"}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    return 0
+
+
 def main():
     from ternary_rank_weight_b200.workloads import HEADLINE, WORKLOADS
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
@@ -348,10 +424,15 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of oracle work per sample")
     ap.add_argument("--mu", type=float, default=None, help="override mu (short runs for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", choices=("factor", "matvec"), default="factor",
+                    help="factor: the factorization (default); matvec: inference with the factors")
+    ap.add_argument("--batch", type=int, default=1, help="input vectors per matvec call (--op matvec)")
     args = ap.parse_args()
     args.ref_budget = min(args.ref_budget, 150.0 / max(args.steps, 1))
     if args.impl == "reference":
         return run_reference(args)
+    if args.op == "matvec":
+        return run_matvec(args)
     if args.all:
         for name in WORKLOADS:
             args.workload = name

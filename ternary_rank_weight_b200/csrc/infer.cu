@@ -11,9 +11,11 @@
 // dots of 2-bit trit rows with a dense fp32 vector:
 //     z_i = D_i * sum_j C[i, j] x_j        (k rows of n trits)
 //     y_r = sum_i B[r, i] z_i              (m rows of k trits)
-// One warp per row; each lane takes 16-byte chunks of the row (64 trits),
-// turns each 32-bit word into nonzero/negative masks and adds the selected
-// entries of the vector (which stays in L1: a few tens of KB).
+// One warp per row.  When the vectors fit in shared memory (NB * len * 4 bytes
+// up to ~200 KB) they are staged there and every trit is one fused multiply-add
+// with its code read as a signed 2-bit integer (rowdot_smem_kernel); otherwise each lane walks
+// the nonzero trits of its 16-byte chunks and reads the vector through L1
+// (rowdot_kernel).
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -84,6 +86,132 @@ __global__ void __launch_bounds__(RD_THREADS) rowdot_kernel(const uint8_t* __res
             const float sc = scale ? __ldg(scale + r) : 1.f;
             #pragma unroll
             for (int b = 0; b < NB; ++b) out[b * ostride + r] = sc * acc[b];
+        }
+    }
+}
+
+// Shared-memory variant: the NB vectors (NB * len fp32) are staged in shared
+// memory.  Each nibble of a trit row (two trits) indexes a 16-entry table of
+// coefficient pairs in {-1, 0, 1} (a 2-bit code read as a signed 2-bit integer is
+// the trit); the table is exactly 128 bytes, so lanes that read the same entry
+// share one access and different entries sit in different banks.  Each trit is
+// then one fused multiply-add per vector, with no divergence.  A warp
+// takes R rows at once: lane l reads the 32-bit words l, l + 32, ... of each (16
+// trits per word, up to G words per row issued before any is used), and every
+// vector value it loads from shared memory serves the R rows.  The staged vector
+// is swizzled: the four 16-byte groups of word w are rotated by (w / 2) % 4, so
+// the eight lanes of a quarter-warp (eight consecutive words) read distinct banks.
+constexpr int RS_THREADS = 128;   // shared-memory row-dot block: 4 warps; several blocks per SM
+
+__device__ __forceinline__ int64_t swz(int64_t j) {    // position of vector entry j in shared memory
+    const int64_t w = j >> 4;
+    const int h = (int)((j >> 2) & 3);
+    return 16 * w + 4 * ((h + (int)(w >> 1)) & 3) + (j & 3);
+}
+
+template <int NB, int R>
+__global__ void __launch_bounds__(RS_THREADS) rowdot_smem_kernel(const uint8_t* __restrict__ T, int64_t rows,
+                                                               int64_t len, int64_t tb, const float* __restrict__ V,
+                                                               int64_t vstride, const float* __restrict__ scale,
+                                                               float* __restrict__ out, int64_t ostride) {
+    extern __shared__ __align__(128) float smem_rd[];
+    float2* lut2 = reinterpret_cast<float2*>(smem_rd);     // 16 entries, 128 bytes: a nibble -> 2 trits
+    float* sv = smem_rd + 32;                               // NB x lenp, lenp = 16 * words, swizzled
+    const int64_t words = tb / 4;
+    const int64_t lenp = words * 16;
+    if (threadIdx.x < 16) {
+        const int v = threadIdx.x;
+        lut2[v] = make_float2((float)((v << 30) >> 30), (float)(((v >> 2) << 30) >> 30));
+    }
+    const bool vec4 = ((len & 3) == 0) && ((vstride & 3) == 0) && ((reinterpret_cast<uintptr_t>(V) & 15) == 0);
+    for (int b = 0; b < NB; ++b) {
+        if (vec4) {   // 16-byte groups copied asynchronously (all in flight at once); the swizzle moves whole groups
+            const float4* V4 = reinterpret_cast<const float4*>(V + b * vstride);
+            for (int64_t g = threadIdx.x; g < lenp / 4; g += RS_THREADS) {
+                float* dst = sv + b * lenp + swz(4 * g);
+                if (4 * g < len) {
+                    const unsigned saddr = (unsigned)__cvta_generic_to_shared(dst);
+                    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr), "l"(V4 + g) : "memory");
+                } else {
+                    *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+        } else {
+            for (int64_t j = threadIdx.x; j < lenp; j += RS_THREADS)
+                sv[b * lenp + swz(j)] = j < len ? __ldg(V + b * vstride + j) : 0.f;
+        }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int64_t groups = (rows + R - 1) / R;
+    const int64_t warps = (int64_t)gridDim.x * (RS_THREADS / 32);
+    constexpr int G = (R >= 4) ? 4 : 8;                     // words per row and lane issued together
+    for (int64_t grp = (int64_t)blockIdx.x * (RS_THREADS / 32) + (threadIdx.x >> 5); grp < groups; grp += warps) {
+        const int64_t r0 = grp * R;
+        float acc[R][NB];
+        #pragma unroll
+        for (int rr = 0; rr < R; ++rr)
+            #pragma unroll
+            for (int b = 0; b < NB; ++b) acc[rr][b] = 0.f;
+        for (int64_t w0 = 0; w0 < words; w0 += 32 * G) {
+            uint32_t q[R][G];
+            #pragma unroll
+            for (int rr = 0; rr < R; ++rr) {
+                const uint32_t* row = reinterpret_cast<const uint32_t*>(T + (r0 + rr) * tb);
+                #pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const int64_t w = w0 + lane + 32 * g;
+                    q[rr][g] = (r0 + rr < rows && w < words) ? __ldg(row + w) : 0u;
+                }
+            }
+            #pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const int64_t w = w0 + lane + 32 * g;
+                if (w >= words) break;
+                const int rot = (int)(w >> 1);
+                #pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const int64_t at = 16 * w + 4 * ((h + rot) & 3);
+                    float x[NB][4];
+                    #pragma unroll
+                    for (int b = 0; b < NB; ++b) {
+                        const float4 t4 = *reinterpret_cast<const float4*>(sv + b * lenp + at);
+                        x[b][0] = t4.x; x[b][1] = t4.y; x[b][2] = t4.z; x[b][3] = t4.w;
+                    }
+                    #pragma unroll
+                    for (int rr = 0; rr < R; ++rr) {
+                        const uint32_t byte = (q[rr][g] >> (8 * h)) & 0xFFu;   // trits 4h .. 4h+3
+                        const float2 c01 = lut2[byte & 15u];
+                        const float2 c23 = lut2[byte >> 4];
+                        #pragma unroll
+                        for (int b = 0; b < NB; ++b) {
+                            acc[rr][b] = fmaf(c01.x, x[b][0], acc[rr][b]);
+                            acc[rr][b] = fmaf(c01.y, x[b][1], acc[rr][b]);
+                            acc[rr][b] = fmaf(c23.x, x[b][2], acc[rr][b]);
+                            acc[rr][b] = fmaf(c23.y, x[b][3], acc[rr][b]);
+                        }
+                    }
+                }
+            }
+        }
+        #pragma unroll
+        for (int rr = 0; rr < R; ++rr)
+            #pragma unroll
+            for (int b = 0; b < NB; ++b) {
+                float a = acc[rr][b];
+                #pragma unroll
+                for (int o = 16; o; o >>= 1) a += __shfl_xor_sync(FULL, a, o);
+                acc[rr][b] = a;
+            }
+        if (lane == 0) {
+            #pragma unroll
+            for (int rr = 0; rr < R; ++rr) {
+                if (r0 + rr >= rows) break;
+                const float sc = scale ? __ldg(scale + r0 + rr) : 1.f;
+                #pragma unroll
+                for (int b = 0; b < NB; ++b) out[b * ostride + r0 + rr] = sc * acc[rr][b];
+            }
         }
     }
 }
@@ -211,11 +339,40 @@ int sms() {
     return v;
 }
 
+constexpr size_t SMEM_CAP = 200 * 1024;   // shared memory for the staged vectors + table
+
+size_t rowdot_smem_bytes(int nb, int64_t tb) { return (32 + (size_t)nb * (size_t)(tb / 4) * 16) * sizeof(float); }
+
+template <int NB, int R>
+bool launch_rowdot_smem(const uint8_t* T, int64_t rows, int64_t len, int64_t tb, const float* V, int64_t vstride,
+                        const float* scale, float* out, int64_t ostride, cudaStream_t s) {
+    const size_t smem = rowdot_smem_bytes(NB, tb);
+    if (smem > SMEM_CAP) return false;
+    static bool attr = false;   // per process; the attribute applies to every device
+    if (!attr) {
+        cudaFuncSetAttribute(rowdot_smem_kernel<NB, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_CAP);
+        attr = true;
+    }
+    const int64_t want = ((rows + R - 1) / R + RS_THREADS / 32 - 1) / (RS_THREADS / 32);
+    const int64_t cap = 16 * (int64_t)sms();
+    const unsigned grid = (unsigned)(want < cap ? (want > 0 ? want : 1) : cap);
+    rowdot_smem_kernel<NB, R><<<grid, RS_THREADS, smem, s>>>(T, rows, len, tb, V, vstride, scale, out, ostride);
+    return true;
+}
+
 template <int NB>
 void launch_rowdot(const uint8_t* T, int64_t rows, int64_t len, int64_t tb, const float* V, int64_t vstride,
                    const float* scale, float* out, int64_t ostride, cudaStream_t s) {
+    // rows per warp: share each staged vector load among R rows, but keep >= 16
+    // warps per SM busy (R = 1 for short matrices)
+    const int64_t nsm = sms();
+    bool done;
+    if (NB == 1 && rows >= 4 * 24 * nsm) done = launch_rowdot_smem<NB, NB == 1 ? 4 : 1>(T, rows, len, tb, V, vstride, scale, out, ostride, s);
+    else if (NB <= 2 && rows >= 2 * 16 * nsm) done = launch_rowdot_smem<NB, NB <= 2 ? 2 : 1>(T, rows, len, tb, V, vstride, scale, out, ostride, s);
+    else done = launch_rowdot_smem<NB, 1>(T, rows, len, tb, V, vstride, scale, out, ostride, s);
+    if (done) return;
     const int64_t want = (rows + 7) / 8;
-    const int64_t cap = (int64_t)sms() * 8;
+    const int64_t cap = nsm * 8;
     const unsigned grid = (unsigned)(want < cap ? (want > 0 ? want : 1) : cap);
     rowdot_kernel<NB><<<grid, RD_THREADS, 0, s>>>(T, rows, len, tb, V, vstride, scale, out, ostride);
 }
@@ -258,8 +415,11 @@ int externd_matvec(const uint8_t* Bt, const float* D, const uint8_t* C, int64_t 
         return EXTERND_EINVAL;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int64_t cb = (int64_t)trit_bytes(n), bb = (int64_t)trit_bytes(k);
-    for (int64_t b0 = 0; b0 < batch; b0 += MAXB) {
-        const int nb = (int)(batch - b0 < MAXB ? batch - b0 : MAXB);
+    // vectors per pass: the most that still fit shared memory for both products
+    int per = MAXB;
+    while (per > 1 && (rowdot_smem_bytes(per, cb) > SMEM_CAP || rowdot_smem_bytes(per, bb) > SMEM_CAP)) per /= 2;
+    for (int64_t b0 = 0; b0 < batch; b0 += per) {
+        const int nb = (int)(batch - b0 < per ? batch - b0 : per);
         // z = diag(D) (C x): k rows of n trits
         rowdot(nb, C, k, n, cb, X + b0 * n, n, D, z_work, k, s);
         // y = B z: m rows of k trits (B transposed)
