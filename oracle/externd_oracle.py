@@ -16,6 +16,9 @@ arXiv 2607.13511), cited below by section and display equation:
 * §2.3 steps 1-3: R <- A; for each component: 15 alternating fits
   v <- T_tau(R^T u), u <- T_tau(R v); scale d = u^T R v / (||u||^2 ||v||^2);
   deflate R <- R - d u v^T; store B[:, i] = u, C[i, :] = v^T.
+* §2.5: importance-weighted ALS minimizes sum_ij h~_j (A - Ahat)^2_ij with
+  h~ = h / max(h) + lambda; the U-step targets W = R diag(h~), the V-step the plain
+  residual R (h~ cancels there), the scale solves the weighted normal equation.
 * §2.6 Cost model: inference computes y = B (diag(D) (C x)); mask+sign packing
   stores one zero/nonzero mask bit per element plus one sign bit per nonzero,
   and Eq. (1): bpw_eff = mu (m + n) / max(m, n) * (2 - sparsity).
@@ -358,3 +361,80 @@ def mask_sign_unpack(mask: np.ndarray, signs: np.ndarray, length: int) -> np.nda
 def mask_sign_bits(B: np.ndarray, C: np.ndarray) -> int:
     """Storage of the factors in mask+sign form: one mask bit per element, one sign bit per nonzero."""
     return int(B.size + C.size + np.count_nonzero(B) + np.count_nonzero(C))
+
+
+# ----------------------------------------------------------------------------
+# §2.5 importance-weighted ALS (sequential, one component at a time)
+# ----------------------------------------------------------------------------
+
+
+def normalized_weights(h: np.ndarray, lam: float) -> np.ndarray:
+    """h~ = h / max(h) + lambda (§2.5), computed in fp64 and held in fp32 like the GPU path
+    (reading: the weights are stored once per matrix in single precision)."""
+    h = np.asarray(h, dtype=np.float64)
+    return (h / np.max(h) + lam).astype(np.float32)
+
+
+def weighted_energy(A: np.ndarray, Ahat: np.ndarray, hw: np.ndarray) -> float:
+    """1 - sum_ij h~_j (A - Ahat)^2_ij / sum_ij h~_j A^2_ij."""
+    A = np.asarray(A, dtype=np.float64)
+    w = np.asarray(hw, dtype=np.float64)[None, :]
+    diff = A - np.asarray(Ahat, dtype=np.float64)
+    return 1.0 - float(np.sum(w * diff * diff)) / float(np.sum(w * A * A))
+
+
+def weighted_ls_scale(R: np.ndarray, u: np.ndarray, v: np.ndarray, hw: np.ndarray) -> float:
+    """argmin_d sum_ij h~_j (R - d u v^T)^2_ij = u^T R (h~ v) / (||u||^2 sum_j h~_j v_j^2)."""
+    u = np.asarray(u, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    w = np.asarray(hw, dtype=np.float64)
+    p = float(u @ (np.asarray(R, dtype=np.float64) @ (w * v)))
+    if p == 0.0:
+        return 0.0
+    return p / (float(u @ u) * float(w @ (v * v)))
+
+
+def greedy_als_weighted(A: np.ndarray, h: np.ndarray, lam: float, k: int, tau: float, iters: int = 15,
+                        seed: int = 0) -> Factorization:
+    """§2.5 with §2.3: V-step on the plain residual (h~ cancels there), U-step on
+    W = R diag(h~), scale from the weighted normal equation, plain deflation.  The
+    energy is the weighted one; the start vectors are those of greedy_als."""
+    hw = normalized_weights(h, lam).astype(np.float64)
+    R = np.array(A, dtype=np.float64, copy=True)
+    m, n = R.shape
+    norm_w = float(np.sum(hw[None, :] * R * R))
+    if norm_w == 0.0:
+        raise ValueError("weighted ||A|| = 0: energy is undefined")
+    B = np.zeros((m, k), dtype=np.int8)
+    C = np.zeros((k, n), dtype=np.int8)
+    D = np.zeros(k, dtype=np.float64)
+    energy = np.zeros(k, dtype=np.float64)
+    margins = np.zeros(k, dtype=np.float64)
+    r2 = norm_w
+    for i in range(k):
+        u, _, _ = ternarize(start_normals(seed, i, m), tau)
+        margin = math.inf
+        y = None
+        v = None
+        for _ in range(iters):
+            x = R.T @ u.astype(np.float64)                    # V-step on R
+            v, tv, _ = ternarize(x, tau)
+            margin = min(margin, relative_margin(x, tv))
+            y = R @ (hw * v.astype(np.float64))               # U-step on W = R diag(h~)
+            u, tu, _ = ternarize(y, tau)
+            margin = min(margin, relative_margin(y, tu))
+        p = float(u.astype(np.float64) @ y)                  # u^T R (h~ v)
+        nu = int(np.count_nonzero(u))
+        sv = float(np.sum(hw[v != 0]))                        # v^T diag(h~) v for ternary v
+        d = 0.0 if p == 0.0 else p / (nu * sv)
+        if d != 0.0:
+            R -= d * np.outer(u.astype(np.float64), v.astype(np.float64))
+        r2 -= (p * p) / (nu * sv)
+        B[:, i] = u
+        C[i, :] = v
+        D[i] = d
+        energy[i] = 1.0 - r2 / norm_w
+        margins[i] = margin
+    e_final = 1.0 - float(np.sum(hw[None, :] * R * R)) / norm_w
+    return Factorization(B=B, C=C, D=D, energy=energy, energy_final=e_final, norm_a2=norm_w,
+                         margins=margins, safeguard_hits=0, residual_norms=None)

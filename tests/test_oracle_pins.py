@@ -345,3 +345,71 @@ def test_mask_sign_storage_matches_eq1():
         f = ora.greedy_als(A, k=k, tau=tau, seed=1)
         bits = ora.mask_sign_bits(f.B, f.C)
         assert bits / (m * n) == pytest.approx(ora.bpw_eff(mu, m, n, f.zero_fraction()), rel=1e-12)
+
+
+# --------------------------------------------------------------------------
+# §2.5 importance-weighted ALS
+# --------------------------------------------------------------------------
+
+def test_weighted_with_uniform_weights_is_the_plain_algorithm():
+    """h constant and lambda = 0 give h~ = 1: the weighted objective is the Frobenius one."""
+    A = np.random.default_rng(41).standard_normal((40, 64)).astype(np.float32) * 0.02
+    k = ora.rank(40, 64, 1.5)
+    f = ora.greedy_als(A, k=k, tau=1.0, seed=3)
+    fw = ora.greedy_als_weighted(A, np.full(64, 2.5), 0.0, k=k, tau=1.0, seed=3)
+    assert np.array_equal(f.B, fw.B) and np.array_equal(f.C, fw.C)
+    assert np.allclose(f.D, fw.D, rtol=1e-13, atol=0)
+    assert np.allclose(f.energy, fw.energy, rtol=0, atol=1e-12)
+
+
+def test_weighted_scale_is_the_weighted_least_squares_minimizer():
+    rng = np.random.default_rng(43)
+    for _ in range(20):
+        m, n = rng.integers(2, 9, size=2)
+        R = rng.standard_normal((m, n))
+        w = rng.uniform(0.05, 2.0, size=n)
+        u = rng.integers(-1, 2, size=m); v = rng.integers(-1, 2, size=n)
+        if not u.any() or not v.any():
+            continue
+        uf, vf = _tf(u), _tf(v)
+        f = lambda d: float(np.sum(w[None, :] * (R - d * np.outer(uf, vf)) ** 2))
+        grid = np.linspace(-6, 6, 24001)
+        vals = np.array([f(d) for d in grid])
+        j = int(np.argmin(vals))
+        d0, d1, d2 = grid[j - 1:j + 2]
+        f0, f1, f2 = vals[j - 1:j + 2]
+        vertex = d1 - 0.5 * ((d1 - d0) ** 2 * (f1 - f2) - (d1 - d2) ** 2 * (f1 - f0)) / \
+            ((d1 - d0) * (f1 - f2) - (d1 - d2) * (f1 - f0))
+        d = ora.weighted_ls_scale(R, u, v, w)
+        assert d == pytest.approx(vertex, rel=1e-8, abs=1e-10)
+        p = uf @ R @ (w * vf)
+        assert f(0.0) - f(d) == pytest.approx(p * p / (np.count_nonzero(u) * np.sum(w[v != 0])), rel=1e-10, abs=1e-12)
+
+
+def test_weights_cancel_in_the_v_step():
+    """§2.5: for a fixed u the column-weighted least-squares v is (R^T u)_j / ||u||^2 whatever h~ is."""
+    rng = np.random.default_rng(44)
+    R = rng.standard_normal((6, 5))
+    u = np.array([1, 0, -1, 1, 1, 0], dtype=np.float64)
+    for w in (np.ones(5), rng.uniform(0.1, 3.0, size=5)):
+        # minimize sum_j w_j sum_i (R_ij - u_i v_j)^2 column by column on a fine grid
+        for j in range(5):
+            grid = np.linspace(-5, 5, 200001)
+            cost = w[j] * np.sum((R[:, j][None, :] - grid[:, None] * u[None, :]) ** 2, axis=1)
+            assert grid[int(np.argmin(cost))] == pytest.approx((R[:, j] @ u) / (u @ u), abs=1e-4)
+
+
+def test_weighted_residual_decreases_and_energy_matches_reconstruction():
+    rng = np.random.default_rng(45)
+    A = (rng.standard_normal((48, 80)) * 0.02).astype(np.float32)
+    h = np.exp(2.0 * rng.standard_normal(80))            # skewed per-channel second moments
+    fw = ora.greedy_als_weighted(A, h, 0.0, k=96, tau=1.0, seed=2)
+    assert np.all(np.diff(fw.energy) >= -1e-12)
+    hw = ora.normalized_weights(h, 0.0)
+    Ahat = ora.reconstruct(fw.B, fw.D, fw.C)
+    assert ora.weighted_energy(A, Ahat, hw) == pytest.approx(fw.energy_final, abs=1e-10)
+    assert fw.energy_final == pytest.approx(fw.energy[-1], abs=1e-10)
+    # weighting helps the weighted objective against the plain algorithm at the same k
+    f = ora.greedy_als(A, k=96, tau=1.0, seed=2)
+    assert ora.weighted_energy(A, ora.reconstruct(f.B, f.D, f.C), hw) < fw.energy_final
+    assert hw.max() == pytest.approx(1.0) and hw.dtype == np.float32
