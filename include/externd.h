@@ -87,6 +87,20 @@ int externd_factor(const float* A, int64_t m, int64_t n, double mu, double tau, 
                    uint64_t seed, uint8_t* B_out, float* D_out, uint8_t* C_out,
                    double* energy_out, void* stream);
 
+/* Importance-weighted factorization (§2.5): minimizes sum_ij h~_j (A - Ahat)^2_ij with
+ * h~ = h / max(h) + lambda (computed in fp64, held in fp32), by the sequential ALS of
+ * §2.3 with the V-step on the plain residual R (h~ cancels there), the U-step on
+ * W = R diag(h~) and the scale d = u^T R (h~ v) / (nnz(u) sum_{v_j != 0} h~_j).
+ *   h          [in]  n per-input-channel (per-column) second moments, fp32, finite and
+ *                    >= 0 with a positive maximum (else EXTERND_EINVAL).
+ *   lambda           >= 0, finite: lambda -> infinity approaches the plain objective.
+ *   energy_out [out] nullable; k doubles, the weighted energy
+ *                    1 - sum h~ (A - Ahat)^2 / sum h~ A^2 after each component.
+ * Other arguments, outputs and conventions are those of externd_factor. */
+int externd_factor_weighted(const float* A, int64_t m, int64_t n, double mu, double tau, int iters,
+                            uint64_t seed, const float* h, double lambda, uint8_t* B_out, float* D_out,
+                            uint8_t* C_out, double* energy_out, void* stream);
+
 /* Allocation-free variant of externd_factor.  The pages have no counterpart:
  * this entry point exists for callers that cannot allocate device memory while
  * it runs -- for example an inference or conversion service whose memory pool

@@ -17,6 +17,7 @@ EXPORTS = (
     "externd_trit_bytes",
     "externd_factor",
     "externd_factor_ex",
+    "externd_factor_weighted",
     "externd_factor_noalloc",
     "externd_factor_batched",
     "externd_reconstruct",
@@ -95,6 +96,8 @@ def load():
     L.externd_factor_ex.argtypes = [vp, i64, i64, dbl, dbl, c_int, u64, vp, vp, vp, vp, vp,
                                     ctypes.POINTER(Options)]
     L.externd_factor_ex.restype = c_int
+    L.externd_factor_weighted.argtypes = [vp, i64, i64, dbl, dbl, c_int, u64, vp, dbl, vp, vp, vp, vp, vp]
+    L.externd_factor_weighted.restype = c_int
     L.externd_factor_noalloc.argtypes = [vp, i64, i64, dbl, dbl, c_int, u64, vp, vp, vp, vp, vp]
     L.externd_factor_noalloc.restype = c_int
     L.externd_factor_batched.argtypes = [c_int, vp, vp, vp, vp, vp, c_int, vp, vp, vp, vp, vp, vp, vp]

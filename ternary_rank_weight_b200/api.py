@@ -153,6 +153,34 @@ def factor(A, mu: float, tau: float, iters: int = 15, seed: int = 0, *, grid: in
                    stats=last_stats())
 
 
+def factor_weighted(A, h, mu: float, tau: float, lam: float = 0.0, iters: int = 15, seed: int = 0, *,
+                    stream=None) -> Factors:
+    """Importance-weighted factorization (externd_factor_weighted, §2.5).
+
+    h: per-column second moments (n,), float32, on the host or the GPU.  The returned
+    energy is the weighted energy."""
+    A = _as_matrix(A)
+    m, n = A.shape
+    if isinstance(h, np.ndarray):
+        h = torch.from_numpy(np.ascontiguousarray(h, dtype=np.float32))
+    if not isinstance(h, torch.Tensor) or h.dtype != torch.float32 or h.numel() != n:
+        raise ValueError("h must hold n float32 values")
+    h = h.contiguous()
+    k = rank(m, n, mu)
+    if k < 1:
+        raise ExterndError(STATUS["EINVAL"], "externd_rank")
+    B = _empty((k, trit_bytes(m)), torch.uint8, A)
+    C = _empty((k, trit_bytes(n)), torch.uint8, A)
+    D = _empty((k,), torch.float32, A)
+    E = _empty((k,), torch.float64, A)
+    with _on_device(A):
+        rc = _lib.load().externd_factor_weighted(_ptr(A), m, n, float(mu), float(tau), int(iters), int(seed), _ptr(h),
+                                                 float(lam), _ptr(B), _ptr(D), _ptr(C), _ptr(E),
+                                                 _stream(stream, A.device))
+    _check(rc, "externd_factor_weighted")
+    return Factors(B=B, D=D, C=C, energy=E, m=m, n=n, k=k, mu=float(mu), tau=float(tau), stats=last_stats())
+
+
 def factor_noalloc(A: torch.Tensor, mu: float, tau: float, iters: int = 15, seed: int = 0, *, out=None,
                    stream=None) -> Factors:
     """externd_factor_noalloc: the same factorization with no device allocation inside the call.

@@ -40,7 +40,7 @@ __global__ void __launch_bounds__(256) setup_kernel(const Prob* __restrict__ pro
         if (r < m && c < n) {
             v = __ldcg(P.A + r * n + c);
             if (!isfinite(v)) ++bad;
-            ss += (double)v * (double)v;
+            ss += (double)v * (double)v * (P.hw ? (double)__ldg(P.hw + c) : 1.0);
             const int q = P.pv.owner(c);
             P.Rv[P.pv.block_offset(q, m) + r * P.pv.pitch(q) + (c - P.pv.start(q))] = v;
         }
@@ -65,6 +65,40 @@ __global__ void __launch_bounds__(256) setup_kernel(const Prob* __restrict__ pro
         P.norm_part[blockIdx.y * tiles_x + blockIdx.x] = s;
     }
     if (bad) atomicAdd(P.nonfinite, bad);
+}
+
+// ---------------------------------------------------------------------------
+// Importance weights of §2.5: h~_j = h_j / max(h) + lambda, computed in fp64 and
+// held in fp32.  h must be finite and non-negative with a positive maximum; a
+// violation raises *bad (the factorization then reports EXTERND_EINVAL).
+// ---------------------------------------------------------------------------
+
+__global__ void __launch_bounds__(1024) weights_kernel(const float* __restrict__ h, int64_t n, double lambda,
+                                                       float* __restrict__ hw, unsigned* bad) {
+    __shared__ float smax[32];
+    __shared__ int sbad[32];
+    float mx = 0.f;
+    int b = 0;
+    for (int64_t j = threadIdx.x; j < n; j += 1024) {
+        const float v = h[j];
+        if (!(v >= 0.f) || !isfinite(v)) b = 1;
+        else mx = fmaxf(mx, v);
+    }
+    #pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
+        b |= __shfl_xor_sync(FULL, b, o);
+    }
+    if ((threadIdx.x & 31) == 0) { smax[threadIdx.x >> 5] = mx; sbad[threadIdx.x >> 5] = b; }
+    __syncthreads();
+    float M = 0.f;
+    int B = 0;
+    for (int w = 0; w < 32; ++w) { M = fmaxf(M, smax[w]); B |= sbad[w]; }
+    if (B || !(M > 0.f) || !isfinite(lambda) || lambda < 0.0) {
+        if (threadIdx.x == 0) *bad = 1u;
+        return;
+    }
+    for (int64_t j = threadIdx.x; j < n; j += 1024) hw[j] = (float)((double)h[j] / (double)M + lambda);
 }
 
 // ---------------------------------------------------------------------------
@@ -140,8 +174,8 @@ __global__ void __launch_bounds__(NTI) init_kernel(const Prob* __restrict__ prob
 // Shared-memory carve of the ALS kernel (host and device use the same layout).
 struct SmemLayout {
     size_t red, pd, coef, coefV, dotU, dotV, scal, wS, wM, wp, gS, gM, wJ, gJ, wc, dotp, sflag, clk, nzU, sgU, nzV, sgV, pnzU, psgU, pnzV,
-        psgV, cnzV, csgV, cnzU, csgU, ulist, vlist, wd, onzU, osgU, onzV, osgV, gV, gU, corr, total;
-    __host__ __device__ SmemLayout(int64_t m_max, int64_t n_max, int Lc, int pv_max, int pu_max) {
+        psgV, cnzV, csgV, cnzU, csgU, ulist, vlist, vwl, wd, onzU, osgU, onzV, osgV, dotVw, dotpw, gV, gU, corr, total;
+    __host__ __device__ SmemLayout(int64_t m_max, int64_t n_max, int Lc, int pv_max, int pu_max, int weighted) {
         const size_t Wm = (size_t)((m_max + 31) / 32), Wn = (size_t)((n_max + 31) / 32);
         size_t o = 0;
         red = o;  o += 8 * (size_t)NT * 5;   // lanes * (pitch + 1) <= NT * (VEC + 1)
@@ -177,12 +211,15 @@ struct SmemLayout {
         csgU = o; o += 4 * (size_t)pu_max;
         ulist = o; o += 4 * (size_t)m_max;
         vlist = o; o += 4 * (size_t)n_max;
+        vwl = o;  o += weighted ? 4 * (size_t)n_max : 0;   // weighted list coefficients of the U-step
         wd = o;   o += 4 * NWARP;
         onzU = o; o += 4 * Wm;
         osgU = o; o += 4 * Wm;
         onzV = o; o += 4 * Wn;
         osgV = o; o += 4 * Wn;
         o = (o + 7) & ~(size_t)7;
+        dotVw = o; o += weighted ? 8 * (size_t)MAX_PENDING : 0;
+        dotpw = o; o += weighted ? 8 * (size_t)NWARP * MAX_PENDING : 0;
         gV = o;   o += 8 * (size_t)pv_max;
         gU = o;   o += 8 * (size_t)pu_max;
         corr = o; o += 8 * (size_t)(pv_max > pu_max ? pv_max : pu_max);
@@ -201,6 +238,8 @@ struct Smem {
     uint32_t *pnzU, *psgU, *pnzV, *psgV;     // pending components (full length, stride W)
     uint32_t *cnzV, *csgV, *cnzU, *csgU;     // pending trits at this CTA's outputs, bit l = component l
     int *ulist, *vlist;                      // compacted trit changes: element offset (index * block pitch) | sign << 31 | (|delta| == 2) << 30
+    float* vwl;                              // weighted objective: coefficient of each vlist entry, delta * h~_c
+    double *dotVw, *dotpw;                   // weighted objective: sum_c h~_c t_l(c) v(c) per pending l; per-warp partials
     int* wd;                                 // per-warp count of changed trits
     uint32_t *onzU, *osgU, *onzV, *osgV;     // masks of the previous u and v of this component
     double *gV, *gU;                         // running GEMV sums R^T u, R v of this CTA's outputs (before lazy-deflation correction)
@@ -238,6 +277,12 @@ __device__ __forceinline__ void load_vec(const float* p, float* v) {
     } else {
         v[0] = __ldcg(p);
     }
+}
+
+// Coefficient of a list entry: -1/+1 from bit 31, doubled by bit 30 (a trit that
+// flipped sign); with importance weights the list carries the coefficients itself.
+__device__ __forceinline__ float entry_coef(int ent) {
+    return (ent < 0 ? -1.f : 1.f) * ((ent & 0x40000000) ? 2.f : 1.f);
 }
 
 // Lazy-deflation correction at one of this CTA's outputs: sum_l coef_l t_l(c),
@@ -282,17 +327,14 @@ __device__ __forceinline__ void emit_tagged(double v, int64_t gi, unsigned long 
 // term (|error| <= (U-1) 2^-24 sum|terms|), then converted and added to the fp64
 // accumulator: this keeps the GEMV at ~2 instructions per element.
 template <int VEC, int U>
-__device__ __forceinline__ void accumulate_batch(double* acc, const int* ent, float (*v)[VEC]) {
+__device__ __forceinline__ void accumulate_batch(double* acc, const float* cf, float (*v)[VEC]) {
     float b[VEC];
     #pragma unroll
     for (int e = 0; e < VEC; ++e) b[e] = 0.f;
     #pragma unroll
     for (int u = 0; u < U; ++u) {
-        // coefficient of the entry: -1/+1 from bit 31, doubled by bit 30 (a trit that
-        // flipped sign); inactive slots hold v = 0
-        const float sgn = (ent[u] < 0 ? -1.f : 1.f) * ((ent[u] & 0x40000000) ? 2.f : 1.f);
         #pragma unroll
-        for (int e = 0; e < VEC; ++e) b[e] = fmaf(sgn, v[u][e], b[e]);
+        for (int e = 0; e < VEC; ++e) b[e] = fmaf(cf[u], v[u][e], b[e]);   // inactive slots hold v = 0
     }
     #pragma unroll
     for (int e = 0; e < VEC; ++e) acc[e] += (double)b[e];
@@ -306,24 +348,26 @@ __host__ __device__ constexpr int GEMV_U() {
 
 // acc += sum over the list entries g, g + lanes, g + 2 lanes, ... of this thread's VEC
 // columns, U entries per batch (every batch issues all its loads before using any).
+
 template <int VEC, int U>
-__device__ __forceinline__ void gemv_rows(double* acc, const float* base, const int* __restrict__ list, int nlist,
-                                          int g, int lanes) {
+__device__ __forceinline__ void gemv_rows(double* acc, const float* base, const int* __restrict__ list,
+                                          const float* __restrict__ wl, int nlist, int g, int lanes) {
     for (int idx = g; idx < nlist; idx += U * lanes) {
-        int ent[U];
+        float cf[U];
         float v[U][VEC];
         #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int ii = idx + u * lanes;
-            ent[u] = ii < nlist ? list[ii] : 0;
+            const int ent = ii < nlist ? list[ii] : 0;
+            cf[u] = ii < nlist ? (wl ? wl[ii] : entry_coef(ent)) : 0.f;
             if (ii < nlist) {
-                load_vec<VEC>(base + (ent[u] & 0x3fffffff), v[u]);
+                load_vec<VEC>(base + (ent & 0x3fffffff), v[u]);
             } else {
                 #pragma unroll
                 for (int e = 0; e < VEC; ++e) v[u][e] = 0.f;
             }
         }
-        accumulate_batch<VEC, U>(acc, ent, v);
+        accumulate_batch<VEC, U>(acc, cf, v);
     }
 }
 
@@ -334,8 +378,9 @@ __device__ __forceinline__ void gemv_rows(double* acc, const float* base, const 
 // lazy-deflation correction is written to gout[out0 + c].  fp64 accumulation of exact fp32 terms, fixed summation order.
 template <int VEC>
 __device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, int64_t out0,
-                          const int* __restrict__ list, int nlist, double* red, unsigned long long* gout,
-                          const HalfCorr& hc, unsigned tag, bool skip, double& S, unsigned long long* clk) {
+                          const int* __restrict__ list, const float* __restrict__ wl, int nlist, double* red,
+                          unsigned long long* gout, const HalfCorr& hc, unsigned tag, bool skip, double& S,
+                          unsigned long long* clk) {
     S = 0.0;
     const int nvec = pitch / VEC;
     if (nvec <= 0) return;
@@ -354,10 +399,10 @@ __device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, i
             // batch width from the longest group (uniform over the CTA): short change
             // lists issue few predicated slots
             const int per = (nlist + lanes - 1) / lanes;
-            if (per <= 1) gemv_rows<VEC, 1>(acc, base, list, nlist, g, lanes);
-            else if (per <= 2) gemv_rows<VEC, 2>(acc, base, list, nlist, g, lanes);
-            else if (per <= 4) gemv_rows<VEC, 4>(acc, base, list, nlist, g, lanes);
-            else gemv_rows<VEC, GEMV_U<VEC>()>(acc, base, list, nlist, g, lanes);
+            if (per <= 1) gemv_rows<VEC, 1>(acc, base, list, wl, nlist, g, lanes);
+            else if (per <= 2) gemv_rows<VEC, 2>(acc, base, list, wl, nlist, g, lanes);
+            else if (per <= 4) gemv_rows<VEC, 4>(acc, base, list, wl, nlist, g, lanes);
+            else gemv_rows<VEC, GEMV_U<VEC>()>(acc, base, list, wl, nlist, g, lanes);
             #pragma unroll
             for (int e = 0; e < VEC; ++e) red[g * rs + j * VEC + e] = acc[e];
         }
@@ -388,20 +433,21 @@ __device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, i
             for (int e = 0; e < VEC; ++e) acc[e] = 0.0;
             const float* base = blk + j * VEC;
             for (int idx = 0; idx < nlist; idx += U) {
-                int ent[U];
+                float cf[U];
                 float v[U][VEC];
                 #pragma unroll
                 for (int u = 0; u < U; ++u) {
                     const int ii = idx + u;
-                    ent[u] = ii < nlist ? list[ii] : 0;
+                    const int ent = ii < nlist ? list[ii] : 0;
+                    cf[u] = ii < nlist ? (wl ? wl[ii] : entry_coef(ent)) : 0.f;
                     if (ii < nlist) {
-                        load_vec<VEC>(base + (ent[u] & 0x3fffffff), v[u]);
+                        load_vec<VEC>(base + (ent & 0x3fffffff), v[u]);
                     } else {
                         #pragma unroll
                         for (int e = 0; e < VEC; ++e) v[u][e] = 0.f;
                     }
                 }
-                accumulate_batch<VEC, U>(acc, ent, v);
+                accumulate_batch<VEC, U>(acc, cf, v);
             }
             #pragma unroll
             for (int e = 0; e < VEC; ++e) {
@@ -417,12 +463,12 @@ __device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, i
 }
 
 __device__ __forceinline__ void gemv_dispatch(int vec, const float* blk, int pitch, int valid, int64_t out0,
-                                              const int* list, int nlist, double* red, unsigned long long* gout,
-                                              const HalfCorr& hc, unsigned tag, bool skip, double& S,
-                                              unsigned long long* clk) {
-    if (vec == 4) gemv_emit<4>(blk, pitch, valid, out0, list, nlist, red, gout, hc, tag, skip, S, clk);
-    else if (vec == 2) gemv_emit<2>(blk, pitch, valid, out0, list, nlist, red, gout, hc, tag, skip, S, clk);
-    else gemv_emit<1>(blk, pitch, valid, out0, list, nlist, red, gout, hc, tag, skip, S, clk);
+                                              const int* list, const float* wl, int nlist, double* red,
+                                              unsigned long long* gout, const HalfCorr& hc, unsigned tag, bool skip,
+                                              double& S, unsigned long long* clk) {
+    if (vec == 4) gemv_emit<4>(blk, pitch, valid, out0, list, wl, nlist, red, gout, hc, tag, skip, S, clk);
+    else if (vec == 2) gemv_emit<2>(blk, pitch, valid, out0, list, wl, nlist, red, gout, hc, tag, skip, S, clk);
+    else gemv_emit<1>(blk, pitch, valid, out0, list, wl, nlist, red, gout, hc, tag, skip, S, clk);
 }
 
 // Fold the L pending components into this CTA's block:
@@ -558,6 +604,28 @@ __device__ void pending_coef(int L, int Ls, int W, const uint32_t* pnz, const ui
     __syncthreads();
 }
 
+// dotw_l = sum_c h~_c t_l(c) t(c) and coef_l = d_l dotw_l for every pending component
+// (weighted objective), fixed order: words by lane, bits in increasing order.
+__device__ void pending_coef_w(int L, int Ls, int W, const uint32_t* pnz, const uint32_t* psg, const uint32_t* nz,
+                               const uint32_t* sg, const double* pd, const float* hw, double* dotw, double* coef) {
+    for (int l = warp_id(); l < L; l += NWARP) {
+        double acc = 0.0;
+        for (int w = lane_id(); w < W; w += 32) {
+            const uint32_t both = pnz[w * Ls + l] & nz[w];
+            const uint32_t neg = psg[w * Ls + l] ^ sg[w];
+            for (uint32_t mk = both; mk; mk &= mk - 1u) {
+                const int b = __ffs(mk) - 1;
+                const double hv = (double)__ldg(hw + ((int64_t)w << 5) + b);
+                acc += ((neg >> b) & 1u) ? -hv : hv;
+            }
+        }
+        #pragma unroll
+        for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(FULL, acc, o);
+        if (lane_id() == 0) { dotw[l] = acc; coef[l] = pd[l] * acc; }
+    }
+    __syncthreads();
+}
+
 __device__ void pack_row(const uint32_t* nz, const uint32_t* sg, int W, uint32_t* out, int64_t out_words) {
     for (int64_t w = threadIdx.x; w < out_words; w += NT) {
         const int64_t mw = w >> 1;
@@ -600,7 +668,8 @@ __device__ __forceinline__ int delta_entry(unsigned idx, int rowpitch, uint32_t 
 // Block-wide: compacted list of the changes (onz, osg) -> (nz, sg) over W mask words,
 // in index order.  Returns the count.
 __device__ int build_delta_list(int W, const uint32_t* onz, const uint32_t* osg, const uint32_t* nz,
-                                const uint32_t* sg, int* list, int rowpitch, const Smem& s) {
+                                const uint32_t* sg, int* list, int rowpitch, const Smem& s,
+                                const float* hw = nullptr, float* wl = nullptr) {
     const int lane = lane_id(), warp = warp_id();
     const int wpw = (W + NWARP - 1) / NWARP;
     const int w0 = min(W, warp * wpw), w1 = min(W, w0 + wpw);
@@ -623,8 +692,12 @@ __device__ int build_delta_list(int W, const uint32_t* onz, const uint32_t* osg,
     for (int w = w0; w < w1; ++w) {
         uint32_t ng, tw;
         const uint32_t ch = delta_mask(onz[w], osg[w], nz[w], sg[w], ng, tw);
-        if ((ch >> lane) & 1u)
-            list[run + __popc(ch & ((1u << lane) - 1u))] = delta_entry(((unsigned)w << 5) + lane, rowpitch, ng, tw, lane);
+        if ((ch >> lane) & 1u) {
+            const int at = run + __popc(ch & ((1u << lane) - 1u));
+            const int e = delta_entry(((unsigned)w << 5) + lane, rowpitch, ng, tw, lane);
+            list[at] = e;
+            if (wl) wl[at] = entry_coef(e) * __ldg(hw + ((int64_t)w << 5) + lane);
+        }
         run += __popc(ch);
     }
     __syncthreads();
@@ -692,7 +765,8 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
                                   uint32_t* nz, uint32_t* sg, uint32_t* onz, uint32_t* osg, int* list, int rowpitch,
                                   const Smem& s, int L, int Ls, const uint32_t* pnz, const uint32_t* psg, int* dots,
                                   double* coef, bool want_p, double& thr_out, int& ndelta, GroupSync* gs,
-                                  uint64_t limit_ns, int* status, bool& ok_out) {
+                                  uint64_t limit_ns, int* status, bool& ok_out, const float* hw = nullptr,
+                                  float* wl = nullptr, double* dotw = nullptr, double* hsum_out = nullptr) {
     const int lane = lane_id(), warp = warp_id();
     // ---- this CTA's partial (fixed butterfly + fixed cross-warp combine)
     #pragma unroll
@@ -766,7 +840,7 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
     //      takes its words in groups of up to 32: first every ballot (registers only),
     //      then lane i handles word base + i (old masks, changes, stores) in parallel.
     int cnt = 0, dcnt = 0, dot = 0;
-    double ps = 0.0;
+    double ps = 0.0, hsum = 0.0, dotw_acc = 0.0;
     for (int base = w0; base < w1; base += 32) {
         const int K = min(32, w1 - base);
         uint32_t my_bz = 0u, my_bs = 0u;
@@ -798,7 +872,7 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
             }
         }
         const int w = base + lane;
-        uint32_t oz = 0u, os = 0u, ch = 0u, dn, dt;
+        uint32_t oz = 0u, os = 0u, ch = 0u, dn = 0u, dt = 0u;
         if (lane < K) {
             oz = nz[w];
             os = sg[w];
@@ -808,7 +882,11 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
         if (lane < K) { nz[w] = my_bz; sg[w] = my_bs; onz[w] = oz; osg[w] = os; }
         cnt += __popc(my_bz);
         dcnt += __popc(ch);
-        // change of t_l . t over the words that changed (lane l = pending component l)
+        if (hw) {   // sum of h~ over the new support (lane = word, bits in increasing order)
+            for (uint32_t mk = my_bz; mk; mk &= mk - 1u) hsum += (double)__ldg(hw + ((int64_t)w << 5) + __ffs(mk) - 1);
+        }
+        // change of t_l . t (weighted: sum h~_c t_l(c) t(c)) over the words that changed
+        // (lane l = pending component l)
         unsigned chw = __ballot_sync(FULL, ch != 0u);
         while (chw) {
             const int i = __ffs(chw) - 1;
@@ -816,11 +894,21 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
             const uint32_t zi = __shfl_sync(FULL, my_bz, i), si = __shfl_sync(FULL, my_bs, i);
             const uint32_t ozi = __shfl_sync(FULL, oz, i), osi = __shfl_sync(FULL, os, i);
             const uint32_t chi = __shfl_sync(FULL, ch, i);
+            const uint32_t dni = __shfl_sync(FULL, dn, i), dti = __shfl_sync(FULL, dt, i);
             if (lane < L) {
                 const uint32_t pz = pnz[(base + i) * Ls + lane], pg = psg[(base + i) * Ls + lane];
-                const uint32_t zn = pz & zi & chi, zo = pz & ozi & chi;
-                const uint32_t sn = pg ^ si, so = pg ^ osi;
-                dot += (__popc(zn & ~sn) - __popc(zn & sn)) - (__popc(zo & ~so) - __popc(zo & so));
+                if (hw) {
+                    for (uint32_t mk = pz & chi; mk; mk &= mk - 1u) {
+                        const int b = __ffs(mk) - 1;
+                        const double hv = (double)__ldg(hw + ((int64_t)(base + i) << 5) + b);
+                        const double dv = (((dni >> b) & 1u) ? -1.0 : 1.0) * (((dti >> b) & 1u) ? 2.0 : 1.0);
+                        dotw_acc += ((pg >> b) & 1u) ? -hv * dv : hv * dv;
+                    }
+                } else {
+                    const uint32_t zn = pz & zi & chi, zo = pz & ozi & chi;
+                    const uint32_t sn = pg ^ si, so = pg ^ osi;
+                    dot += (__popc(zn & ~sn) - __popc(zn & sn)) - (__popc(zo & ~so) - __popc(zo & so));
+                }
             }
         }
     }
@@ -828,6 +916,12 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
     dcnt = __reduce_add_sync(FULL, dcnt);
     #pragma unroll
     for (int o = 16; o; o >>= 1) ps += __shfl_xor_sync(FULL, ps, o);
+    if (hw) {
+        #pragma unroll
+        for (int o = 16; o; o >>= 1) hsum += __shfl_xor_sync(FULL, hsum, o);
+        if (lane == 0) s.wM[warp] = hsum;
+        if (lane < L) s.dotpw[warp * MAX_PENDING + lane] = dotw_acc;
+    }
     if (lane == 0) { s.wc[warp] = cnt; s.wd[warp] = dcnt; s.wp[warp] = ps; }
     if (lane < L) s.dotp[warp * MAX_PENDING + lane] = dot;
     ok = __syncthreads_and(ok);
@@ -848,15 +942,32 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
     const int total = cw;
     #pragma unroll
     for (int o = 16; o; o >>= 1) p += __shfl_xor_sync(FULL, p, o);
+    if (hw && hsum_out) {
+        double hs = lane < NWARP ? s.wM[lane] : 0.0;
+        #pragma unroll
+        for (int o = 16; o; o >>= 1) hs += __shfl_xor_sync(FULL, hs, o);
+        *hsum_out = hs;
+    }
     if (total > 0) {
         for (int l = warp; l < L; l += NWARP) {
-            int d = lane < NWARP ? s.dotp[lane * MAX_PENDING + l] : 0;
-            #pragma unroll
-            for (int o = 16; o; o >>= 1) d += __shfl_xor_sync(FULL, d, o);
-            if (lane == 0) {
-                d += dots[l];
-                dots[l] = d;
-                coef[l] = s.pd[l] * (double)d;
+            if (hw) {
+                double d = lane < NWARP ? s.dotpw[lane * MAX_PENDING + l] : 0.0;
+                #pragma unroll
+                for (int o = 16; o; o >>= 1) d += __shfl_xor_sync(FULL, d, o);
+                if (lane == 0) {
+                    d += dotw[l];
+                    dotw[l] = d;
+                    coef[l] = s.pd[l] * d;
+                }
+            } else {
+                int d = lane < NWARP ? s.dotp[lane * MAX_PENDING + l] : 0;
+                #pragma unroll
+                for (int o = 16; o; o >>= 1) d += __shfl_xor_sync(FULL, d, o);
+                if (lane == 0) {
+                    d += dots[l];
+                    dots[l] = d;
+                    coef[l] = s.pd[l] * (double)d;
+                }
             }
         }
         int run = off;
@@ -874,7 +985,9 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
             int at = run + incl - c;
             for (uint32_t mk = ch; mk; mk &= mk - 1u) {
                 const int b = __ffs(mk) - 1;
-                list[at++] = delta_entry(((unsigned)w << 5) + b, rowpitch, ng, tw, b);
+                const int e = delta_entry(((unsigned)w << 5) + b, rowpitch, ng, tw, b);
+                if (wl) wl[at] = entry_coef(e) * __ldg(hw + ((int64_t)w << 5) + b);
+                list[at++] = e;
             }
             run += __shfl_sync(FULL, incl, 31);
         }
@@ -903,8 +1016,12 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
             s.scal[1] = 1.0;
         }
         __syncthreads();
-        ndelta = build_delta_list((int)((len + 31) >> 5), onz, osg, nz, sg, list, rowpitch, s);
-        if (L > 0) pending_coef(L, Ls, (int)((len + 31) >> 5), pnz, psg, nz, sg, s.pd, dots, coef);
+        ndelta = build_delta_list((int)((len + 31) >> 5), onz, osg, nz, sg, list, rowpitch, s, hw, wl);
+        if (L > 0) {
+            if (hw) pending_coef_w(L, Ls, (int)((len + 31) >> 5), pnz, psg, nz, sg, s.pd, hw, dotw, coef);
+            else pending_coef(L, Ls, (int)((len + 31) >> 5), pnz, psg, nz, sg, s.pd, dots, coef);
+        }
+        if (hw && hsum_out) *hsum_out = (double)__ldg(hw + Jc);
     }
     __syncthreads();
     phase_mark(s, 6);
@@ -936,6 +1053,7 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
     const int tid = threadIdx.x;
     const bool lead = (q == 0);
     const bool skip = (cfg.fault_skip == q);
+    const bool wtd = (P.hw != nullptr);   // §2.5 importance-weighted objective
     const int Ls = cfg.Lcap > 0 ? cfg.Lcap : 1;   // stride of the word-major pending masks
 
     float* blkV = P.Rv + P.pv.block_offset(q, m);
@@ -949,6 +1067,10 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
 
     if (__ldcg(P.nonfinite) != 0u) {
         if (lead && tid == 0) atomicExch(P.status, ST_ENONFINITE);
+        return true;
+    }
+    if (__ldcg(P.nonfinite + 1) != 0u) {   // importance weights not finite, negative or all zero
+        if (lead && tid == 0) atomicExch(P.status, ST_EINVAL);
         return true;
     }
     double N0 = 1.0;
@@ -970,6 +1092,7 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
     unsigned long long sum_nu = 0, sum_nv = 0, sum_du = 0, sum_dv = 0, sum_nunv = 0, hs = 0, fb = 0;
     const int64_t kk = (mode == MODE_FACTOR) ? P.k : 1;
     int nU = 0, nV = 0, dU = 0, dV = 0;   // support sizes and list lengths (trit changes)
+    double hsv = 0.0;                     // weighted objective: sum of h~ over the support of v
     double p = 0.0, thr;
     unsigned gen = 0;   // half-step counter of this matrix (tags of the exchanged words)
     HalfCorr hcV{s.coef, s.cnzV, s.csgV, s.corr, s.gV, 0};
@@ -989,7 +1112,11 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
             nU = build_from_trits(P.start + i * P.start_words, P.start_words, m, s.nzU, s.sgU, s.ulist, pitchV, s);
             dU = nU;
             if (L > 0) pending_coef(L, Ls, Wm, s.pnzU, s.psgU, s.nzU, s.sgU, s.pd, s.dotU, s.coef);
-            for (int l = tid; l < L; l += NT) { s.dotV[l] = 0; s.coefV[l] = 0.0; }
+            for (int l = tid; l < L; l += NT) {
+                s.dotV[l] = 0;
+                s.coefV[l] = 0.0;
+                if (wtd) s.dotVw[l] = 0.0;
+            }
         } else {
             for (int w = tid; w < Wm; w += NT) { s.nzU[w] = 0u; s.sgU[w] = 0u; }
             nV = build_from_trits(P.start, P.start_words, n, s.nzV, s.sgV, s.vlist, pitchU, s);
@@ -1003,12 +1130,13 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
                 const unsigned tg = gen_tag(++gen);
                 double S;
                 hcV.L = L;
-                gemv_dispatch(P.pv.vec, blkV, pitchV, validV, c0, s.ulist, dU, s.red, P.xbuf, hcV, tg, skip, S, s.clk);
+                gemv_dispatch(P.pv.vec, blkV, pitchV, validV, c0, s.ulist, nullptr, dU, s.red, P.xbuf, hcV, tg, skip, S, s.clk);
                 phase_mark(s, 1);
                 bool ok = true;
                 const int nv2 = exchange_threshold(P.partV, q, Gg, tg, arrivals, skip, S, P.xbuf, n, P.tau, s.nzV,
                                                    s.sgV, s.onzV, s.osgV, s.vlist, pitchU, s, L, Ls, s.pnzV, s.psgV,
-                                                   s.dotV, s.coefV, false, thr, dV, gs, cfg.limit_ns, P.status, ok);
+                                                   s.dotV, s.coefV, false, thr, dV, gs, cfg.limit_ns, P.status, ok,
+                                                   wtd ? P.hw : nullptr, wtd ? s.vwl : nullptr, s.dotVw, &hsv);
                 if (!ok) return false;
                 fb += (s.scal[1] != 0.0) ? 1 : 0;
                 sum_nu += (unsigned long long)nU;
@@ -1031,7 +1159,8 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
             const unsigned tg = gen_tag(++gen);
             double S;
             hcU.L = L;
-            gemv_dispatch(P.pu.vec, blkU, pitchU, validU, r0, s.vlist, dV, s.red, P.ybuf, hcU, tg, skip, S, s.clk);
+            gemv_dispatch(P.pu.vec, blkU, pitchU, validU, r0, s.vlist, wtd ? s.vwl : nullptr, dV, s.red, P.ybuf, hcU, tg, skip,
+                          S, s.clk);
             phase_mark(s, 1);
             bool ok = true;
             sum_nv += (unsigned long long)nV;
@@ -1054,8 +1183,9 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
                 return true;
             }
         }
-        // ---- scale (§2.3 step 2): d = u^T R v / (nnz(u) nnz(v)), with u^T R v = u^T y = p
-        const double d = (p == 0.0) ? 0.0 : p / ((double)nU * (double)nV);
+        // ---- scale (§2.3 step 2): d = u^T R v / (nnz(u) nnz(v)), with u^T R v = u^T y = p;
+        //      weighted (§2.5): d = u^T R (h~ v) / (nnz(u) sum_{v != 0} h~), the decrease p d
+        const double d = (p == 0.0) ? 0.0 : p / ((double)nU * (wtd ? hsv : (double)nV));
         RN2 -= p * d;
         sum_nunv += (unsigned long long)nU * (unsigned long long)nV;
         if (lead) {
@@ -1111,7 +1241,7 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
             const int64_t r = t / validV;
             const int c = (int)(t - r * validV);
             const double v = (double)__ldcg(blkV + r * pitchV + c);
-            rs += v * v;
+            rs += v * v * (wtd ? (double)__ldg(P.hw + c0 + c) : 1.0);
         }
     }
     double R2 = 0.0;
@@ -1140,7 +1270,7 @@ __global__ void __launch_bounds__(NT, 1) als_kernel(const KCfg cfg) {
     const int grp = blockIdx.x / cfg.Gg;
     const int q = blockIdx.x - grp * cfg.Gg;
     const int Lc = cfg.Lcap > 0 ? cfg.Lcap : 1;
-    const SmemLayout lay(cfg.m_max, cfg.n_max, Lc, cfg.pv_max, cfg.pu_max);
+    const SmemLayout lay(cfg.m_max, cfg.n_max, Lc, cfg.pv_max, cfg.pu_max, cfg.weighted);
     Smem s;
     s.red = reinterpret_cast<double*>(smem_raw + lay.red);
     s.pd = reinterpret_cast<double*>(smem_raw + lay.pd);
@@ -1179,6 +1309,9 @@ __global__ void __launch_bounds__(NT, 1) als_kernel(const KCfg cfg) {
     s.osgU = reinterpret_cast<uint32_t*>(smem_raw + lay.osgU);
     s.onzV = reinterpret_cast<uint32_t*>(smem_raw + lay.onzV);
     s.osgV = reinterpret_cast<uint32_t*>(smem_raw + lay.osgV);
+    s.vwl = reinterpret_cast<float*>(smem_raw + lay.vwl);
+    s.dotVw = reinterpret_cast<double*>(smem_raw + lay.dotVw);
+    s.dotpw = reinterpret_cast<double*>(smem_raw + lay.dotpw);
     s.gV = reinterpret_cast<double*>(smem_raw + lay.gV);
     s.gU = reinterpret_cast<double*>(smem_raw + lay.gU);
     s.corr = reinterpret_cast<double*>(smem_raw + lay.corr);
@@ -1346,12 +1479,14 @@ Part make_part(int64_t len, int G, int vec) {
     return p;
 }
 
-size_t als_smem_bytes(int64_t m_max, int64_t n_max, int L, int pv_max, int pu_max) {
-    return SmemLayout(m_max, n_max, L > 0 ? L : 1, pv_max, pu_max).total;
+size_t als_smem_bytes(int64_t m_max, int64_t n_max, int L, int pv_max, int pu_max, int weighted) {
+    return SmemLayout(m_max, n_max, L > 0 ? L : 1, pv_max, pu_max, weighted).total;
 }
 
 struct ProbIn {
     const float* A;
+    const float* h;       // §2.5 per-column second moments (n), or null for the plain objective
+    double lambda;
     int64_t m, n, k;
     double tau;
     int iters;
@@ -1451,9 +1586,11 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
     for (int b = 0; b < np; ++b)
         if ((double)in[b].m * pv_max >= 1073741824.0 || (double)in[b].n * pu_max >= 1073741824.0) return EXTERND_ELIMIT;
     int Lcap = MAX_PENDING;
-    while (Lcap > 1 && als_smem_bytes(m_max, n_max, Lcap, pv_max, pu_max) > di.smem_optin) --Lcap;
+    int weighted = 0;
+    for (int b = 0; b < np; ++b) weighted |= (in[b].h != nullptr);
+    while (Lcap > 1 && als_smem_bytes(m_max, n_max, Lcap, pv_max, pu_max, weighted) > di.smem_optin) --Lcap;
     if (opt.pending > 0 && opt.pending < Lcap) Lcap = opt.pending;
-    const size_t smem = als_smem_bytes(m_max, n_max, Lcap, pv_max, pu_max);
+    const size_t smem = als_smem_bytes(m_max, n_max, Lcap, pv_max, pu_max, weighted);
     if (smem > di.smem_optin) return EXTERND_ELIMIT;
 
     int nb = 0;
@@ -1466,14 +1603,14 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
     // ---- plan the workspace
     std::vector<Prob> probs(np);
     std::vector<size_t> off_rv(np), off_ru(np), off_x(np), off_y(np), off_sums(np), off_start(np), off_norm(np), off_A(np),
-        off_B(np), off_C(np), off_D(np), off_E(np), off_d64(np), off_pre(np), off_thr(np), off_tro(np);
+        off_B(np), off_C(np), off_D(np), off_E(np), off_d64(np), off_pre(np), off_thr(np), off_tro(np), off_hw(np), off_h(np);
     size_t ctl = 0;
     const size_t off_gsync = ctl;
     ctl += round_up(sizeof(GroupSync) * NG, 256);
     const size_t off_status = ctl;
     ctl += round_up(sizeof(int) * np, 256);
     const size_t off_nonfin = ctl;
-    ctl += round_up(sizeof(unsigned) * np, 256);
+    ctl += round_up(sizeof(unsigned) * 2 * np, 256);
     const size_t off_stats = ctl;
     ctl += round_up(sizeof(DevStats) * np, 256);
     const size_t off_probs = ctl;
@@ -1506,6 +1643,11 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
         const int64_t srows = (I.mode == MODE_FACTOR) ? I.k : 1;
         off_start[b] = ws; ws += round_up(sizeof(uint32_t) * (size_t)(P.start_words * srows), 256);
         off_norm[b] = ws; ws += round_up(sizeof(double) * (size_t)P.n_norm_part, 256);
+        off_hw[b] = off_h[b] = SIZE_MAX;
+        if (I.h) {
+            off_hw[b] = ws; ws += round_up(sizeof(float) * (size_t)I.n, 256);
+            if (!is_device_ptr(I.h)) { off_h[b] = ws; ws += round_up(sizeof(float) * (size_t)I.n, 256); }
+        }
         // staging for host pointers
         off_A[b] = SIZE_MAX;
         if (I.A && !is_device_ptr(I.A)) { off_A[b] = ws; ws += round_up(sizeof(float) * (size_t)(I.m * I.n), 256); }
@@ -1555,6 +1697,7 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
         const ProbIn& I = in[b];
         Prob& P = probs[b];
         P.A = off_A[b] == SIZE_MAX ? I.A : reinterpret_cast<const float*>(dws + off_A[b]);
+        P.hw = off_hw[b] == SIZE_MAX ? nullptr : reinterpret_cast<const float*>(dws + off_hw[b]);
         P.Rv = reinterpret_cast<float*>(dws + off_rv[b]);
         P.Ru = reinterpret_cast<float*>(dws + off_ru[b]);
         P.xbuf = reinterpret_cast<unsigned long long*>(dws + off_x[b]);
@@ -1564,7 +1707,7 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
         P.partU = P.sums + 2 * Gg;
         P.start = reinterpret_cast<uint32_t*>(dws + off_start[b]);
         P.norm_part = reinterpret_cast<double*>(dws + off_norm[b]);
-        P.nonfinite = reinterpret_cast<unsigned*>(dws + off_nonfin) + b;
+        P.nonfinite = reinterpret_cast<unsigned*>(dws + off_nonfin) + 2 * b;
         P.status = reinterpret_cast<int*>(dws + off_status) + b;
         P.stats = reinterpret_cast<DevStats*>(dws + off_stats) + b;
         if (I.mode == MODE_FACTOR) {
@@ -1597,6 +1740,15 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
         const ProbIn& I = in[b];
         if (off_A[b] != SIZE_MAX)
             CK(cudaMemcpyAsync(dws + off_A[b], I.A, sizeof(float) * (size_t)(I.m * I.n), cudaMemcpyHostToDevice, stream));
+        if (off_h[b] != SIZE_MAX)
+            CK(cudaMemcpyAsync(dws + off_h[b], I.h, sizeof(float) * (size_t)I.n, cudaMemcpyHostToDevice, stream));
+        if (off_hw[b] != SIZE_MAX) {
+            const float* hsrc = off_h[b] == SIZE_MAX ? I.h : reinterpret_cast<const float*>(dws + off_h[b]);
+            weights_kernel<<<1, 1024, 0, stream>>>(hsrc, I.n, I.lambda, reinterpret_cast<float*>(dws + off_hw[b]),
+                                                   reinterpret_cast<unsigned*>(dws + off_nonfin) + 2 * b + 1);
+            CK(cudaGetLastError());
+            ++launches;
+        }
         if (I.mode != MODE_FACTOR) {
             // debug input trits -> start row
             const bool dev_in = is_device_ptr(I.dbg_in);
@@ -1643,6 +1795,7 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
             const double lim = opt.wait_limit_s > 0 ? opt.wait_limit_s : 2.0;
             cfg.limit_ns = (uint64_t)(lim * 1e9);
             cfg.fault_skip = opt.fault_skip;
+            cfg.weighted = weighted;
             void* args[] = {&cfg};
             CK(cudaLaunchCooperativeKernel((void*)als_kernel, dim3((unsigned)(NG * Gg)), dim3(NT), args, smem, stream));
             ++launches;
@@ -1816,6 +1969,22 @@ int externd_factor_ex(const float* A, int64_t m, int64_t n, double mu, double ta
         ro.fault_skip = opt->fault_inject ? opt->fault_skip_cta : -1;
         I.d64 = opt->d64_out;
     }
+    int st = 0;
+    return run(&I, 1, ro, reinterpret_cast<cudaStream_t>(stream), &st);
+}
+
+int externd_factor_weighted(const float* A, int64_t m, int64_t n, double mu, double tau, int iters, uint64_t seed,
+                            const float* h, double lambda, uint8_t* B_out, float* D_out, uint8_t* C_out,
+                            double* energy_out, void* stream) {
+    int64_t k = 0;
+    int rc = validate_factor(A, m, n, mu, tau, iters, B_out, D_out, C_out, &k);
+    if (rc != EXTERND_OK) return rc;
+    if (!h || !std::isfinite(lambda) || lambda < 0.0) return EXTERND_EINVAL;
+    ProbIn I = {};
+    I.A = A; I.m = m; I.n = n; I.k = k; I.tau = tau; I.iters = iters; I.seed = seed;
+    I.h = h; I.lambda = lambda;
+    I.B = B_out; I.D = D_out; I.C = C_out; I.energy = energy_out; I.mode = MODE_FACTOR;
+    RunOpts ro;
     int st = 0;
     return run(&I, 1, ro, reinterpret_cast<cudaStream_t>(stream), &st);
 }

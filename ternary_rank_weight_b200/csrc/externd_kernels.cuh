@@ -57,6 +57,7 @@ constexpr unsigned FULL = 0xffffffffu;
 
 // Status codes written by kernels (mirror externd_status).
 constexpr int ST_OK = 0;
+constexpr int ST_EINVAL = -1;
 constexpr int ST_EZERO = -2;
 constexpr int ST_ENONFINITE = -3;
 constexpr int ST_ETIMEOUT = -7;
@@ -108,6 +109,7 @@ enum Mode { MODE_FACTOR = 0, MODE_HALF_V = 1, MODE_HALF_U = 2 };
 
 struct Prob {
     const float* A;
+    const float* hw;          // importance weights h~ (n, fp32) of §2.5, or null for the plain objective
     int64_t m, n, k;
     double tau;
     int iters;
@@ -151,6 +153,7 @@ struct KCfg {
     int pv_max, pu_max;       // largest stripe pitch of the two layouts
     uint64_t limit_ns;
     int fault_skip;           // CTA rank (within group) that never arrives; -1 = off
+    int weighted;             // problems carry importance weights (single-matrix launches only)
 };
 
 // ---------------------------------------------------------------------------

@@ -61,6 +61,18 @@ def llm_matrix(m: int, n: int, seed: int, outliers: int = 8, std: float = 0.02,
     return a
 
 
+def importance_weights(n: int, seed: int, sigma: float = 1.5, hot: int = 8, hot_scale: float = 30.0) -> np.ndarray:
+    """Per-input-channel second moments standing in for a llama.cpp importance matrix
+    (the pages' §2.5 input, not available here): log-normal with spread ``sigma`` and
+    ``hot`` distinct channels scaled by ``hot_scale`` (activation outlier channels)."""
+    rng = np.random.default_rng(seed)
+    h = np.exp(sigma * rng.standard_normal(n))
+    k = min(hot, n)
+    if k > 0:
+        h[rng.choice(n, size=k, replace=False)] *= hot_scale
+    return h.astype(np.float32)
+
+
 @dataclass(frozen=True)
 class Workload:
     """One named factorization job: matrices plus the method's parameters."""
