@@ -149,7 +149,7 @@ def _config(w, extra=None):
            "shape": list(shapes[0]) if len(shapes) == 1 else [list(s) for s in shapes],
            "mu": w.mu[0] if len(set(w.mu)) == 1 else list(w.mu),
            "tau": w.tau[0] if len(set(w.tau)) == 1 else list(w.tau),
-           "iters": w.iters, "recipe": w.recipe + ("+bf16" if w.bf16 else ""),
+           "iters": w.iters, "recipe": w.recipe + ("+bf16" if w.bf16 else "") + ("+importance weights" if w.weighted else ""),
            "l2": "inputs larger than L2 (A + two residual copies exceed 126 MB); no flush"}
     if extra:
         cfg.update(extra)
@@ -237,7 +237,12 @@ def run_ours(args):
 
     from ternary_rank_weight_b200 import dist
 
+    hw = [torch.from_numpy(w.weights(b)).to(dev) for b in range(w.count)] if w.weighted else None
+
     def step(inputs):
+        if w.weighted:
+            f = ext.factor_weighted(inputs[0], hw[0], w.mu[0], w.tau[0], lam=w.lam, iters=w.iters, seed=w.seeds[0])
+            return [f], f.stats
         if w.count == 1:
             f = ext.factor(inputs[0], w.mu[0], w.tau[0], iters=w.iters, seed=w.seeds[0],
                            grid=args.grid, pending=args.pending)

@@ -349,7 +349,7 @@ __host__ __device__ constexpr int GEMV_U() {
 // acc += sum over the list entries g, g + lanes, g + 2 lanes, ... of this thread's VEC
 // columns, U entries per batch (every batch issues all its loads before using any).
 
-template <int VEC, int U>
+template <int VEC, int U, bool WL>
 __device__ __forceinline__ void gemv_rows(double* acc, const float* base, const int* __restrict__ list,
                                           const float* __restrict__ wl, int nlist, int g, int lanes) {
     for (int idx = g; idx < nlist; idx += U * lanes) {
@@ -359,7 +359,8 @@ __device__ __forceinline__ void gemv_rows(double* acc, const float* base, const 
         for (int u = 0; u < U; ++u) {
             const int ii = idx + u * lanes;
             const int ent = ii < nlist ? list[ii] : 0;
-            cf[u] = ii < nlist ? (wl ? wl[ii] : entry_coef(ent)) : 0.f;
+            if constexpr (WL) cf[u] = ii < nlist ? wl[ii] : 0.f;
+            else cf[u] = entry_coef(ent);
             if (ii < nlist) {
                 load_vec<VEC>(base + (ent & 0x3fffffff), v[u]);
             } else {
@@ -376,7 +377,7 @@ __device__ __forceinline__ void gemv_rows(double* acc, const float* base, const 
 // them in the first one, where g starts at 0), so g[c] += sum_{e in list} s_e blk[r_e][c]
 // keeps g = R^T t (or R t) for the current input trits t; out[c] = g[c] minus the
 // lazy-deflation correction is written to gout[out0 + c].  fp64 accumulation of exact fp32 terms, fixed summation order.
-template <int VEC>
+template <int VEC, bool WL>
 __device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, int64_t out0,
                           const int* __restrict__ list, const float* __restrict__ wl, int nlist, double* red,
                           unsigned long long* gout, const HalfCorr& hc, unsigned tag, bool skip, double& S,
@@ -399,10 +400,10 @@ __device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, i
             // batch width from the longest group (uniform over the CTA): short change
             // lists issue few predicated slots
             const int per = (nlist + lanes - 1) / lanes;
-            if (per <= 1) gemv_rows<VEC, 1>(acc, base, list, wl, nlist, g, lanes);
-            else if (per <= 2) gemv_rows<VEC, 2>(acc, base, list, wl, nlist, g, lanes);
-            else if (per <= 4) gemv_rows<VEC, 4>(acc, base, list, wl, nlist, g, lanes);
-            else gemv_rows<VEC, GEMV_U<VEC>()>(acc, base, list, wl, nlist, g, lanes);
+            if (per <= 1) gemv_rows<VEC, 1, WL>(acc, base, list, wl, nlist, g, lanes);
+            else if (per <= 2) gemv_rows<VEC, 2, WL>(acc, base, list, wl, nlist, g, lanes);
+            else if (per <= 4) gemv_rows<VEC, 4, WL>(acc, base, list, wl, nlist, g, lanes);
+            else gemv_rows<VEC, GEMV_U<VEC>(), WL>(acc, base, list, wl, nlist, g, lanes);
             #pragma unroll
             for (int e = 0; e < VEC; ++e) red[g * rs + j * VEC + e] = acc[e];
         }
@@ -439,7 +440,8 @@ __device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, i
                 for (int u = 0; u < U; ++u) {
                     const int ii = idx + u;
                     const int ent = ii < nlist ? list[ii] : 0;
-                    cf[u] = ii < nlist ? (wl ? wl[ii] : entry_coef(ent)) : 0.f;
+                    if constexpr (WL) cf[u] = ii < nlist ? wl[ii] : 0.f;
+                    else cf[u] = entry_coef(ent);
                     if (ii < nlist) {
                         load_vec<VEC>(base + (ent & 0x3fffffff), v[u]);
                     } else {
@@ -462,13 +464,14 @@ __device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, i
     }
 }
 
+template <bool WL>
 __device__ __forceinline__ void gemv_dispatch(int vec, const float* blk, int pitch, int valid, int64_t out0,
                                               const int* list, const float* wl, int nlist, double* red,
                                               unsigned long long* gout, const HalfCorr& hc, unsigned tag, bool skip,
                                               double& S, unsigned long long* clk) {
-    if (vec == 4) gemv_emit<4>(blk, pitch, valid, out0, list, wl, nlist, red, gout, hc, tag, skip, S, clk);
-    else if (vec == 2) gemv_emit<2>(blk, pitch, valid, out0, list, wl, nlist, red, gout, hc, tag, skip, S, clk);
-    else gemv_emit<1>(blk, pitch, valid, out0, list, wl, nlist, red, gout, hc, tag, skip, S, clk);
+    if (vec == 4) gemv_emit<4, WL>(blk, pitch, valid, out0, list, wl, nlist, red, gout, hc, tag, skip, S, clk);
+    else if (vec == 2) gemv_emit<2, WL>(blk, pitch, valid, out0, list, wl, nlist, red, gout, hc, tag, skip, S, clk);
+    else gemv_emit<1, WL>(blk, pitch, valid, out0, list, wl, nlist, red, gout, hc, tag, skip, S, clk);
 }
 
 // Fold the L pending components into this CTA's block:
@@ -667,6 +670,7 @@ __device__ __forceinline__ int delta_entry(unsigned idx, int rowpitch, uint32_t 
 
 // Block-wide: compacted list of the changes (onz, osg) -> (nz, sg) over W mask words,
 // in index order.  Returns the count.
+template <bool WL>
 __device__ int build_delta_list(int W, const uint32_t* onz, const uint32_t* osg, const uint32_t* nz,
                                 const uint32_t* sg, int* list, int rowpitch, const Smem& s,
                                 const float* hw = nullptr, float* wl = nullptr) {
@@ -696,7 +700,7 @@ __device__ int build_delta_list(int W, const uint32_t* onz, const uint32_t* osg,
             const int at = run + __popc(ch & ((1u << lane) - 1u));
             const int e = delta_entry(((unsigned)w << 5) + lane, rowpitch, ng, tw, lane);
             list[at] = e;
-            if (wl) wl[at] = entry_coef(e) * __ldg(hw + ((int64_t)w << 5) + lane);
+            if constexpr (WL) wl[at] = entry_coef(e) * __ldg(hw + ((int64_t)w << 5) + lane);
         }
         run += __popc(ch);
     }
@@ -760,6 +764,7 @@ __device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned* p) {
 // one fixed order, so every CTA of the group derives identical results.  Arrival
 // needs no fence: the tags validate every word that is read.
 // Returns nnz; ok = false if a wait ran out.
+template <bool WTD>
 __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, unsigned tag, unsigned& arrivals,
                                   bool skip, double S, const unsigned long long* gvec, int64_t len, double tau,
                                   uint32_t* nz, uint32_t* sg, uint32_t* onz, uint32_t* osg, int* list, int rowpitch,
@@ -882,7 +887,7 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
         if (lane < K) { nz[w] = my_bz; sg[w] = my_bs; onz[w] = oz; osg[w] = os; }
         cnt += __popc(my_bz);
         dcnt += __popc(ch);
-        if (hw) {   // sum of h~ over the new support (lane = word, bits in increasing order)
+        if constexpr (WTD) {   // sum of h~ over the new support (lane = word, bits in increasing order)
             for (uint32_t mk = my_bz; mk; mk &= mk - 1u) hsum += (double)__ldg(hw + ((int64_t)w << 5) + __ffs(mk) - 1);
         }
         // change of t_l . t (weighted: sum h~_c t_l(c) t(c)) over the words that changed
@@ -894,10 +899,11 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
             const uint32_t zi = __shfl_sync(FULL, my_bz, i), si = __shfl_sync(FULL, my_bs, i);
             const uint32_t ozi = __shfl_sync(FULL, oz, i), osi = __shfl_sync(FULL, os, i);
             const uint32_t chi = __shfl_sync(FULL, ch, i);
-            const uint32_t dni = __shfl_sync(FULL, dn, i), dti = __shfl_sync(FULL, dt, i);
+            uint32_t dni = 0u, dti = 0u;
+            if constexpr (WTD) { dni = __shfl_sync(FULL, dn, i); dti = __shfl_sync(FULL, dt, i); }
             if (lane < L) {
                 const uint32_t pz = pnz[(base + i) * Ls + lane], pg = psg[(base + i) * Ls + lane];
-                if (hw) {
+                if constexpr (WTD) {
                     for (uint32_t mk = pz & chi; mk; mk &= mk - 1u) {
                         const int b = __ffs(mk) - 1;
                         const double hv = (double)__ldg(hw + ((int64_t)(base + i) << 5) + b);
@@ -916,7 +922,7 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
     dcnt = __reduce_add_sync(FULL, dcnt);
     #pragma unroll
     for (int o = 16; o; o >>= 1) ps += __shfl_xor_sync(FULL, ps, o);
-    if (hw) {
+    if constexpr (WTD) {
         #pragma unroll
         for (int o = 16; o; o >>= 1) hsum += __shfl_xor_sync(FULL, hsum, o);
         if (lane == 0) s.wM[warp] = hsum;
@@ -942,7 +948,7 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
     const int total = cw;
     #pragma unroll
     for (int o = 16; o; o >>= 1) p += __shfl_xor_sync(FULL, p, o);
-    if (hw && hsum_out) {
+    if constexpr (WTD) {
         double hs = lane < NWARP ? s.wM[lane] : 0.0;
         #pragma unroll
         for (int o = 16; o; o >>= 1) hs += __shfl_xor_sync(FULL, hs, o);
@@ -950,7 +956,7 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
     }
     if (total > 0) {
         for (int l = warp; l < L; l += NWARP) {
-            if (hw) {
+            if constexpr (WTD) {
                 double d = lane < NWARP ? s.dotpw[lane * MAX_PENDING + l] : 0.0;
                 #pragma unroll
                 for (int o = 16; o; o >>= 1) d += __shfl_xor_sync(FULL, d, o);
@@ -986,7 +992,7 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
             for (uint32_t mk = ch; mk; mk &= mk - 1u) {
                 const int b = __ffs(mk) - 1;
                 const int e = delta_entry(((unsigned)w << 5) + b, rowpitch, ng, tw, b);
-                if (wl) wl[at] = entry_coef(e) * __ldg(hw + ((int64_t)w << 5) + b);
+                if constexpr (WTD) wl[at] = entry_coef(e) * __ldg(hw + ((int64_t)w << 5) + b);
                 list[at++] = e;
             }
             run += __shfl_sync(FULL, incl, 31);
@@ -1016,12 +1022,12 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
             s.scal[1] = 1.0;
         }
         __syncthreads();
-        ndelta = build_delta_list((int)((len + 31) >> 5), onz, osg, nz, sg, list, rowpitch, s, hw, wl);
+        ndelta = build_delta_list<WTD>((int)((len + 31) >> 5), onz, osg, nz, sg, list, rowpitch, s, hw, wl);
         if (L > 0) {
-            if (hw) pending_coef_w(L, Ls, (int)((len + 31) >> 5), pnz, psg, nz, sg, s.pd, hw, dotw, coef);
+            if constexpr (WTD) pending_coef_w(L, Ls, (int)((len + 31) >> 5), pnz, psg, nz, sg, s.pd, hw, dotw, coef);
             else pending_coef(L, Ls, (int)((len + 31) >> 5), pnz, psg, nz, sg, s.pd, dots, coef);
         }
-        if (hw && hsum_out) *hsum_out = (double)__ldg(hw + Jc);
+        if constexpr (WTD) *hsum_out = (double)__ldg(hw + Jc);
     }
     __syncthreads();
     phase_mark(s, 6);
@@ -1045,6 +1051,7 @@ __device__ bool exchange_sum(unsigned long long* sums, int q, int Gg, double v, 
 
 // Factor (or run one debug half-step of) one matrix with this CTA group.
 // Returns false if the group aborted.
+template <bool WTD>
 __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s, GroupSync* gs, unsigned& arrivals) {
     const int64_t m = P.m, n = P.n;
     const int Wm = (int)((m + 31) >> 5), Wn = (int)((n + 31) >> 5);
@@ -1053,7 +1060,7 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
     const int tid = threadIdx.x;
     const bool lead = (q == 0);
     const bool skip = (cfg.fault_skip == q);
-    const bool wtd = (P.hw != nullptr);   // §2.5 importance-weighted objective
+    constexpr bool wtd = WTD;   // §2.5 importance-weighted objective (P.hw set)
     const int Ls = cfg.Lcap > 0 ? cfg.Lcap : 1;   // stride of the word-major pending masks
 
     float* blkV = P.Rv + P.pv.block_offset(q, m);
@@ -1130,10 +1137,10 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
                 const unsigned tg = gen_tag(++gen);
                 double S;
                 hcV.L = L;
-                gemv_dispatch(P.pv.vec, blkV, pitchV, validV, c0, s.ulist, nullptr, dU, s.red, P.xbuf, hcV, tg, skip, S, s.clk);
+                gemv_dispatch<false>(P.pv.vec, blkV, pitchV, validV, c0, s.ulist, nullptr, dU, s.red, P.xbuf, hcV, tg, skip, S, s.clk);
                 phase_mark(s, 1);
                 bool ok = true;
-                const int nv2 = exchange_threshold(P.partV, q, Gg, tg, arrivals, skip, S, P.xbuf, n, P.tau, s.nzV,
+                const int nv2 = exchange_threshold<WTD>(P.partV, q, Gg, tg, arrivals, skip, S, P.xbuf, n, P.tau, s.nzV,
                                                    s.sgV, s.onzV, s.osgV, s.vlist, pitchU, s, L, Ls, s.pnzV, s.psgV,
                                                    s.dotV, s.coefV, false, thr, dV, gs, cfg.limit_ns, P.status, ok,
                                                    wtd ? P.hw : nullptr, wtd ? s.vwl : nullptr, s.dotVw, &hsv);
@@ -1159,13 +1166,13 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
             const unsigned tg = gen_tag(++gen);
             double S;
             hcU.L = L;
-            gemv_dispatch(P.pu.vec, blkU, pitchU, validU, r0, s.vlist, wtd ? s.vwl : nullptr, dV, s.red, P.ybuf, hcU, tg, skip,
+            gemv_dispatch<WTD>(P.pu.vec, blkU, pitchU, validU, r0, s.vlist, wtd ? s.vwl : nullptr, dV, s.red, P.ybuf, hcU, tg, skip,
                           S, s.clk);
             phase_mark(s, 1);
             bool ok = true;
             sum_nv += (unsigned long long)nV;
             sum_dv += (unsigned long long)dV;
-            nU = exchange_threshold(P.partU, q, Gg, tg, arrivals, skip, S, P.ybuf, m, P.tau, s.nzU, s.sgU, s.onzU,
+            nU = exchange_threshold<false>(P.partU, q, Gg, tg, arrivals, skip, S, P.ybuf, m, P.tau, s.nzU, s.sgU, s.onzU,
                                     s.osgU, s.ulist, pitchV, s, L, Ls, s.pnzU, s.psgU, s.dotU, s.coef, true, thr, dU,
                                     gs, cfg.limit_ns, P.status, ok);
             if (!ok) return false;
@@ -1265,6 +1272,7 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
     return true;
 }
 
+template <bool WTD>
 __global__ void __launch_bounds__(NT, 1) als_kernel(const KCfg cfg) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int grp = blockIdx.x / cfg.Gg;
@@ -1319,7 +1327,7 @@ __global__ void __launch_bounds__(NT, 1) als_kernel(const KCfg cfg) {
     GroupSync* gs = cfg.gsync + grp;
     unsigned arrivals = 0;   // exchanges this CTA took part in (counter targets)
     for (int pi = grp; pi < cfg.nprob; pi += cfg.NG) {
-        if (!run_problem(cfg.probs[pi], q, cfg, s, gs, arrivals)) return;
+        if (!run_problem<WTD>(cfg.probs[pi], q, cfg, s, gs, arrivals)) return;
     }
 }
 
@@ -1421,7 +1429,8 @@ int dev_info(DevInfo& out) {
         d.smem_optin = (size_t)v;
         if (cudaDeviceGetAttribute(&v, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess) { cudaGetLastError(); return EXTERND_ECUDA; }
         d.coop = v;
-        if (cudaFuncSetAttribute(als_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)d.smem_optin) != cudaSuccess) {
+        if (cudaFuncSetAttribute(als_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)d.smem_optin) != cudaSuccess ||
+            cudaFuncSetAttribute(als_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)d.smem_optin) != cudaSuccess) {
             cudaGetLastError();
             return EXTERND_ECUDA;
         }
@@ -1586,15 +1595,19 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
     for (int b = 0; b < np; ++b)
         if ((double)in[b].m * pv_max >= 1073741824.0 || (double)in[b].n * pu_max >= 1073741824.0) return EXTERND_ELIMIT;
     int Lcap = MAX_PENDING;
+    // one launch runs one objective: every problem weighted, or none
     int weighted = 0;
-    for (int b = 0; b < np; ++b) weighted |= (in[b].h != nullptr);
+    for (int b = 0; b < np; ++b) weighted += (in[b].h != nullptr);
+    if (weighted != 0 && weighted != np) return EXTERND_EINVAL;
+    weighted = weighted ? 1 : 0;
     while (Lcap > 1 && als_smem_bytes(m_max, n_max, Lcap, pv_max, pu_max, weighted) > di.smem_optin) --Lcap;
     if (opt.pending > 0 && opt.pending < Lcap) Lcap = opt.pending;
     const size_t smem = als_smem_bytes(m_max, n_max, Lcap, pv_max, pu_max, weighted);
     if (smem > di.smem_optin) return EXTERND_ELIMIT;
 
     int nb = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, als_kernel, NT, smem) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, weighted ? als_kernel<true> : als_kernel<false>, NT, smem) !=
+        cudaSuccess) {
         cudaGetLastError();
         return EXTERND_ECUDA;
     }
@@ -1797,7 +1810,7 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
             cfg.fault_skip = opt.fault_skip;
             cfg.weighted = weighted;
             void* args[] = {&cfg};
-            CK(cudaLaunchCooperativeKernel((void*)als_kernel, dim3((unsigned)(NG * Gg)), dim3(NT), args, smem, stream));
+            CK(cudaLaunchCooperativeKernel(weighted ? (void*)als_kernel<true> : (void*)als_kernel<false>, dim3((unsigned)(NG * Gg)), dim3(NT), args, smem, stream));
             ++launches;
         }
         if (ev[3]) CK(cudaEventRecord(ev[3], stream));

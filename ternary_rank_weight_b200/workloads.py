@@ -86,6 +86,11 @@ class Workload:
     bf16: bool = False
     iters: int = 15
     mu_sweep: tuple = field(default=())   # extra mu read off one run (prefix property)
+    weighted: bool = False                # §2.5 objective with importance_weights(n, seed)
+    lam: float = 0.0
+
+    def weights(self, b: int) -> np.ndarray:
+        return importance_weights(self.shapes[b][1], self.seeds[b])
 
     def matrix(self, b: int) -> np.ndarray:
         m, n = self.shapes[b]
@@ -113,6 +118,8 @@ WORKLOADS = {
         "attn_16x1536x1536_mu2.5_tau_cycle", tuple((1536, 1536) for _ in range(16)),
         tuple(range(100, 116)), tuple(2.5 for _ in range(16)),
         tuple((0.7, 1.0, 2.0)[b % 3] for b in range(16))),
+    "mlp_2560x6912_bf16_mu3_tau1.0_weighted": Workload(
+        "mlp_2560x6912_bf16_mu3_tau1.0_weighted", ((2560, 6912),), (2,), (3.0,), (1.0,), bf16=True, weighted=True),
     "llm_4096x4096_mu3.5_tau0.7": Workload(
         "llm_4096x4096_mu3.5_tau0.7", ((4096, 4096),), (4,), (3.5,), (0.7,), outliers=32,
         mu_sweep=(1.0, 2.0, 3.0, 3.5)),
