@@ -19,6 +19,14 @@ arXiv 2607.13511), cited below by section and display equation:
 * §2.5: importance-weighted ALS minimizes sum_ij h~_j (A - Ahat)^2_ij with
   h~ = h / max(h) + lambda; the U-step targets W = R diag(h~), the V-step the plain
   residual R (h~ cancels there), the scale solves the weighted normal equation.
+* §2.4 "Refinement sweeps": after extraction, revisit each block (add its
+  contribution back to R, re-run the fit, re-deflate); here blocks of one
+  component.  Readings: the refit starts from the stored u and runs the same
+  alternation as extraction; it replaces the stored component only if its
+  least-squares decrease of the added-back residual is at least that of the
+  stored pair with its own least-squares scale (otherwise the stored pair stays,
+  rescaled), which makes every visit non-increasing in the residual, as the
+  pages report the sweeps to be.
 * §2.6 Cost model: inference computes y = B (diag(D) (C x)); mask+sign packing
   stores one zero/nonzero mask bit per element plus one sign bit per nonzero,
   and Eq. (1): bpw_eff = mu (m + n) / max(m, n) * (2 - sparsity).
@@ -438,3 +446,93 @@ def greedy_als_weighted(A: np.ndarray, h: np.ndarray, lam: float, k: int, tau: f
     e_final = 1.0 - float(np.sum(hw[None, :] * R * R)) / norm_w
     return Factorization(B=B, C=C, D=D, energy=energy, energy_final=e_final, norm_a2=norm_w,
                          margins=margins, safeguard_hits=0, residual_norms=None)
+
+
+# ----------------------------------------------------------------------------
+# §2.4 refinement sweeps (blocks of one component)
+# ----------------------------------------------------------------------------
+
+
+@dataclass
+class Refinement:
+    B: np.ndarray              # m x k int8
+    C: np.ndarray              # k x n int8
+    D: np.ndarray              # k float64
+    sweep_energy: np.ndarray   # per sweep, incremental (weighted when h is given): 1 - r2 / ||A||^2
+    energy_final: float        # explicit energy of the final residual
+    kept: int                  # visits that kept the stored pair (rescaled)
+    margins: np.ndarray        # sweeps x k: closest approach of the refit's half-steps to a threshold tie
+    decision_margins: np.ndarray  # sweeps x k: |dec_refit - dec_stored| / max(dec_refit, dec_stored)
+    visit_residuals: np.ndarray = field(default=None)  # sweeps x k explicit residual norms after each visit
+
+
+def refine_sweeps(A: np.ndarray, B: np.ndarray, D: np.ndarray, C: np.ndarray, sweeps: int, tau: float,
+                  iters: int = 15, h: np.ndarray | None = None, lam: float = 0.0,
+                  track_residual: bool = False) -> Refinement:
+    """§2.4 refinement sweeps with b = 1 on the factors (B, D, C) of A, for the plain
+    objective (h None) or the §2.5 weighted one.  Each visit of component i:
+    R <- R + d_i u_i v_i^T; refit from u_i with `iters` (V-step, U-step) pairs;
+    take the refit or the stored pair, whichever decreases the residual more with
+    its least-squares scale (ties go to the refit); R <- R - d u v^T."""
+    A = np.asarray(A, dtype=np.float64)
+    m, n = A.shape
+    k = int(np.asarray(D).shape[0])
+    hw = np.ones(n) if h is None else normalized_weights(h, lam).astype(np.float64)
+    B = np.array(B, dtype=np.int8, copy=True)
+    C = np.array(C, dtype=np.int8, copy=True)
+    D = np.array(D, dtype=np.float64, copy=True)
+    R = residual_after(A, B, D, C, k)
+    norm = float(np.sum(hw[None, :] * A * A))
+    r2 = float(np.sum(hw[None, :] * R * R))
+    sweep_energy = np.zeros(sweeps)
+    margins = np.zeros((sweeps, k))
+    dmargins = np.zeros((sweeps, k))
+    res = np.zeros((sweeps, k)) if track_residual else None
+    kept = 0
+    for s in range(sweeps):
+        for i in range(k):
+            ui = B[:, i].astype(np.float64)
+            vi = C[i, :].astype(np.float64)
+            di = float(D[i])
+            # add the stored contribution back
+            R += di * np.outer(ui, vi)
+            p_old = float(ui @ (R @ (hw * vi)))
+            n_old = float(np.count_nonzero(ui)) * float(np.sum(hw[vi != 0]))
+            r2 += 2.0 * di * p_old - di * di * n_old
+            d_old = 0.0 if (p_old == 0.0 or n_old == 0.0) else p_old / n_old
+            dec_old = p_old * d_old
+            # refit from the stored u
+            u = B[:, i].copy()
+            v = None
+            y = None
+            margin = math.inf
+            for _ in range(iters):
+                x = R.T @ u.astype(np.float64)
+                v, tv, _ = ternarize(x, tau)
+                margin = min(margin, relative_margin(x, tv))
+                y = R @ (hw * v.astype(np.float64))
+                u, tu, _ = ternarize(y, tau)
+                margin = min(margin, relative_margin(y, tu))
+            p = float(u.astype(np.float64) @ y)
+            nn = float(np.count_nonzero(u)) * float(np.sum(hw[v != 0]))
+            d = 0.0 if p == 0.0 else p / nn
+            dec = p * d
+            margins[s, i] = margin
+            top = max(dec, dec_old)
+            dmargins[s, i] = abs(dec - dec_old) / top if top > 0.0 else math.inf
+            if dec >= dec_old:
+                B[:, i] = u
+                C[i, :] = v
+                D[i] = d
+                r2 -= dec
+            else:
+                D[i] = d_old
+                kept += 1
+                r2 -= dec_old
+            R -= float(D[i]) * np.outer(B[:, i].astype(np.float64), C[i, :].astype(np.float64))
+            if track_residual:
+                res[s, i] = float(np.sum(hw[None, :] * R * R))
+        sweep_energy[s] = 1.0 - r2 / norm
+    e_final = 1.0 - float(np.sum(hw[None, :] * R * R)) / norm
+    return Refinement(B=B, C=C, D=D, sweep_energy=sweep_energy, energy_final=e_final, kept=kept,
+                      margins=margins, decision_margins=dmargins, visit_residuals=res)

@@ -413,3 +413,105 @@ def test_weighted_residual_decreases_and_energy_matches_reconstruction():
     f = ora.greedy_als(A, k=96, tau=1.0, seed=2)
     assert ora.weighted_energy(A, ora.reconstruct(f.B, f.D, f.C), hw) < fw.energy_final
     assert hw.max() == pytest.approx(1.0) and hw.dtype == np.float32
+
+
+# --------------------------------------------------------------------------
+# §2.4 refinement sweeps (blocks of one component)
+# --------------------------------------------------------------------------
+
+def _orthogonal_ternary_factors(m, n, k, seed):
+    """k components with disjoint row and column supports: A = B diag(D) C exactly."""
+    rng = np.random.default_rng(seed)
+    B = np.zeros((m, k), dtype=np.int8)
+    C = np.zeros((k, n), dtype=np.int8)
+    rows = np.array_split(rng.permutation(m), k)
+    cols = np.array_split(rng.permutation(n), k)
+    for i in range(k):
+        B[rows[i], i] = rng.choice([-1, 1], size=len(rows[i]))
+        C[i, cols[i]] = rng.choice([-1, 1], size=len(cols[i]))
+    D = rng.uniform(0.5, 2.0, size=k) * rng.choice([-1, 1], size=k)
+    return B, D, C
+
+
+def test_refinement_of_an_exact_orthogonal_factorization_is_a_fixed_point():
+    """Closed form: with R = 0 the add-back leaves d_i u_i v_i^T alone, whose refit from
+    u_i returns u_i, sign(d_i) v_i and |d_i| whenever tau * nnz < length (the V-step sees
+    d_i nnz(u_i) v_i); every rank-1 term must stay what it was."""
+    B, D, C = _orthogonal_ternary_factors(24, 30, 4, seed=3)
+    A = ora.reconstruct(B, D, C)
+    r = ora.refine_sweeps(A, B, D, C, sweeps=2, tau=1.0)
+    assert np.array_equal(r.B, B)
+    assert np.array_equal(r.C, (np.sign(D)[:, None] * C).astype(np.int8))
+    assert np.allclose(r.D, np.abs(D), rtol=1e-14, atol=0)
+    assert r.kept == 0
+    assert r.energy_final == pytest.approx(1.0, abs=1e-14)
+    assert np.allclose(r.sweep_energy, 1.0, atol=1e-12)
+
+
+def test_refinement_with_zero_sweeps_returns_the_input():
+    A = np.random.default_rng(2).standard_normal((12, 9))
+    f = ora.greedy_als(A, k=9, tau=0.7, seed=1)
+    r = ora.refine_sweeps(A, f.B, f.D, f.C, sweeps=0, tau=0.7)
+    assert np.array_equal(r.B, f.B) and np.array_equal(r.C, f.C) and np.array_equal(r.D, f.D)
+    assert r.energy_final == pytest.approx(f.energy_final, abs=1e-13)
+
+
+def test_refinement_visit_is_bounded_by_brute_force_over_all_ternary_pairs():
+    """k = 1: the add-back restores A itself, so the visit's decrease of ||A||^2 must lie
+    between the stored pair's least-squares decrease and the best over every ternary pair
+    (enumerated), and the new residual must follow from the chosen factors."""
+    rng = np.random.default_rng(5)
+    pairs = [(np.array(u), np.array(v)) for u in itertools.product((-1, 0, 1), repeat=3)
+             for v in itertools.product((-1, 0, 1), repeat=4) if any(u) and any(v)]
+    for trial in range(6):
+        A = rng.standard_normal((3, 4))
+        f = ora.greedy_als(A, k=1, tau=0.7, seed=trial)
+        r = ora.refine_sweeps(A, f.B, f.D, f.C, sweeps=1, tau=0.7)
+        na = float(np.sum(A * A))
+
+        def best_decrease(u, v):   # 1-D least squares in the Frobenius inner product: <A,M>^2 / <M,M>
+            M = np.outer(_tf(u), _tf(v))
+            return float(np.sum(A * M)) ** 2 / float(np.sum(M * M))
+
+        top = max(best_decrease(u, v) for u, v in pairs)
+        stored = best_decrease(f.B[:, 0], f.C[0])
+        got = na - float(np.sum((A - ora.reconstruct(r.B, r.D, r.C)) ** 2))
+        assert stored - 1e-7 <= got <= top + 1e-9
+        assert 1.0 - float(np.sum((A - ora.reconstruct(r.B, r.D, r.C)) ** 2)) / na == \
+            pytest.approx(r.energy_final, abs=1e-12)
+
+
+@pytest.mark.parametrize("weighted", [False, True])
+def test_refinement_never_increases_the_residual(weighted):
+    """Every visit is non-increasing (the property the pages report for the sweeps);
+    the incremental energy equals the explicit one; sweeps gain energy on a Gaussian matrix."""
+    rng = np.random.default_rng(47)
+    A = rng.standard_normal((40, 56)) * 0.02
+    h = np.exp(1.5 * rng.standard_normal(56)) if weighted else None
+    k = ora.rank(40, 56, 1.5)
+    if weighted:
+        f = ora.greedy_als_weighted(A, h, 0.0, k=k, tau=1.0, seed=4)
+        hw = ora.normalized_weights(h, 0.0).astype(np.float64)
+    else:
+        f = ora.greedy_als(A, k=k, tau=1.0, seed=4)
+        hw = np.ones(56)
+    r = ora.refine_sweeps(A, f.B, f.D, f.C, sweeps=3, tau=1.0, h=h, track_residual=True)
+    before = float(np.sum(hw[None, :] * ora.residual_after(A, f.B, f.D, f.C, k) ** 2))
+    seq = np.concatenate([[before], r.visit_residuals.ravel()])
+    assert np.all(np.diff(seq) <= 1e-14 * before)
+    assert np.all(np.diff(np.concatenate([[f.energy_final], r.sweep_energy])) >= -1e-12)
+    assert r.sweep_energy[-1] == pytest.approx(r.energy_final, abs=1e-12)
+    assert r.energy_final > f.energy_final + 1e-4
+    Ahat = ora.reconstruct(r.B, r.D, r.C)
+    assert 1.0 - float(np.sum(hw[None, :] * (A - Ahat) ** 2)) / float(np.sum(hw[None, :] * A * A)) == \
+        pytest.approx(r.energy_final, abs=1e-12)
+
+
+def test_weighted_refinement_with_uniform_weights_is_the_plain_one():
+    A = np.random.default_rng(48).standard_normal((20, 28)) * 0.02
+    f = ora.greedy_als(A, k=30, tau=0.7, seed=2)
+    r = ora.refine_sweeps(A, f.B, f.D, f.C, sweeps=2, tau=0.7)
+    rw = ora.refine_sweeps(A, f.B, f.D, f.C, sweeps=2, tau=0.7, h=np.full(28, 4.0))
+    assert np.array_equal(r.B, rw.B) and np.array_equal(r.C, rw.C)
+    assert np.allclose(r.D, rw.D, rtol=1e-13, atol=0)
+    assert np.allclose(r.sweep_energy, rw.sweep_energy, rtol=0, atol=1e-12)
