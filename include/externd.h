@@ -218,6 +218,20 @@ typedef struct {
     int fault_skip_cta;    /* test hook, used only if fault_inject != 0: this CTA never signals */
     int fault_inject;
     double* d64_out;       /* nullable: k fp64 scales */
+    /* Refinement sweeps ("ExTernD: Expanded-Rank Ternary Decomposition", §2.4, "Refinement
+     * sweeps"), blocks of one component: after extraction every component i is revisited
+     * `sweeps` times in order: its term d_i u_i v_i^T is added back to the residual, refitted
+     * by the same alternation started from the stored u_i, and re-deflated.  The refit
+     * replaces the stored component only if its least-squares decrease of the added-back
+     * residual is at least that of the stored pair with its least-squares scale; otherwise
+     * the stored trits stay with that scale.  Every visit is therefore non-increasing in
+     * ||R||.  energy_out keeps the extraction energies; D/B/C hold the refined factors.
+     * Needs a lazy-deflation depth of at least 2 (EXTERND_ELIMIT otherwise). */
+    int sweeps;                /* 0 = none; at most 1000 */
+    double* sweep_energy_out;  /* nullable: `sweeps` doubles, the energy after each sweep */
+    /* Importance weights of §2.5 (see externd_factor_weighted); h = NULL: plain objective. */
+    const float* h;
+    double lambda;
 } externd_options;
 
 /* externd_factor with options (opt may be NULL). */
@@ -249,6 +263,7 @@ typedef struct {
     int pending;               /* lazy-deflation depth used */
     size_t smem_bytes;         /* dynamic shared memory per CTA */
     size_t workspace_bytes;
+    int64_t sweep_kept;        /* refinement visits that kept the stored pair (matrix 0) */
     int64_t phase_cycles[11];  /* [10]: exchanged words found not yet visible by CTA 0; [0..9]: SM cycles of CTA 0 of matrix 0 (diagnostics): GEMV loads, GEMV reduce +
                                   emit, publish, wait, partials + first loads, threshold, compaction,
                                   start vector, output + pending push, deflation fold */

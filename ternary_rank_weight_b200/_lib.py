@@ -39,6 +39,10 @@ class Options(ctypes.Structure):
         ("fault_skip_cta", ctypes.c_int),
         ("fault_inject", ctypes.c_int),
         ("d64_out", ctypes.c_void_p),
+        ("sweeps", ctypes.c_int),
+        ("sweep_energy_out", ctypes.c_void_p),
+        ("h", ctypes.c_void_p),
+        ("lambda_", ctypes.c_double),
     ]
 
 
@@ -63,6 +67,7 @@ class Stats(ctypes.Structure):
         ("pending", ctypes.c_int),
         ("smem_bytes", ctypes.c_size_t),
         ("workspace_bytes", ctypes.c_size_t),
+        ("sweep_kept", ctypes.c_int64),
         ("phase_cycles", ctypes.c_int64 * 11),
     ]
 

@@ -115,6 +115,7 @@ class Factors:
     tau: float
     d64: Optional[torch.Tensor] = None
     stats: dict = field(default_factory=dict)
+    sweep_energy: Optional[torch.Tensor] = None   # float64 [sweeps]: energy after each refinement sweep
 
     def trits(self):
         """Unpacked (B as m x k int8, C as k x n int8) on the host."""
@@ -125,10 +126,16 @@ class Factors:
 
 def factor(A, mu: float, tau: float, iters: int = 15, seed: int = 0, *, grid: int = 0, pending: int = 0,
            wait_limit_s: float = 0.0, fault_skip_cta: Optional[int] = None, want_d64: bool = False,
-           want_energy: bool = True, stream=None) -> Factors:
-    """Factor one matrix (externd_factor_ex).  Outputs are allocated where A lives."""
+           want_energy: bool = True, sweeps: int = 0, h=None, lam: float = 0.0, stream=None) -> Factors:
+    """Factor one matrix (externd_factor_ex).  Outputs are allocated where A lives.
+
+    sweeps: §2.4 refinement sweeps after extraction (``energy`` keeps the extraction
+    energies, ``sweep_energy`` the energy after each sweep).  h, lam: §2.5 importance
+    weights (per-column second moments, n float32 values), or None for the plain objective."""
     A = _as_matrix(A)
     m, n = A.shape
+    if h is not None:
+        h = _weights(h, n)
     k = rank(m, n, mu)
     if k < 1:
         raise ExterndError(STATUS["EINVAL"], "externd_rank")
@@ -144,13 +151,26 @@ def factor(A, mu: float, tau: float, iters: int = 15, seed: int = 0, *, grid: in
     opt.fault_inject = 1 if fault_skip_cta is not None else 0
     opt.fault_skip_cta = int(fault_skip_cta) if fault_skip_cta is not None else -1
     opt.d64_out = _ptr(d64)
+    SE = _empty((int(sweeps),), torch.float64, A) if sweeps > 0 else None
+    opt.sweeps = int(sweeps)
+    opt.sweep_energy_out = _ptr(SE)
+    opt.h = _ptr(h)
+    opt.lambda_ = float(lam)
     with _on_device(A):
         rc = _lib.load().externd_factor_ex(_ptr(A), m, n, float(mu), float(tau), int(iters), int(seed),
                                            _ptr(B), _ptr(D), _ptr(C), _ptr(E),
                                            _stream(stream, A.device), ctypes.byref(opt))
     _check(rc, "externd_factor")
     return Factors(B=B, D=D, C=C, energy=E, m=m, n=n, k=k, mu=float(mu), tau=float(tau), d64=d64,
-                   stats=last_stats())
+                   stats=last_stats(), sweep_energy=SE)
+
+
+def _weights(h, n: int) -> torch.Tensor:
+    if isinstance(h, np.ndarray):
+        h = torch.from_numpy(np.ascontiguousarray(h, dtype=np.float32))
+    if not isinstance(h, torch.Tensor) or h.dtype != torch.float32 or h.numel() != n:
+        raise ValueError("h must hold n float32 values")
+    return h.contiguous()
 
 
 def factor_weighted(A, h, mu: float, tau: float, lam: float = 0.0, iters: int = 15, seed: int = 0, *,
@@ -158,14 +178,10 @@ def factor_weighted(A, h, mu: float, tau: float, lam: float = 0.0, iters: int = 
     """Importance-weighted factorization (externd_factor_weighted, §2.5).
 
     h: per-column second moments (n,), float32, on the host or the GPU.  The returned
-    energy is the weighted energy."""
+    energy is the weighted energy.  (Refinement sweeps with weights: ``factor(..., h=h, sweeps=S)``.)"""
     A = _as_matrix(A)
     m, n = A.shape
-    if isinstance(h, np.ndarray):
-        h = torch.from_numpy(np.ascontiguousarray(h, dtype=np.float32))
-    if not isinstance(h, torch.Tensor) or h.dtype != torch.float32 or h.numel() != n:
-        raise ValueError("h must hold n float32 values")
-    h = h.contiguous()
+    h = _weights(h, n)
     k = rank(m, n, mu)
     if k < 1:
         raise ExterndError(STATUS["EINVAL"], "externd_rank")

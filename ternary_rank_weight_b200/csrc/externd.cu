@@ -1036,22 +1036,103 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
 }
 
 // Sum of one fp64 value per CTA of the group (fixed order), exchanged as tagged words.
+// `use` counts the calls of this group: consecutive calls alternate between two
+// buffers of Gg words and carry different tags, so a CTA that is already in call
+// j + 1 cannot overwrite a word another CTA still waits for in call j.  Every
+// exchange also orders: a CTA leaves it only after every CTA has entered it.
 __device__ bool exchange_sum(unsigned long long* sums, int q, int Gg, double v, const Smem& s, GroupSync* gs,
-                             uint64_t limit_ns, int* status, bool skip, double& out) {
+                             uint64_t limit_ns, int* status, bool skip, unsigned& use, double& out) {
+    ++use;
+    const unsigned tag = gen_tag(use);
+    unsigned long long* buf = sums + (size_t)(use & 1u) * Gg;
     const double t = block_sum(v, s.red);
-    if (threadIdx.x == 0 && !skip) st_relaxed_u64(sums + q, tag_value(t, 1u));
+    if (threadIdx.x == 0 && !skip) st_relaxed_u64(buf + q, tag_value(t, tag));
     int ok = 1;
     double x = 0.0;
-    if ((int)threadIdx.x < Gg) x = untag(wait_tagged(sums + threadIdx.x, 1u, gs, limit_ns, status, ok));
+    if ((int)threadIdx.x < Gg) x = untag(wait_tagged(buf + threadIdx.x, tag, gs, limit_ns, status, ok));
     ok = __syncthreads_and(ok);
     if (!ok) return false;
     out = block_sum(x, s.red);
     return true;
 }
 
+// Append the rank-1 term d u v^T (u, v: the masks nzU/sgU, nzV/sgV) as pending
+// lazy-deflation component L: full-length word-major masks for the dot products and
+// per-output bits for the corrections of this CTA's columns and rows.
+__device__ void push_pending(const Smem& s, int L, int Ls, double d, int Wm, int Wn, int64_t c0, int validV,
+                             int64_t r0, int validU) {
+    const int tid = threadIdx.x;
+    if (tid == 0) s.pd[L] = d;
+    for (int w = tid; w < Wm; w += NT) { s.pnzU[w * Ls + L] = s.nzU[w]; s.psgU[w * Ls + L] = s.sgU[w]; }
+    for (int w = tid; w < Wn; w += NT) { s.pnzV[w * Ls + L] = s.nzV[w]; s.psgV[w * Ls + L] = s.sgV[w]; }
+    for (int c = tid; c < validV; c += NT) {
+        const int64_t gc = c0 + c;
+        const uint32_t b = 1u << (gc & 31);
+        if (s.nzV[gc >> 5] & b) {
+            s.cnzV[c] |= 1u << L;
+            if (s.sgV[gc >> 5] & b) s.csgV[c] |= 1u << L;
+        }
+    }
+    for (int r = tid; r < validU; r += NT) {
+        const int64_t gr = r0 + r;
+        const uint32_t b = 1u << (gr & 31);
+        if (s.nzU[gr >> 5] & b) {
+            s.cnzU[r] |= 1u << L;
+            if (s.sgU[gr >> 5] & b) s.csgU[r] |= 1u << L;
+        }
+    }
+    __syncthreads();
+}
+
+// Start of a refinement visit of component i (§2.4, "Refinement sweeps"): load the
+// stored u_i, v_i (packed rows of B and C) and d_i, record d_i, n_old and the pending
+// slot in s.scal[8], [9], [11], and append the added-back term d_i u_i v_i^T as pending
+// component L with coefficient -d_i.  Leaves u = u_i in nzU/sgU/ulist and v = 0.
+// Returns nnz(u_i), or -1 if the group aborted.  Kept out of line: it runs once per
+// visit and would otherwise crowd the registers of the half-step loop.
+__device__ __noinline__ int refine_begin(const Prob& P, int64_t i, int q, int Gg, const KCfg& cfg, const Smem& s,
+                                         GroupSync* gs, bool skip, unsigned& sum_use, int L, int Ls, int Wm, int Wn,
+                                         int64_t c0, int validV, int64_t r0, int validU, int pitchU, int pitchV,
+                                         bool wtd) {
+    const int tid = threadIdx.x;
+    const int64_t m = P.m, n = P.n;
+    const int64_t kk = P.k;
+    // the stored component (written by the lead CTA at least one exchange ago;
+    // with k = 1 one more exchange orders it), read through L2
+    if (kk == 1) {
+        double unused;
+        if (!exchange_sum(P.sums, q, Gg, 0.0, s, gs, cfg.limit_ns, P.status, skip, sum_use, unused))
+            return -1;
+    }
+    __threadfence();
+    const int nV0 = build_from_trits(reinterpret_cast<const uint32_t*>(P.C + i * P.c_bytes), P.c_bytes / 4, n, s.nzV,
+                                     s.sgV, s.vlist, pitchU, s);
+    const int nU0 = build_from_trits(reinterpret_cast<const uint32_t*>(P.B + i * P.b_bytes), P.b_bytes / 4, m, s.nzU,
+                                     s.sgU, s.ulist, pitchV, s);
+    double hv0 = (double)nV0;   // v_i^T diag(h~) v_i (nnz(v_i) for the plain objective)
+    if (wtd) {
+        double acc = 0.0;
+        for (int w = tid; w < Wn; w += NT)
+            for (uint32_t mk = s.nzV[w]; mk; mk &= mk - 1u)
+                acc += (double)__ldg(P.hw + ((int64_t)w << 5) + __ffs(mk) - 1);
+        hv0 = block_sum(acc, s.red);
+    }
+    const double di = __ldcg(P.dk + i);
+    if (tid == 0) {
+        s.scal[8] = di;
+        s.scal[9] = (double)nU0 * hv0;
+        s.scal[11] = (double)L;
+    }
+    // add d_i u_i v_i^T back: a pending term with coefficient -d_i
+    push_pending(s, L, Ls, -di, Wm, Wn, c0, validV, r0, validU);
+    for (int w = tid; w < Wn; w += NT) { s.nzV[w] = 0u; s.sgV[w] = 0u; }
+    __syncthreads();
+    return nU0;
+}
+
 // Factor (or run one debug half-step of) one matrix with this CTA group.
 // Returns false if the group aborted.
-template <bool WTD>
+template <bool WTD, bool SWP>
 __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s, GroupSync* gs, unsigned& arrivals) {
     const int64_t m = P.m, n = P.n;
     const int Wm = (int)((m + 31) >> 5), Wn = (int)((n + 31) >> 5);
@@ -1098,6 +1179,11 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
     int L = 0;
     unsigned long long sum_nu = 0, sum_nv = 0, sum_du = 0, sum_dv = 0, sum_nunv = 0, hs = 0, fb = 0;
     const int64_t kk = (mode == MODE_FACTOR) ? P.k : 1;
+    // §2.4 refinement sweeps: visits kk .. nvis-1 revisit components 0 .. kk-1 in order
+    const int S = (SWP && mode == MODE_FACTOR) ? P.sweeps : 0;
+    const int64_t nvis = kk * (int64_t)(1 + S);
+    unsigned sum_use = 0;                  // calls of exchange_sum by this group
+    unsigned long long kept = 0;           // refinement visits that kept the stored pair
     int nU = 0, nV = 0, dU = 0, dV = 0;   // support sizes and list lengths (trit changes)
     double hsv = 0.0;                     // weighted objective: sum of h~ over the support of v
     double p = 0.0, thr;
@@ -1109,14 +1195,27 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
         s.clk[11] = (unsigned long long)clock64();
     }
 
-    for (int64_t i = 0; i < kk; ++i) {
+    for (int64_t vis = 0; vis < nvis; ++vis) {
+        const int64_t i = vis % kk;
+        const bool refine = SWP && vis >= kk;   // a refinement visit of component i
+        // refinement state in shared memory (s.scal[8..11]): d_i, n_old = nnz(u_i) v_i^T diag(h~) v_i,
+        // this CTA's part of p_old, and the pending slot of the added-back term
         // a new component: the GEMV sums restart from zero and the previous trits
         // of the output vectors are zero, so the first lists hold whole supports
         for (int c = tid; c < pitchV; c += NT) s.gV[c] = 0.0;
         for (int c = tid; c < pitchU; c += NT) s.gU[c] = 0.0;
         if (mode != MODE_HALF_U) {
-            for (int w = tid; w < Wn; w += NT) { s.nzV[w] = 0u; s.sgV[w] = 0u; }
-            nU = build_from_trits(P.start + i * P.start_words, P.start_words, m, s.nzU, s.sgU, s.ulist, pitchV, s);
+            if constexpr (SWP) if (refine) {
+                const int nU0 = refine_begin(P, i, q, Gg, cfg, s, gs, skip, sum_use, L, Ls, Wm, Wn, c0, validV, r0,
+                                             validU, pitchU, pitchV, wtd);
+                if (nU0 < 0) return false;
+                ++L;
+                nU = nU0;   // the refit starts from the stored u
+            }
+            if (!refine) {
+                for (int w = tid; w < Wn; w += NT) { s.nzV[w] = 0u; s.sgV[w] = 0u; }
+                nU = build_from_trits(P.start + i * P.start_words, P.start_words, m, s.nzU, s.sgU, s.ulist, pitchV, s);
+            }
             dU = nU;
             if (L > 0) pending_coef(L, Ls, Wm, s.pnzU, s.psgU, s.nzU, s.sgU, s.pd, s.dotU, s.coef);
             for (int l = tid; l < L; l += NT) {
@@ -1145,6 +1244,20 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
                                                    s.dotV, s.coefV, false, thr, dV, gs, cfg.limit_ns, P.status, ok,
                                                    wtd ? P.hw : nullptr, wtd ? s.vwl : nullptr, s.dotVw, &hsv);
                 if (!ok) return false;
+                if constexpr (SWP) if (refine && it == 0) {
+                    // u_i^T R (h~ v_i) of the added-back residual: x = R^T u_i at this CTA's columns
+                    const int La = (int)s.scal[11];
+                    double pold_part = 0.0;
+                    for (int c = tid; c < validV; c += NT) {
+                        if ((s.cnzV[c] >> La) & 1u) {
+                            double x = untag(ld_relaxed_u64(P.xbuf + c0 + c));
+                            if (wtd) x *= (double)__ldg(P.hw + c0 + c);
+                            pold_part += ((s.csgV[c] >> La) & 1u) ? -x : x;
+                        }
+                    }
+                    pold_part = block_sum(pold_part, s.red);
+                    if (tid == 0) s.scal[10] = pold_part;
+                }
                 fb += (s.scal[1] != 0.0) ? 1 : 0;
                 sum_nu += (unsigned long long)nU;
                 sum_du += (unsigned long long)dU;
@@ -1192,42 +1305,59 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
         }
         // ---- scale (§2.3 step 2): d = u^T R v / (nnz(u) nnz(v)), with u^T R v = u^T y = p;
         //      weighted (§2.5): d = u^T R (h~ v) / (nnz(u) sum_{v != 0} h~), the decrease p d
-        const double d = (p == 0.0) ? 0.0 : p / ((double)nU * (wtd ? hsv : (double)nV));
-        RN2 -= p * d;
+        const double dnew = (p == 0.0) ? 0.0 : p / ((double)nU * (wtd ? hsv : (double)nV));
+        double d = dnew;
+        bool take = true;   // store the refit (always, outside refinement)
+        if constexpr (SWP) if (refine) {
+            // §2.4 refinement: the residual grew by the added-back term,
+            // ||R + d_i u_i v_i^T||^2 = ||R||^2 + 2 d_i p_old - d_i^2 n_old with p_old = u_i^T R_added (h~ v_i);
+            // keep the refit if its decrease p dnew is at least the stored pair's p_old^2 / n_old
+            const double di = s.scal[8], n_old = s.scal[9];
+            const int La = (int)s.scal[11];
+            double pold = 0.0;
+            if (!exchange_sum(P.sums, q, Gg, tid == 0 ? s.scal[10] : 0.0, s, gs, cfg.limit_ns, P.status, skip, sum_use,
+                              pold))
+                return false;
+            RN2 += 2.0 * di * pold - di * di * n_old;
+            const double dold = (pold == 0.0 || n_old == 0.0) ? 0.0 : pold / n_old;
+            take = (p * dnew >= pold * dold);
+            if (take) {
+                RN2 -= p * dnew;
+            } else {
+                RN2 -= pold * dold;
+                d = dold;
+                ++kept;
+                if (tid == 0) s.pd[La] = dold - di;   // net pending term of the stored pair
+            }
+        }
+        if (!refine) RN2 -= p * dnew;
         sum_nunv += (unsigned long long)nU * (unsigned long long)nV;
         if (lead) {
-            pack_row(s.nzU, s.sgU, Wm, reinterpret_cast<uint32_t*>(P.B + i * P.b_bytes), P.b_bytes / 4);
-            pack_row(s.nzV, s.sgV, Wn, reinterpret_cast<uint32_t*>(P.C + i * P.c_bytes), P.c_bytes / 4);
+            if (take) {
+                pack_row(s.nzU, s.sgU, Wm, reinterpret_cast<uint32_t*>(P.B + i * P.b_bytes), P.b_bytes / 4);
+                pack_row(s.nzV, s.sgV, Wn, reinterpret_cast<uint32_t*>(P.C + i * P.c_bytes), P.c_bytes / 4);
+            }
             if (tid == 0) {
                 P.D[i] = (float)d;
-                if (P.energy) P.energy[i] = 1.0 - RN2 / N0;
+                if (P.energy && !refine) P.energy[i] = 1.0 - RN2 / N0;
                 if (P.d64) P.d64[i] = d;
+                if (P.dk) P.dk[i] = d;
+                if (refine && i == kk - 1 && P.sweep_energy) P.sweep_energy[vis / kk - 1] = 1.0 - RN2 / N0;
             }
+            if (S > 0) __threadfence();   // the other CTAs re-read this component in the next sweep
         }
         // ---- deflation (§2.3 step 3), held lazily as a pending rank-1 term
-        if (tid == 0) s.pd[L] = d;
-        for (int w = tid; w < Wm; w += NT) { s.pnzU[w * Ls + L] = s.nzU[w]; s.psgU[w * Ls + L] = s.sgU[w]; }
-        for (int w = tid; w < Wn; w += NT) { s.pnzV[w * Ls + L] = s.nzV[w]; s.psgV[w * Ls + L] = s.sgV[w]; }
-        for (int c = tid; c < validV; c += NT) {
-            const int64_t gc = c0 + c;
-            const uint32_t b = 1u << (gc & 31);
-            if (s.nzV[gc >> 5] & b) {
-                s.cnzV[c] |= 1u << L;
-                if (s.sgV[gc >> 5] & b) s.csgV[c] |= 1u << L;
-            }
+        if (take) {
+            push_pending(s, L, Ls, d, Wm, Wn, c0, validV, r0, validU);
+            ++L;
+        } else {
+            __syncthreads();
         }
-        for (int r = tid; r < validU; r += NT) {
-            const int64_t gr = r0 + r;
-            const uint32_t b = 1u << (gr & 31);
-            if (s.nzU[gr >> 5] & b) {
-                s.cnzU[r] |= 1u << L;
-                if (s.sgU[gr >> 5] & b) s.csgU[r] |= 1u << L;
-            }
-        }
-        ++L;
-        __syncthreads();
         phase_mark(s, 8);
-        if (L == cfg.Lcap || i == kk - 1) {
+        // room for the next visit's terms (two during refinement; extraction folds on the
+        // plain schedule, so its rounding is that of a run without sweeps), and R folded
+        // at the end of the extraction and of the run
+        if (L + (vis + 1 >= kk ? 2 : 1) > cfg.Lcap || vis == kk - 1 || vis == nvis - 1) {
             uint32_t* scratch = reinterpret_cast<uint32_t*>(s.red);
             flush_dispatch(P.pv.vec, blkV, pitchV, m, validV, L, Ls, s.pd, s.pnzU, s.psgU, s.cnzV, s.csgV, scratch);
             flush_dispatch(P.pu.vec, blkU, pitchU, n, validU, L, Ls, s.pd, s.pnzV, s.psgV, s.cnzU, s.csgU, scratch);
@@ -1252,7 +1382,7 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
         }
     }
     double R2 = 0.0;
-    if (!exchange_sum(P.sums, q, Gg, rs, s, gs, cfg.limit_ns, P.status, skip, R2)) return false;
+    if (!exchange_sum(P.sums, q, Gg, rs, s, gs, cfg.limit_ns, P.status, skip, sum_use, R2)) return false;
     if (lead && tid == 0) {
         P.stats->sum_nu = sum_nu;
         P.stats->sum_nv = sum_nv;
@@ -1263,6 +1393,7 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
         P.stats->fallbacks = fb;
         P.stats->residual2 = R2;
         P.stats->norm_a2 = N0;
+        P.stats->sweep_kept = kept;
         phase_mark(s, 7);
         for (int k2 = 0; k2 < 11; ++k2) P.stats->phase[k2] = s.clk[k2];
         __threadfence();
@@ -1272,7 +1403,7 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
     return true;
 }
 
-template <bool WTD>
+template <bool WTD, bool SWP>
 __global__ void __launch_bounds__(NT, 1) als_kernel(const KCfg cfg) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int grp = blockIdx.x / cfg.Gg;
@@ -1327,11 +1458,17 @@ __global__ void __launch_bounds__(NT, 1) als_kernel(const KCfg cfg) {
     GroupSync* gs = cfg.gsync + grp;
     unsigned arrivals = 0;   // exchanges this CTA took part in (counter targets)
     for (int pi = grp; pi < cfg.nprob; pi += cfg.NG) {
-        if (!run_problem<WTD>(cfg.probs[pi], q, cfg, s, gs, arrivals)) return;
+        if (!run_problem<WTD, SWP>(cfg.probs[pi], q, cfg, s, gs, arrivals)) return;
     }
 }
 
 // Writes one problem descriptor and its running status into a caller-fixed workspace.
+// The four instantiations: importance weights (§2.5) x refinement sweeps (§2.4).
+static const void* als_fn(int weighted, int sweeping) {
+    if (weighted) return sweeping ? (const void*)als_kernel<true, true> : (const void*)als_kernel<true, false>;
+    return sweeping ? (const void*)als_kernel<false, true> : (const void*)als_kernel<false, false>;
+}
+
 __global__ void init_control_kernel(const Prob p, Prob* dst, int* status) {
     if (threadIdx.x == 0) {
         *dst = p;
@@ -1429,8 +1566,12 @@ int dev_info(DevInfo& out) {
         d.smem_optin = (size_t)v;
         if (cudaDeviceGetAttribute(&v, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess) { cudaGetLastError(); return EXTERND_ECUDA; }
         d.coop = v;
-        if (cudaFuncSetAttribute(als_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)d.smem_optin) != cudaSuccess ||
-            cudaFuncSetAttribute(als_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)d.smem_optin) != cudaSuccess) {
+        bool attr_ok = true;
+        for (int w = 0; w < 2; ++w)
+            for (int sw = 0; sw < 2; ++sw)
+                attr_ok = attr_ok && cudaFuncSetAttribute(als_fn(w, sw), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                          (int)d.smem_optin) == cudaSuccess;
+        if (!attr_ok) {
             cudaGetLastError();
             return EXTERND_ECUDA;
         }
@@ -1505,6 +1646,8 @@ struct ProbIn {
     uint8_t* C;
     double* energy;
     double* d64;
+    int sweeps;           // §2.4 refinement sweeps (MODE_FACTOR only)
+    double* sweep_energy; // nullable, sweeps values
     int mode;
     const uint8_t* dbg_in;
     double* pre_out;
@@ -1602,12 +1745,15 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
     weighted = weighted ? 1 : 0;
     while (Lcap > 1 && als_smem_bytes(m_max, n_max, Lcap, pv_max, pu_max, weighted) > di.smem_optin) --Lcap;
     if (opt.pending > 0 && opt.pending < Lcap) Lcap = opt.pending;
+    for (int b = 0; b < np; ++b)
+        if (in[b].mode == MODE_FACTOR && in[b].sweeps > 0 && Lcap < 2) return EXTERND_ELIMIT;   // add-back + refit
     const size_t smem = als_smem_bytes(m_max, n_max, Lcap, pv_max, pu_max, weighted);
     if (smem > di.smem_optin) return EXTERND_ELIMIT;
 
     int nb = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, weighted ? als_kernel<true> : als_kernel<false>, NT, smem) !=
-        cudaSuccess) {
+    int sweeping = 0;
+    for (int b = 0; b < np; ++b) sweeping |= (in[b].mode == MODE_FACTOR && in[b].sweeps > 0);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, als_fn(weighted, sweeping), NT, smem) != cudaSuccess) {
         cudaGetLastError();
         return EXTERND_ECUDA;
     }
@@ -1616,7 +1762,8 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
     // ---- plan the workspace
     std::vector<Prob> probs(np);
     std::vector<size_t> off_rv(np), off_ru(np), off_x(np), off_y(np), off_sums(np), off_start(np), off_norm(np), off_A(np),
-        off_B(np), off_C(np), off_D(np), off_E(np), off_d64(np), off_pre(np), off_thr(np), off_tro(np), off_hw(np), off_h(np);
+        off_B(np), off_C(np), off_D(np), off_E(np), off_d64(np), off_pre(np), off_thr(np), off_tro(np), off_hw(np), off_h(np),
+        off_dk(np), off_SE(np);
     size_t ctl = 0;
     const size_t off_gsync = ctl;
     ctl += round_up(sizeof(GroupSync) * NG, 256);
@@ -1647,7 +1794,7 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
         // exchange buffers: zero = "no half-step yet" (tags are 1..255)
         off_x[b] = ws; ws += round_up(sizeof(unsigned long long) * (size_t)I.n, 256);
         off_y[b] = ws; ws += round_up(sizeof(unsigned long long) * (size_t)I.m, 256);
-        off_sums[b] = ws; ws += round_up(sizeof(unsigned long long) * (size_t)Gg * 3, 256);
+        off_sums[b] = ws; ws += round_up(sizeof(unsigned long long) * (size_t)Gg * 4, 256);   // sums x2, partV, partU
     }
     const size_t zero_to = ws;
     for (int b = 0; b < np; ++b) {
@@ -1665,6 +1812,13 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
         off_A[b] = SIZE_MAX;
         if (I.A && !is_device_ptr(I.A)) { off_A[b] = ws; ws += round_up(sizeof(float) * (size_t)(I.m * I.n), 256); }
         off_B[b] = off_C[b] = off_D[b] = off_E[b] = off_d64[b] = off_pre[b] = off_thr[b] = off_tro[b] = SIZE_MAX;
+        off_dk[b] = off_SE[b] = SIZE_MAX;
+        if (I.mode == MODE_FACTOR && !opt.init_only && I.sweeps > 0) {
+            off_dk[b] = ws; ws += round_up(sizeof(double) * (size_t)I.k, 256);
+            if (I.sweep_energy && !is_device_ptr(I.sweep_energy)) {
+                off_SE[b] = ws; ws += round_up(sizeof(double) * (size_t)I.sweeps, 256);
+            }
+        }
         if (I.mode == MODE_FACTOR && !opt.init_only) {
             if (!is_device_ptr(I.B)) { off_B[b] = ws; ws += round_up((size_t)(I.k * P.b_bytes), 256); }
             if (!is_device_ptr(I.C)) { off_C[b] = ws; ws += round_up((size_t)(I.k * P.c_bytes), 256); }
@@ -1685,7 +1839,7 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
         for (int b = 0; b < np; ++b)
             if (off_A[b] != SIZE_MAX || off_B[b] != SIZE_MAX || off_C[b] != SIZE_MAX || off_D[b] != SIZE_MAX ||
                 off_E[b] != SIZE_MAX || off_d64[b] != SIZE_MAX || off_pre[b] != SIZE_MAX || off_thr[b] != SIZE_MAX ||
-                off_tro[b] != SIZE_MAX)
+                off_tro[b] != SIZE_MAX || off_SE[b] != SIZE_MAX)
                 return EXTERND_EINVAL;   // host buffers would need staging memory
         if (ws > fixed->cap) return EXTERND_ELIMIT;
     }
@@ -1716,8 +1870,8 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
         P.xbuf = reinterpret_cast<unsigned long long*>(dws + off_x[b]);
         P.ybuf = reinterpret_cast<unsigned long long*>(dws + off_y[b]);
         P.sums = reinterpret_cast<unsigned long long*>(dws + off_sums[b]);
-        P.partV = P.sums + Gg;
-        P.partU = P.sums + 2 * Gg;
+        P.partV = P.sums + 2 * Gg;
+        P.partU = P.sums + 3 * Gg;
         P.start = reinterpret_cast<uint32_t*>(dws + off_start[b]);
         P.norm_part = reinterpret_cast<double*>(dws + off_norm[b]);
         P.nonfinite = reinterpret_cast<unsigned*>(dws + off_nonfin) + 2 * b;
@@ -1729,6 +1883,10 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
             P.D = off_D[b] == SIZE_MAX ? I.D : reinterpret_cast<float*>(dws + off_D[b]);
             P.energy = off_E[b] == SIZE_MAX ? I.energy : reinterpret_cast<double*>(dws + off_E[b]);
             P.d64 = off_d64[b] == SIZE_MAX ? I.d64 : reinterpret_cast<double*>(dws + off_d64[b]);
+            P.sweeps = off_dk[b] == SIZE_MAX ? 0 : I.sweeps;
+            P.dk = off_dk[b] == SIZE_MAX ? nullptr : reinterpret_cast<double*>(dws + off_dk[b]);
+            P.sweep_energy = off_SE[b] == SIZE_MAX ? (P.sweeps ? I.sweep_energy : nullptr)
+                                                   : reinterpret_cast<double*>(dws + off_SE[b]);
         } else {
             P.pre_out = off_pre[b] == SIZE_MAX ? I.pre_out : reinterpret_cast<double*>(dws + off_pre[b]);
             P.thr_out = off_thr[b] == SIZE_MAX ? I.thr_out : reinterpret_cast<double*>(dws + off_thr[b]);
@@ -1810,7 +1968,7 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
             cfg.fault_skip = opt.fault_skip;
             cfg.weighted = weighted;
             void* args[] = {&cfg};
-            CK(cudaLaunchCooperativeKernel(weighted ? (void*)als_kernel<true> : (void*)als_kernel<false>, dim3((unsigned)(NG * Gg)), dim3(NT), args, smem, stream));
+            CK(cudaLaunchCooperativeKernel(als_fn(weighted, sweeping), dim3((unsigned)(NG * Gg)), dim3(NT), args, smem, stream));
             ++launches;
         }
         if (ev[3]) CK(cudaEventRecord(ev[3], stream));
@@ -1830,6 +1988,8 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
         if (off_D[b] != SIZE_MAX) CK(cudaMemcpyAsync(I.D, P.D, sizeof(float) * (size_t)I.k, cudaMemcpyDeviceToHost, stream));
         if (off_E[b] != SIZE_MAX) CK(cudaMemcpyAsync(I.energy, P.energy, sizeof(double) * (size_t)I.k, cudaMemcpyDeviceToHost, stream));
         if (off_d64[b] != SIZE_MAX) CK(cudaMemcpyAsync(I.d64, P.d64, sizeof(double) * (size_t)I.k, cudaMemcpyDeviceToHost, stream));
+        if (off_SE[b] != SIZE_MAX)
+            CK(cudaMemcpyAsync(I.sweep_energy, P.sweep_energy, sizeof(double) * (size_t)I.sweeps, cudaMemcpyDeviceToHost, stream));
         if (I.mode != MODE_FACTOR) {
             const int64_t lout = I.mode == MODE_HALF_V ? I.n : I.m;
             if (off_pre[b] != SIZE_MAX) CK(cudaMemcpyAsync(I.pre_out, P.pre_out, sizeof(double) * (size_t)lout, cudaMemcpyDeviceToHost, stream));
@@ -1878,6 +2038,7 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
             if (b == 0) {
                 st.residual_energy = d.norm_a2 > 0 ? 1.0 - d.residual2 / d.norm_a2 : 0.0;
                 for (int k2 = 0; k2 < 11; ++k2) st.phase_cycles[k2] = (int64_t)d.phase[k2];
+                st.sweep_kept = (int64_t)d.sweep_kept;
             }
         }
     }
@@ -1981,6 +2142,14 @@ int externd_factor_ex(const float* A, int64_t m, int64_t n, double mu, double ta
         if (opt->wait_limit_s > 0) ro.wait_limit_s = opt->wait_limit_s;
         ro.fault_skip = opt->fault_inject ? opt->fault_skip_cta : -1;
         I.d64 = opt->d64_out;
+        if (opt->sweeps < 0 || opt->sweeps > 1000) return EXTERND_EINVAL;
+        I.sweeps = opt->sweeps;
+        I.sweep_energy = opt->sweep_energy_out;
+        if (opt->h) {
+            if (!std::isfinite(opt->lambda) || opt->lambda < 0.0) return EXTERND_EINVAL;
+            I.h = opt->h;
+            I.lambda = opt->lambda;
+        }
     }
     int st = 0;
     return run(&I, 1, ro, reinterpret_cast<cudaStream_t>(stream), &st);

@@ -103,6 +103,7 @@ struct DevStats {
     double norm_a2;
     double pad;
     unsigned long long phase[11];   // SM cycles of CTA 0 per phase (see run_problem); [10] stale words seen
+    unsigned long long sweep_kept;  // refinement visits that kept the stored pair (rescaled)
 };
 
 enum Mode { MODE_FACTOR = 0, MODE_HALF_V = 1, MODE_HALF_U = 2 };
@@ -120,12 +121,15 @@ struct Prob {
     uint8_t* C;               // k rows of c_bytes
     double* energy;           // nullable
     double* d64;              // nullable
+    int sweeps;               // §2.4 refinement sweeps after extraction (0 = none)
+    double* dk;               // k fp64 scales every CTA re-reads during sweeps (workspace; null without sweeps)
+    double* sweep_energy;     // nullable: energy after each sweep
     int64_t b_bytes, c_bytes;
     float* Rv;                // V-layout blocks
     float* Ru;                // U-layout blocks
     unsigned long long* xbuf; // n, published V-step outputs (tagged fp64 words, zero-initialised)
     unsigned long long* ybuf; // m, published U-step outputs (tagged fp64 words, zero-initialised)
-    unsigned long long* sums; // G, per-CTA partial sums of the final residual (tagged, zero-initialised)
+    unsigned long long* sums; // 2 G, per-CTA partial sums, double-buffered by use (tagged, zero-initialised)
     unsigned long long* partV;// G, per-CTA sum |out| of the V-step (tagged, zero-initialised)
     unsigned long long* partU;// G, same for the U-step
     const uint32_t* start;    // start trits (k rows of start_words) or debug input (1 row)

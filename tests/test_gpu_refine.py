@@ -1,0 +1,132 @@
+"""Parity of the refinement sweeps (§2.4, blocks of one component) with the oracle.
+
+Teacher forcing: the kernel is deterministic, so the extraction inside a run with
+sweeps equals a run without them (checked); the oracle's sweeps start from those
+GPU factors (fp64 scales).  A component is compared as a rank-1 term, so (u, v, d)
+and (u, -v, -d) are the same.  Tolerances are the extraction's: trits equal and d
+within 1e-4 relative until the first visit that differs, which must start at a
+near-tie of the oracle (a threshold margin below 1e-3 relative, or a refit/stored
+decision within 1e-6 relative); energies within 2e-3 (1e-5 before any divergence).
+"""
+import numpy as np
+import pytest
+import torch
+
+import ternary_rank_weight_b200 as ext
+from oracle import externd_oracle as ora
+from ternary_rank_weight_b200.workloads import importance_weights, llm_matrix
+
+pytestmark = pytest.mark.gpu
+
+
+def _canonical(B, D, C):
+    """Flip (u, v, d) with d < 0 to (u, -v, -d)."""
+    sgn = np.where(np.asarray(D) < 0, -1, 1)
+    return B.copy(), np.abs(np.asarray(D, dtype=np.float64)), (C * sgn[:, None].astype(np.int8))
+
+
+def _run(A, mu, tau, seed, sweeps, h=None):
+    Ag = torch.from_numpy(A).cuda()
+    base = ext.factor(Ag, mu, tau, seed=seed, want_d64=True, h=h)
+    ref = ext.factor(Ag, mu, tau, seed=seed, want_d64=True, sweeps=sweeps, h=h)
+    return base, ref
+
+
+def _check_one_sweep(A, base, ref, tau, h=None):
+    B0, C0 = base.trits()
+    D0 = base.d64.cpu().numpy()
+    want = ora.refine_sweeps(A, B0, D0, C0, sweeps=1, tau=tau, h=h)
+    B1, C1 = ref.trits()
+    gb, gd, gc = _canonical(B1, ref.d64.cpu().numpy(), C1)
+    ob, od, oc = _canonical(want.B, want.D, want.C)
+    k = base.k
+    div = k
+    for i in range(k):
+        if not (np.array_equal(gb[:, i], ob[:, i]) and np.array_equal(gc[i], oc[i])):
+            div = i
+            break
+    if div > 0:
+        assert np.allclose(gd[:div], od[:div], rtol=1e-4, atol=1e-12)
+    if div < k:
+        near = want.margins[0, div] < 1e-3 or want.decision_margins[0, div] < 1e-6
+        assert near, (div, want.margins[0, div], want.decision_margins[0, div])
+        assert abs(ref.sweep_energy[0].item() - want.sweep_energy[0]) < 2e-3
+    else:
+        assert abs(ref.sweep_energy[0].item() - want.sweep_energy[0]) < 1e-5
+    return want, div
+
+
+@pytest.mark.parametrize("m,n,mu,tau", [(7, 5, 2.0, 0.7), (33, 65, 1.5, 1.0), (96, 160, 2.0, 1.0),
+                                        (160, 96, 1.0, 0.7), (256, 256, 2.0, 0.7)])
+def test_one_sweep_matches_oracle(m, n, mu, tau):
+    A = llm_matrix(m, n, seed=m * 3 + n, outliers=min(2, n))
+    base, ref = _run(A, mu, tau, seed=5, sweeps=1)
+    # the extraction inside the refined run is the plain one, bit for bit
+    assert torch.equal(base.energy, ref.energy)
+    _, div = _check_one_sweep(A, base, ref, tau)
+    assert ref.sweep_energy[0].item() >= base.energy[-1].item() - 1e-9
+    # the refined factors reproduce the reported energy
+    Ah = ext.reconstruct(ref.B, ref.D, ref.C, m, n).cpu().numpy()
+    assert ora.energy(A, Ah) == pytest.approx(ref.sweep_energy[-1].item(), abs=1e-4)
+    assert ref.stats["residual_energy"] == pytest.approx(ref.sweep_energy[-1].item(), abs=1e-5)
+
+
+def test_weighted_sweep_matches_oracle():
+    m, n = 128, 192
+    A = llm_matrix(m, n, seed=21, outliers=2)
+    h = importance_weights(n, seed=22)
+    base, ref = _run(A, 1.5, 1.0, seed=3, sweeps=1, h=h)
+    assert torch.equal(base.energy, ref.energy)
+    _check_one_sweep(A, base, ref, 1.0, h=h.astype(np.float64))
+    hw = ora.normalized_weights(h.astype(np.float64), 0.0)
+    Ah = ext.reconstruct(ref.B, ref.D, ref.C, m, n).cpu().numpy()
+    assert ora.weighted_energy(A, Ah, hw) == pytest.approx(ref.sweep_energy[-1].item(), abs=1e-4)
+
+
+@pytest.mark.parametrize("m,n", [(4, 4), (1, 9), (40, 3)])
+def test_single_component_sweeps(m, n):
+    """k = 1: every visit re-reads the component written by the previous one."""
+    A = llm_matrix(m, n, seed=m + 7 * n, outliers=0)
+    mu = 1.0 / min(m, n)
+    base, ref = _run(A, mu, 1.0, seed=1, sweeps=3)
+    assert base.k == 1
+    B0, C0 = base.trits()
+    want = ora.refine_sweeps(A, B0, base.d64.cpu().numpy(), C0, sweeps=3, tau=1.0)
+    np.testing.assert_allclose(ref.sweep_energy.cpu().numpy(), want.sweep_energy, atol=1e-6)
+    B1, C1 = ref.trits()
+    gb, gd, gc = _canonical(B1, ref.d64.cpu().numpy(), C1)
+    ob, od, oc = _canonical(want.B, want.D, want.C)
+    assert np.array_equal(gb, ob) and np.array_equal(gc, oc)
+    assert np.allclose(gd, od, rtol=1e-6)
+
+
+def test_several_sweeps_are_monotone_and_track_the_oracle():
+    m, n = 192, 256
+    A = llm_matrix(m, n, seed=31, outliers=2)
+    base, ref = _run(A, 1.5, 1.0, seed=2, sweeps=4)
+    se = ref.sweep_energy.cpu().numpy()
+    assert np.all(np.diff(np.concatenate([[base.energy[-1].item()], se])) >= -1e-9)
+    B0, C0 = base.trits()
+    want = ora.refine_sweeps(A, B0, base.d64.cpu().numpy(), C0, sweeps=4, tau=1.0)
+    assert np.max(np.abs(se - want.sweep_energy)) < 2e-3
+    assert ref.stats["sweep_kept"] >= 0
+    Ah = ext.reconstruct(ref.B, ref.D, ref.C, m, n).cpu().numpy()
+    assert ora.energy(A, Ah) == pytest.approx(se[-1], abs=1e-4)
+
+
+def test_sweeps_with_small_pending_depth_and_host_buffers():
+    """Depth 2 folds after every visit; host (pinned) inputs stage through the call."""
+    A = llm_matrix(64, 80, seed=41, outliers=1)
+    Ah = torch.from_numpy(A).pin_memory()
+    f2 = ext.factor(Ah, 1.5, 0.7, seed=4, sweeps=2, pending=2, want_d64=True)
+    fd = ext.factor(torch.from_numpy(A).cuda(), 1.5, 0.7, seed=4, sweeps=2, want_d64=True)
+    assert f2.sweep_energy is not None and not f2.sweep_energy.is_cuda
+    # a different fold schedule changes fp32 rounding only
+    assert np.max(np.abs(f2.sweep_energy.numpy() - fd.sweep_energy.cpu().numpy())) < 2e-3
+    with pytest.raises(ext.ExterndError) as e:
+        ext.factor(Ah, 1.5, 0.7, sweeps=1, pending=1)
+    assert e.value.status == ext.STATUS["ELIMIT"]
+    for bad in (-1, 1001):
+        with pytest.raises(ext.ExterndError) as e:
+            ext.factor(Ah, 1.5, 0.7, sweeps=bad)
+        assert e.value.status == ext.STATUS["EINVAL"]
