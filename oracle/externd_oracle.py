@@ -466,14 +466,59 @@ class Refinement:
     visit_residuals: np.ndarray = field(default=None)  # sweeps x k explicit residual norms after each visit
 
 
+@dataclass
+class Visit:
+    u: np.ndarray
+    v: np.ndarray
+    d: float
+    kept: bool             # the stored pair stayed (with its least-squares scale)
+    p_old: float           # u_i^T R (h~ v_i) of the added-back residual
+    n_old: float           # nnz(u_i) * sum_{v_i != 0} h~
+    decrease: float        # decrease of the (weighted) squared residual by the chosen term
+    margin: float          # closest approach of the refit's half-steps to a threshold tie
+    decision_margin: float
+
+
+def refine_visit(R: np.ndarray, ui: np.ndarray, vi: np.ndarray, tau: float, iters: int, hw: np.ndarray) -> Visit:
+    """One §2.4 visit on the added-back residual R = R_prev + d_i u_i v_i^T: refit from u_i
+    (V-step on R, U-step on R diag(h~)), then take the refit or the stored pair, whichever
+    decreases the residual more with its least-squares scale (ties go to the refit)."""
+    uf = np.asarray(ui, dtype=np.float64)
+    vf = np.asarray(vi, dtype=np.float64)
+    p_old = float(uf @ (R @ (hw * vf)))
+    n_old = float(np.count_nonzero(ui)) * float(np.sum(hw[vf != 0]))
+    d_old = 0.0 if (p_old == 0.0 or n_old == 0.0) else p_old / n_old
+    dec_old = p_old * d_old
+    u = np.asarray(ui, dtype=np.int8).copy()
+    v = None
+    y = None
+    margin = math.inf
+    for _ in range(iters):
+        x = R.T @ u.astype(np.float64)
+        v, tv, _ = ternarize(x, tau)
+        margin = min(margin, relative_margin(x, tv))
+        y = R @ (hw * v.astype(np.float64))
+        u, tu, _ = ternarize(y, tau)
+        margin = min(margin, relative_margin(y, tu))
+    p = float(u.astype(np.float64) @ y)
+    nn = float(np.count_nonzero(u)) * float(np.sum(hw[v != 0]))
+    d = 0.0 if p == 0.0 else p / nn
+    dec = p * d
+    top = max(dec, dec_old)
+    dm = abs(dec - dec_old) / top if top > 0.0 else math.inf
+    if dec >= dec_old:
+        return Visit(u=u, v=v, d=d, kept=False, p_old=p_old, n_old=n_old, decrease=dec, margin=margin,
+                     decision_margin=dm)
+    return Visit(u=np.asarray(ui, dtype=np.int8).copy(), v=np.asarray(vi, dtype=np.int8).copy(), d=d_old, kept=True,
+                 p_old=p_old, n_old=n_old, decrease=dec_old, margin=margin, decision_margin=dm)
+
+
 def refine_sweeps(A: np.ndarray, B: np.ndarray, D: np.ndarray, C: np.ndarray, sweeps: int, tau: float,
                   iters: int = 15, h: np.ndarray | None = None, lam: float = 0.0,
                   track_residual: bool = False) -> Refinement:
     """§2.4 refinement sweeps with b = 1 on the factors (B, D, C) of A, for the plain
     objective (h None) or the §2.5 weighted one.  Each visit of component i:
-    R <- R + d_i u_i v_i^T; refit from u_i with `iters` (V-step, U-step) pairs;
-    take the refit or the stored pair, whichever decreases the residual more with
-    its least-squares scale (ties go to the refit); R <- R - d u v^T."""
+    R <- R + d_i u_i v_i^T, refine_visit, R <- R - d u v^T with the chosen term."""
     A = np.asarray(A, dtype=np.float64)
     m, n = A.shape
     k = int(np.asarray(D).shape[0])
@@ -491,45 +536,18 @@ def refine_sweeps(A: np.ndarray, B: np.ndarray, D: np.ndarray, C: np.ndarray, sw
     kept = 0
     for s in range(sweeps):
         for i in range(k):
-            ui = B[:, i].astype(np.float64)
-            vi = C[i, :].astype(np.float64)
             di = float(D[i])
-            # add the stored contribution back
-            R += di * np.outer(ui, vi)
-            p_old = float(ui @ (R @ (hw * vi)))
-            n_old = float(np.count_nonzero(ui)) * float(np.sum(hw[vi != 0]))
-            r2 += 2.0 * di * p_old - di * di * n_old
-            d_old = 0.0 if (p_old == 0.0 or n_old == 0.0) else p_old / n_old
-            dec_old = p_old * d_old
-            # refit from the stored u
-            u = B[:, i].copy()
-            v = None
-            y = None
-            margin = math.inf
-            for _ in range(iters):
-                x = R.T @ u.astype(np.float64)
-                v, tv, _ = ternarize(x, tau)
-                margin = min(margin, relative_margin(x, tv))
-                y = R @ (hw * v.astype(np.float64))
-                u, tu, _ = ternarize(y, tau)
-                margin = min(margin, relative_margin(y, tu))
-            p = float(u.astype(np.float64) @ y)
-            nn = float(np.count_nonzero(u)) * float(np.sum(hw[v != 0]))
-            d = 0.0 if p == 0.0 else p / nn
-            dec = p * d
-            margins[s, i] = margin
-            top = max(dec, dec_old)
-            dmargins[s, i] = abs(dec - dec_old) / top if top > 0.0 else math.inf
-            if dec >= dec_old:
-                B[:, i] = u
-                C[i, :] = v
-                D[i] = d
-                r2 -= dec
-            else:
-                D[i] = d_old
-                kept += 1
-                r2 -= dec_old
-            R -= float(D[i]) * np.outer(B[:, i].astype(np.float64), C[i, :].astype(np.float64))
+            R += di * np.outer(B[:, i].astype(np.float64), C[i, :].astype(np.float64))   # add back
+            vis = refine_visit(R, B[:, i], C[i, :], tau, iters, hw)
+            r2 += 2.0 * di * vis.p_old - di * di * vis.n_old
+            r2 -= vis.decrease
+            B[:, i] = vis.u
+            C[i, :] = vis.v
+            D[i] = vis.d
+            kept += int(vis.kept)
+            margins[s, i] = vis.margin
+            dmargins[s, i] = vis.decision_margin
+            R -= vis.d * np.outer(vis.u.astype(np.float64), vis.v.astype(np.float64))
             if track_residual:
                 res[s, i] = float(np.sum(hw[None, :] * R * R))
         sweep_energy[s] = 1.0 - r2 / norm
