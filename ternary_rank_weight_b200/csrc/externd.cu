@@ -1036,13 +1036,12 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
 }
 
 // Sum of one fp64 value per CTA of the group (fixed order), exchanged as tagged words.
-// `use` counts the calls of this group: consecutive calls alternate between two
-// buffers of Gg words and carry different tags, so a CTA that is already in call
+// `use` numbers the calls of this group from 1: consecutive calls alternate between
+// two buffers of Gg words and carry different tags, so a CTA that is already in call
 // j + 1 cannot overwrite a word another CTA still waits for in call j.  Every
 // exchange also orders: a CTA leaves it only after every CTA has entered it.
 __device__ bool exchange_sum(unsigned long long* sums, int q, int Gg, double v, const Smem& s, GroupSync* gs,
-                             uint64_t limit_ns, int* status, bool skip, unsigned& use, double& out) {
-    ++use;
+                             uint64_t limit_ns, int* status, bool skip, unsigned use, double& out) {
     const unsigned tag = gen_tag(use);
     unsigned long long* buf = sums + (size_t)(use & 1u) * Gg;
     const double t = block_sum(v, s.red);
@@ -1084,14 +1083,19 @@ __device__ void push_pending(const Smem& s, int L, int Ls, double d, int Wm, int
     __syncthreads();
 }
 
+// Calls of exchange_sum during refinement, numbered from 1 by visit: per refinement
+// visit r = 0, 1, ... one at its end (p_old) and, with k = 1, one at its start.
+__device__ __forceinline__ unsigned sum_use_start(int64_t r) { return (unsigned)(2 * r + 1); }
+__device__ __forceinline__ unsigned sum_use_end(int64_t r, int64_t kk) { return (unsigned)(kk == 1 ? 2 * r + 2 : r + 1); }
+
 // Start of a refinement visit of component i (§2.4, "Refinement sweeps"): load the
 // stored u_i, v_i (packed rows of B and C) and d_i, record d_i, n_old and the pending
 // slot in s.scal[8], [9], [11], and append the added-back term d_i u_i v_i^T as pending
 // component L with coefficient -d_i.  Leaves u = u_i in nzU/sgU/ulist and v = 0.
 // Returns nnz(u_i), or -1 if the group aborted.  Kept out of line: it runs once per
 // visit and would otherwise crowd the registers of the half-step loop.
-__device__ __noinline__ int refine_begin(const Prob& P, int64_t i, int q, int Gg, const KCfg& cfg, const Smem& s,
-                                         GroupSync* gs, bool skip, unsigned& sum_use, int L, int Ls, int Wm, int Wn,
+__device__ __forceinline__ int refine_begin(const Prob& P, int64_t i, int q, int Gg, const KCfg& cfg, const Smem& s,
+                                         GroupSync* gs, bool skip, unsigned sum_use, int L, int Ls, int Wm, int Wn,
                                          int64_t c0, int validV, int64_t r0, int validU, int pitchU, int pitchV,
                                          bool wtd) {
     const int tid = threadIdx.x;
@@ -1179,11 +1183,12 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
     int L = 0;
     unsigned long long sum_nu = 0, sum_nv = 0, sum_du = 0, sum_dv = 0, sum_nunv = 0, hs = 0, fb = 0;
     const int64_t kk = (mode == MODE_FACTOR) ? P.k : 1;
-    // §2.4 refinement sweeps: visits kk .. nvis-1 revisit components 0 .. kk-1 in order
-    const int S = (SWP && mode == MODE_FACTOR) ? P.sweeps : 0;
-    const int64_t nvis = kk * (int64_t)(1 + S);
-    unsigned sum_use = 0;                  // calls of exchange_sum by this group
-    unsigned long long kept = 0;           // refinement visits that kept the stored pair
+    // §2.4 refinement sweeps: visits kk .. nvis-1 revisit components 0 .. kk-1 in order.
+    // (Little of this is held in registers across the visit loop: the half-steps already
+    // use all 64 of a 1024-thread CTA's.)  s.scal[12] counts the visits that kept the
+    // stored pair.
+    const int64_t nvis = kk * (int64_t)(1 + ((SWP && mode == MODE_FACTOR) ? P.sweeps : 0));
+    if constexpr (SWP) if (tid == 0) s.scal[12] = 0.0;
     int nU = 0, nV = 0, dU = 0, dV = 0;   // support sizes and list lengths (trit changes)
     double hsv = 0.0;                     // weighted objective: sum of h~ over the support of v
     double p = 0.0, thr;
@@ -1206,7 +1211,7 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
         for (int c = tid; c < pitchU; c += NT) s.gU[c] = 0.0;
         if (mode != MODE_HALF_U) {
             if constexpr (SWP) if (refine) {
-                const int nU0 = refine_begin(P, i, q, Gg, cfg, s, gs, skip, sum_use, L, Ls, Wm, Wn, c0, validV, r0,
+                const int nU0 = refine_begin(P, i, q, Gg, cfg, s, gs, skip, sum_use_start(vis - kk), L, Ls, Wm, Wn, c0, validV, r0,
                                              validU, pitchU, pitchV, wtd);
                 if (nU0 < 0) return false;
                 ++L;
@@ -1302,6 +1307,14 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
                 }
                 return true;
             }
+            // A U-step that changed no trit of u ends the alternation: the next V-step would
+            // see the same u (an empty change list, unchanged sums and corrections), hence give
+            // the same x, v, y and u, and so would every later iteration.  Stopping here yields
+            // exactly the factors of all `iters` iterations.  (dU is the same in every CTA.)
+            // Refits start next to their fixed point, so this matters in the instantiation with
+            // refinement sweeps; first fits rarely settle within 15 iterations, and in the plain
+            // instantiations the extra exit costs registers, so they run every iteration.
+            if (SWP && dU == 0) break;
         }
         // ---- scale (§2.3 step 2): d = u^T R v / (nnz(u) nnz(v)), with u^T R v = u^T y = p;
         //      weighted (§2.5): d = u^T R (h~ v) / (nnz(u) sum_{v != 0} h~), the decrease p d
@@ -1315,28 +1328,26 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
             const double di = s.scal[8], n_old = s.scal[9];
             const int La = (int)s.scal[11];
             double pold = 0.0;
-            if (!exchange_sum(P.sums, q, Gg, tid == 0 ? s.scal[10] : 0.0, s, gs, cfg.limit_ns, P.status, skip, sum_use,
+            if (!exchange_sum(P.sums, q, Gg, tid == 0 ? s.scal[10] : 0.0, s, gs, cfg.limit_ns, P.status, skip,
+                              sum_use_end(vis - kk, kk),
                               pold))
                 return false;
             RN2 += 2.0 * di * pold - di * di * n_old;
             const double dold = (pold == 0.0 || n_old == 0.0) ? 0.0 : pold / n_old;
             take = (p * dnew >= pold * dold);
-            if (take) {
-                RN2 -= p * dnew;
-            } else {
-                RN2 -= pold * dold;
-                d = dold;
-                ++kept;
-                if (tid == 0) s.pd[La] = dold - di;   // net pending term of the stored pair
+            RN2 -= take ? p * dnew : pold * dold;
+            d = take ? dnew : dold;
+            if (tid == 0 && !take) {
+                s.scal[12] += 1.0;
+                s.pd[La] = dold - di;   // net pending term of the stored pair
             }
         }
         if (!refine) RN2 -= p * dnew;
         sum_nunv += (unsigned long long)nU * (unsigned long long)nV;
         if (lead) {
-            if (take) {
-                pack_row(s.nzU, s.sgU, Wm, reinterpret_cast<uint32_t*>(P.B + i * P.b_bytes), P.b_bytes / 4);
-                pack_row(s.nzV, s.sgV, Wn, reinterpret_cast<uint32_t*>(P.C + i * P.c_bytes), P.c_bytes / 4);
-            }
+            // (selects rather than branches on `take` keep the half-step loop's register allocation)
+            pack_row(s.nzU, s.sgU, Wm, reinterpret_cast<uint32_t*>(P.B + i * P.b_bytes), take ? P.b_bytes / 4 : 0);
+            pack_row(s.nzV, s.sgV, Wn, reinterpret_cast<uint32_t*>(P.C + i * P.c_bytes), take ? P.c_bytes / 4 : 0);
             if (tid == 0) {
                 P.D[i] = (float)d;
                 if (P.energy && !refine) P.energy[i] = 1.0 - RN2 / N0;
@@ -1344,15 +1355,13 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
                 if (P.dk) P.dk[i] = d;
                 if (refine && i == kk - 1 && P.sweep_energy) P.sweep_energy[vis / kk - 1] = 1.0 - RN2 / N0;
             }
-            if (S > 0) __threadfence();   // the other CTAs re-read this component in the next sweep
+            if (SWP) __threadfence();   // the other CTAs re-read this component in the next sweep
         }
-        // ---- deflation (§2.3 step 3), held lazily as a pending rank-1 term
-        if (take) {
-            push_pending(s, L, Ls, d, Wm, Wn, c0, validV, r0, validU);
-            ++L;
-        } else {
-            __syncthreads();
-        }
+        // ---- deflation (§2.3 step 3), held lazily as a pending rank-1 term; a refinement
+        //      visit that kept the stored pair pushes the refit with coefficient 0 (the
+        //      pair's new scale sits in its added-back slot)
+        push_pending(s, L, Ls, take ? d : 0.0, Wm, Wn, c0, validV, r0, validU);
+        ++L;
         phase_mark(s, 8);
         // room for the next visit's terms (two during refinement; extraction folds on the
         // plain schedule, so its rounding is that of a run without sweeps), and R folded
@@ -1382,7 +1391,9 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
         }
     }
     double R2 = 0.0;
-    if (!exchange_sum(P.sums, q, Gg, rs, s, gs, cfg.limit_ns, P.status, skip, sum_use, R2)) return false;
+    // the final sum follows the refinement visits' calls
+    const unsigned last_use = (nvis > kk) ? sum_use_end(nvis - kk - 1, kk) : 0u;
+    if (!exchange_sum(P.sums, q, Gg, rs, s, gs, cfg.limit_ns, P.status, skip, last_use + 1u, R2)) return false;
     if (lead && tid == 0) {
         P.stats->sum_nu = sum_nu;
         P.stats->sum_nv = sum_nv;
@@ -1393,7 +1404,7 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
         P.stats->fallbacks = fb;
         P.stats->residual2 = R2;
         P.stats->norm_a2 = N0;
-        P.stats->sweep_kept = kept;
+        P.stats->sweep_kept = SWP ? (unsigned long long)s.scal[12] : 0ull;
         phase_mark(s, 7);
         for (int k2 = 0; k2 < 11; ++k2) P.stats->phase[k2] = s.clk[k2];
         __threadfence();

@@ -88,6 +88,7 @@ class Workload:
     mu_sweep: tuple = field(default=())   # extra mu read off one run (prefix property)
     weighted: bool = False                # §2.5 objective with importance_weights(n, seed)
     lam: float = 0.0
+    sweeps: int = 0                       # §2.4 refinement sweeps after extraction
 
     def weights(self, b: int) -> np.ndarray:
         return importance_weights(self.shapes[b][1], self.seeds[b])
@@ -120,6 +121,10 @@ WORKLOADS = {
         tuple((0.7, 1.0, 2.0)[b % 3] for b in range(16))),
     "mlp_2560x6912_bf16_mu3_tau1.0_weighted": Workload(
         "mlp_2560x6912_bf16_mu3_tau1.0_weighted", ((2560, 6912),), (2,), (3.0,), (1.0,), bf16=True, weighted=True),
+    "mlp_2560x6912_bf16_mu3_tau1.0_sweep1": Workload(
+        "mlp_2560x6912_bf16_mu3_tau1.0_sweep1", ((2560, 6912),), (2,), (3.0,), (1.0,), bf16=True, sweeps=1),
+    "llm_1024x1024_mu2_tau0.7_sweep10": Workload(
+        "llm_1024x1024_mu2_tau0.7_sweep10", ((1024, 1024),), (1,), (2.0,), (0.7,), sweeps=10),
     "llm_4096x4096_mu3.5_tau0.7": Workload(
         "llm_4096x4096_mu3.5_tau0.7", ((4096, 4096),), (4,), (3.5,), (0.7,), outliers=32,
         mu_sweep=(1.0, 2.0, 3.0, 3.5)),

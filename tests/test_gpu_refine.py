@@ -14,7 +14,7 @@ import torch
 
 import ternary_rank_weight_b200 as ext
 from oracle import externd_oracle as ora
-from ternary_rank_weight_b200.workloads import importance_weights, llm_matrix
+from ternary_rank_weight_b200.workloads import WORKLOADS, importance_weights, llm_matrix
 
 pytestmark = pytest.mark.gpu
 
@@ -130,3 +130,35 @@ def test_sweeps_with_small_pending_depth_and_host_buffers():
         with pytest.raises(ext.ExterndError) as e:
             ext.factor(Ah, 1.5, 0.7, sweeps=bad)
         assert e.value.status == ext.STATUS["EINVAL"]
+
+
+def test_refinement_headline_workload_full_size_sampled():
+    """2560 x 6912 (k = 7680), one sweep: sampled visits teacher-forced.  Visit i sees
+    A minus the refined components before i and the extracted ones after it (component
+    i added back); the oracle's visit on that residual must give the GPU's term."""
+    w = WORKLOADS["mlp_2560x6912_bf16_mu3_tau1.0_sweep1"]
+    A = w.matrix(0)
+    base, ref = _run(A, w.mu[0], w.tau[0], seed=w.seeds[0], sweeps=1)
+    assert base.k == 7680 and torch.equal(base.energy, ref.energy)
+    assert ref.sweep_energy[0].item() >= base.energy[-1].item() - 1e-9
+    assert ref.stats["residual_energy"] == pytest.approx(ref.sweep_energy[0].item(), abs=1e-4)
+    B0, C0 = base.trits()
+    B1, C1 = ref.trits()
+    D0 = base.d64.cpu().numpy()
+    D1 = ref.d64.cpu().numpy()
+    hw = np.ones(A.shape[1])
+    mism = 0
+    for i in (0, 1, 700, 7679):
+        Bm = np.concatenate([B1[:, :i], B0[:, i + 1:]], axis=1).astype(np.float64)
+        Cm = np.concatenate([C1[:i], C0[i + 1:]], axis=0).astype(np.float64)
+        Dm = np.concatenate([D1[:i], D0[i + 1:]])
+        R = A.astype(np.float64) - (Bm * Dm) @ Cm
+        vis = ora.refine_visit(R, B0[:, i], C0[i], w.tau[0], 15, hw)
+        gb, gd, gc = _canonical(B1[:, i:i + 1], D1[i:i + 1], C1[i:i + 1])
+        ob, od, oc = _canonical(vis.u[:, None], np.array([vis.d]), vis.v[None, :])
+        if np.array_equal(gb, ob) and np.array_equal(gc, oc):
+            assert gd[0] == pytest.approx(od[0], rel=1e-4)
+        else:
+            assert vis.margin < 1e-3 or vis.decision_margin < 1e-6, (i, vis.margin, vis.decision_margin)
+            mism += 1
+    assert mism <= 1
