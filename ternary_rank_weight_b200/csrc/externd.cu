@@ -171,6 +171,10 @@ __global__ void __launch_bounds__(NTI) init_kernel(const Prob* __restrict__ prob
 // ALS kernel pieces
 // ---------------------------------------------------------------------------
 
+// Stride of the per-warp partial dot products, [l * DSTR + warp]: odd, so a warp's
+// lanes (l = lane) write and read distinct banks.
+constexpr int DSTR = NWARP + 1;
+
 // Shared-memory carve of the ALS kernel (host and device use the same layout).
 struct SmemLayout {
     size_t red, pd, coef, coefV, dotU, dotV, scal, wS, wM, wp, gS, gM, wJ, gJ, wc, dotp, sflag, clk, nzU, sgU, nzV, sgV, pnzU, psgU, pnzV,
@@ -194,7 +198,7 @@ struct SmemLayout {
         wJ = o;   o += 8 * NWARP;
         gJ = o;   o += 8 * NWARP;
         wc = o;   o += 4 * NWARP;
-        dotp = o; o += 4 * NWARP * MAX_PENDING;
+        dotp = o; o += 4 * DSTR * MAX_PENDING;
         sflag = o; o += 16;
         clk = o;  o += 8 * 12;
         nzU = o;  o += 4 * Wm;
@@ -219,7 +223,7 @@ struct SmemLayout {
         osgV = o; o += 4 * Wn;
         o = (o + 7) & ~(size_t)7;
         dotVw = o; o += weighted ? 8 * (size_t)MAX_PENDING : 0;
-        dotpw = o; o += weighted ? 8 * (size_t)NWARP * MAX_PENDING : 0;
+        dotpw = o; o += weighted ? 8 * (size_t)DSTR * MAX_PENDING : 0;
         gV = o;   o += 8 * (size_t)pv_max;
         gU = o;   o += 8 * (size_t)pu_max;
         corr = o; o += 8 * (size_t)(pv_max > pu_max ? pv_max : pu_max);
@@ -296,20 +300,18 @@ struct HalfCorr {
     int L;
 };
 
-// corr[c] = sum_l coef_l t_l(c) for this CTA's outputs: one thread per output, the
-// pending components that touch it added in increasing l.
+// corr[c] = sum_l coef_l t_l(c) for this CTA's outputs: one warp per output, lane l
+// taking pending component l, summed by a fixed butterfly.
 __device__ __forceinline__ void corrections(int valid, const HalfCorr& hc) {
     if (hc.L <= 0) return;
-    for (int c = threadIdx.x; c < valid; c += NT) {
-        uint32_t z = hc.cnz[c];
-        const uint32_t g = hc.csg[c];
-        double t = 0.0;
-        while (z) {
-            const int l = __ffs(z) - 1;
-            z &= z - 1u;
-            t += ((g >> l) & 1u) ? -hc.coef[l] : hc.coef[l];
-        }
-        hc.corr[c] = t;
+    const int lane = lane_id();
+    const double cl = lane < hc.L ? hc.coef[lane] : 0.0;
+    for (int c = warp_id(); c < valid; c += NWARP) {
+        const uint32_t z = hc.cnz[c], g = hc.csg[c];
+        double t = ((z >> lane) & 1u) ? (((g >> lane) & 1u) ? -cl : cl) : 0.0;
+        #pragma unroll
+        for (int o = 16; o; o >>= 1) t += __shfl_xor_sync(FULL, t, o);
+        if (lane == 0) hc.corr[c] = t;
     }
 }
 
@@ -385,7 +387,7 @@ __device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, i
     S = 0.0;
     const int nvec = pitch / VEC;
     if (nvec <= 0) return;
-    corrections(valid, hc);   // read after the CTA barrier below (or in the same thread)
+    corrections(valid, hc);   // read after the CTA barrier below
     if (nvec <= NT) {
         const int lanes = NT / nvec;
         const int act = min(lanes, nlist);   // row groups that get at least one entry
@@ -766,7 +768,7 @@ __device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned* p) {
 // Returns nnz; ok = false if a wait ran out.
 template <bool WTD>
 __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, unsigned tag, unsigned& arrivals,
-                                  bool skip, double S, const unsigned long long* gvec, int64_t len, double tau,
+                                  bool skip, double S, const unsigned long long* gvec, int64_t len, double tau_len,
                                   uint32_t* nz, uint32_t* sg, uint32_t* onz, uint32_t* osg, int* list, int rowpitch,
                                   const Smem& s, int L, int Ls, const uint32_t* pnz, const uint32_t* psg, int* dots,
                                   double* coef, bool want_p, double& thr_out, int& ndelta, GroupSync* gs,
@@ -827,18 +829,19 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
         const int64_t idx = ((int64_t)w << 5) + lane;
         wb[i] = (w < w1 && idx < len) ? ld_relaxed_u64(gvec + idx) : (unsigned long long)tag;
     }
-    double Sq = 0.0;
-    if ((int)threadIdx.x < Gg) Sq = untag(wait_tagged(partials + threadIdx.x, tag, gs, limit_ns, status, ok));
-    #pragma unroll
-    for (int o = 16; o; o >>= 1) Sq += __shfl_xor_sync(FULL, Sq, o);
-    if (lane == 0) s.gS[warp] = Sq;
+    if (warp * 32 < Gg) {   // the warps that hold partials
+        double Sq = 0.0;
+        if ((int)threadIdx.x < Gg) Sq = untag(wait_tagged(partials + threadIdx.x, tag, gs, limit_ns, status, ok));
+        #pragma unroll
+        for (int o = 16; o; o >>= 1) Sq += __shfl_xor_sync(FULL, Sq, o);
+        if (lane == 0) s.gS[warp] = Sq;
+    }
     ok = __syncthreads_and(ok);
     phase_mark(s, 4);
     if (!ok) { ok_out = false; return 0; }
-    double St = lane < NWARP ? s.gS[lane] : 0.0;
-    #pragma unroll
-    for (int o = 16; o; o >>= 1) St += __shfl_xor_sync(FULL, St, o);
-    const double thr = tau * St / (double)len;
+    double St = 0.0;   // the same fixed order in every thread
+    for (int w = 0; w < Gg; w += 32) St += s.gS[w >> 5];
+    const double thr = St * tau_len;   // tau * mean |x|, with tau / len computed once per matrix
     thr_out = thr;
 
     // ---- one pass over the vector: threshold, masks, counts, pending dots.  The warp
@@ -858,11 +861,16 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
                     wb[i] = (c0 + i < K && idx < len) ? ld_relaxed_u64(gvec + idx) : (unsigned long long)tag;
                 }
             }
+            bool stale = false;
             #pragma unroll
-            for (int i = 0; i < CH; ++i) {
-                if ((unsigned)(wb[i] & 0xFFull) != tag)
-                    wb[i] = wait_tagged(gvec + ((int64_t)(base + c0 + i) << 5) + lane, tag, gs, limit_ns, status, ok,
-                                        s.clk + 10);
+            for (int i = 0; i < CH; ++i) stale |= (unsigned)(wb[i] & 0xFFull) != tag;
+            if (__any_sync(FULL, stale)) {   // rare: a word not yet visible here, re-poll it
+                #pragma unroll
+                for (int i = 0; i < CH; ++i) {
+                    if ((unsigned)(wb[i] & 0xFFull) != tag)
+                        wb[i] = wait_tagged(gvec + ((int64_t)(base + c0 + i) << 5) + lane, tag, gs, limit_ns, status,
+                                            ok, s.clk + 10);
+                }
             }
             #pragma unroll
             for (int i = 0; i < CH; ++i) {
@@ -920,34 +928,31 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
     }
     cnt = __reduce_add_sync(FULL, cnt);
     dcnt = __reduce_add_sync(FULL, dcnt);
-    #pragma unroll
-    for (int o = 16; o; o >>= 1) ps += __shfl_xor_sync(FULL, ps, o);
+    if (want_p) {
+        #pragma unroll
+        for (int o = 16; o; o >>= 1) ps += __shfl_xor_sync(FULL, ps, o);
+    }
     if constexpr (WTD) {
         #pragma unroll
         for (int o = 16; o; o >>= 1) hsum += __shfl_xor_sync(FULL, hsum, o);
         if (lane == 0) s.wM[warp] = hsum;
-        if (lane < L) s.dotpw[warp * MAX_PENDING + lane] = dotw_acc;
+        if (lane < L) s.dotpw[lane * DSTR + warp] = dotw_acc;
     }
     if (lane == 0) { s.wc[warp] = cnt; s.wd[warp] = dcnt; s.wp[warp] = ps; }
-    if (lane < L) s.dotp[warp * MAX_PENDING + lane] = dot;
+    if (lane < L) s.dotp[lane * DSTR + warp] = dot;
     ok = __syncthreads_and(ok);
     phase_mark(s, 5);
     if (!ok) { ok_out = false; return 0; }
-    int cw = lane < NWARP ? s.wc[lane] : 0;
     const int dw = lane < NWARP ? s.wd[lane] : 0;
-    double p = lane < NWARP ? s.wp[lane] : 0.0;
-    int incl = dw;
-    #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(FULL, incl, o);
-        if (lane >= o) incl += t;
-        cw += __shfl_xor_sync(FULL, cw, o);
+    const int total = __reduce_add_sync(FULL, lane < NWARP ? s.wc[lane] : 0);
+    const int off = __reduce_add_sync(FULL, lane < warp ? dw : 0);   // this warp's place in the list
+    const int dtotal = __reduce_add_sync(FULL, dw);
+    double p = 0.0;   // needed by thread 0 only
+    if (warp == 0 && want_p) {
+        p = lane < NWARP ? s.wp[lane] : 0.0;
+        #pragma unroll
+        for (int o = 16; o; o >>= 1) p += __shfl_xor_sync(FULL, p, o);
     }
-    const int off = __shfl_sync(FULL, incl - dw, warp);
-    const int dtotal = __shfl_sync(FULL, incl, 31);
-    const int total = cw;
-    #pragma unroll
-    for (int o = 16; o; o >>= 1) p += __shfl_xor_sync(FULL, p, o);
     if constexpr (WTD) {
         double hs = lane < NWARP ? s.wM[lane] : 0.0;
         #pragma unroll
@@ -957,7 +962,7 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
     if (total > 0) {
         for (int l = warp; l < L; l += NWARP) {
             if constexpr (WTD) {
-                double d = lane < NWARP ? s.dotpw[lane * MAX_PENDING + l] : 0.0;
+                double d = lane < NWARP ? s.dotpw[l * DSTR + lane] : 0.0;
                 #pragma unroll
                 for (int o = 16; o; o >>= 1) d += __shfl_xor_sync(FULL, d, o);
                 if (lane == 0) {
@@ -966,9 +971,8 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
                     coef[l] = s.pd[l] * d;
                 }
             } else {
-                int d = lane < NWARP ? s.dotp[lane * MAX_PENDING + l] : 0;
-                #pragma unroll
-                for (int o = 16; o; o >>= 1) d += __shfl_xor_sync(FULL, d, o);
+                int d = lane < NWARP ? s.dotp[l * DSTR + lane] : 0;
+                d = __reduce_add_sync(FULL, d);
                 if (lane == 0) {
                     d += dots[l];
                     dots[l] = d;
@@ -1146,6 +1150,7 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
     const bool lead = (q == 0);
     const bool skip = (cfg.fault_skip == q);
     constexpr bool wtd = WTD;   // §2.5 importance-weighted objective (P.hw set)
+    const double tauV = P.tau / (double)n, tauU = P.tau / (double)m;   // T_tau: tau / length, times sum |x|
     const int Ls = cfg.Lcap > 0 ? cfg.Lcap : 1;   // stride of the word-major pending masks
 
     float* blkV = P.Rv + P.pv.block_offset(q, m);
@@ -1244,7 +1249,7 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
                 gemv_dispatch<false>(P.pv.vec, blkV, pitchV, validV, c0, s.ulist, nullptr, dU, s.red, P.xbuf, hcV, tg, skip, S, s.clk);
                 phase_mark(s, 1);
                 bool ok = true;
-                const int nv2 = exchange_threshold<WTD>(P.partV, q, Gg, tg, arrivals, skip, S, P.xbuf, n, P.tau, s.nzV,
+                const int nv2 = exchange_threshold<WTD>(P.partV, q, Gg, tg, arrivals, skip, S, P.xbuf, n, tauV, s.nzV,
                                                    s.sgV, s.onzV, s.osgV, s.vlist, pitchU, s, L, Ls, s.pnzV, s.psgV,
                                                    s.dotV, s.coefV, false, thr, dV, gs, cfg.limit_ns, P.status, ok,
                                                    wtd ? P.hw : nullptr, wtd ? s.vwl : nullptr, s.dotVw, &hsv);
@@ -1290,7 +1295,7 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
             bool ok = true;
             sum_nv += (unsigned long long)nV;
             sum_dv += (unsigned long long)dV;
-            nU = exchange_threshold<false>(P.partU, q, Gg, tg, arrivals, skip, S, P.ybuf, m, P.tau, s.nzU, s.sgU, s.onzU,
+            nU = exchange_threshold<false>(P.partU, q, Gg, tg, arrivals, skip, S, P.ybuf, m, tauU, s.nzU, s.sgU, s.onzU,
                                     s.osgU, s.ulist, pitchV, s, L, Ls, s.pnzU, s.psgU, s.dotU, s.coef, true, thr, dU,
                                     gs, cfg.limit_ns, P.status, ok);
             if (!ok) return false;
