@@ -300,18 +300,34 @@ struct HalfCorr {
     int L;
 };
 
-// corr[c] = sum_l coef_l t_l(c) for this CTA's outputs: one warp per output, lane l
-// taking pending component l, summed by a fixed butterfly.
+// corr[c] = sum_l coef_l t_l(c) for this CTA's outputs.  Few outputs (a CTA of a large
+// group): one warp per output, lane l taking pending component l, summed by a fixed
+// butterfly.  Many outputs (a small group): one thread per output, the components that
+// touch it added in increasing l.
 __device__ __forceinline__ void corrections(int valid, const HalfCorr& hc) {
     if (hc.L <= 0) return;
-    const int lane = lane_id();
-    const double cl = lane < hc.L ? hc.coef[lane] : 0.0;
-    for (int c = warp_id(); c < valid; c += NWARP) {
-        const uint32_t z = hc.cnz[c], g = hc.csg[c];
-        double t = ((z >> lane) & 1u) ? (((g >> lane) & 1u) ? -cl : cl) : 0.0;
-        #pragma unroll
-        for (int o = 16; o; o >>= 1) t += __shfl_xor_sync(FULL, t, o);
-        if (lane == 0) hc.corr[c] = t;
+    if (valid <= 2 * NWARP) {
+        const int lane = lane_id();
+        const double cl = lane < hc.L ? hc.coef[lane] : 0.0;
+        for (int c = warp_id(); c < valid; c += NWARP) {
+            const uint32_t z = hc.cnz[c], g = hc.csg[c];
+            double t = ((z >> lane) & 1u) ? (((g >> lane) & 1u) ? -cl : cl) : 0.0;
+            #pragma unroll
+            for (int o = 16; o; o >>= 1) t += __shfl_xor_sync(FULL, t, o);
+            if (lane == 0) hc.corr[c] = t;
+        }
+    } else {
+        for (int c = threadIdx.x; c < valid; c += NT) {
+            uint32_t z = hc.cnz[c];
+            const uint32_t g = hc.csg[c];
+            double t = 0.0;
+            while (z) {
+                const int l = __ffs(z) - 1;
+                z &= z - 1u;
+                t += ((g >> l) & 1u) ? -hc.coef[l] : hc.coef[l];
+            }
+            hc.corr[c] = t;
+        }
     }
 }
 
