@@ -99,3 +99,49 @@ def test_inference_entry_points_reject_bad_arguments_before_device_work():
     assert L.externd_matvec(p, p, p, 2, 2, 2, p, 1, p, p, None) == einval   # host memory is refused
     assert L.externd_pack_mask_sign(p, 1, 1, p, p, 0, p, None) == einval    # no room for signs
     assert L.externd_pack_mask_sign(None, 1, 1, p, p, 1, p, None) == einval
+
+
+def _c_layout(struct, fields):
+    """sizeof and offsetof of a struct of include/externd.h, from the C compiler."""
+    import shutil
+    import subprocess
+    import tempfile
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    body = "".join(f'    printf("%zu\\n", offsetof({struct}, {f}));\n' for f in fields)
+    src = ("#include <stddef.h>\n#include <stdio.h>\n#include \"externd.h\"\nint main(void) {\n"
+           f'    printf("%zu\\n", sizeof({struct}));\n{body}    return 0;\n}}\n')
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "layout.c")
+        exe = os.path.join(d, "layout")
+        open(c, "w").write(src)
+        subprocess.run([cc, "-I", os.path.join(ROOT, "include"), c, "-o", exe], check=True)
+        out = [int(x) for x in subprocess.run([exe], check=True, capture_output=True, text=True).stdout.split()]
+    return out[0], out[1:]
+
+
+@pytest.mark.parametrize("cls,struct,rename", [(_lib.Options, "externd_options", {"lambda_": "lambda"}),
+                                               (_lib.Stats, "externd_stats", {})])
+def test_ctypes_structs_match_the_header(cls, struct, rename):
+    names = [n for n, _ in cls._fields_]
+    size, offs = _c_layout(struct, [rename.get(n, n) for n in names])
+    assert ctypes.sizeof(cls) == size
+    for n, off in zip(names, offs):
+        assert getattr(cls, n).offset == off, n
+
+
+def test_factor_options_are_validated_before_device_work():
+    L = _lib.load()
+    buf = (ctypes.c_uint8 * 64)()
+    A = (ctypes.c_float * 4)(1, 2, 3, 4)
+    h = (ctypes.c_float * 2)(1, 1)
+    einval = ext.STATUS["EINVAL"]
+    for kw in ({"sweeps": -1}, {"sweeps": 1001}, {"h": ctypes.addressof(h), "lambda_": -1.0},
+               {"h": ctypes.addressof(h), "lambda_": float("nan")}):
+        opt = _lib.Options()
+        for k, v in kw.items():
+            setattr(opt, k, v)
+        rc = L.externd_factor_ex(ctypes.addressof(A), 2, 2, 1.0, 0.7, 15, 0, ctypes.addressof(buf),
+                                 ctypes.addressof(buf), ctypes.addressof(buf), None, None, ctypes.byref(opt))
+        assert rc == einval, kw
