@@ -49,10 +49,15 @@ def _peaks():
 
 
 def _kernel_source_hash() -> str:
+    """Hash of the ALS kernel's code (line comments and blank lines removed, so editing a
+    comment does not invalidate the recorded ncu traffic)."""
     h = hashlib.sha256()
     for name in ("externd.cu", "externd_kernels.cuh"):
-        with open(os.path.join(ROOT, "ternary_rank_weight_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "ternary_rank_weight_b200", "csrc", name), encoding="utf-8") as f:
+            for line in f:
+                code = line.split("//", 1)[0].rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()
 
 

@@ -331,8 +331,8 @@ __device__ __forceinline__ void corrections(int valid, const HalfCorr& hc) {
     }
 }
 
-// Publish one output word and fold its (published, 44-bit) value into this thread's
-// partial |.| sum and max.
+// Publish one output word and add its (published, 44-bit) magnitude to this thread's
+// partial sum of |out|.
 __device__ __forceinline__ void emit_tagged(double v, int64_t gi, unsigned long long* gout, unsigned tag, bool skip,
                                             double& S) {
     const unsigned long long w = tag_value(v, tag);
@@ -775,7 +775,8 @@ __device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned* p) {
 // partials[q] and count its arrival on counter q % NCTR; wait until every CTA of
 // the group has arrived (NCTR threads poll one counter each, bounded), read all
 // partials (tag-checked), read the whole output vector (tag-checked, re-polling any
-// word not yet visible), threshold it (T_tau of §2.2 with the all-zero fallback),
+// word not yet visible), threshold it (T_tau of §2.2 with the all-zero fallback;
+// tau_len = tau / len, so the threshold is tau_len * sum |out|),
 // write its masks and compacted support list, the coefficients d_l (t_l . t) of the
 // pending components for the next half-step, and p = sum over the support of |x|
 // into s.scal[0] (s.scal[1] = 1 if the fallback was taken).  Sums are combined in
