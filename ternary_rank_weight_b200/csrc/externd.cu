@@ -912,8 +912,12 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
         if (lane < K) { nz[w] = my_bz; sg[w] = my_bs; onz[w] = oz; osg[w] = os; }
         cnt += __popc(my_bz);
         dcnt += __popc(ch);
-        if constexpr (WTD) {   // sum of h~ over the new support (lane = word, bits in increasing order)
-            for (uint32_t mk = my_bz; mk; mk &= mk - 1u) hsum += (double)__ldg(hw + ((int64_t)w << 5) + __ffs(mk) - 1);
+        if constexpr (WTD) {   // sum of h~ over the new support: lane b takes bit b of each word, in word order
+            for (int i = 0; i < K; ++i) {
+                const uint32_t zi = __shfl_sync(FULL, my_bz, i);
+                const int64_t c = ((int64_t)(base + i) << 5) + lane;
+                if ((zi >> lane) & 1u) hsum += (double)__ldg(hw + c);
+            }
         }
         // change of t_l . t (weighted: sum h~_c t_l(c) t(c)) over the words that changed
         // (lane l = pending component l)
@@ -924,18 +928,25 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
             const uint32_t zi = __shfl_sync(FULL, my_bz, i), si = __shfl_sync(FULL, my_bs, i);
             const uint32_t ozi = __shfl_sync(FULL, oz, i), osi = __shfl_sync(FULL, os, i);
             const uint32_t chi = __shfl_sync(FULL, ch, i);
-            uint32_t dni = 0u, dti = 0u;
-            if constexpr (WTD) { dni = __shfl_sync(FULL, dn, i); dti = __shfl_sync(FULL, dt, i); }
-            if (lane < L) {
-                const uint32_t pz = pnz[(base + i) * Ls + lane], pg = psg[(base + i) * Ls + lane];
-                if constexpr (WTD) {
-                    for (uint32_t mk = pz & chi; mk; mk &= mk - 1u) {
-                        const int b = __ffs(mk) - 1;
-                        const double hv = (double)__ldg(hw + ((int64_t)(base + i) << 5) + b);
+            if constexpr (WTD) {
+                // sum over the changed bits b of h~_b t_l(b) (new - old trit), lane l = component l;
+                // the word's 32 weights are loaded once (lane b: bit b) and broadcast per bit
+                const uint32_t dni = __shfl_sync(FULL, dn, i), dti = __shfl_sync(FULL, dt, i);
+                const int64_t cb = ((int64_t)(base + i) << 5) + lane;
+                const float hword = cb < len ? __ldg(hw + cb) : 0.f;
+                const uint32_t pz = lane < L ? pnz[(base + i) * Ls + lane] : 0u;
+                const uint32_t pg = lane < L ? psg[(base + i) * Ls + lane] : 0u;
+                for (uint32_t mk = chi; mk; mk &= mk - 1u) {
+                    const int b = __ffs(mk) - 1;
+                    const double hv = (double)__shfl_sync(FULL, hword, b);
+                    if ((pz >> b) & 1u) {
                         const double dv = (((dni >> b) & 1u) ? -1.0 : 1.0) * (((dti >> b) & 1u) ? 2.0 : 1.0);
                         dotw_acc += ((pg >> b) & 1u) ? -hv * dv : hv * dv;
                     }
-                } else {
+                }
+            } else if (lane < L) {
+                const uint32_t pz = pnz[(base + i) * Ls + lane], pg = psg[(base + i) * Ls + lane];
+                {
                     const uint32_t zn = pz & zi & chi, zo = pz & ozi & chi;
                     const uint32_t sn = pg ^ si, so = pg ^ osi;
                     dot += (__popc(zn & ~sn) - __popc(zn & sn)) - (__popc(zo & ~so) - __popc(zo & so));
@@ -998,7 +1009,19 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
             }
         }
         int run = off;
-        for (int base = w0; base < w1; base += 32) {
+        if constexpr (WTD) {   // one word at a time across the lanes (lane b: bit b), in index order
+            for (int w = w0; w < w1; ++w) {
+                uint32_t ng, tw;
+                const uint32_t ch = delta_mask(onz[w], osg[w], nz[w], sg[w], ng, tw);
+                if ((ch >> lane) & 1u) {
+                    const int at = run + __popc(ch & ((1u << lane) - 1u));
+                    const int e = delta_entry(((unsigned)w << 5) + lane, rowpitch, ng, tw, lane);
+                    wl[at] = entry_coef(e) * __ldg(hw + ((int64_t)w << 5) + lane);
+                    list[at] = e;
+                }
+                run += __popc(ch);
+            }
+        } else for (int base = w0; base < w1; base += 32) {
             const int w = base + lane;
             uint32_t ch = 0u, ng = 0u, tw = 0u;
             if (w < w1) ch = delta_mask(onz[w], osg[w], nz[w], sg[w], ng, tw);
@@ -1013,7 +1036,6 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
             for (uint32_t mk = ch; mk; mk &= mk - 1u) {
                 const int b = __ffs(mk) - 1;
                 const int e = delta_entry(((unsigned)w << 5) + b, rowpitch, ng, tw, b);
-                if constexpr (WTD) wl[at] = entry_coef(e) * __ldg(hw + ((int64_t)w << 5) + b);
                 list[at++] = e;
             }
             run += __shfl_sync(FULL, incl, 31);
