@@ -891,7 +891,8 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
             }
             #pragma unroll
             for (int i = 0; i < CH; ++i) {
-                if (c0 + i < K) {
+                if (c0 + i >= K) break;   // K is the same in every lane: skip the unused slots
+                {
                     const double x = untag(wb[i]);           // padding words untag to 0
                     const bool z = fabs(x) > thr;
                     const unsigned bz = __ballot_sync(FULL, z);
