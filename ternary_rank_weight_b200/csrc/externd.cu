@@ -395,6 +395,7 @@ __device__ __forceinline__ void gemv_rows(double* acc, const float* base, const 
 // them in the first one, where g starts at 0), so g[c] += sum_{e in list} s_e blk[r_e][c]
 // keeps g = R^T t (or R t) for the current input trits t; out[c] = g[c] minus the
 // lazy-deflation correction is written to gout[out0 + c].  fp64 accumulation of exact fp32 terms, fixed summation order.
+// S returns this warp's sum of the published |out| in lane 0 (a fixed butterfly).
 template <int VEC, bool WL>
 __device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, int64_t out0,
                           const int* __restrict__ list, const float* __restrict__ wl, int nlist, double* red,
@@ -443,6 +444,9 @@ __device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, i
                 emit_tagged(hc.L > 0 ? gc - hc.corr[c] : gc, out0 + c, gout, tag, skip, S);
             }
         }
+        // this warp's sum of |out| into lane 0: only lanes that are multiples of tpc emitted,
+        // so the butterfly rounds below tpc would add exact zeros
+        for (int o = 16; o >= tpc; o >>= 1) S += __shfl_xor_sync(FULL, S, o);
     } else {
         constexpr int U = GEMV_U<VEC>();
         __syncthreads();   // corrections
@@ -479,6 +483,8 @@ __device__ void gemv_emit(const float* __restrict__ blk, int pitch, int valid, i
                 }
             }
         }
+        #pragma unroll
+        for (int o = 16; o; o >>= 1) S += __shfl_xor_sync(FULL, S, o);   // this warp's sum into lane 0
     }
 }
 
@@ -792,9 +798,8 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
                                   uint64_t limit_ns, int* status, bool& ok_out, const float* hw = nullptr,
                                   float* wl = nullptr, double* dotw = nullptr, double* hsum_out = nullptr) {
     const int lane = lane_id(), warp = warp_id();
-    // ---- this CTA's partial (fixed butterfly + fixed cross-warp combine)
-    #pragma unroll
-    for (int o = 16; o; o >>= 1) S += __shfl_xor_sync(FULL, S, o);
+    // ---- this CTA's partial: S holds each warp's sum in lane 0 (summed by the GEMV's
+    //      fixed butterfly), combined across warps in a fixed order
     if (lane == 0) s.wS[warp] = S;
     __syncthreads();
     if (warp == 0) {

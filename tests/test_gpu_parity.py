@@ -244,6 +244,18 @@ def test_bounded_wait_reports_timeout_and_context_stays_usable():
     assert f.energy[-1].item() > 0.5
 
 
+@pytest.mark.parametrize("kw", [{"sweeps": 1}, {"h": np.linspace(0.5, 2.0, 256).astype(np.float32)},
+                                {"sweeps": 2, "h": np.linspace(0.5, 2.0, 256).astype(np.float32)}])
+def test_bounded_wait_in_the_weighted_and_sweep_kernels(kw):
+    """The other instantiations of the ALS kernel end the same way when a CTA never signals."""
+    A = torch.from_numpy(llm_matrix(256, 256, seed=4)).cuda()
+    with pytest.raises(ext.ExterndError) as e:
+        ext.factor(A, 1.0, 0.7, grid=4, fault_skip_cta=1, wait_limit_s=0.2, **kw)
+    assert e.value.status == ext.STATUS["ETIMEOUT"]
+    f = ext.factor(A, 1.0, 0.7, grid=4, **kw)
+    assert f.energy[-1].item() > 0.5
+
+
 # ---------------------------------------------------------------------------
 # full size: the headline workload in the launch configuration the bench times
 # ---------------------------------------------------------------------------
