@@ -1,0 +1,107 @@
+"""Full-size parity for the remaining workload configurations.
+
+* 1024 x 1024, mu = 2, tau = 0.7 (k = 2048): end to end against the oracle's whole
+  run, with the extraction's tolerances (energy within 2e-3, zero fraction within 0.5
+  points, trits equal until the first divergence, which must start at a near-tie of
+  the oracle, d within 1e-4 relative before it).
+* 16 x 1536 x 1536, mu = 2.5, tau cycling (the batched entry point): every matrix
+  succeeds, two matrices equal single calls with the same group size bit for bit,
+  and sampled components of matrix 0 are teacher-forced against the oracle.
+* 4096 x 4096, mu = 3.5, tau = 0.7 (k = 14336): the prefix property (the start vector
+  of component i depends only on the seed and i, so the first k components of a run
+  at larger mu are the run at smaller mu, bit for bit) and teacher-forced samples up
+  to the last component.
+"""
+import numpy as np
+import pytest
+import torch
+
+import ternary_rank_weight_b200 as ext
+from oracle import externd_oracle as ora
+from ternary_rank_weight_b200.workloads import WORKLOADS
+
+pytestmark = pytest.mark.gpu
+
+
+def _zero_fraction(B, C):
+    return (np.count_nonzero(B == 0) + np.count_nonzero(C == 0)) / (B.size + C.size)
+
+
+def _teacher_forced(A, Bg, Cg, d64, seed, tau, samples):
+    """For each sampled component: refit it on the residual the GPU's own earlier
+    components leave; returns the number of samples whose trits differ (each must sit
+    at a near-tie)."""
+    m = A.shape[0]
+    mism = 0
+    for i in samples:
+        R = ora.residual_after(A, Bg, d64, Cg, i)
+        u0, _, _ = ora.ternarize(ora.start_normals(seed, i, m), tau)
+        fit = ora.fit_component(R, u0, tau, 15)
+        if np.array_equal(fit.u, Bg[:, i]) and np.array_equal(fit.v, Cg[i]):
+            assert d64[i] == pytest.approx(fit.d, rel=1e-4), i
+        else:
+            mism += 1
+            assert fit.min_margin < 1e-3, (i, fit.min_margin)
+    return mism
+
+
+def test_llm_1024_end_to_end_matches_oracle():
+    w = WORKLOADS["llm_1024x1024_mu2_tau0.7"]
+    A = w.matrix(0)
+    f = ext.factor(torch.from_numpy(A).cuda(), w.mu[0], w.tau[0], seed=w.seeds[0], want_d64=True)
+    assert f.k == 2048
+    ref = ora.greedy_als(A, k=f.k, tau=w.tau[0], seed=w.seeds[0])
+    Bg, Cg = f.trits()
+    e = f.energy.cpu().numpy()
+    assert np.max(np.abs(e - ref.energy)) < 2e-3
+    assert abs(_zero_fraction(Bg, Cg) - ref.zero_fraction()) < 0.005
+    div = f.k
+    for i in range(f.k):
+        if not (np.array_equal(Bg[:, i], ref.B[:, i]) and np.array_equal(Cg[i], ref.C[i])):
+            div = i
+            break
+    d64 = f.d64.cpu().numpy()
+    if div > 0:
+        assert np.allclose(d64[:div], ref.D[:div], rtol=1e-4, atol=0)
+    if div < f.k:
+        assert ref.margins[div] < 1e-3, (div, ref.margins[div])
+    assert div >= 16, div
+
+
+def test_batched_attention_workload_full_size():
+    w = WORKLOADS["attn_16x1536x1536_mu2.5_tau_cycle"]
+    mats = [w.matrix(b) for b in range(w.count)]
+    res, st = ext.factor_batched([torch.from_numpy(a).cuda() for a in mats], list(w.mu), list(w.tau),
+                                 seeds=list(w.seeds))
+    assert st == [0] * w.count
+    G = res[0].stats["group"]
+    for r in res:
+        assert r.k == 3840
+        e = r.energy.cpu().numpy()
+        assert np.all(np.diff(e) >= -1e-12) and 0.5 < e[-1] < 1.0
+    for b in (0, 7):
+        f = ext.factor(torch.from_numpy(mats[b]).cuda(), w.mu[b], w.tau[b], seed=w.seeds[b], grid=G)
+        assert torch.equal(f.B, res[b].B) and torch.equal(f.C, res[b].C) and torch.equal(f.D, res[b].D)
+        assert torch.equal(f.energy, res[b].energy)
+    f0 = ext.factor(torch.from_numpy(mats[0]).cuda(), w.mu[0], w.tau[0], seed=w.seeds[0], grid=G, want_d64=True)
+    Bg, Cg = f0.trits()
+    mism = _teacher_forced(mats[0], Bg, Cg, f0.d64.cpu().numpy(), w.seeds[0], w.tau[0], (0, 1, 1919, 3839))
+    assert mism <= 1
+
+
+def test_llm_4096_prefix_property_and_sampled_parity():
+    w = WORKLOADS["llm_4096x4096_mu3.5_tau0.7"]
+    A = w.matrix(0)
+    Ag = torch.from_numpy(A).cuda()
+    big = ext.factor(Ag, w.mu[0], w.tau[0], seed=w.seeds[0], want_d64=True)
+    small = ext.factor(Ag, 1.0, w.tau[0], seed=w.seeds[0])
+    assert big.k == 14336 and small.k == 4096
+    k = small.k
+    assert torch.equal(big.B[:k], small.B) and torch.equal(big.C[:k], small.C) and torch.equal(big.D[:k], small.D)
+    assert torch.equal(big.energy[:k], small.energy)
+    e = big.energy.cpu().numpy()
+    assert np.all(np.diff(e) >= -1e-12)
+    assert big.stats["residual_energy"] == pytest.approx(e[-1], abs=1e-4)
+    Bg, Cg = big.trits()
+    mism = _teacher_forced(A, Bg, Cg, big.d64.cpu().numpy(), w.seeds[0], w.tau[0], (0, 4096, 14335))
+    assert mism <= 1
