@@ -141,6 +141,29 @@ int externd_factor_batched(int count, const float* const* A, const int64_t* m, c
                            uint8_t* const* B_out, float* const* D_out, uint8_t* const* C_out,
                            double* const* energy_out, int* status_out, void* stream);
 
+/* Per-matrix extensions of a batched call (zero-initialise, set what is needed).
+ *   h         NULL, or `count` pointers to per-column importance weights (n_b fp32 values each):
+ *             the §2.5 objective ("ExTernD: Expanded-Rank Ternary Decomposition", §2.5, see
+ *             externd_factor_weighted).  One launch runs one objective, so either every entry is
+ *             non-NULL or h is NULL (EXTERND_EINVAL otherwise).
+ *   lambda    with h: `count` values of lambda (finite, >= 0); NULL means 0 for every matrix.
+ *   sweeps    refinement sweeps after extraction for every matrix (§2.4, see externd_options),
+ *             0 .. 1000.
+ *   sweep_energy_out  NULL, or `count` pointers (entries may be NULL) to `sweeps` doubles each. */
+typedef struct {
+    const float* const* h;
+    const double* lambda;
+    int sweeps;
+    double* const* sweep_energy_out;
+} externd_batch_options;
+
+/* externd_factor_batched with per-matrix extensions (opt may be NULL: the plain call). */
+int externd_factor_batched_ex(int count, const float* const* A, const int64_t* m, const int64_t* n,
+                              const double* mu, const double* tau, int iters, const uint64_t* seed,
+                              uint8_t* const* B_out, float* const* D_out, uint8_t* const* C_out,
+                              double* const* energy_out, int* status_out, void* stream,
+                              const externd_batch_options* opt);
+
 /* Ahat = B diag(D) C (§2.1) with fp64 accumulation, written as fp32 m x n
  * row-major.  B, C packed as produced by externd_factor. */
 int externd_reconstruct(const uint8_t* B, const float* D, const uint8_t* C, int64_t m, int64_t n,

@@ -20,6 +20,7 @@ EXPORTS = (
     "externd_factor_weighted",
     "externd_factor_noalloc",
     "externd_factor_batched",
+    "externd_factor_batched_ex",
     "externd_reconstruct",
     "externd_strerror",
     "externd_debug_halfstep",
@@ -43,6 +44,15 @@ class Options(ctypes.Structure):
         ("sweep_energy_out", ctypes.c_void_p),
         ("h", ctypes.c_void_p),
         ("lambda_", ctypes.c_double),
+    ]
+
+
+class BatchOptions(ctypes.Structure):
+    _fields_ = [
+        ("h", ctypes.c_void_p),
+        ("lambda_", ctypes.c_void_p),
+        ("sweeps", ctypes.c_int),
+        ("sweep_energy_out", ctypes.c_void_p),
     ]
 
 
@@ -107,6 +117,8 @@ def load():
     L.externd_factor_noalloc.restype = c_int
     L.externd_factor_batched.argtypes = [c_int, vp, vp, vp, vp, vp, c_int, vp, vp, vp, vp, vp, vp, vp]
     L.externd_factor_batched.restype = c_int
+    L.externd_factor_batched_ex.argtypes = [c_int, vp, vp, vp, vp, vp, c_int, vp, vp, vp, vp, vp, vp, vp, vp]
+    L.externd_factor_batched_ex.restype = c_int
     L.externd_reconstruct.argtypes = [vp, vp, vp, i64, i64, i64, vp, vp]
     L.externd_reconstruct.restype = c_int
     L.externd_strerror.argtypes = [c_int]

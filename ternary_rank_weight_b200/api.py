@@ -231,9 +231,12 @@ NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
 def factor_batched(As: Sequence, mus: Sequence[float], taus: Sequence[float], iters: int = 15,
-                   seeds: Optional[Sequence[int]] = None, *, stream=None):
-    """Factor independent matrices in one launch (externd_factor_batched).
+                   seeds: Optional[Sequence[int]] = None, *, hs: Optional[Sequence] = None,
+                   lams: Optional[Sequence[float]] = None, sweeps: int = 0, stream=None):
+    """Factor independent matrices in one launch (externd_factor_batched_ex).
 
+    hs: per-matrix importance weights (§2.5; every matrix or none), lams their lambdas;
+    sweeps: refinement sweeps (§2.4) for every matrix.
     Returns (list of Factors, list of per-matrix status codes)."""
     mats = [_as_matrix(a) for a in As]
     cnt = len(mats)
@@ -259,18 +262,35 @@ def factor_batched(As: Sequence, mus: Sequence[float], taus: Sequence[float], it
     tau_a = (ctypes.c_double * cnt)(*[float(x) for x in taus])
     seed_a = (ctypes.c_uint64 * cnt)(*[int(s) for s in seeds])
     st = (ctypes.c_int * cnt)()
+    opt = _lib.BatchOptions()
+    keep = []   # ctypes arrays and tensors that must outlive the call
+    if hs is not None:
+        hts = [_weights(h, A.shape[1]) for h, A in zip(hs, mats)]
+        harr = P(*[_ptr(h) for h in hts])
+        keep += [hts, harr]
+        opt.h = ctypes.cast(harr, ctypes.c_void_p)
+        if lams is not None:
+            larr = (ctypes.c_double * cnt)(*[float(x) for x in lams])
+            keep.append(larr)
+            opt.lambda_ = ctypes.cast(larr, ctypes.c_void_p)
+    SEs = [_empty((int(sweeps),), torch.float64, A) if sweeps > 0 else None for A in mats]
+    opt.sweeps = int(sweeps)
+    if sweeps > 0:
+        sarr = P(*[_ptr(x) for x in SEs])
+        keep.append(sarr)
+        opt.sweep_energy_out = ctypes.cast(sarr, ctypes.c_void_p)
     with _on_device(mats[0]):
-        rc = _lib.load().externd_factor_batched(cnt, a_ptrs, ms, ns, mu_a, tau_a, int(iters), seed_a,
-                                                b_ptrs, d_ptrs, c_ptrs, e_ptrs, st,
-                                                _stream(stream, mats[0].device))
+        rc = _lib.load().externd_factor_batched_ex(cnt, a_ptrs, ms, ns, mu_a, tau_a, int(iters), seed_a,
+                                                   b_ptrs, d_ptrs, c_ptrs, e_ptrs, st,
+                                                   _stream(stream, mats[0].device), ctypes.byref(opt))
     stats = last_stats()
     res = []
-    for A, mu, tau, o in zip(mats, mus, taus, outs):
+    for A, mu, tau, o, se in zip(mats, mus, taus, outs, SEs):
         res.append(Factors(B=o[0], D=o[1], C=o[2], energy=o[3], m=A.shape[0], n=A.shape[1], k=o[4],
-                           mu=float(mu), tau=float(tau), stats=stats))
+                           mu=float(mu), tau=float(tau), stats=stats, sweep_energy=se))
     statuses = list(st)
     if rc != 0 and all(s == 0 for s in statuses):
-        _check(rc, "externd_factor_batched")
+        _check(rc, "externd_factor_batched_ex")
     return res, statuses
 
 

@@ -2259,8 +2259,32 @@ int externd_factor_batched(int count, const float* const* A, const int64_t* m, c
                            const double* tau, int iters, const uint64_t* seed, uint8_t* const* B_out,
                            float* const* D_out, uint8_t* const* C_out, double* const* energy_out, int* status_out,
                            void* stream) {
+    return externd_factor_batched_ex(count, A, m, n, mu, tau, iters, seed, B_out, D_out, C_out, energy_out,
+                                     status_out, stream, nullptr);
+}
+
+int externd_factor_batched_ex(int count, const float* const* A, const int64_t* m, const int64_t* n,
+                              const double* mu, const double* tau, int iters, const uint64_t* seed,
+                              uint8_t* const* B_out, float* const* D_out, uint8_t* const* C_out,
+                              double* const* energy_out, int* status_out, void* stream,
+                              const externd_batch_options* opt) {
     if (count < 1 || !A || !m || !n || !mu || !tau || !seed || !B_out || !D_out || !C_out || !status_out)
         return EXTERND_EINVAL;
+    if (opt) {
+        bool bad = opt->sweeps < 0 || opt->sweeps > 1000;
+        if (opt->h) {
+            for (int b = 0; b < count; ++b) {
+                const double lam = opt->lambda ? opt->lambda[b] : 0.0;
+                bad = bad || !opt->h[b] || !std::isfinite(lam) || lam < 0.0;
+            }
+        } else {
+            bad = bad || opt->lambda != nullptr;
+        }
+        if (bad) {
+            for (int c = 0; c < count; ++c) status_out[c] = EXTERND_EINVAL;
+            return EXTERND_EINVAL;
+        }
+    }
     std::vector<ProbIn> ins(count);
     for (int b = 0; b < count; ++b) {
         int64_t k = 0;
@@ -2274,6 +2298,14 @@ int externd_factor_batched(int count, const float* const* A, const int64_t* m, c
         I.A = A[b]; I.m = m[b]; I.n = n[b]; I.k = k; I.tau = tau[b]; I.iters = iters; I.seed = seed[b];
         I.B = B_out[b]; I.D = D_out[b]; I.C = C_out[b]; I.energy = energy_out ? energy_out[b] : nullptr;
         I.mode = MODE_FACTOR;
+        if (opt) {
+            if (opt->h) {
+                I.h = opt->h[b];
+                I.lambda = opt->lambda ? opt->lambda[b] : 0.0;
+            }
+            I.sweeps = opt->sweeps;
+            I.sweep_energy = opt->sweep_energy_out ? opt->sweep_energy_out[b] : nullptr;
+        }
     }
     RunOpts ro;
     return run(ins.data(), count, ro, reinterpret_cast<cudaStream_t>(stream), status_out);

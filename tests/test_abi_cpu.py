@@ -122,7 +122,8 @@ def _c_layout(struct, fields):
 
 
 @pytest.mark.parametrize("cls,struct,rename", [(_lib.Options, "externd_options", {"lambda_": "lambda"}),
-                                               (_lib.Stats, "externd_stats", {})])
+                                               (_lib.Stats, "externd_stats", {}),
+                                               (_lib.BatchOptions, "externd_batch_options", {"lambda_": "lambda"})])
 def test_ctypes_structs_match_the_header(cls, struct, rename):
     names = [n for n, _ in cls._fields_]
     size, offs = _c_layout(struct, [rename.get(n, n) for n in names])
@@ -145,3 +146,28 @@ def test_factor_options_are_validated_before_device_work():
         rc = L.externd_factor_ex(ctypes.addressof(A), 2, 2, 1.0, 0.7, 15, 0, ctypes.addressof(buf),
                                  ctypes.addressof(buf), ctypes.addressof(buf), None, None, ctypes.byref(opt))
         assert rc == einval, kw
+
+
+def test_batched_options_are_validated_before_device_work():
+    L = _lib.load()
+    einval = ext.STATUS["EINVAL"]
+    buf = (ctypes.c_uint8 * 64)()
+    A = (ctypes.c_float * 4)(1, 2, 3, 4)
+    h = (ctypes.c_float * 2)(1, 1)
+    P2 = ctypes.c_void_p * 2
+    a = P2(ctypes.addressof(A), ctypes.addressof(A))
+    bp = P2(ctypes.addressof(buf), ctypes.addressof(buf))
+    m = (ctypes.c_int64 * 2)(2, 2)
+    mu = (ctypes.c_double * 2)(1.0, 1.0)
+    tau = (ctypes.c_double * 2)(0.7, 0.7)
+    seed = (ctypes.c_uint64 * 2)(0, 1)
+    for kw in ({"h": P2(ctypes.addressof(h), None)},                 # weights for one matrix only
+               {"h": P2(ctypes.addressof(h), ctypes.addressof(h)), "lambda_": (ctypes.c_double * 2)(0.0, -1.0)},
+               {"lambda_": (ctypes.c_double * 2)(0.0, 0.0)},        # lambda without weights
+               {"sweeps": -1}, {"sweeps": 1001}):
+        opt = _lib.BatchOptions()
+        for k, v in kw.items():
+            setattr(opt, k, ctypes.cast(v, ctypes.c_void_p) if not isinstance(v, int) else v)
+        st = (ctypes.c_int * 2)()
+        rc = L.externd_factor_batched_ex(2, a, m, m, mu, tau, 15, seed, bp, bp, bp, None, st, None, ctypes.byref(opt))
+        assert rc == einval and list(st) == [einval, einval], kw
