@@ -248,7 +248,7 @@ def run_ours(args):
     fits = k_total * (1 + w.sweeps)
 
     def step(inputs):
-        if w.weighted and not w.sweeps:
+        if w.weighted and not w.sweeps and w.count == 1:
             f = ext.factor_weighted(inputs[0], hw[0], w.mu[0], w.tau[0], lam=w.lam, iters=w.iters, seed=w.seeds[0])
             return [f], f.stats
         if w.count == 1:
@@ -256,7 +256,8 @@ def run_ours(args):
                            grid=args.grid, pending=args.pending, sweeps=w.sweeps,
                            h=hw[0] if w.weighted else None, lam=w.lam)
             return [f], f.stats
-        res, st = ext.factor_batched(inputs, w.mu, w.tau, iters=w.iters, seeds=list(w.seeds))
+        res, st = ext.factor_batched(inputs, w.mu, w.tau, iters=w.iters, seeds=list(w.seeds), hs=hw,
+                                     lams=[w.lam] * w.count if w.weighted else None, sweeps=w.sweeps)
         assert all(s == 0 for s in st), st
         return res, res[0].stats
 

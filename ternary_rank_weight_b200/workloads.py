@@ -119,6 +119,10 @@ WORKLOADS = {
         "attn_16x1536x1536_mu2.5_tau_cycle", tuple((1536, 1536) for _ in range(16)),
         tuple(range(100, 116)), tuple(2.5 for _ in range(16)),
         tuple((0.7, 1.0, 2.0)[b % 3] for b in range(16))),
+    "attn_16x1536x1536_mu2.5_tau_cycle_weighted_sweep1": Workload(
+        "attn_16x1536x1536_mu2.5_tau_cycle_weighted_sweep1", tuple((1536, 1536) for _ in range(16)),
+        tuple(range(100, 116)), tuple(2.5 for _ in range(16)),
+        tuple((0.7, 1.0, 2.0)[b % 3] for b in range(16)), weighted=True, sweeps=1),
     "mlp_2560x6912_bf16_mu3_tau1.0_weighted": Workload(
         "mlp_2560x6912_bf16_mu3_tau1.0_weighted", ((2560, 6912),), (2,), (3.0,), (1.0,), bf16=True, weighted=True),
     "mlp_2560x6912_bf16_mu3_tau1.0_sweep1": Workload(
