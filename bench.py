@@ -49,12 +49,15 @@ def _peaks():
 
 
 def _kernel_source_hash() -> str:
-    """Hash of the ALS kernel's code (line comments and blank lines removed, so editing a
-    comment does not invalidate the recorded ncu traffic)."""
+    """Hash of the device code: externd_kernels.cuh and externd.cu up to its host half (which
+    starts at `struct ProbIn`), line comments and blank lines removed, so editing a comment or
+    the host entry points does not invalidate the recorded ncu traffic."""
     h = hashlib.sha256()
     for name in ("externd.cu", "externd_kernels.cuh"):
         with open(os.path.join(ROOT, "ternary_rank_weight_b200", "csrc", name), encoding="utf-8") as f:
             for line in f:
+                if line.startswith("struct ProbIn"):
+                    break
                 code = line.split("//", 1)[0].rstrip()
                 if code:
                     h.update(code.encode() + b"\n")
