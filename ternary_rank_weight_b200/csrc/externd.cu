@@ -942,12 +942,17 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
                 const float hword = cb < len ? __ldg(hw + cb) : 0.f;
                 const uint32_t pz = lane < L ? pnz[(base + i) * Ls + lane] : 0u;
                 const uint32_t pg = lane < L ? psg[(base + i) * Ls + lane] : 0u;
-                for (uint32_t mk = chi; mk; mk &= mk - 1u) {
-                    const int b = __ffs(mk) - 1;
+                // each lane walks its own bits (pz & chi) in increasing order; every lane takes
+                // part in each shuffle, so the loop runs the warp's largest count
+                uint32_t mine = pz & chi;
+                const int rounds = (int)__reduce_max_sync(FULL, (unsigned)__popc(mine));
+                for (int t = 0; t < rounds; ++t) {
+                    const int b = mine ? __ffs(mine) - 1 : 0;
                     const double hv = (double)__shfl_sync(FULL, hword, b);
-                    if ((pz >> b) & 1u) {
+                    if (mine) {
                         const double dv = (((dni >> b) & 1u) ? -1.0 : 1.0) * (((dti >> b) & 1u) ? 2.0 : 1.0);
                         dotw_acc += ((pg >> b) & 1u) ? -hv * dv : hv * dv;
+                        mine &= mine - 1u;
                     }
                 }
             } else if (lane < L) {
