@@ -515,3 +515,31 @@ def test_weighted_refinement_with_uniform_weights_is_the_plain_one():
     assert np.array_equal(r.B, rw.B) and np.array_equal(r.C, rw.C)
     assert np.allclose(r.D, rw.D, rtol=1e-13, atol=0)
     assert np.allclose(r.sweep_energy, rw.sweep_energy, rtol=0, atol=1e-12)
+
+
+def test_weighted_refinement_visit_is_bounded_by_brute_force():
+    """k = 1 under column weights h~: the visit's decrease of sum h~_j A_ij^2 lies between the
+    stored pair's weighted least-squares decrease and the best over every ternary pair, each
+    from the weighted Frobenius inner product <X, Y> = sum_ij h~_j X_ij Y_ij."""
+    rng = np.random.default_rng(9)
+    pairs = [(np.array(u), np.array(v)) for u in itertools.product((-1, 0, 1), repeat=3)
+             for v in itertools.product((-1, 0, 1), repeat=4) if any(u) and any(v)]
+    for trial in range(5):
+        A = rng.standard_normal((3, 4))
+        h = rng.uniform(0.05, 3.0, size=4)
+        hw = ora.normalized_weights(h, 0.0).astype(np.float64)
+        inner = lambda X, Y: float(np.sum(hw[None, :] * X * Y))
+        f = ora.greedy_als_weighted(A, h, 0.0, k=1, tau=0.7, seed=trial)
+        r = ora.refine_sweeps(A, f.B, f.D, f.C, sweeps=1, tau=0.7, h=h)
+        na = inner(A, A)
+
+        def best(u, v):
+            M = np.outer(_tf(u), _tf(v))
+            return inner(A, M) ** 2 / inner(M, M)
+
+        top = max(best(u, v) for u, v in pairs)
+        stored = best(f.B[:, 0], f.C[0])
+        R = A - ora.reconstruct(r.B, r.D, r.C)
+        got = na - inner(R, R)
+        assert stored - 1e-9 <= got <= top + 1e-9
+        assert 1.0 - inner(R, R) / na == pytest.approx(r.energy_final, abs=1e-12)
