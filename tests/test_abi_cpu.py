@@ -171,3 +171,18 @@ def test_batched_options_are_validated_before_device_work():
         st = (ctypes.c_int * 2)()
         rc = L.externd_factor_batched_ex(2, a, m, m, mu, tau, 15, seed, bp, bp, bp, None, st, None, ctypes.byref(opt))
         assert rc == einval and list(st) == [einval, einval], kw
+
+
+def test_binding_rejects_bad_inputs_before_the_library_call():
+    import torch
+    with pytest.raises(ValueError):
+        ext.factor(torch.zeros(3, 4, dtype=torch.float64), 1.0, 0.7)       # not float32
+    with pytest.raises(ValueError):
+        ext.factor(np.zeros(5, dtype=np.float32), 1.0, 0.7)                # not a matrix
+    with pytest.raises(ValueError):
+        ext.factor_weighted(np.ones((3, 4), dtype=np.float32), np.ones(3, dtype=np.float32), 1.0, 0.7)
+    with pytest.raises(ValueError):
+        ext.factor(np.ones((3, 4), dtype=np.float32), 1.0, 0.7, h=np.ones(5, dtype=np.float32))
+    with pytest.raises(ext.ExterndError) as e:
+        ext.factor(np.ones((3, 4), dtype=np.float32), 0.01, 0.7)          # k rounds to 0
+    assert e.value.status == ext.STATUS["EINVAL"]
