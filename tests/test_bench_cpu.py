@@ -80,3 +80,26 @@ def test_traffic_record_applies_only_to_its_source(bench, tmp_path, monkeypatch)
     rec["source_sha256"] = "0" * 64
     (root / "profiles" / "als_kernel_traffic.json").write_text(json.dumps(rec))
     assert bench._ncu_traffic("wl") is None
+
+
+def test_reference_arm_prints_once_on_rank_zero(tmp_path):
+    """`bench.py --impl reference` under several ranks: rank 0 times the oracle on a bounded
+    sample and prints one JSON line with the contract's keys; every other rank exits 0 silently."""
+    import subprocess
+    import sys
+    base = dict(os.environ, WORLD_SIZE="2", MASTER_ADDR="127.0.0.1", MASTER_PORT="29555")
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1", "--warmup", "0",
+           "--workload", "iid_256x256_mu2_tau0.7", "--ref-budget", "1"]
+    r1 = subprocess.run(cmd, env=dict(base, RANK="1", LOCAL_RANK="1"), capture_output=True, text=True, timeout=300)
+    assert r1.returncode == 0 and r1.stdout.strip() == ""
+    r0 = subprocess.run(cmd, env=dict(base, RANK="0", LOCAL_RANK="0"), capture_output=True, text=True, timeout=300)
+    assert r0.returncode == 0
+    lines = [l for l in r0.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
