@@ -1146,8 +1146,8 @@ __device__ __forceinline__ unsigned sum_use_end(int64_t r, int64_t kk) { return 
 // stored u_i, v_i (packed rows of B and C) and d_i, record d_i, n_old and the pending
 // slot in s.scal[8], [9], [11], and append the added-back term d_i u_i v_i^T as pending
 // component L with coefficient -d_i.  Leaves u = u_i in nzU/sgU/ulist and v = 0.
-// Returns nnz(u_i), or -1 if the group aborted.  Kept out of line: it runs once per
-// visit and would otherwise crowd the registers of the half-step loop.
+// Returns nnz(u_i), or -1 if the group aborted.  (Inlined: as a call, the registers
+// the half-step loop keeps live across it spilled more than the inlined code does.)
 __device__ __forceinline__ int refine_begin(const Prob& P, int64_t i, int q, int Gg, const KCfg& cfg, const Smem& s,
                                          GroupSync* gs, bool skip, unsigned sum_use, int L, int Ls, int Wm, int Wn,
                                          int64_t c0, int validV, int64_t r0, int validU, int pitchU, int pitchV,
