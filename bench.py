@@ -362,7 +362,7 @@ def run_ours(args):
 def run_matvec(args):
     """Time externd_matvec on the factors of the workload's matrix 0 (factorization untimed).
 
-    Between timed calls a 256 MiB buffer is overwritten (L2 is 126 MB), so every call
+    Before every timed call a 1 GiB buffer is overwritten (L2 is 126 MB), so every call
     streams the packed factors from HBM; each call is timed alone with CUDA events."""
     import torch
     import ternary_rank_weight_b200 as ext
