@@ -117,8 +117,13 @@ int externd_factor_weighted(const float* A, int64_t m, int64_t n, double mu, dou
  *   - A matrix whose scratch would exceed EXTERND_NOALLOC_SCRATCH_BYTES is
  *     rejected with EXTERND_ELIMIT (about 8 m n + k ceil(m/4) bytes; e.g.
  *     1024 x 1024 at mu = 2 needs ~8.6 MiB).
- *   - The first call on a device looks up the array's device address; make that
- *     first call before any stream capture.
+ *   - Every call looks up the array's device address (cudaGetSymbolAddress, with
+ *     the caller's device current), so the address stays right after a
+ *     cudaDeviceReset.  The first call on a device may load the library's device
+ *     code there: make that first call before any stream capture on the device.
+ *   - Like every entry point of this library the call is synchronous: it waits
+ *     for `stream` before returning, because the return code carries the device
+ *     status (also when it fails after queueing work on the array).
  *   - All calls share the one array and it keeps the previous call's contents
  *     (each call clears what must start at zero).  Calls that overlap on the GPU
  *     (e.g. on two streams, or from two host threads) race and corrupt each

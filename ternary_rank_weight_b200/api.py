@@ -209,7 +209,9 @@ def factor_noalloc(A: torch.Tensor, mu: float, tau: float, iters: int = 15, seed
     Python side too.  Calls share the scratch and must not overlap on the GPU."""
     if not (isinstance(A, torch.Tensor) and A.is_cuda and A.dtype == torch.float32 and A.dim() == 2):
         raise ValueError("A must be a 2-D float32 CUDA tensor")
-    A = A.contiguous()
+    if not A.is_contiguous():
+        # a contiguous copy would be an allocation on the caller's side
+        raise ValueError("A must be contiguous (row-major): factor_noalloc makes no copies")
     m, n = A.shape
     k = rank(m, n, mu)
     if k < 1:

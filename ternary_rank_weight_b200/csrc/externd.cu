@@ -2114,10 +2114,13 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
 
 done:
     if (dws && !fixed) { cudaFreeAsync(dws, stream); cudaStreamSynchronize(stream); }
+    // fixed scratch: work already queued on the shared array must end before the
+    // call returns, also when a later queueing step failed
+    if (fixed && rc != EXTERND_OK) cudaStreamSynchronize(stream);
     for (int i = 0; i < 5; ++i)
         if (ev[i]) cudaEventDestroy(ev[i]);
     cudaGetLastError();
-    g_last = st;
+    if (!fixed) g_last = st;   // the allocation-free call records no events and leaves the stats alone
     return rc;
 }
 
@@ -2144,28 +2147,21 @@ int validate_factor(const float* A, int64_t m, int64_t n, double mu, double tau,
 // Scratch memory of externd_factor_noalloc: one file-scope device array,
 // EXTERND_NOALLOC_SCRATCH_BYTES on every device that loads this library, kept
 // until the process exits.  Host code may not use the array's name as a device
-// address: the address is looked up once per device with cudaGetSymbolAddress.
+// address (it names a host-side shadow).  The address is looked up with
+// cudaGetSymbolAddress on every call, with the caller's device current: a cached
+// address could outlive its context (after cudaDeviceReset the module is loaded
+// again and the array may sit elsewhere).
 // ---------------------------------------------------------------------------
 static __device__ __align__(256) unsigned char g_noalloc_scratch[EXTERND_NOALLOC_SCRATCH_BYTES];
 
 namespace {
 
-std::mutex g_noalloc_mu;
-unsigned char* g_noalloc_base[64] = {};
-
-// Device address of the scratch array on the current device (set up on first use).
+// Device address of the scratch array in the current context.
 int noalloc_scratch(unsigned char** out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return EXTERND_ECUDA; }
-    if (dev < 0 || dev >= 64) return EXTERND_ECUDA;
-    std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (!g_noalloc_base[dev]) {
-        void* ptr = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-        if (e != cudaSuccess || ptr == nullptr) { cudaGetLastError(); return EXTERND_ECUDA; }
-        g_noalloc_base[dev] = static_cast<unsigned char*>(ptr);
-    }
-    *out = g_noalloc_base[dev];
+    void* ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess || ptr == nullptr) { cudaGetLastError(); return EXTERND_ECUDA; }
+    *out = static_cast<unsigned char*>(ptr);
     return EXTERND_OK;
 }
 

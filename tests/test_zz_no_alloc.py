@@ -53,3 +53,14 @@ def test_noalloc_rejects_what_it_cannot_do_without_memory():
     rc = _lib.load().externd_factor_noalloc(host.ctypes.data, 8, 8, 1.0, 0.7, 15, 0, B.data_ptr(), D.data_ptr(),
                                             C.data_ptr(), None, torch.cuda.current_stream().cuda_stream)
     assert rc == ext.STATUS["EINVAL"]
+
+
+def test_noalloc_refuses_a_copy_and_leaves_the_stats_alone():
+    A = torch.from_numpy(llm_matrix(128, 96, seed=9)).cuda()
+    ref = ext.factor(A, 1.0, 0.7, seed=1)
+    before = ext.last_stats()
+    f = ext.factor_noalloc(A, 1.0, 0.7, seed=1)
+    assert torch.equal(f.B, ref.B) and torch.equal(f.D, ref.D)
+    assert ext.last_stats() == before          # this entry point records no figures
+    with pytest.raises(ValueError):
+        ext.factor_noalloc(A.t(), 1.0, 0.7)    # non-contiguous: would need a copy
