@@ -238,7 +238,7 @@ class Factorization:
     energy_final: float        # explicit 1 - ||A - Ahat||^2 / ||A||^2 at the end
     norm_a2: float
     margins: np.ndarray        # per component min relative threshold margin
-    safeguard_hits: int        # components whose decrease fell below max_rc R_rc^2
+    safeguard_hits: int        # components whose decrease fell below the single-entry bound ||R||^2 / (m n)
     residual_norms: np.ndarray = field(default=None)  # ||R_i||^2 explicit, per component
 
     @property
@@ -271,10 +271,12 @@ def greedy_als(A: np.ndarray, k: int, tau: float, iters: int = 15, seed: int = 0
     for i in range(k):
         u0, _, _ = ternarize(start_normals(seed, i, m), tau)
         fit = fit_component(R, u0, tau, iters)
-        # Appendix 7 reading: the single-entry component (one residual entry of
-        # largest magnitude) decreases ||R||^2 by max R_rc^2; count components
-        # where ALS did worse (the pages say this never happens in practice).
-        if fit.decrease < float(np.max(R * R)):
+        # §7 "Monotone residual decrease and convergence": a single-entry component
+        # (u = e_r, v = e_c at the largest |R_rc|) removes max R_rc^2 >= ||R||^2 / (m n),
+        # the single-entry bound behind the geometric rate in m n; the safeguard steps in
+        # when the ALS decrease falls below that bound.  Count those components (the
+        # pages say it never happens in practice); no substitution is made.
+        if fit.decrease < float(np.sum(R * R)) / (m * n):
             hits += 1
         if fit.d != 0.0:
             R -= fit.d * np.outer(fit.u.astype(np.float64), fit.v.astype(np.float64))

@@ -15,6 +15,7 @@ import numpy as np
 import pytest
 
 from oracle import externd_oracle as ora
+from ternary_rank_weight_b200.workloads import llm_matrix
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -231,6 +232,41 @@ def test_safeguard_never_activates_on_small_workload():
     A = np.random.default_rng(0).standard_normal((96, 80)).astype(np.float32) * 0.02
     f = ora.greedy_als(A, k=160, tau=1.0, seed=0)
     assert f.safeguard_hits == 0
+
+
+def test_safeguard_counts_an_isolated_entry_that_als_cannot_reach():
+    """§7: the safeguard bound is the single-entry decrease ||R||^2 / (m n).
+
+    An entry alone in its row and column (R[r, :] = R[:, c] = 0 elsewhere) that the
+    start vector misses (u0_r = 0) is invisible to the alternation: u_r = 0 gives
+    x_c = 0, hence v_c = 0, hence y_r = 0 and u_r = 0 again.  The ALS decrease then
+    comes from the noise alone, far below the bound set by the big entry."""
+    m, n, tau, seed = 12, 10, 0.7, 3
+    u0, _, _ = ora.ternarize(ora.start_normals(seed, 0, m), tau)
+    r = int(np.nonzero(u0 == 0)[0][0])
+    c = 4
+    A = (np.random.default_rng(5).standard_normal((m, n)) * 0.01).astype(np.float32)
+    A[r, :] = 0.0
+    A[:, c] = 0.0
+    A[r, c] = 50.0
+    f = ora.greedy_als(A, k=1, tau=tau, seed=seed)
+    assert f.B[r, 0] == 0 and f.C[0, c] == 0
+    decrease = f.energy[0] * f.norm_a2
+    assert decrease < f.norm_a2 / (m * n)
+    assert f.safeguard_hits == 1
+
+
+def test_safeguard_bound_is_the_mean_not_the_largest_entry():
+    """On the LLM-like generator (heavy-tailed outlier columns) the ALS decrease of late
+    components is smaller than the largest squared residual entry but far above the
+    single-entry bound ||R||^2 / (m n): the count stays 0, as the pages state."""
+    A = llm_matrix(160, 128, seed=3, outliers=4)
+    k = 256
+    f = ora.greedy_als(A, k=k, tau=0.7, seed=1)
+    assert f.safeguard_hits == 0
+    R = ora.residual_after(A, f.B, f.D, f.C, k - 1)
+    last_decrease = (f.energy[k - 1] - f.energy[k - 2]) * f.norm_a2
+    assert float(np.max(R * R)) > last_decrease > 10 * float(np.sum(R * R)) / R.size
 
 
 def test_v_step_threshold_uses_output_length():
