@@ -23,9 +23,10 @@
  * - `stream` is a cudaStream_t (NULL = legacy default stream) of the current
  *   device.  Every call is stream-ordered and SYNCHRONOUS: it returns after
  *   the work finished, because the return code carries the device status.
- * - The library keeps no pointer after return.  Workspace (a copy of the
- *   residual in two layouts, exchange buffers, start trits) is allocated
- *   stream-ordered inside the call and released before it returns.
+ * - The library keeps no pointer after return.  Workspace (the residual in
+ *   two layouts, each entry an fp32 pair hi + lo; exchange buffers, start
+ *   trits) is allocated stream-ordered inside the call and released before it
+ *   returns.
  * - Ternary outputs are packed 2 bits per trit: 00 = 0, 01 = +1, 11 = -1
  *   (10 is never written).  Trit j of a row sits in byte j/4, bits 2*(j%4).
  *   A row of `len` trits occupies externd_trit_bytes(len) bytes (ceil(len/4)
@@ -115,8 +116,8 @@ int externd_factor_weighted(const float* A, int64_t m, int64_t n, double mu, dou
  *   - A, B_out, D_out, C_out, energy_out must be DEVICE pointers (EXTERND_EINVAL
  *     otherwise: host buffers would need staging memory).
  *   - A matrix whose scratch would exceed EXTERND_NOALLOC_SCRATCH_BYTES is
- *     rejected with EXTERND_ELIMIT (about 8 m n + k ceil(m/4) bytes; e.g.
- *     1024 x 1024 at mu = 2 needs ~8.6 MiB).
+ *     rejected with EXTERND_ELIMIT (about 16 m n + k ceil(m/4) bytes: the residual
+ *     in two layouts, each as an fp32 pair; e.g. 1024 x 1024 at mu = 2 needs ~16.5 MiB).
  *   - Every call looks up the array's device address (cudaGetSymbolAddress, with
  *     the caller's device current), so the address stays right after a
  *     cudaDeviceReset.  The first call on a device may load the library's device
@@ -237,6 +238,27 @@ int externd_debug_halfstep(const float* R, int64_t m, int64_t n, int transpose,
 int externd_debug_start_trits(int64_t m, int64_t k, double tau, uint64_t seed, uint8_t* out,
                               void* stream);
 
+/* Test hook: ONE component of §2.3 (15 alternating fits, scale) run by the kernel of
+ * externd_factor on a caller-given residual state, with a trace of every half-step.
+ *   R          [in]  m x n fp32 row-major: the residual as stored (device or host).
+ *   u0         [in]  packed start trits of the component (externd_trit_bytes(m) bytes).
+ *   n_pend           0 .. 31 rank-1 terms d_j u_j v_j^T held pending, i.e. applied as the
+ *                    corrections the factorization uses for deflations not yet folded into R:
+ *                    the component is fitted to R - sum_j d_j u_j v_j^T.  EXTERND_ELIMIT above
+ *                    the lazy-deflation depth of the launch minus one.
+ *   pend_d     [in]  n_pend fp64 scales; pend_u [in] n_pend rows of externd_trit_bytes(m);
+ *                    pend_v [in] n_pend rows of externd_trit_bytes(n) (DEVICE pointers).
+ *   pre_v, thr_v, trit_v, pre_u, thr_u, trit_u  [out]  the trace of externd_options with
+ *                    trace_count = 1 (DEVICE pointers).
+ *   D_out, d64_out   [out] the scale d in fp32 and fp64; u_out, v_out [out] the final trits.
+ *   grid             CTAs serving the matrix (0 = the factorization's automatic choice).
+ * Returns EXTERND_OK or a negative externd_status. */
+int externd_debug_component(const float* R, int64_t m, int64_t n, double tau, int iters, const uint8_t* u0,
+                            int n_pend, const double* pend_d, const uint8_t* pend_u, const uint8_t* pend_v,
+                            double* pre_v, double* thr_v, uint8_t* trit_v, double* pre_u, double* thr_u,
+                            uint8_t* trit_u, float* D_out, double* d64_out, uint8_t* u_out, uint8_t* v_out,
+                            int grid, void* stream);
+
 /* Knobs and extra outputs for externd_factor_ex.  Zero-initialise and set
  * only what is needed. */
 typedef struct {
@@ -260,6 +282,28 @@ typedef struct {
     /* Importance weights of §2.5 (see externd_factor_weighted); h = NULL: plain objective. */
     const float* h;
     double lambda;
+    /* Test hook: a trace of visits [trace_first, trace_first + trace_count) of this
+     * factorization, written by the kernel that computes it.  Visit i < k is the extraction of
+     * component i; with refinement sweeps, visit (s + 1) k + i is sweep s's refit of component i
+     * (a refit that reaches a fixed point stops early and leaves its later rows unwritten).
+     * For every V-step (x = R^T u, §2.3 step 1) and U-step (y = R v) of a traced visit it stores
+     * the output vector exactly
+     * as the threshold saw it (after the corrections of deflations not yet folded into R, rounded
+     * to the 44 significant bits the kernel exchanges), the threshold tau * mean |.| and the
+     * resulting trits.  DEVICE pointers; trace_pre_v = NULL turns the trace off.  The window must
+     * lie inside [0, k (1 + sweeps)), trit rows 16-byte aligned (EXTERND_EINVAL otherwise).
+     *   trace_pre_v  [trace_count][iters][n] fp64     trace_pre_u  [trace_count][iters][m] fp64
+     *   trace_thr_v  [trace_count][iters] fp64        trace_thr_u  [trace_count][iters] fp64
+     *   trace_trit_v [trace_count][iters] rows of externd_trit_bytes(n)
+     *   trace_trit_u [trace_count][iters] rows of externd_trit_bytes(m) */
+    int64_t trace_first;
+    int64_t trace_count;
+    double* trace_pre_v;
+    double* trace_thr_v;
+    uint8_t* trace_trit_v;
+    double* trace_pre_u;
+    double* trace_thr_u;
+    uint8_t* trace_trit_u;
 } externd_options;
 
 /* externd_factor with options (opt may be NULL). */
@@ -295,6 +339,9 @@ typedef struct {
     int64_t phase_cycles[11];  /* [10]: exchanged words found not yet visible by CTA 0; [0..9]: SM cycles of CTA 0 of matrix 0 (diagnostics): GEMV loads, GEMV reduce +
                                   emit, publish, wait, partials + first loads, threshold, compaction,
                                   start vector, output + pending push, deflation fold */
+    int64_t safeguard_hits;    /* extraction components whose ALS decrease p^2 / (nnz(u) nnz(v)) fell below the
+                                  single-entry bound ||R||^2 / (m n) of §7 ("Monotone residual decrease and
+                                  convergence"), summed over matrices; counted only, no component is replaced */
 } externd_stats;
 
 int externd_last_stats(externd_stats* out);

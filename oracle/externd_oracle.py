@@ -404,6 +404,21 @@ def weighted_ls_scale(R: np.ndarray, u: np.ndarray, v: np.ndarray, hw: np.ndarra
     return p / (float(u @ u) * float(w @ (v * v)))
 
 
+def half_step_weighted(R: np.ndarray, trits_in: np.ndarray, tau: float, transpose: bool, hw: np.ndarray):
+    """One half of §2.3 step 1 under the §2.5 objective.
+
+    transpose=True : x = R^T u, v = T_tau(x)         (V-step on the plain residual: h~ cancels)
+    transpose=False: y = R (h~ v), u = T_tau(y)      (U-step on the weighted target W = R diag(h~))
+    Returns (pre-threshold vector, threshold, output trits, fallback_used)."""
+    if transpose:
+        return half_step(R, trits_in, tau, True)
+    R = np.asarray(R, dtype=np.float64)
+    w = np.asarray(trits_in, dtype=np.float64) * np.asarray(hw, dtype=np.float64)
+    pre = R @ w
+    out, thr, fb = ternarize(pre, tau)
+    return pre, thr, out, fb
+
+
 def greedy_als_weighted(A: np.ndarray, h: np.ndarray, lam: float, k: int, tau: float, iters: int = 15,
                         seed: int = 0) -> Factorization:
     """§2.5 with §2.3: V-step on the plain residual (h~ cancels there), U-step on

@@ -25,6 +25,7 @@ EXPORTS = (
     "externd_strerror",
     "externd_debug_halfstep",
     "externd_debug_start_trits",
+    "externd_debug_component",
     "externd_last_stats",
     "externd_transpose_trits",
     "externd_matvec",
@@ -44,6 +45,14 @@ class Options(ctypes.Structure):
         ("sweep_energy_out", ctypes.c_void_p),
         ("h", ctypes.c_void_p),
         ("lambda_", ctypes.c_double),
+        ("trace_first", ctypes.c_int64),
+        ("trace_count", ctypes.c_int64),
+        ("trace_pre_v", ctypes.c_void_p),
+        ("trace_thr_v", ctypes.c_void_p),
+        ("trace_trit_v", ctypes.c_void_p),
+        ("trace_pre_u", ctypes.c_void_p),
+        ("trace_thr_u", ctypes.c_void_p),
+        ("trace_trit_u", ctypes.c_void_p),
     ]
 
 
@@ -79,6 +88,7 @@ class Stats(ctypes.Structure):
         ("workspace_bytes", ctypes.c_size_t),
         ("sweep_kept", ctypes.c_int64),
         ("phase_cycles", ctypes.c_int64 * 11),
+        ("safeguard_hits", ctypes.c_int64),
     ]
 
     def as_dict(self):
@@ -127,6 +137,9 @@ def load():
     L.externd_debug_halfstep.restype = c_int
     L.externd_debug_start_trits.argtypes = [i64, i64, dbl, u64, vp, vp]
     L.externd_debug_start_trits.restype = c_int
+    L.externd_debug_component.argtypes = [vp, i64, i64, dbl, c_int, vp, c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                          vp, vp, vp, vp, c_int, vp]
+    L.externd_debug_component.restype = c_int
     L.externd_last_stats.argtypes = [ctypes.POINTER(Stats)]
     L.externd_last_stats.restype = c_int
     L.externd_transpose_trits.argtypes = [vp, i64, i64, vp, vp]

@@ -116,6 +116,7 @@ class Factors:
     d64: Optional[torch.Tensor] = None
     stats: dict = field(default_factory=dict)
     sweep_energy: Optional[torch.Tensor] = None   # float64 [sweeps]: energy after each refinement sweep
+    trace: Optional["Trace"] = None               # test hook: traced half-steps (factor(..., trace=...))
 
     def trits(self):
         """Unpacked (B as m x k int8, C as k x n int8) on the host."""
@@ -124,14 +125,45 @@ class Factors:
         return Bu, Cu
 
 
+@dataclass
+class Trace:
+    """Half-steps of components [first, first + count) as the kernel saw them (test hook).
+
+    pre_v[c, t] / pre_u[c, t]: the published output of the t-th V-step (x = R^T u, length n)
+    and U-step (y = R v, length m) of component first + c; thr_*: the thresholds; trit_*:
+    the packed trits those half-steps produced."""
+    first: int
+    count: int
+    pre_v: torch.Tensor
+    thr_v: torch.Tensor
+    trit_v: torch.Tensor
+    pre_u: torch.Tensor
+    thr_u: torch.Tensor
+    trit_u: torch.Tensor
+
+    @staticmethod
+    def alloc(first: int, count: int, iters: int, m: int, n: int, device) -> "Trace":
+        """Buffers pre-filled with NaN, so half-steps a visit did not run stay recognisable."""
+        nan = dict(fill_value=float("nan"), dtype=torch.float64, device=device)
+        return Trace(first, count,
+                     torch.full((count, iters, n), **nan), torch.full((count, iters), **nan),
+                     torch.zeros((count, iters, trit_bytes(n)), dtype=torch.uint8, device=device),
+                     torch.full((count, iters, m), **nan), torch.full((count, iters), **nan),
+                     torch.zeros((count, iters, trit_bytes(m)), dtype=torch.uint8, device=device))
+
+
 def factor(A, mu: float, tau: float, iters: int = 15, seed: int = 0, *, grid: int = 0, pending: int = 0,
            wait_limit_s: float = 0.0, fault_skip_cta: Optional[int] = None, want_d64: bool = False,
-           want_energy: bool = True, sweeps: int = 0, h=None, lam: float = 0.0, stream=None) -> Factors:
+           want_energy: bool = True, sweeps: int = 0, h=None, lam: float = 0.0, trace=None,
+           stream=None) -> Factors:
     """Factor one matrix (externd_factor_ex).  Outputs are allocated where A lives.
 
     sweeps: §2.4 refinement sweeps after extraction (``energy`` keeps the extraction
     energies, ``sweep_energy`` the energy after each sweep).  h, lam: §2.5 importance
-    weights (per-column second moments, n float32 values), or None for the plain objective."""
+    weights (per-column second moments, n float32 values), or None for the plain objective.
+    trace: (first, count) -- test hook, records the half-steps of those visits: visit
+    i < k extracts component i, visit (s + 1) k + i is sweep s's refit of component i
+    (``Factors.trace``; A must be on the GPU)."""
     A = _as_matrix(A)
     m, n = A.shape
     if h is not None:
@@ -156,13 +188,21 @@ def factor(A, mu: float, tau: float, iters: int = 15, seed: int = 0, *, grid: in
     opt.sweep_energy_out = _ptr(SE)
     opt.h = _ptr(h)
     opt.lambda_ = float(lam)
+    tr = None
+    if trace is not None:
+        if not A.is_cuda:
+            raise ValueError("trace needs A on the GPU")
+        tr = Trace.alloc(int(trace[0]), int(trace[1]), int(iters), m, n, A.device)
+        opt.trace_first, opt.trace_count = tr.first, tr.count
+        opt.trace_pre_v, opt.trace_thr_v, opt.trace_trit_v = _ptr(tr.pre_v), _ptr(tr.thr_v), _ptr(tr.trit_v)
+        opt.trace_pre_u, opt.trace_thr_u, opt.trace_trit_u = _ptr(tr.pre_u), _ptr(tr.thr_u), _ptr(tr.trit_u)
     with _on_device(A):
         rc = _lib.load().externd_factor_ex(_ptr(A), m, n, float(mu), float(tau), int(iters), int(seed),
                                            _ptr(B), _ptr(D), _ptr(C), _ptr(E),
                                            _stream(stream, A.device), ctypes.byref(opt))
     _check(rc, "externd_factor")
     return Factors(B=B, D=D, C=C, energy=E, m=m, n=n, k=k, mu=float(mu), tau=float(tau), d64=d64,
-                   stats=last_stats(), sweep_energy=SE)
+                   stats=last_stats(), sweep_energy=SE, trace=tr)
 
 
 def _weights(h, n: int) -> torch.Tensor:
@@ -322,6 +362,31 @@ def debug_halfstep(R, trits_in: torch.Tensor, tau: float, transpose: bool, *, st
                                                 _ptr(pre), _ptr(thr), _ptr(out), _stream(stream, R.device))
     _check(rc, "externd_debug_halfstep")
     return pre, float(thr[0].item()), out
+
+
+def debug_component(R, u0: torch.Tensor, tau: float, iters: int = 15, *, pend_d=None, pend_u=None, pend_v=None,
+                    grid: int = 0, stream=None):
+    """One component of §2.3 on a given residual state (externd_debug_component, test hook).
+
+    R: m x n float32 (GPU); u0: packed start trits (GPU); pend_d / pend_u / pend_v: pending
+    rank-1 terms (fp64 scales, packed u rows, packed v rows, all on the GPU) that the kernel
+    applies as lazy-deflation corrections.  Returns (Trace with count 1, d64, packed u, packed v)."""
+    R = _as_matrix(R)
+    m, n = R.shape
+    dev = R.device
+    tr = Trace.alloc(0, 1, int(iters), m, n, dev)
+    D = torch.empty((1,), dtype=torch.float32, device=dev)
+    d64 = torch.empty((1,), dtype=torch.float64, device=dev)
+    uo = torch.empty((1, trit_bytes(m)), dtype=torch.uint8, device=dev)
+    vo = torch.empty((1, trit_bytes(n)), dtype=torch.uint8, device=dev)
+    npend = 0 if pend_d is None else int(pend_d.shape[0])
+    with _on_device(R):
+        rc = _lib.load().externd_debug_component(
+            _ptr(R), m, n, float(tau), int(iters), _ptr(u0), npend, _ptr(pend_d), _ptr(pend_u), _ptr(pend_v),
+            _ptr(tr.pre_v), _ptr(tr.thr_v), _ptr(tr.trit_v), _ptr(tr.pre_u), _ptr(tr.thr_u), _ptr(tr.trit_u),
+            _ptr(D), _ptr(d64), _ptr(uo), _ptr(vo), int(grid), _stream(stream, dev))
+    _check(rc, "externd_debug_component")
+    return tr, float(d64[0].item()), uo[0], vo[0]
 
 
 def debug_start_trits(m: int, k: int, tau: float, seed: int, device="cuda", *, stream=None) -> torch.Tensor:

@@ -110,7 +110,7 @@ constexpr int NTI = 256;
 
 __global__ void __launch_bounds__(NTI) init_kernel(const Prob* __restrict__ probs) {
     const Prob& P = probs[blockIdx.y];
-    if (P.mode != MODE_FACTOR) return;
+    if (P.mode != MODE_FACTOR || P.start_given) return;
     const int64_t m = P.m;
     __shared__ double shd[NTI / 32 + 1];
     __shared__ double shm[NTI / 32 + 1];
@@ -340,22 +340,18 @@ __device__ __forceinline__ void emit_tagged(double v, int64_t gi, unsigned long 
     S += fabs(__longlong_as_double((long long)(w & ~0xFFull)));
 }
 
-// acc += sum_u s_u v_u for one batch of loaded rows (s_u = +1/-1 from the sign bit
-// of the list entry).  The batch is summed in fp32 with one fused multiply-add per
-// term (|error| <= (U-1) 2^-24 sum|terms|), then converted and added to the fp64
-// accumulator: this keeps the GEMV at ~2 instructions per element.
+// acc += sum_u c_u v_u for one batch of loaded rows, in fp64: every term c_u v_u is
+// exact in fp64 (c_u is +-1, +-2, or an fp32 weight times that; v_u is fp32, so the
+// product has at most 48 significant bits) and each fused multiply-add rounds once,
+// so a running sum of N terms is within (N - 1) 2^-53 sum|terms| of the exact sum.
 template <int VEC, int U>
 __device__ __forceinline__ void accumulate_batch(double* acc, const float* cf, float (*v)[VEC]) {
-    float b[VEC];
-    #pragma unroll
-    for (int e = 0; e < VEC; ++e) b[e] = 0.f;
     #pragma unroll
     for (int u = 0; u < U; ++u) {
+        const double c = (double)cf[u];
         #pragma unroll
-        for (int e = 0; e < VEC; ++e) b[e] = fmaf(cf[u], v[u][e], b[e]);   // inactive slots hold v = 0
+        for (int e = 0; e < VEC; ++e) acc[e] = fma(c, (double)v[u][e], acc[e]);   // inactive slots hold v = 0
     }
-    #pragma unroll
-    for (int e = 0; e < VEC; ++e) acc[e] += (double)b[e];
 }
 
 // Rows per batch of the GEMV: enough loads in flight per thread within the register budget.
@@ -505,7 +501,7 @@ __device__ __forceinline__ void gemv_dispatch(int vec, const float* blk, int pit
 // lane b holds row b's mask over the components; tC_l(c) comes from the
 // per-output masks cnz/csg.  scratch: 64 words per warp.
 template <int VEC>
-__device__ void flush_block(float* blk, int pitch, int64_t rows, int valid, int L, int Ls, const double* pd,
+__device__ void flush_block(float* blk, float* blo, int pitch, int64_t rows, int valid, int L, int Ls, const double* pd,
                             const uint32_t* pnzR, const uint32_t* psgR, const uint32_t* cnz, const uint32_t* csg,
                             uint32_t* scratch) {
     const int nvec = pitch / VEC;
@@ -535,9 +531,7 @@ __device__ void flush_block(float* blk, int pitch, int64_t rows, int valid, int 
             if (!rnz) continue;
             const uint32_t rsn = my[32 + b];
             float* p = blk + ((wr << 5) + b) * pitch + j * VEC;
-            float v[VEC];
-            load_vec<VEC>(p, v);
-            bool changed = false;
+            float* plo = blo + ((wr << 5) + b) * pitch + j * VEC;
             #pragma unroll
             for (int e = 0; e < VEC; ++e) {
                 const int c = j * VEC + e;
@@ -551,24 +545,24 @@ __device__ void flush_block(float* blk, int pitch, int64_t rows, int valid, int 
                     bits &= bits - 1u;
                     corr += ((neg >> l) & 1u) ? -pd[l] : pd[l];
                 }
-                v[e] = (float)((double)v[e] - corr);
-                changed = true;
-            }
-            if (changed) {
-                #pragma unroll
-                for (int e = 0; e < VEC; ++e) p[e] = v[e];
+                // hi + lo is exact in fp64; the new value rounds once in fp64, then splits
+                // into its nearest fp32 (hi) and the fp32 rounding of the rest (lo)
+                const double nv = ((double)__ldcg(p + e) + (double)__ldcg(plo + e)) - corr;
+                const float hi = (float)nv;
+                p[e] = hi;
+                plo[e] = (float)(nv - (double)hi);
             }
         }
         __syncwarp();
     }
 }
 
-__device__ __forceinline__ void flush_dispatch(int vec, float* blk, int pitch, int64_t rows, int valid, int L, int Ls,
-                                               const double* pd, const uint32_t* pnzR, const uint32_t* psgR,
+__device__ __forceinline__ void flush_dispatch(int vec, float* blk, float* blo, int pitch, int64_t rows, int valid, int L,
+                                               int Ls, const double* pd, const uint32_t* pnzR, const uint32_t* psgR,
                                                const uint32_t* cnz, const uint32_t* csg, uint32_t* scratch) {
-    if (vec == 4) flush_block<4>(blk, pitch, rows, valid, L, Ls, pd, pnzR, psgR, cnz, csg, scratch);
-    else if (vec == 2) flush_block<2>(blk, pitch, rows, valid, L, Ls, pd, pnzR, psgR, cnz, csg, scratch);
-    else flush_block<1>(blk, pitch, rows, valid, L, Ls, pd, pnzR, psgR, cnz, csg, scratch);
+    if (vec == 4) flush_block<4>(blk, blo, pitch, rows, valid, L, Ls, pd, pnzR, psgR, cnz, csg, scratch);
+    else if (vec == 2) flush_block<2>(blk, blo, pitch, rows, valid, L, Ls, pd, pnzR, psgR, cnz, csg, scratch);
+    else flush_block<1>(blk, blo, pitch, rows, valid, L, Ls, pd, pnzR, psgR, cnz, csg, scratch);
 }
 
 // Start trits (2-bit packed words) -> masks and list; returns nnz.
@@ -1188,6 +1182,18 @@ __device__ __forceinline__ int refine_begin(const Prob& P, int64_t i, int q, int
     return nU0;
 }
 
+// Test-hook trace of one half-step (lead CTA): the published output vector (the
+// values the threshold saw), the threshold and the resulting trits.
+// (Kept out of line: inlined at its two call sites it made the half-step loop spill
+// several times more.)
+__device__ __noinline__ void trace_halfstep(const unsigned long long* gvec, int64_t len, double thr, const uint32_t* nz,
+                                            const uint32_t* sg, double* pre, double* thr_out, uint8_t* trits,
+                                            int64_t row_bytes) {
+    for (int64_t t = threadIdx.x; t < len; t += NT) pre[t] = untag(ld_relaxed_u64(gvec + t));
+    if (threadIdx.x == 0) *thr_out = thr;
+    pack_row(nz, sg, (int)((len + 31) >> 5), reinterpret_cast<uint32_t*>(trits), row_bytes / 4);
+}
+
 // Factor (or run one debug half-step of) one matrix with this CTA group.
 // Returns false if the group aborted.
 template <bool WTD, bool SWP>
@@ -1236,7 +1242,15 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
 
     double RN2 = N0;
     int L = 0;
-    unsigned long long sum_nu = 0, sum_nv = 0, sum_du = 0, sum_dv = 0, sum_nunv = 0, hs = 0, fb = 0;
+    // test hook: rank-1 terms d_j u_j v_j^T supplied by the caller, held pending (not yet
+    // folded into R) exactly as the factorization holds its own recent components
+    for (int j = 0; j < P.n_pend; ++j) {
+        build_from_trits(P.pend_u + j * (P.b_bytes / 4), P.b_bytes / 4, m, s.nzU, s.sgU, s.ulist, pitchV, s);
+        build_from_trits(P.pend_v + j * (P.c_bytes / 4), P.c_bytes / 4, n, s.nzV, s.sgV, s.vlist, pitchU, s);
+        push_pending(s, L, Ls, P.pend_d[j], Wm, Wn, c0, validV, r0, validU);
+        ++L;
+    }
+    unsigned long long sum_nu = 0, sum_nv = 0, sum_du = 0, sum_dv = 0, sum_nunv = 0, hs = 0, fb = 0, sgh = 0;
     const int64_t kk = (mode == MODE_FACTOR) ? P.k : 1;
     // §2.4 refinement sweeps: visits kk .. nvis-1 revisit components 0 .. kk-1 in order.
     // (Little of this is held in registers across the visit loop: the half-steps already
@@ -1258,6 +1272,7 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
     for (int64_t vis = 0; vis < nvis; ++vis) {
         const int64_t i = vis % kk;
         const bool refine = SWP && vis >= kk;   // a refinement visit of component i
+        const bool trv = P.tr_pre_v != nullptr && lead && vis >= P.tr_first && vis - P.tr_first < P.tr_count;
         // refinement state in shared memory (s.scal[8..11]): d_i, n_old = nnz(u_i) v_i^T diag(h~) v_i,
         // this CTA's part of p_old, and the pending slot of the added-back term
         // a new component: the GEMV sums restart from zero and the previous trits
@@ -1318,6 +1333,11 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
                     pold_part = block_sum(pold_part, s.red);
                     if (tid == 0) s.scal[10] = pold_part;
                 }
+                if (trv) {
+                    const int64_t at = (vis - P.tr_first) * P.iters + it;
+                    trace_halfstep(P.xbuf, n, thr, s.nzV, s.sgV, P.tr_pre_v + at * n, P.tr_thr_v + at,
+                                   P.tr_trit_v + at * P.c_bytes, P.c_bytes);
+                }
                 fb += (s.scal[1] != 0.0) ? 1 : 0;
                 sum_nu += (unsigned long long)nU;
                 sum_du += (unsigned long long)dU;
@@ -1349,6 +1369,11 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
                                     s.osgU, s.ulist, pitchV, s, L, Ls, s.pnzU, s.psgU, s.dotU, s.coef, true, thr, dU,
                                     gs, cfg.limit_ns, P.status, ok);
             if (!ok) return false;
+            if (trv) {
+                const int64_t at = (vis - P.tr_first) * P.iters + it;
+                trace_halfstep(P.ybuf, m, thr, s.nzU, s.sgU, P.tr_pre_u + at * m, P.tr_thr_u + at,
+                               P.tr_trit_u + at * P.b_bytes, P.b_bytes);
+            }
             p = s.scal[0];
             fb += (s.scal[1] != 0.0) ? 1 : 0;
             ++hs;
@@ -1397,7 +1422,12 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
                 s.pd[La] = dold - di;   // net pending term of the stored pair
             }
         }
-        if (!refine) RN2 -= p * dnew;
+        // §7 safeguard condition: the ALS decrease p d below the single-entry bound ||R||^2 / (m n)
+        // (counted, not substituted; RN2 is ||R||^2 before this component)
+        if (!refine) {
+            sgh += (p * dnew < RN2 / ((double)m * (double)n)) ? 1ull : 0ull;
+            RN2 -= p * dnew;
+        }
         sum_nunv += (unsigned long long)nU * (unsigned long long)nV;
         if (lead) {
             // (selects rather than branches on `take` keep the half-step loop's register allocation)
@@ -1423,8 +1453,10 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
         // at the end of the extraction and of the run
         if (L + (vis + 1 >= kk ? 2 : 1) > cfg.Lcap || vis == kk - 1 || vis == nvis - 1) {
             uint32_t* scratch = reinterpret_cast<uint32_t*>(s.red);
-            flush_dispatch(P.pv.vec, blkV, pitchV, m, validV, L, Ls, s.pd, s.pnzU, s.psgU, s.cnzV, s.csgV, scratch);
-            flush_dispatch(P.pu.vec, blkU, pitchU, n, validU, L, Ls, s.pd, s.pnzV, s.psgV, s.cnzU, s.csgU, scratch);
+            flush_dispatch(P.pv.vec, blkV, P.Rv_lo + P.pv.block_offset(q, m), pitchV, m, validV, L, Ls, s.pd, s.pnzU,
+                           s.psgU, s.cnzV, s.csgV, scratch);
+            flush_dispatch(P.pu.vec, blkU, P.Ru_lo + P.pu.block_offset(q, n), pitchU, n, validU, L, Ls, s.pd, s.pnzV,
+                           s.psgV, s.cnzU, s.csgU, scratch);
             __syncthreads();
             for (int c = tid; c < pitchV; c += NT) { s.cnzV[c] = 0u; s.csgV[c] = 0u; }
             for (int c = tid; c < pitchU; c += NT) { s.cnzU[c] = 0u; s.csgU[c] = 0u; }
@@ -1434,14 +1466,15 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
         phase_mark(s, 9);
     }
 
-    // ---- explicit ||R_k||^2 from the folded fp32 residual (V-layout covers all of R)
+    // ---- explicit ||R_k||^2 from the folded residual hi + lo (V-layout covers all of R)
     double rs = 0.0;
     if (validV > 0) {
+        const float* bloV = P.Rv_lo + P.pv.block_offset(q, m);
         const int64_t tot = m * (int64_t)validV;
         for (int64_t t = tid; t < tot; t += NT) {
             const int64_t r = t / validV;
             const int c = (int)(t - r * validV);
-            const double v = (double)__ldcg(blkV + r * pitchV + c);
+            const double v = (double)__ldcg(blkV + r * pitchV + c) + (double)__ldcg(bloV + r * pitchV + c);
             rs += v * v * (wtd ? (double)__ldg(P.hw + c0 + c) : 1.0);
         }
     }
@@ -1460,6 +1493,7 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
         P.stats->residual2 = R2;
         P.stats->norm_a2 = N0;
         P.stats->sweep_kept = SWP ? (unsigned long long)s.scal[12] : 0ull;
+        P.stats->safeguard = sgh;
         phase_mark(s, 7);
         for (int k2 = 0; k2 < 11; ++k2) P.stats->phase[k2] = s.clk[k2];
         __threadfence();
@@ -1719,6 +1753,15 @@ struct ProbIn {
     double* pre_out;
     double* thr_out;
     uint8_t* trit_out;
+    // test hooks (device pointers)
+    const uint8_t* start_in;  // caller-given start trits of component 0 (k = 1), or null
+    int n_pend;
+    const double* pend_d;
+    const uint8_t* pend_u;
+    const uint8_t* pend_v;
+    int64_t tr_first, tr_count;
+    double *tr_pre_v, *tr_thr_v, *tr_pre_u, *tr_thr_u;
+    uint8_t *tr_trit_v, *tr_trit_u;
 };
 
 struct RunOpts {
@@ -1811,8 +1854,10 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
     weighted = weighted ? 1 : 0;
     while (Lcap > 1 && als_smem_bytes(m_max, n_max, Lcap, pv_max, pu_max, weighted) > di.smem_optin) --Lcap;
     if (opt.pending > 0 && opt.pending < Lcap) Lcap = opt.pending;
-    for (int b = 0; b < np; ++b)
+    for (int b = 0; b < np; ++b) {
         if (in[b].mode == MODE_FACTOR && in[b].sweeps > 0 && Lcap < 2) return EXTERND_ELIMIT;   // add-back + refit
+        if (in[b].n_pend > 0 && in[b].n_pend + 1 > Lcap) return EXTERND_ELIMIT;   // caller's terms + the component
+    }
     const size_t smem = als_smem_bytes(m_max, n_max, Lcap, pv_max, pu_max, weighted);
     if (smem > di.smem_optin) return EXTERND_ELIMIT;
 
@@ -1827,7 +1872,7 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
 
     // ---- plan the workspace
     std::vector<Prob> probs(np);
-    std::vector<size_t> off_rv(np), off_ru(np), off_x(np), off_y(np), off_sums(np), off_start(np), off_norm(np), off_A(np),
+    std::vector<size_t> off_rv(np), off_ru(np), off_rvl(np), off_rul(np), off_x(np), off_y(np), off_sums(np), off_start(np), off_norm(np), off_A(np),
         off_B(np), off_C(np), off_D(np), off_E(np), off_d64(np), off_pre(np), off_thr(np), off_tro(np), off_hw(np), off_h(np),
         off_dk(np), off_SE(np);
     size_t ctl = 0;
@@ -1854,9 +1899,21 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
         P.b_bytes = (int64_t)trit_bytes(I.m);
         P.c_bytes = (int64_t)trit_bytes(I.n);
         P.start_words = (int64_t)trit_bytes(I.mode == MODE_HALF_U ? I.n : I.m) / 4;
+        P.start_given = I.start_in != nullptr;
+        P.n_pend = I.n_pend;
+        P.pend_d = I.pend_d;
+        P.pend_u = reinterpret_cast<const uint32_t*>(I.pend_u);
+        P.pend_v = reinterpret_cast<const uint32_t*>(I.pend_v);
+        P.tr_first = I.tr_first;
+        P.tr_count = I.tr_count;
+        P.tr_pre_v = I.tr_pre_v; P.tr_thr_v = I.tr_thr_v; P.tr_trit_v = I.tr_trit_v;
+        P.tr_pre_u = I.tr_pre_u; P.tr_thr_u = I.tr_thr_u; P.tr_trit_u = I.tr_trit_u;
         P.n_norm_part = ((I.m + 31) / 32) * ((I.n + 31) / 32);
         off_rv[b] = ws; ws += round_up(sizeof(float) * (size_t)P.pv.total(I.m), 256);
         off_ru[b] = ws; ws += round_up(sizeof(float) * (size_t)P.pu.total(I.n), 256);
+        // low halves of the residual (zero until the first fold)
+        off_rvl[b] = ws; ws += round_up(sizeof(float) * (size_t)P.pv.total(I.m), 256);
+        off_rul[b] = ws; ws += round_up(sizeof(float) * (size_t)P.pu.total(I.n), 256);
         // exchange buffers: zero = "no half-step yet" (tags are 1..255)
         off_x[b] = ws; ws += round_up(sizeof(unsigned long long) * (size_t)I.n, 256);
         off_y[b] = ws; ws += round_up(sizeof(unsigned long long) * (size_t)I.m, 256);
@@ -1933,6 +1990,8 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
         P.hw = off_hw[b] == SIZE_MAX ? nullptr : reinterpret_cast<const float*>(dws + off_hw[b]);
         P.Rv = reinterpret_cast<float*>(dws + off_rv[b]);
         P.Ru = reinterpret_cast<float*>(dws + off_ru[b]);
+        P.Rv_lo = reinterpret_cast<float*>(dws + off_rvl[b]);
+        P.Ru_lo = reinterpret_cast<float*>(dws + off_rul[b]);
         P.xbuf = reinterpret_cast<unsigned long long*>(dws + off_x[b]);
         P.ybuf = reinterpret_cast<unsigned long long*>(dws + off_y[b]);
         P.sums = reinterpret_cast<unsigned long long*>(dws + off_sums[b]);
@@ -1985,6 +2044,11 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
                                                    reinterpret_cast<unsigned*>(dws + off_nonfin) + 2 * b + 1);
             CK(cudaGetLastError());
             ++launches;
+        }
+        if (I.start_in) {
+            // caller-given start trits -> start row of component 0
+            CK(cudaMemcpyAsync(dws + off_start[b], I.start_in, (size_t)probs[b].start_words * 4,
+                               is_device_ptr(I.start_in) ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice, stream));
         }
         if (I.mode != MODE_FACTOR) {
             // debug input trits -> start row
@@ -2106,6 +2170,7 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
                 for (int k2 = 0; k2 < 11; ++k2) st.phase_cycles[k2] = (int64_t)d.phase[k2];
                 st.sweep_kept = (int64_t)d.sweep_kept;
             }
+            st.safeguard_hits += (int64_t)d.safeguard;
         }
     }
     rc = EXTERND_OK;
@@ -2122,6 +2187,18 @@ done:
     cudaGetLastError();
     if (!fixed) g_last = st;   // the allocation-free call records no events and leaves the stats alone
     return rc;
+}
+
+// Trace buffers of the test hooks: all device memory, trit rows 16-byte aligned, the
+// window inside [0, visits) (k extraction visits, then k per refinement sweep).
+int check_trace(int64_t first, int64_t count, int64_t k, const double* pv, const double* tv, const uint8_t* rv,
+                const double* pu, const double* tu, const uint8_t* ru) {
+    if (first < 0 || count < 1 || first + count > k) return EXTERND_EINVAL;
+    const void* ptrs[6] = {pv, tv, rv, pu, tu, ru};
+    for (const void* q : ptrs)
+        if (!q || !is_device_ptr(q)) return EXTERND_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(rv) & 15u) || (reinterpret_cast<uintptr_t>(ru) & 15u)) return EXTERND_EINVAL;
+    return EXTERND_OK;
 }
 
 int check_rows_aligned(const void* p) {
@@ -2211,6 +2288,15 @@ int externd_factor_ex(const float* A, int64_t m, int64_t n, double mu, double ta
             if (!std::isfinite(opt->lambda) || opt->lambda < 0.0) return EXTERND_EINVAL;
             I.h = opt->h;
             I.lambda = opt->lambda;
+        }
+        if (opt->trace_pre_v) {
+            if ((rc = check_trace(opt->trace_first, opt->trace_count, k * (1 + (int64_t)opt->sweeps), opt->trace_pre_v, opt->trace_thr_v,
+                                  opt->trace_trit_v, opt->trace_pre_u, opt->trace_thr_u, opt->trace_trit_u)) != EXTERND_OK)
+                return rc;
+            I.tr_first = opt->trace_first;
+            I.tr_count = opt->trace_count;
+            I.tr_pre_v = opt->trace_pre_v; I.tr_thr_v = opt->trace_thr_v; I.tr_trit_v = opt->trace_trit_v;
+            I.tr_pre_u = opt->trace_pre_u; I.tr_thr_u = opt->trace_thr_u; I.tr_trit_u = opt->trace_trit_u;
         }
     }
     int st = 0;
@@ -2334,6 +2420,37 @@ int externd_debug_start_trits(int64_t m, int64_t k, double tau, uint64_t seed, u
     I.B = out;
     RunOpts ro;
     ro.init_only = true;
+    int st = 0;
+    return run(&I, 1, ro, reinterpret_cast<cudaStream_t>(stream), &st);
+}
+
+int externd_debug_component(const float* R, int64_t m, int64_t n, double tau, int iters, const uint8_t* u0,
+                            int n_pend, const double* pend_d, const uint8_t* pend_u, const uint8_t* pend_v,
+                            double* pre_v, double* thr_v, uint8_t* trit_v, double* pre_u, double* thr_u,
+                            uint8_t* trit_u, float* D_out, double* d64_out, uint8_t* u_out, uint8_t* v_out, int grid,
+                            void* stream) {
+    if (!R || !u0 || !D_out || !d64_out || !u_out || !v_out) return EXTERND_EINVAL;
+    if (m < 1 || n < 1 || iters < 1 || !std::isfinite(tau) || tau < 0 || grid < 0) return EXTERND_EINVAL;
+    if (m > INT_MAX / 2 || n > INT_MAX / 2) return EXTERND_ELIMIT;
+    if (n_pend < 0 || n_pend >= MAX_PENDING) return n_pend < 0 ? EXTERND_EINVAL : EXTERND_ELIMIT;
+    if (n_pend > 0) {
+        if (!pend_d || !pend_u || !pend_v || !is_device_ptr(pend_d) || !is_device_ptr(pend_u) || !is_device_ptr(pend_v))
+            return EXTERND_EINVAL;
+        if (check_rows_aligned(pend_u) || check_rows_aligned(pend_v)) return EXTERND_EINVAL;
+    }
+    int rc = check_trace(0, 1, 1, pre_v, thr_v, trit_v, pre_u, thr_u, trit_u);
+    if (rc != EXTERND_OK) return rc;
+    if (check_rows_aligned(u_out) || check_rows_aligned(v_out)) return EXTERND_EINVAL;
+    ProbIn I = {};
+    I.A = R; I.m = m; I.n = n; I.k = 1; I.tau = tau; I.iters = iters; I.mode = MODE_FACTOR;
+    I.B = u_out; I.C = v_out; I.D = D_out; I.d64 = d64_out;
+    I.start_in = u0;
+    I.n_pend = n_pend; I.pend_d = pend_d; I.pend_u = pend_u; I.pend_v = pend_v;
+    I.tr_first = 0; I.tr_count = 1;
+    I.tr_pre_v = pre_v; I.tr_thr_v = thr_v; I.tr_trit_v = trit_v;
+    I.tr_pre_u = pre_u; I.tr_thr_u = thr_u; I.tr_trit_u = trit_u;
+    RunOpts ro;
+    ro.grid = grid;
     int st = 0;
     return run(&I, 1, ro, reinterpret_cast<cudaStream_t>(stream), &st);
 }

@@ -33,11 +33,16 @@
 //    bit masks in shared memory and applied as rank-1 corrections to each
 //    GEMV output (x -= sum_j d_j (u_j . u) v_j, the integer dot products kept
 //    up to date from the changed trits); every L components each CTA folds
-//    them into its own two blocks in one pass (fp64 sum, one fp32 rounding
-//    per entry).
-//  * Accumulation: batches of at most 16 signed fp32 residual entries are
-//    summed in fp32 with fused multiply-adds, batch sums are added in fp64,
-//    and the threshold decisions are taken on fp64 values like the oracle.
+//    them into its own two blocks in one pass.  Each residual entry is held as
+//    an fp32 pair hi + lo: a fold computes hi + lo - sum_j ... in fp64 and
+//    splits the result again, so the pair tracks the exact residual to ~2^-48
+//    of its magnitude however many folds it went through, and the GEMVs read
+//    hi alone, which is within 2^-24 of the current residual entry (a plain
+//    fp32 residual would keep the rounding errors of early folds, made at the
+//    scale of A, while the residual shrinks).
+//  * Accumulation: every signed fp32 residual entry is added to an fp64 sum
+//    (each term is exact in fp64, each add rounds once), and the threshold
+//    decisions are taken on fp64 values like the oracle.
 //  * Every device-side wait is bounded by %globaltimer; a wait that runs out
 //    raises a status word and the kernel returns.
 #pragma once
@@ -104,6 +109,7 @@ struct DevStats {
     double pad;
     unsigned long long phase[11];   // SM cycles of CTA 0 per phase (see run_problem); [10] stale words seen
     unsigned long long sweep_kept;  // refinement visits that kept the stored pair (rescaled)
+    unsigned long long safeguard;   // components whose ALS decrease fell below ||R||^2 / (m n)
 };
 
 enum Mode { MODE_FACTOR = 0, MODE_HALF_V = 1, MODE_HALF_U = 2 };
@@ -127,6 +133,8 @@ struct Prob {
     int64_t b_bytes, c_bytes;
     float* Rv;                // V-layout blocks
     float* Ru;                // U-layout blocks
+    float* Rv_lo;             // low halves of the V-layout residual: R = Rv + Rv_lo (see the fold)
+    float* Ru_lo;             // low halves of the U-layout residual
     unsigned long long* xbuf; // n, published V-step outputs (tagged fp64 words, zero-initialised)
     unsigned long long* ybuf; // m, published U-step outputs (tagged fp64 words, zero-initialised)
     unsigned long long* sums; // 2 G, per-CTA partial sums, double-buffered by use (tagged, zero-initialised)
@@ -139,6 +147,19 @@ struct Prob {
     unsigned* nonfinite;
     int* status;
     DevStats* stats;
+    int start_given;          // 1: the start trits were supplied by the caller (no generated start vector)
+    int n_pend;               // pending rank-1 terms supplied by the caller, applied before component 0
+    const double* pend_d;     // their scales (n_pend)
+    const uint32_t* pend_u;   // their u trits (n_pend rows of b_bytes)
+    const uint32_t* pend_v;   // their v trits (n_pend rows of c_bytes)
+    int64_t tr_first, tr_count;   // traced visits [tr_first, tr_first + tr_count): components 0 .. k-1, then
+                                  // sweep s revisits component i as visit (s + 1) k + i
+    double* tr_pre_v;         // [tr_count][iters][n] published V-step outputs
+    double* tr_thr_v;         // [tr_count][iters]
+    double* tr_pre_u;         // [tr_count][iters][m] published U-step outputs
+    double* tr_thr_u;         // [tr_count][iters]
+    uint8_t* tr_trit_v;       // [tr_count][iters] rows of c_bytes: the V-step trits
+    uint8_t* tr_trit_u;       // [tr_count][iters] rows of b_bytes: the U-step trits
     double* pre_out;          // debug half-step outputs
     double* thr_out;
     uint8_t* trit_out;

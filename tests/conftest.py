@@ -25,3 +25,13 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_sessionfinish(session, exitstatus):
+    """Write the divergences the parity tests recorded to $EXTERND_DIVERGENCE_REPORT (if set)."""
+    path = os.environ.get("EXTERND_DIVERGENCE_REPORT")
+    if not path:
+        return
+    mod = sys.modules.get("_parity")   # the module the tests imported (tests/ is on sys.path)
+    if mod is not None:
+        mod.write_report(path)

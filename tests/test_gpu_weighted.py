@@ -1,10 +1,11 @@
 """Parity of the importance-weighted factorization (§2.5) with the oracle.
 
 Same tolerances as the plain path (the arithmetic is the same plus one fp32
-weight per U-step term, exact in the fp32 batch sums' error bound): trits equal
-away from threshold ties (1e-5 relative), d within 1e-4 relative until the first
-divergence, which must start at a near-tie of the oracle's trajectory; weighted
-energy within 2e-3.
+weight per U-step term, whose product with an fp32 residual entry is exact in
+fp64): trits equal away from threshold ties (1e-5 relative), d within 1e-4
+relative until the first divergence; the first divergent component is traced
+and replayed by the oracle, and its first differing half-step may differ only at
+entries within 1e-5 relative of the threshold; weighted energy within 2e-3.
 """
 import numpy as np
 import pytest
@@ -13,6 +14,8 @@ import torch
 import ternary_rank_weight_b200 as ext
 from oracle import externd_oracle as ora
 from ternary_rank_weight_b200.workloads import WORKLOADS, importance_weights, llm_matrix
+
+import _parity
 
 pytestmark = pytest.mark.gpu
 
@@ -37,7 +40,7 @@ def test_uniform_weights_reproduce_the_plain_factorization_bit_for_bit():
 def test_weighted_matches_oracle(m, n, mu, tau, lam):
     A = llm_matrix(m, n, seed=m + n, outliers=min(2, n))
     h = importance_weights(n, seed=n)
-    fw = ext.factor_weighted(torch.from_numpy(A).cuda(), h, mu, tau, lam=lam, seed=3)
+    fw = ext.factor(torch.from_numpy(A).cuda(), mu, tau, seed=3, h=h, lam=lam, want_d64=True)
     Bg, Cg = fw.trits()
     ref = ora.greedy_als_weighted(A, h.astype(np.float64), lam, k=fw.k, tau=tau, seed=3)
     e = fw.energy.cpu().numpy()
@@ -48,7 +51,9 @@ def test_weighted_matches_oracle(m, n, mu, tau, lam):
     if div > 0:
         assert np.allclose(D[:div], ref.D[:div].astype(np.float32), rtol=1e-4, atol=0)
     if div < ref.k:
-        assert ref.margins[div] < 1e-3, (div, ref.margins[div])
+        hwn = ora.normalized_weights(h.astype(np.float64), lam).astype(np.float64)
+        nd = _parity.teacher_forced(A, fw, 3, tau, [div], ("weighted first divergence", m, n), hw=hwn, h=h, lam=lam)
+        assert nd == 1
     # the weighted energy of the reconstruction agrees with the incremental one
     hw = ora.normalized_weights(h.astype(np.float64), lam)
     Ah = ext.reconstruct(fw.B, fw.D, fw.C, m, n).cpu().numpy()
@@ -86,24 +91,11 @@ def test_weighted_headline_workload_full_size_sampled():
     w = WORKLOADS["mlp_2560x6912_bf16_mu3_tau1.0"]
     A = w.matrix(0)
     h = importance_weights(6912, seed=2)
-    fw = ext.factor_weighted(torch.from_numpy(A).cuda(), h, w.mu[0], w.tau[0], lam=0.0, seed=w.seeds[0])
+    fw = ext.factor(torch.from_numpy(A).cuda(), w.mu[0], w.tau[0], seed=w.seeds[0], h=h, lam=0.0, want_d64=True)
     e = fw.energy.cpu().numpy()
     assert fw.k == 7680 and np.all(np.diff(e) >= -1e-12) and 0.5 < e[-1] < 1.0
     assert fw.stats["residual_energy"] == pytest.approx(e[-1], abs=1e-4)
-    Bg, Cg = fw.trits()
-    D = fw.D.cpu().numpy().astype(np.float64)
     hw = ora.normalized_weights(h.astype(np.float64), 0.0).astype(np.float64)
-    mism = 0
-    for i in (0, 1, 700, 7679):
-        R = ora.residual_after(A, Bg, D, Cg, i)
-        u, _, _ = ora.ternarize(ora.start_normals(w.seeds[0], i, 2560), w.tau[0])
-        for _ in range(15):
-            v, _, _ = ora.ternarize(R.T @ u.astype(np.float64), w.tau[0])
-            y = R @ (hw * v.astype(np.float64))
-            u, _, _ = ora.ternarize(y, w.tau[0])
-        if np.array_equal(u, Bg[:, i]) and np.array_equal(v, Cg[i]):
-            d = float(u.astype(np.float64) @ y) / (np.count_nonzero(u) * hw[v != 0].sum())
-            assert D[i] == pytest.approx(d, rel=1e-4)
-        else:
-            mism += 1
-    assert mism <= 1
+    ndiv = _parity.teacher_forced(A, fw, w.seeds[0], w.tau[0], (0, 1, 700, 7679), "weighted mlp 2560x6912 samples",
+                                  hw=hw, h=h, lam=0.0)
+    assert ndiv <= 1

@@ -579,3 +579,42 @@ def test_weighted_refinement_visit_is_bounded_by_brute_force():
         got = na - inner(R, R)
         assert stored - 1e-9 <= got <= top + 1e-9
         assert 1.0 - inner(R, R) / na == pytest.approx(r.energy_final, abs=1e-12)
+
+
+def test_weighted_half_step_brute_force_and_special_cases():
+    """§2.5: the U-step thresholds y_r = sum_c R_rc h~_c v_c, the V-step ignores h~."""
+    rng = np.random.default_rng(17)
+    R = rng.standard_normal((5, 7))
+    hw = rng.uniform(0.1, 2.0, 7)
+    v = rng.integers(-1, 2, 7).astype(np.int8)
+    u = rng.integers(-1, 2, 5).astype(np.int8)
+    pre, thr, out, _ = ora.half_step_weighted(R, v, 0.7, False, hw)
+    for r in range(5):
+        acc = 0.0
+        for c in range(7):
+            acc += R[r, c] * hw[c] * float(v[c])
+        assert pre[r] == pytest.approx(acc, rel=1e-14, abs=1e-15)
+    assert thr == pytest.approx(0.7 * sum(abs(x) for x in pre) / 5, rel=1e-14)
+    # V-step: the weights cancel (the same as the plain half-step)
+    a = ora.half_step_weighted(R, u, 0.7, True, hw)
+    b = ora.half_step(R, u, 0.7, True)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[2], b[2])
+    # uniform weights: the plain U-step
+    c = ora.half_step_weighted(R, v, 0.7, False, np.ones(7))
+    d = ora.half_step(R, v, 0.7, False)
+    assert np.array_equal(c[0], d[0]) and np.array_equal(c[2], d[2])
+
+
+def test_weighted_half_steps_reproduce_the_weighted_factorization():
+    """Alternating half_step_weighted from the start vector gives greedy_als_weighted's first component."""
+    A = llm_matrix(40, 56, seed=6, outliers=2)
+    h = np.random.default_rng(3).uniform(0.2, 3.0, 56)
+    f = ora.greedy_als_weighted(A, h, 0.05, k=1, tau=1.0, seed=2)
+    hw = ora.normalized_weights(h, 0.05).astype(np.float64)
+    u, _, _ = ora.ternarize(ora.start_normals(2, 0, 40), 1.0)
+    R = A.astype(np.float64)
+    for _ in range(15):
+        _, _, v, _ = ora.half_step_weighted(R, u, 1.0, True, hw)
+        _, _, u, _ = ora.half_step_weighted(R, v, 1.0, False, hw)
+    assert np.array_equal(u, f.B[:, 0]) and np.array_equal(v, f.C[0])
+    assert ora.weighted_ls_scale(R, u, v, hw) == pytest.approx(f.D[0], rel=1e-12)

@@ -37,7 +37,7 @@ def test_noalloc_matches_the_allocating_entry_point_on_two_calls():
 
 
 def test_noalloc_rejects_what_it_cannot_do_without_memory():
-    big = torch.zeros((2048, 4096), device="cuda")      # 8 m n = 64 MiB of residual copies > scratch
+    big = torch.zeros((2048, 4096), device="cuda")      # 16 m n = 128 MiB of residual copies > scratch
     big[0, 0] = 1.0
     with pytest.raises(ext.ExterndError) as e:
         ext.factor_noalloc(big, 1.0, 0.7)
