@@ -237,13 +237,30 @@ def run_ours(args):
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
 
-    w, mats = _workload_arrays(args.workload, rank, args.mu)
+    from ternary_rank_weight_b200 import dist
+
+    strong = args.scaling == "strong"
+    plan = {"grid": args.grid, "cluster": args.cluster}
+    if strong:
+        # one fixed batch split over the ranks: every rank takes a contiguous slice of the SAME
+        # matrices and runs it with the plan of the whole batch on one GPU, so each matrix gets
+        # the bits a single-GPU batched call gives
+        w_full, mats_full = _workload_arrays(args.workload, 0, args.mu)
+        if w_full.count < 2:
+            raise SystemExit("--scaling strong needs a batched workload")
+        _, pst = ext.factor_batched([torch.from_numpy(a) for a in mats_full], list(w_full.mu), list(w_full.tau),
+                                    iters=w_full.iters, seeds=list(w_full.seeds), sweeps=w_full.sweeps,
+                                    hs=[w_full.weights(b) for b in range(w_full.count)] if w_full.weighted else None,
+                                    grid=args.grid, cluster=args.cluster, plan_only=True)
+        plan = {"grid": pst["group"], "cluster": pst["cluster"]}
+        w, idx = dist.slice_workload(w_full, ws, rank)
+        mats = [mats_full[i] for i in idx]
+    else:
+        w, mats = _workload_arrays(args.workload, rank, args.mu)
     As = [torch.from_numpy(a).to(dev) for a in mats]
     host_As = [torch.from_numpy(a).pin_memory() for a in mats]
     k_total = sum(ext.rank(a.shape[0], a.shape[1], mu) for a, mu in zip(mats, w.mu))
     stream = torch.cuda.current_stream(dev)
-
-    from ternary_rank_weight_b200 import dist
 
     hw = [torch.from_numpy(w.weights(b)).to(dev) for b in range(w.count)] if w.weighted else None
 
@@ -251,16 +268,23 @@ def run_ours(args):
     fits = k_total * (1 + w.sweeps)
 
     def step(inputs):
+        if strong:
+            res, st = ext.factor_batched(inputs, w.mu, w.tau, iters=w.iters, seeds=list(w.seeds), hs=hw,
+                                         lams=[w.lam] * w.count if w.weighted else None, sweeps=w.sweeps,
+                                         grid=plan["grid"], cluster=plan["cluster"])
+            assert all(x == 0 for x in st), st
+            return res, res[0].stats
         if w.weighted and not w.sweeps and w.count == 1:
             f = ext.factor_weighted(inputs[0], hw[0], w.mu[0], w.tau[0], lam=w.lam, iters=w.iters, seed=w.seeds[0])
             return [f], f.stats
         if w.count == 1:
             f = ext.factor(inputs[0], w.mu[0], w.tau[0], iters=w.iters, seed=w.seeds[0],
                            grid=args.grid, pending=args.pending, sweeps=w.sweeps,
-                           h=hw[0] if w.weighted else None, lam=w.lam)
+                           h=hw[0] if w.weighted else None, lam=w.lam, cluster=args.cluster)
             return [f], f.stats
         res, st = ext.factor_batched(inputs, w.mu, w.tau, iters=w.iters, seeds=list(w.seeds), hs=hw,
-                                     lams=[w.lam] * w.count if w.weighted else None, sweeps=w.sweeps)
+                                     lams=[w.lam] * w.count if w.weighted else None, sweeps=w.sweeps,
+                                     grid=args.grid, cluster=args.cluster)
         assert all(s == 0 for s in st), st
         return res, res[0].stats
 
@@ -324,15 +348,22 @@ def run_ours(args):
         e = res[0].energy.cpu()
         m0, n0 = w.shapes[0]
         energy_curve = {str(mu): float(e[ext.rank(m0, n0, mu) - 1].item()) for mu in w.mu_sweep}
+    kernel = "externd::als2_kernel (clusters of %d)" % st["cluster"] if st.get("cluster", 1) > 1 else "externd::als_kernel"
+    parallelism = (f"batch split over {ws} GPUs (contiguous slices, plan of the whole batch: {plan['grid']} CTAs per "
+                   f"matrix, clusters of {plan['cluster']})" if strong
+                   else f"replicas x{ws} (independent matrices per rank)")
     out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
-           "warmup": args.warmup, "ms_per_step": t_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+           "warmup": args.warmup, "ms_per_step": t_ms / args.steps, "higher_is_better": True,
+           "scaling": "strong" if strong else "weak",
            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-           "config": _config(w, {"k": k_total, "sweeps": w.sweeps, "grid": st["grid"], "group": st["group"], "block": st["block"],
-                                 "pending": st["pending"], "vec": [st["vec_v"], st["vec_u"]],
-                                 "parallelism": f"replicas x{ws} (independent matrices per rank)"}),
+           "config": _config(w_full if strong else w,
+                             {"k": k_total, "sweeps": w.sweeps, "grid": st["grid"], "group": st["group"],
+                              "block": st["block"], "cluster": st.get("cluster", 1),
+                              "pending": st["pending"], "vec": [st["vec_v"], st["vec_u"]],
+                              "parallelism": parallelism}),
            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                         "frac": achieved / peak, "traffic": traffic,
-                        "kernel": "externd::als_kernel", "peak_kind": f"{peak_kind} copy bandwidth",
+                        "kernel": kernel, "peak_kind": f"{peak_kind} copy bandwidth",
                         "alg_bytes_per_launch": mean_bytes, "kernel_ms": mean_als,
                         "bytes_read_per_launch": statistics.mean(read_bytes),
                         "note": "alg bytes: direct-evaluation count per component; the kernel reads only "
@@ -342,8 +373,8 @@ def run_ours(args):
            "clocks": clocks,
            "energy": energy_final,
            "energy_vs_mu": energy_curve,
-           "components_per_step": ws * k_total,
-           "fits_per_step": ws * fits,
+           "components_per_step": dist.sum_over_ranks(k_total, dev),
+           "fits_per_step": dist.sum_over_ranks(fits, dev),
            "wall_s_per_matrix": (t_ms / 1000.0) / args.steps / w.count}
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = time_oracle(w, mats, budget_s=args.ref_budget)
@@ -441,6 +472,10 @@ def main():
     ap.add_argument("--workload", default=HEADLINE, choices=sorted(WORKLOADS))
     ap.add_argument("--all", action="store_true", help="one line per workload (reporting, not the driver's line)")
     ap.add_argument("--grid", type=int, default=0)
+    ap.add_argument("--cluster", type=int, default=0,
+                    help="ALS kernel: 0 automatic, 1 one CTA per stripe, 2/4/8/16 clustered with that cluster size")
+    ap.add_argument("--scaling", choices=("weak", "strong"), default="weak",
+                    help="N > 1: weak = each rank its own matrices; strong = one batch split over the ranks")
     ap.add_argument("--pending", type=int, default=0)
     ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of oracle work per sample")
     ap.add_argument("--mu", type=float, default=None, help="override mu (short runs for profiling)")

@@ -155,12 +155,23 @@ int externd_factor_batched(int count, const float* const* A, const int64_t* m, c
  *   lambda    with h: `count` values of lambda (finite, >= 0); NULL means 0 for every matrix.
  *   sweeps    refinement sweeps after extraction for every matrix (§2.4, see externd_options),
  *             0 .. 1000.
- *   sweep_energy_out  NULL, or `count` pointers (entries may be NULL) to `sweeps` doubles each. */
+ *   sweep_energy_out  NULL, or `count` pointers (entries may be NULL) to `sweeps` doubles each.
+ *   grid      CTAs per matrix (0: automatic), as externd_options.grid.
+ *   cluster   kernel choice, as externd_options.cluster.  A matrix gets the same bits from
+ *             any launch with the same grid and cluster size -- e.g. one slice of a batch per
+ *             GPU, run with the plan of the whole batch.
+ *   plan_only nonzero: validate the arguments, choose the launch (CTAs per matrix, cluster
+ *             size, lazy-deflation depth) exactly as the call would, record it for
+ *             externd_last_stats (grid, group, cluster, pending, smem_bytes) and return
+ *             without device work. */
 typedef struct {
     const float* const* h;
     const double* lambda;
     int sweeps;
     double* const* sweep_energy_out;
+    int grid;
+    int cluster;
+    int plan_only;
 } externd_batch_options;
 
 /* externd_factor_batched with per-matrix extensions (opt may be NULL: the plain call). */
@@ -304,6 +315,12 @@ typedef struct {
     double* trace_pre_u;
     double* trace_thr_u;
     uint8_t* trace_trit_u;
+    /* Kernel choice: 0 = automatic (currently the one-CTA-per-stripe kernel); 1 = one CTA per
+     * residual stripe (the kernel that also runs refinement sweeps); 2, 4, 8 or 16 = the
+     * clustered kernel with clusters of that many CTAs, for factorizations without sweeps
+     * (EXTERND_ELAUNCH if they cannot all be resident, EXTERND_EINVAL for other values).
+     * Results depend on the partition: the same grid and cluster size give the same bits. */
+    int cluster;
 } externd_options;
 
 /* externd_factor with options (opt may be NULL). */
@@ -342,6 +359,8 @@ typedef struct {
     int64_t safeguard_hits;    /* extraction components whose ALS decrease p^2 / (nnz(u) nnz(v)) fell below the
                                   single-entry bound ||R||^2 / (m n) of §7 ("Monotone residual decrease and
                                   convergence"), summed over matrices; counted only, no component is replaced */
+    int cluster;               /* CTAs per cluster of the ALS launch (1: the one-CTA-per-stripe kernel) */
+    int reserved;
 } externd_stats;
 
 int externd_last_stats(externd_stats* out);

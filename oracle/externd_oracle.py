@@ -27,6 +27,13 @@ arXiv 2607.13511), cited below by section and display equation:
   stored pair with its own least-squares scale (otherwise the stored pair stays,
   rescaled), which makes every visit non-increasing in the residual, as the
   pages report the sweeps to be.
+* §2.4 "Batched block ALS": blocks of b components (default 256, capped at
+  floor(min(m, n)/8)); V <- T_tau([(U^T U + eps I)^-1 U^T R]^T),
+  U <- T_tau(R V (V^T V + eps I)^-1) column-wise, then the scales solve
+  [(U^T U) o (V^T V)] d = diag(U^T R V) and R <- R - U diag(d) V^T.  Readings: eps
+  (unspecified) = 1e-6 x the Gram matrix's mean diagonal; the start block holds the
+  sequential method's start vectors of its components; the alternation runs `iters`
+  times like the sequential fit.
 * §2.6 Cost model: inference computes y = B (diag(D) (C x)); mask+sign packing
   stores one zero/nonzero mask bit per element plus one sign bit per nonzero,
   and Eq. (1): bpw_eff = mu (m + n) / max(m, n) * (2 - sparsity).
@@ -291,6 +298,90 @@ def greedy_als(A: np.ndarray, k: int, tau: float, iters: int = 15, seed: int = 0
     e_final = 1.0 - float(np.sum(R * R)) / norm_a2
     return Factorization(B=B, C=C, D=D, energy=energy, energy_final=e_final, norm_a2=norm_a2,
                          margins=margins, safeguard_hits=hits, residual_norms=res)
+
+
+# ----------------------------------------------------------------------------
+# §2.4 batched block ALS with decorrelated targets
+# ----------------------------------------------------------------------------
+
+BLOCK_EPS_REL = 1e-6   # reading: the ridge epsilon, unspecified on the pages, is 1e-6 x the mean
+                       # diagonal of the Gram matrix it regularizes (nnz of the block's vectors)
+
+
+def block_width(m: int, n: int, b: int = 256) -> int:
+    """§2.4: blocks of b components (default 256), capped at floor(min(m, n) / 8), at least 1."""
+    return max(1, min(int(b), min(m, n) // 8))
+
+
+def ternarize_columns(X: np.ndarray, tau: float) -> np.ndarray:
+    """T_tau of §2.2 applied to every column of X on its own (mean and fallback per column)."""
+    X = np.asarray(X, dtype=np.float64)
+    out = np.zeros(X.shape, dtype=np.int8)
+    for j in range(X.shape[1]):
+        out[:, j], _, _ = ternarize(X[:, j], tau)
+    return out
+
+
+def _ridge(G: np.ndarray) -> np.ndarray:
+    eps = BLOCK_EPS_REL * float(np.mean(np.diag(G)))
+    return G + eps * np.eye(G.shape[0])
+
+
+def block_scales(R: np.ndarray, U: np.ndarray, V: np.ndarray) -> np.ndarray:
+    """§2.4 joint scale solve: [(U^T U) o (V^T V)] d = diag(U^T R V) (the least-squares scales
+    of the block for fixed trits).  A singular system (repeated components) takes the
+    minimum-norm solution (reading: the pages say "solved jointly and exactly")."""
+    U = np.asarray(U, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    H = (U.T @ U) * (V.T @ V)
+    rhs = np.einsum("rj,rc,cj->j", U, np.asarray(R, dtype=np.float64), V)
+    d, *_ = np.linalg.lstsq(H, rhs, rcond=None)
+    return d
+
+
+def block_fit(R: np.ndarray, U0: np.ndarray, tau: float, iters: int):
+    """§2.4 block fit from start trits U0 (m x b): `iters` times
+    V <- T_tau([(U^T U + eps I)^-1 U^T R]^T), U <- T_tau(R V (V^T V + eps I)^-1), column-wise,
+    then the joint scales.  Returns (U int8 m x b, V int8 n x b, d)."""
+    R = np.asarray(R, dtype=np.float64)
+    U = np.asarray(U0, dtype=np.float64)
+    V = None
+    for _ in range(iters):
+        Gu = U.T @ U
+        V = ternarize_columns(np.linalg.solve(_ridge(Gu), U.T @ R).T, tau).astype(np.float64)
+        Gv = V.T @ V
+        U = ternarize_columns(np.linalg.solve(_ridge(Gv), (R @ V).T).T, tau).astype(np.float64)
+    d = block_scales(R, U, V)
+    return U.astype(np.int8), V.astype(np.int8), d
+
+
+def block_als(A: np.ndarray, k: int, tau: float, iters: int = 15, seed: int = 0, b: int | None = None) -> Factorization:
+    """§2.4 batched block ALS: components in blocks of b (the last one shorter), each block
+    fitted by block_fit from the start vectors of its components (those of greedy_als, so
+    that b = 1 is the sequential method), then R <- R - U diag(d) V^T; deflation across
+    blocks is sequential.  energy[i] is the energy after the block holding component i."""
+    R = np.array(A, dtype=np.float64, copy=True)
+    m, n = R.shape
+    norm_a2 = float(np.sum(R * R))
+    if norm_a2 == 0.0:
+        raise ValueError("||A||_F = 0: energy is undefined")
+    bw = block_width(m, n) if b is None else int(b)
+    B = np.zeros((m, k), dtype=np.int8)
+    C = np.zeros((k, n), dtype=np.int8)
+    D = np.zeros(k, dtype=np.float64)
+    energy = np.zeros(k, dtype=np.float64)
+    for s0 in range(0, k, bw):
+        nb = min(bw, k - s0)
+        U0 = np.stack([ternarize(start_normals(seed, s0 + j, m), tau)[0] for j in range(nb)], axis=1)
+        U, V, d = block_fit(R, U0, tau, iters)
+        R -= (U.astype(np.float64) * d) @ V.astype(np.float64).T
+        B[:, s0:s0 + nb] = U
+        C[s0:s0 + nb, :] = V.T
+        D[s0:s0 + nb] = d
+        energy[s0:s0 + nb] = 1.0 - float(np.sum(R * R)) / norm_a2
+    e_final = 1.0 - float(np.sum(R * R)) / norm_a2
+    return Factorization(B=B, C=C, D=D, energy=energy, energy_final=e_final, norm_a2=norm_a2,
+                         margins=np.full(k, np.inf), safeguard_hits=0, residual_norms=None)
 
 
 def residual_after(A: np.ndarray, B: np.ndarray, D: np.ndarray, C: np.ndarray, upto: int) -> np.ndarray:

@@ -53,6 +53,7 @@ class Options(ctypes.Structure):
         ("trace_pre_u", ctypes.c_void_p),
         ("trace_thr_u", ctypes.c_void_p),
         ("trace_trit_u", ctypes.c_void_p),
+        ("cluster", ctypes.c_int),
     ]
 
 
@@ -62,6 +63,9 @@ class BatchOptions(ctypes.Structure):
         ("lambda_", ctypes.c_void_p),
         ("sweeps", ctypes.c_int),
         ("sweep_energy_out", ctypes.c_void_p),
+        ("grid", ctypes.c_int),
+        ("cluster", ctypes.c_int),
+        ("plan_only", ctypes.c_int),
     ]
 
 
@@ -89,6 +93,8 @@ class Stats(ctypes.Structure):
         ("sweep_kept", ctypes.c_int64),
         ("phase_cycles", ctypes.c_int64 * 11),
         ("safeguard_hits", ctypes.c_int64),
+        ("cluster", ctypes.c_int),
+        ("reserved", ctypes.c_int),
     ]
 
     def as_dict(self):

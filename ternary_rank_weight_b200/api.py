@@ -154,7 +154,7 @@ class Trace:
 
 def factor(A, mu: float, tau: float, iters: int = 15, seed: int = 0, *, grid: int = 0, pending: int = 0,
            wait_limit_s: float = 0.0, fault_skip_cta: Optional[int] = None, want_d64: bool = False,
-           want_energy: bool = True, sweeps: int = 0, h=None, lam: float = 0.0, trace=None,
+           want_energy: bool = True, sweeps: int = 0, h=None, lam: float = 0.0, trace=None, cluster: int = 0,
            stream=None) -> Factors:
     """Factor one matrix (externd_factor_ex).  Outputs are allocated where A lives.
 
@@ -163,7 +163,8 @@ def factor(A, mu: float, tau: float, iters: int = 15, seed: int = 0, *, grid: in
     weights (per-column second moments, n float32 values), or None for the plain objective.
     trace: (first, count) -- test hook, records the half-steps of those visits: visit
     i < k extracts component i, visit (s + 1) k + i is sweep s's refit of component i
-    (``Factors.trace``; A must be on the GPU)."""
+    (``Factors.trace``; A must be on the GPU).  cluster: kernel choice (0 automatic, 1 one
+    CTA per residual stripe, 2/4/8/16 the clustered kernel with that cluster size)."""
     A = _as_matrix(A)
     m, n = A.shape
     if h is not None:
@@ -188,6 +189,7 @@ def factor(A, mu: float, tau: float, iters: int = 15, seed: int = 0, *, grid: in
     opt.sweep_energy_out = _ptr(SE)
     opt.h = _ptr(h)
     opt.lambda_ = float(lam)
+    opt.cluster = int(cluster)
     tr = None
     if trace is not None:
         if not A.is_cuda:
@@ -274,11 +276,13 @@ NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 def factor_batched(As: Sequence, mus: Sequence[float], taus: Sequence[float], iters: int = 15,
                    seeds: Optional[Sequence[int]] = None, *, hs: Optional[Sequence] = None,
-                   lams: Optional[Sequence[float]] = None, sweeps: int = 0, stream=None):
+                   lams: Optional[Sequence[float]] = None, sweeps: int = 0, grid: int = 0, cluster: int = 0,
+                   plan_only: bool = False, stream=None):
     """Factor independent matrices in one launch (externd_factor_batched_ex).
 
     hs: per-matrix importance weights (§2.5; every matrix or none), lams their lambdas;
-    sweeps: refinement sweeps (§2.4) for every matrix.
+    sweeps: refinement sweeps (§2.4) for every matrix; grid, cluster: the launch (0:
+    automatic).  plan_only: return (None, stats of the plan) without device work.
     Returns (list of Factors, list of per-matrix status codes)."""
     mats = [_as_matrix(a) for a in As]
     cnt = len(mats)
@@ -317,6 +321,9 @@ def factor_batched(As: Sequence, mus: Sequence[float], taus: Sequence[float], it
             opt.lambda_ = ctypes.cast(larr, ctypes.c_void_p)
     SEs = [_empty((int(sweeps),), torch.float64, A) if sweeps > 0 else None for A in mats]
     opt.sweeps = int(sweeps)
+    opt.grid = int(grid)
+    opt.cluster = int(cluster)
+    opt.plan_only = 1 if plan_only else 0
     if sweeps > 0:
         sarr = P(*[_ptr(x) for x in SEs])
         keep.append(sarr)
@@ -326,6 +333,9 @@ def factor_batched(As: Sequence, mus: Sequence[float], taus: Sequence[float], it
                                                    b_ptrs, d_ptrs, c_ptrs, e_ptrs, st,
                                                    _stream(stream, mats[0].device), ctypes.byref(opt))
     stats = last_stats()
+    if plan_only:
+        _check(rc, "externd_factor_batched_ex")
+        return None, stats
     res = []
     for A, mu, tau, o, se in zip(mats, mus, taus, outs, SEs):
         res.append(Factors(B=o[0], D=o[1], C=o[2], energy=o[3], m=A.shape[0], n=A.shape[1], k=o[4],

@@ -4,6 +4,7 @@
 // §2.1 (factorization, energy), §2.2 (T_tau), §2.3 (greedy sequential ALS).
 // The data layout and the synchronisation scheme are described at the top of
 // externd_kernels.cuh.
+#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 
 #include <climits>
@@ -1088,18 +1089,18 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
 // two buffers of Gg words and carry different tags, so a CTA that is already in call
 // j + 1 cannot overwrite a word another CTA still waits for in call j.  Every
 // exchange also orders: a CTA leaves it only after every CTA has entered it.
-__device__ bool exchange_sum(unsigned long long* sums, int q, int Gg, double v, const Smem& s, GroupSync* gs,
+__device__ bool exchange_sum(unsigned long long* sums, int q, int Gg, double v, double* red, GroupSync* gs,
                              uint64_t limit_ns, int* status, bool skip, unsigned use, double& out) {
     const unsigned tag = gen_tag(use);
     unsigned long long* buf = sums + (size_t)(use & 1u) * Gg;
-    const double t = block_sum(v, s.red);
+    const double t = block_sum(v, red);
     if (threadIdx.x == 0 && !skip) st_relaxed_u64(buf + q, tag_value(t, tag));
     int ok = 1;
     double x = 0.0;
     if ((int)threadIdx.x < Gg) x = untag(wait_tagged(buf + threadIdx.x, tag, gs, limit_ns, status, ok));
     ok = __syncthreads_and(ok);
     if (!ok) return false;
-    out = block_sum(x, s.red);
+    out = block_sum(x, red);
     return true;
 }
 
@@ -1153,7 +1154,7 @@ __device__ __forceinline__ int refine_begin(const Prob& P, int64_t i, int q, int
     // with k = 1 one more exchange orders it), read through L2
     if (kk == 1) {
         double unused;
-        if (!exchange_sum(P.sums, q, Gg, 0.0, s, gs, cfg.limit_ns, P.status, skip, sum_use, unused))
+        if (!exchange_sum(P.sums, q, Gg, 0.0, s.red, gs, cfg.limit_ns, P.status, skip, sum_use, unused))
             return -1;
     }
     __threadfence();
@@ -1408,7 +1409,7 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
             const double di = s.scal[8], n_old = s.scal[9];
             const int La = (int)s.scal[11];
             double pold = 0.0;
-            if (!exchange_sum(P.sums, q, Gg, tid == 0 ? s.scal[10] : 0.0, s, gs, cfg.limit_ns, P.status, skip,
+            if (!exchange_sum(P.sums, q, Gg, tid == 0 ? s.scal[10] : 0.0, s.red, gs, cfg.limit_ns, P.status, skip,
                               sum_use_end(vis - kk, kk),
                               pold))
                 return false;
@@ -1481,7 +1482,7 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
     double R2 = 0.0;
     // the final sum follows the refinement visits' calls
     const unsigned last_use = (nvis > kk) ? sum_use_end(nvis - kk - 1, kk) : 0u;
-    if (!exchange_sum(P.sums, q, Gg, rs, s, gs, cfg.limit_ns, P.status, skip, last_use + 1u, R2)) return false;
+    if (!exchange_sum(P.sums, q, Gg, rs, s.red, gs, cfg.limit_ns, P.status, skip, last_use + 1u, R2)) return false;
     if (lead && tid == 0) {
         P.stats->sum_nu = sum_nu;
         P.stats->sum_nv = sum_nv;
@@ -1562,8 +1563,18 @@ __global__ void __launch_bounds__(NT, 1) als_kernel(const KCfg cfg) {
     }
 }
 
+}  // namespace externd
+
+#include "als_cluster.cuh"
+
+namespace externd {
+
 // Writes one problem descriptor and its running status into a caller-fixed workspace.
 // The four instantiations: importance weights (§2.5) x refinement sweeps (§2.4).
+static const void* als2_fn(int weighted) {
+    return weighted ? (const void*)als2_kernel<true> : (const void*)als2_kernel<false>;
+}
+
 static const void* als_fn(int weighted, int sweeping) {
     if (weighted) return sweeping ? (const void*)als_kernel<true, true> : (const void*)als_kernel<true, false>;
     return sweeping ? (const void*)als_kernel<false, true> : (const void*)als_kernel<false, false>;
@@ -1671,6 +1682,13 @@ int dev_info(DevInfo& out) {
             for (int sw = 0; sw < 2; ++sw)
                 attr_ok = attr_ok && cudaFuncSetAttribute(als_fn(w, sw), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                           (int)d.smem_optin) == cudaSuccess;
+        for (int w = 0; w < 2; ++w) {
+            attr_ok = attr_ok && cudaFuncSetAttribute(als2_fn(w), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                      (int)d.smem_optin) == cudaSuccess;
+            // clusters of 16 CTAs need the non-portable size
+            if (cudaFuncSetAttribute(als2_fn(w), cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+                cudaGetLastError();
+        }
         if (!attr_ok) {
             cudaGetLastError();
             return EXTERND_ECUDA;
@@ -1770,7 +1788,96 @@ struct RunOpts {
     double wait_limit_s = 2.0;
     int fault_skip = -1;
     bool init_only = false;
+    bool plan_only = false;   // fill the stats with the launch plan and return (no device work)
+    int cluster = 0;          // 0: automatic; 1: the one-CTA-per-stripe kernel; 2, 4, 8, 16: clusters of that size
 };
+
+// Plan of the clustered kernel for one launch (see als_cluster.cuh).
+struct Plan2 {
+    bool ok = false;
+    int c = 0, Gg = 0, Lcap = 0, ncl = 0;
+    size_t smem = 0;
+    int qr_max = 1, qc_max = 1, sv_max = 1, su_max = 1, wpm = 1;
+    std::vector<Grid2> g;
+    std::vector<int64_t> bsv, bsu;
+};
+
+// Try clusters of size c for groups of G CTAs (a multiple of c).  pl.ncl reports how many
+// such clusters can be resident at once.
+Plan2 plan_cluster(const ProbIn* in, int np, int NG, int G, int c, int Lreq, int weighted, const DevInfo& di) {
+    Plan2 pl;
+    if (G < c || G % c != 0 || G > NT) return pl;
+    const int NC = G / c;
+    int64_t m_max = 1, n_max = 1;
+    pl.g.resize(np);
+    pl.bsv.resize(np);
+    pl.bsu.resize(np);
+    for (int b = 0; b < np; ++b) {
+        Grid2& g = pl.g[b];
+        g.m = in[b].m;
+        g.n = in[b].n;
+        g.c = c;
+        g.NC = NC;
+        g.vecv = 4;   // the clustered kernel reads its blocks in 16-byte vectors
+        g.vecu = 4;
+        m_max = in[b].m > m_max ? in[b].m : m_max;
+        n_max = in[b].n > n_max ? in[b].n : n_max;
+        const Part QR = g.qr(), QC = g.qc();
+        int64_t bsv = 1, bsu = 1;
+        for (int r = 0; r < c; ++r) {
+            pl.qr_max = (int)std::max<int64_t>(pl.qr_max, QR.end(r) - QR.start(r));
+            pl.qc_max = (int)std::max<int64_t>(pl.qc_max, QC.end(r) - QC.start(r));
+            for (int q = 0; q < NC; ++q) {
+                pl.wpm = std::max(pl.wpm, std::max(g.pcol(r).pitch(q), g.prow(r).pitch(q)));
+            }
+        }
+        for (int q = 0; q < NC; ++q) {
+            const int pv = g.pitchV(q), pu = g.pitchU(q);
+            pl.sv_max = std::max(pl.sv_max, pv);
+            pl.su_max = std::max(pl.su_max, pu);
+            for (int r = 0; r < c; ++r) {
+                bsv = std::max<int64_t>(bsv, (QR.end(r) - QR.start(r)) * (int64_t)pv);
+                bsu = std::max<int64_t>(bsu, (QC.end(r) - QC.start(r)) * (int64_t)pu);
+            }
+        }
+        // list entries hold element offsets below 2^30
+        if ((double)bsv >= 1073741824.0 || (double)bsu >= 1073741824.0) return pl;
+        pl.bsv[b] = (bsv + 63) / 64 * 64;
+        pl.bsu[b] = (bsu + 63) / 64 * 64;
+    }
+    int L = MAX_PENDING;
+    auto smem_of = [&](int Lc) {
+        return SmemLayout2(m_max, n_max, pl.qr_max, pl.qc_max, pl.sv_max, pl.su_max, pl.wpm, pl.wpm, c, Lc, weighted).total;
+    };
+    while (L > 1 && smem_of(L) > di.smem_optin) --L;
+    if (Lreq > 0 && Lreq < L) L = Lreq;
+    if (smem_of(L) > di.smem_optin) return pl;
+    pl.smem = smem_of(L);
+    // every cluster of the launch must be resident at once
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(NG * G));
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = pl.smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)c;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int ncl = 0;
+    if (cudaOccupancyMaxActiveClusters(&ncl, als2_fn(weighted), &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return pl;
+    }
+    pl.ncl = ncl;
+    if ((int64_t)ncl < (int64_t)NG * NC) return pl;
+    pl.ok = true;
+    pl.c = c;
+    pl.Gg = G;
+    pl.Lcap = L;
+    return pl;
+}
 
 struct Buf {  // device staging for a possibly-host pointer
     void* host = nullptr;
@@ -1858,7 +1965,7 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
         if (in[b].mode == MODE_FACTOR && in[b].sweeps > 0 && Lcap < 2) return EXTERND_ELIMIT;   // add-back + refit
         if (in[b].n_pend > 0 && in[b].n_pend + 1 > Lcap) return EXTERND_ELIMIT;   // caller's terms + the component
     }
-    const size_t smem = als_smem_bytes(m_max, n_max, Lcap, pv_max, pu_max, weighted);
+    size_t smem = als_smem_bytes(m_max, n_max, Lcap, pv_max, pu_max, weighted);
     if (smem > di.smem_optin) return EXTERND_ELIMIT;
 
     int nb = 0;
@@ -1869,6 +1976,59 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
         return EXTERND_ECUDA;
     }
     if ((int64_t)nb * sms < (int64_t)NG * Gg) return EXTERND_ELAUNCH;
+
+    // ---- the clustered kernel (factorizations without refinement sweeps), where its
+    //      clusters can all be resident; the largest cluster size that keeps at least 85 %
+    //      of the CTAs asked for (small matrices: a group of up to 16 CTAs, one word of
+    //      32 indices per quarter at least)
+    Plan2 pl;
+    if (!opt.init_only && opt.cluster > 1 && !sweeping) {
+        bool all_factor = true;
+        int64_t mn_min = INT64_MAX;
+        for (int b = 0; b < np; ++b) {
+            all_factor = all_factor && in[b].mode == MODE_FACTOR;
+            mn_min = std::min<int64_t>(mn_min, std::min(in[b].m, in[b].n));
+        }
+        if (all_factor) {
+            int Gt = Gg;
+            if (opt.grid <= 0 && Gt < 16) {
+                const int64_t want = std::min<int64_t>(16, std::max<int64_t>(2, (mn_min + 31) / 32));
+                if ((int64_t)NG * want <= sms) Gt = (int)want;
+            }
+            for (int c : {16, 8, 4, 2}) {
+                if (opt.cluster > 1 && c != opt.cluster) continue;
+                if (c > Gt) continue;
+                Plan2 t = plan_cluster(in, np, NG, (Gt / c) * c, c, opt.pending, weighted, di);
+                if (!t.ok && opt.grid <= 0 && t.ncl >= NG) {   // fewer clusters per matrix, as many as fit
+                    const int G1 = (t.ncl / NG) * c;
+                    if (G1 >= c && G1 < (Gt / c) * c) t = plan_cluster(in, np, NG, G1, c, opt.pending, weighted, di);
+                }
+                if (t.ok && (opt.cluster > 1 || opt.grid > 0 || t.Gg * 100 >= Gt * 85)) {
+                    pl = t;
+                    break;
+                }
+            }
+            if (opt.cluster > 1 && !pl.ok) return EXTERND_ELAUNCH;   // the size asked for does not fit
+        }
+    }
+    const bool clustered = pl.ok;
+    if (clustered) {
+        Gg = pl.Gg;
+        Lcap = pl.Lcap;
+        smem = pl.smem;
+    }
+
+    if (opt.plan_only) {
+        st.grid = NG * Gg;
+        st.group = Gg;
+        st.block = NT;
+        st.pending = Lcap;
+        st.cluster = clustered ? pl.c : 1;
+        st.smem_bytes = smem;
+        g_last = st;
+        for (int b = 0; b < np; ++b) statuses[b] = EXTERND_OK;
+        return EXTERND_OK;
+    }
 
     // ---- plan the workspace
     std::vector<Prob> probs(np);
@@ -1909,11 +2069,18 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
         P.tr_pre_v = I.tr_pre_v; P.tr_thr_v = I.tr_thr_v; P.tr_trit_v = I.tr_trit_v;
         P.tr_pre_u = I.tr_pre_u; P.tr_thr_u = I.tr_thr_u; P.tr_trit_u = I.tr_trit_u;
         P.n_norm_part = ((I.m + 31) / 32) * ((I.n + 31) / 32);
-        off_rv[b] = ws; ws += round_up(sizeof(float) * (size_t)P.pv.total(I.m), 256);
-        off_ru[b] = ws; ws += round_up(sizeof(float) * (size_t)P.pu.total(I.n), 256);
+        if (clustered) {
+            P.g2 = pl.g[b];
+            P.bsv = pl.bsv[b];
+            P.bsu = pl.bsu[b];
+        }
+        const size_t rv_elems = clustered ? (size_t)Gg * (size_t)pl.bsv[b] : (size_t)P.pv.total(I.m);
+        const size_t ru_elems = clustered ? (size_t)Gg * (size_t)pl.bsu[b] : (size_t)P.pu.total(I.n);
+        off_rv[b] = ws; ws += round_up(sizeof(float) * rv_elems, 256);
+        off_ru[b] = ws; ws += round_up(sizeof(float) * ru_elems, 256);
         // low halves of the residual (zero until the first fold)
-        off_rvl[b] = ws; ws += round_up(sizeof(float) * (size_t)P.pv.total(I.m), 256);
-        off_rul[b] = ws; ws += round_up(sizeof(float) * (size_t)P.pu.total(I.n), 256);
+        off_rvl[b] = ws; ws += round_up(sizeof(float) * rv_elems, 256);
+        off_rul[b] = ws; ws += round_up(sizeof(float) * ru_elems, 256);
         // exchange buffers: zero = "no half-step yet" (tags are 1..255)
         off_x[b] = ws; ws += round_up(sizeof(unsigned long long) * (size_t)I.n, 256);
         off_y[b] = ws; ws += round_up(sizeof(unsigned long long) * (size_t)I.m, 256);
@@ -2067,7 +2234,10 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
             kmax = in[b].k > kmax ? in[b].k : kmax;
         }
         if (!opt.init_only) {
-            setup_kernel<<<dim3((unsigned)tx, (unsigned)ty, (unsigned)np), dim3(32, 8), 0, stream>>>(dprobs);
+            if (clustered)
+                setup2_kernel<<<dim3((unsigned)tx, (unsigned)ty, (unsigned)np), dim3(32, 8), 0, stream>>>(dprobs);
+            else
+                setup_kernel<<<dim3((unsigned)tx, (unsigned)ty, (unsigned)np), dim3(32, 8), 0, stream>>>(dprobs);
             CK(cudaGetLastError());
             ++launches;
         }
@@ -2097,8 +2267,33 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
             cfg.limit_ns = (uint64_t)(lim * 1e9);
             cfg.fault_skip = opt.fault_skip;
             cfg.weighted = weighted;
-            void* args[] = {&cfg};
-            CK(cudaLaunchCooperativeKernel(als_fn(weighted, sweeping), dim3((unsigned)(NG * Gg)), dim3(NT), args, smem, stream));
+            if (clustered) {
+                cfg.pv_max = pl.sv_max;
+                cfg.pu_max = pl.su_max;
+                cfg.qr_max = pl.qr_max;
+                cfg.qc_max = pl.qc_max;
+                cfg.wpm = pl.wpm;
+                cudaLaunchConfig_t lc = {};
+                lc.gridDim = dim3((unsigned)(NG * Gg));
+                lc.blockDim = dim3(NT);
+                lc.dynamicSmemBytes = smem;
+                lc.stream = stream;
+                cudaLaunchAttribute attr[2];
+                attr[0].id = cudaLaunchAttributeClusterDimension;
+                attr[0].val.clusterDim.x = (unsigned)pl.c;
+                attr[0].val.clusterDim.y = 1;
+                attr[0].val.clusterDim.z = 1;
+                attr[1].id = cudaLaunchAttributeCooperative;   // all CTAs resident at once
+                attr[1].val.cooperative = 1;
+                lc.attrs = attr;
+                lc.numAttrs = 2;
+                void* args[] = {&cfg};
+                CK(cudaLaunchKernelExC(&lc, als2_fn(weighted), args));
+            } else {
+                void* args[] = {&cfg};
+                CK(cudaLaunchCooperativeKernel(als_fn(weighted, sweeping), dim3((unsigned)(NG * Gg)), dim3(NT), args, smem,
+                                               stream));
+            }
             ++launches;
         }
         if (ev[3]) CK(cudaEventRecord(ev[3], stream));
@@ -2149,6 +2344,7 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
     st.vec_v = probs[0].pv.vec;
     st.vec_u = probs[0].pu.vec;
     st.pending = Lcap;
+    st.cluster = clustered ? pl.c : 1;
     st.smem_bytes = smem;
     st.workspace_bytes = ws;
     for (int b = 0; b < np; ++b) {
@@ -2280,6 +2476,9 @@ int externd_factor_ex(const float* A, int64_t m, int64_t n, double mu, double ta
         ro.pending = opt->pending;
         if (opt->wait_limit_s > 0) ro.wait_limit_s = opt->wait_limit_s;
         ro.fault_skip = opt->fault_inject ? opt->fault_skip_cta : -1;
+        if (opt->cluster < 0 || opt->cluster > 16 || (opt->cluster > 1 && (opt->cluster & (opt->cluster - 1))))
+            return EXTERND_EINVAL;
+        ro.cluster = opt->cluster;
         I.d64 = opt->d64_out;
         if (opt->sweeps < 0 || opt->sweeps > 1000) return EXTERND_EINVAL;
         I.sweeps = opt->sweeps;
@@ -2395,6 +2594,15 @@ int externd_factor_batched_ex(int count, const float* const* A, const int64_t* m
         }
     }
     RunOpts ro;
+    if (opt) {
+        if (opt->grid < 0 || opt->cluster < 0 || opt->cluster > 16 || (opt->cluster > 1 && (opt->cluster & (opt->cluster - 1)))) {
+            for (int c = 0; c < count; ++c) status_out[c] = EXTERND_EINVAL;
+            return EXTERND_EINVAL;
+        }
+        ro.grid = opt->grid;
+        ro.cluster = opt->cluster;
+        ro.plan_only = opt->plan_only != 0;
+    }
     return run(ins.data(), count, ro, reinterpret_cast<cudaStream_t>(stream), status_out);
 }
 

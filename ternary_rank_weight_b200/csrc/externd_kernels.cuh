@@ -88,6 +88,38 @@ struct Part {
     __host__ __device__ int64_t total(int64_t other) const { return other * vec * units; }
 };
 
+// 2-D partition of one matrix.
+struct Grid2 {
+    int64_t m, n;
+    int c, NC, vecv, vecu;
+    __host__ __device__ static Part mk(int64_t len, int G, int vec) {
+        Part p;
+        p.len = len;
+        p.vec = vec;
+        p.G = G;
+        p.units = (len + vec - 1) / vec;
+        return p;
+    }
+    __host__ __device__ Part qr() const { return mk(m, c, 32); }      // row quarters
+    __host__ __device__ Part qc() const { return mk(n, c, 32); }      // column quarters
+    // pieces of column quarter s (V-step outputs) and of row quarter s (U-step outputs)
+    __host__ __device__ Part pcol(int s) const { const Part Q = qc(); return mk(Q.end(s) - Q.start(s), NC, vecv); }
+    __host__ __device__ Part prow(int s) const { const Part Q = qr(); return mk(Q.end(s) - Q.start(s), NC, vecu); }
+    // offset of piece (q, s) inside cluster q's stripe, and the stripe's width
+    __host__ __device__ int soffV(int q, int s) const {
+        int o = 0;
+        for (int t = 0; t < s; ++t) o += pcol(t).pitch(q);
+        return o;
+    }
+    __host__ __device__ int soffU(int q, int s) const {
+        int o = 0;
+        for (int t = 0; t < s; ++t) o += prow(t).pitch(q);
+        return o;
+    }
+    __host__ __device__ int pitchV(int q) const { return soffV(q, c); }
+    __host__ __device__ int pitchU(int q) const { return soffU(q, c); }
+};
+
 constexpr int NCTR = 8;       // arrival counters per group (spread over L2 lines)
 
 struct GroupSync {            // one per CTA group
@@ -165,6 +197,8 @@ struct Prob {
     uint8_t* trit_out;
     Part pv;                  // column stripes (len n)
     Part pu;                  // row stripes (len m)
+    Grid2 g2;                 // clustered kernel: 2-D partition over the group's clusters
+    int64_t bsv, bsu;         // clustered kernel: elements per CTA block of the V- and U-layout
 };
 
 struct KCfg {
@@ -179,6 +213,8 @@ struct KCfg {
     uint64_t limit_ns;
     int fault_skip;           // CTA rank (within group) that never arrives; -1 = off
     int weighted;             // problems carry importance weights (single-matrix launches only)
+    int qr_max, qc_max;       // clustered kernel: longest row / column quarter
+    int wpm;                  // clustered kernel: widest output piece (pitch)
 };
 
 // ---------------------------------------------------------------------------

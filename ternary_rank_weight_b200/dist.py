@@ -7,8 +7,8 @@ timed region and for the max-over-ranks time (NCCL on GPUs, gloo on CPU).
 
 A rank's matrices are the workload's shapes and recipe with seeds offset by
 ``rank * SEED_STRIDE`` (weak scaling: per-rank work is fixed as ranks are
-added); ``partition`` instead splits one fixed batch into contiguous slices
-(strong scaling of a batch).
+added); ``partition`` / ``slice_workload`` instead split one fixed batch into
+contiguous slices (strong scaling of a batch: the total work stays fixed).
 """
 from __future__ import annotations
 
@@ -41,6 +41,15 @@ def rank_seeds(seeds, rank: int):
 def rank_workload(workload, rank: int):
     """The workload a rank factors under weak scaling (same shapes, own seeds)."""
     return replace(workload, seeds=rank_seeds(workload.seeds, rank))
+
+
+def slice_workload(workload, world: int, rank: int):
+    """This rank's contiguous slice of a batch (strong scaling): the same matrices (same seeds)
+    as in the whole batch.  Returns (sliced workload, indices into the batch)."""
+    idx = partition(workload.count, world, rank)
+    pick = lambda t: tuple(t[i] for i in idx)   # noqa: E731
+    return replace(workload, shapes=pick(workload.shapes), seeds=pick(workload.seeds), mu=pick(workload.mu),
+                   tau=pick(workload.tau)), idx
 
 
 def partition(count: int, world: int, rank: int) -> range:

@@ -99,3 +99,47 @@ def test_partition_and_rank_workload_host_logic():
     assert dist.throughput(100, 500.0) == pytest.approx(200.0)
     with pytest.raises(ValueError):
         dist.throughput(1, 0.0)
+
+
+def _strong_worker(rank, world, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world), RANK=str(rank),
+                      LOCAL_RANK=str(rank))
+    from datetime import timedelta
+    tdist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        from oracle import externd_oracle as ora
+        base = Workload("tiny batch", ((24, 40), (32, 16), (20, 20), (16, 48), (40, 24)), (7, 8, 9, 10, 11),
+                        (1.0, 1.5, 1.0, 2.0, 1.0), (0.7, 1.0, 2.0, 0.7, 1.0))
+        w, idx = dist.slice_workload(base, world, rank)
+        energies = []
+        for b in range(w.count):
+            A = w.matrix(b)
+            f = ora.greedy_als(A, k=ora.rank(*A.shape, w.mu[b]), tau=w.tau[b], iters=15, seed=w.seeds[b])
+            energies.append(f.energy_final)
+        units = dist.sum_over_ranks(sum(ora.rank(*sh, mu) for sh, mu in zip(w.shapes, w.mu)))
+        t_max = dist.max_over_ranks(5.0 * (rank + 1))
+        np.save(os.path.join(out_dir, f"strong{rank}.npy"),
+                np.array([idx.start, idx.stop, units, t_max] + energies, dtype=np.float64))
+    finally:
+        tdist.destroy_process_group()
+
+
+def test_two_gloo_ranks_split_one_batch():
+    """Strong scaling of a batch: contiguous slices of the SAME matrices; together the ranks
+    process the whole batch once, and each matrix gets what a single process gets."""
+    import tempfile
+    world = 2
+    with tempfile.TemporaryDirectory() as d:
+        mp.start_processes(_strong_worker, args=(world, _free_port(), d), nprocs=world, start_method="spawn")
+        recs = [np.load(os.path.join(d, f"strong{r}.npy")) for r in range(world)]
+    from oracle import externd_oracle as ora
+    base = Workload("tiny batch", ((24, 40), (32, 16), (20, 20), (16, 48), (40, 24)), (7, 8, 9, 10, 11),
+                    (1.0, 1.5, 1.0, 2.0, 1.0), (0.7, 1.0, 2.0, 0.7, 1.0))
+    assert [(int(r[0]), int(r[1])) for r in recs] == [(0, 2), (2, 5)]
+    total = sum(ora.rank(*sh, mu) for sh, mu in zip(base.shapes, base.mu))
+    assert all(r[2] == total for r in recs) and all(r[3] == 10.0 for r in recs)
+    got = [e for r in recs for e in r[4:]]
+    for b in range(base.count):
+        A = base.matrix(b)
+        f = ora.greedy_als(A, k=ora.rank(*A.shape, base.mu[b]), tau=base.tau[b], iters=15, seed=base.seeds[b])
+        assert got[b] == f.energy_final

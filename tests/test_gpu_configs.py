@@ -68,11 +68,11 @@ def test_batched_attention_workload_full_size():
         e = r.energy.cpu().numpy()
         assert np.all(np.diff(e) >= -1e-12) and 0.5 < e[-1] < 1.0
     for b in (0, 7):
-        f = ext.factor(torch.from_numpy(mats[b]).cuda(), w.mu[b], w.tau[b], seed=w.seeds[b], grid=G)
+        f = ext.factor(torch.from_numpy(mats[b]).cuda(), w.mu[b], w.tau[b], seed=w.seeds[b], grid=G, cluster=res[0].stats["cluster"])
         assert torch.equal(f.B, res[b].B) and torch.equal(f.C, res[b].C) and torch.equal(f.D, res[b].D)
         assert torch.equal(f.energy, res[b].energy)
-    f0 = ext.factor(torch.from_numpy(mats[0]).cuda(), w.mu[0], w.tau[0], seed=w.seeds[0], grid=G, want_d64=True)
-    ndiv = _parity.teacher_forced(mats[0], f0, w.seeds[0], w.tau[0], (0, 1, 1919, 3839), "attn 1536 matrix 0", grid=G)
+    f0 = ext.factor(torch.from_numpy(mats[0]).cuda(), w.mu[0], w.tau[0], seed=w.seeds[0], grid=G, cluster=res[0].stats["cluster"], want_d64=True)
+    ndiv = _parity.teacher_forced(mats[0], f0, w.seeds[0], w.tau[0], (0, 1, 1919, 3839), "attn 1536 matrix 0", grid=G, cluster=res[0].stats["cluster"])
     assert ndiv <= 1
 
 
@@ -91,3 +91,26 @@ def test_llm_4096_prefix_property_and_sampled_parity():
     assert big.stats["residual_energy"] == pytest.approx(e[-1], abs=1e-4)
     ndiv = _parity.teacher_forced(A, big, w.seeds[0], w.tau[0], (0, 4096, 14335), "llm 4096 samples")
     assert ndiv <= 1
+
+
+def test_batch_slices_run_with_the_batch_plan_equal_the_whole_batch():
+    """Strong scaling of a batch over GPUs: each rank runs a contiguous slice of the same matrices
+    with the plan of the whole batch (CTAs per matrix, cluster size), so every matrix gets the
+    bits of the single-GPU batched call.  Checked here on one GPU, slice by slice."""
+    from ternary_rank_weight_b200 import dist
+    w = WORKLOADS["attn_16x1536x1536_mu2.5_tau_cycle"]
+    mats = [torch.from_numpy(w.matrix(b)).cuda() for b in range(w.count)]
+    res, st = ext.factor_batched(mats, list(w.mu), list(w.tau), seeds=list(w.seeds))
+    assert st == [0] * w.count
+    _, plan = ext.factor_batched(mats, list(w.mu), list(w.tau), seeds=list(w.seeds), plan_only=True)
+    G, cl = res[0].stats["group"], res[0].stats["cluster"]
+    assert (plan["group"], plan["cluster"], plan["pending"]) == (G, cl, res[0].stats["pending"])
+    for world in (2, 3):
+        for rank in range(world):
+            ws, idx = dist.slice_workload(w, world, rank)
+            part, st2 = ext.factor_batched([mats[i] for i in idx], list(ws.mu), list(ws.tau), seeds=list(ws.seeds),
+                                           grid=G, cluster=cl)
+            assert st2 == [0] * len(idx)
+            for j, i in enumerate(idx):
+                assert torch.equal(part[j].B, res[i].B) and torch.equal(part[j].C, res[i].C), (world, rank, i)
+                assert torch.equal(part[j].D, res[i].D) and torch.equal(part[j].energy, res[i].energy)

@@ -230,7 +230,7 @@ def test_batched_equals_single_calls_with_the_same_group_size():
     assert st == [0, 0, 0, 0]
     G = res[0].stats["group"]
     for A, mu, tau, sd, r in zip(mats, mus, taus, seeds, res):
-        f = ext.factor(torch.from_numpy(A).cuda(), mu, tau, seed=sd, grid=G)
+        f = ext.factor(torch.from_numpy(A).cuda(), mu, tau, seed=sd, grid=G, cluster=res[0].stats["cluster"])
         assert torch.equal(f.B, r.B) and torch.equal(f.C, r.C) and torch.equal(f.D, r.D)
         assert torch.equal(f.energy, r.energy)
 

@@ -618,3 +618,70 @@ def test_weighted_half_steps_reproduce_the_weighted_factorization():
         _, _, u, _ = ora.half_step_weighted(R, v, 1.0, False, hw)
     assert np.array_equal(u, f.B[:, 0]) and np.array_equal(v, f.C[0])
     assert ora.weighted_ls_scale(R, u, v, hw) == pytest.approx(f.D[0], rel=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# §2.4 batched block ALS with decorrelated targets
+# ---------------------------------------------------------------------------
+
+def test_block_width_default_and_cap():
+    """§2.4: default 256, capped at floor(min(m, n) / 8)."""
+    assert ora.block_width(4096, 4096) == 256
+    assert ora.block_width(1024, 1536) == 128
+    assert ora.block_width(256, 300) == 32
+    assert ora.block_width(7, 5) == 1
+
+
+def test_block_of_one_is_the_sequential_method():
+    """For b = 1 the decorrelated targets are positive multiples of R^T u and R v, and T_tau is
+    scale-invariant, so the block method is the sequential one (§2.4 reduces to §2.3)."""
+    A = llm_matrix(48, 40, seed=3, outliers=2)
+    seq = ora.greedy_als(A, k=24, tau=0.7, seed=1)
+    blk = ora.block_als(A, k=24, tau=0.7, seed=1, b=1)
+    assert np.array_equal(seq.B, blk.B) and np.array_equal(seq.C, blk.C)
+    assert np.allclose(blk.D, seq.D, rtol=1e-12, atol=0)
+
+
+def test_joint_scales_are_the_least_squares_scales():
+    """[(U^T U) o (V^T V)] d = diag(U^T R V) against a generic least-squares solve of
+    min_d ||R - sum_j d_j u_j v_j^T||_F over the vectorized rank-1 terms."""
+    rng = np.random.default_rng(11)
+    for m, n, b in ((6, 5, 3), (9, 7, 4)):
+        R = rng.standard_normal((m, n))
+        U = rng.integers(-1, 2, size=(m, b)).astype(np.int8)
+        V = rng.integers(-1, 2, size=(n, b)).astype(np.int8)
+        U[0, :] = 1            # no empty component
+        V[0, :] = 1
+        M = np.stack([np.outer(U[:, j], V[:, j]).ravel() for j in range(b)], axis=1).astype(np.float64)
+        want, *_ = np.linalg.lstsq(M, R.ravel(), rcond=None)
+        assert np.allclose(ora.block_scales(R, U, V), want, rtol=1e-10, atol=1e-12)
+
+
+def test_decorrelated_targets_avoid_the_collapse_of_naive_batching():
+    """§2.4: ternarizing R^T U column by column makes every column chase the same dominant
+    direction; the decorrelated targets do not.  At b = min(m, n)/8 the naive block fit ends
+    far below the decorrelated one."""
+    A = llm_matrix(256, 256, seed=7)
+    tau, k, b = 0.7, 256, 32
+    blk = ora.block_als(A, k=k, tau=tau, seed=2, b=b)
+    R = A.astype(np.float64)
+    for s0 in range(0, k, b):
+        U = np.stack([ora.ternarize(ora.start_normals(2, s0 + j, 256), tau)[0] for j in range(b)], 1).astype(np.float64)
+        for _ in range(15):
+            V = ora.ternarize_columns(R.T @ U, tau).astype(np.float64)
+            U = ora.ternarize_columns(R @ V, tau).astype(np.float64)
+        R = R - (U * ora.block_scales(R, U, V)) @ V.T
+    naive = 1.0 - float(np.sum(R * R)) / blk.norm_a2
+    assert blk.energy_final > naive + 0.05
+
+
+def test_block_energy_tracks_the_sequential_method():
+    """§1 / Table 1 caption: at b <= min(m, n)/8 the batched energy is within ~0.2 points of
+    the sequential one; energy never decreases from block to block."""
+    A = llm_matrix(256, 256, seed=7)
+    seq = ora.greedy_als(A, k=512, tau=0.7, seed=2)
+    blk = ora.block_als(A, k=512, tau=0.7, seed=2)
+    assert ora.block_width(256, 256) == 32
+    assert abs(blk.energy_final - seq.energy_final) <= 0.002
+    assert np.all(np.diff(blk.energy) >= -1e-12)
+    assert ora.energy(A, ora.reconstruct(blk.B, blk.D, blk.C)) == pytest.approx(blk.energy_final, abs=1e-12)
