@@ -562,20 +562,46 @@ struct Tot {
 };
 static_assert(sizeof(Tot) <= 64, "shared-memory slot of the totals");
 
+// Lane s of warp 0 takes rank s's message; fixed butterflies combine them (the same order in
+// every CTA of every cluster).
 __device__ __forceinline__ void totals(const Msg* msg, int c, int hb, Tot* out) {
-    if (threadIdx.x == 0) {
-        Tot t{0, 0, 0, 0, 0.0, 0.0, -1.0, 0.0, LLONG_MAX};
-        for (int s = 0; s < c; ++s) {
-            const Msg& m = msg[hb * c + s];
-            t.cnt += m.cnt;
-            t.nch += m.nch;
-            t.fail |= m.fail;
-            t.p += m.p;
-            t.hs += m.hs;
-            if (m.jx != LLONG_MAX && (m.mx > t.mx || (m.mx == t.mx && m.jx < t.jx))) { t.mx = m.mx; t.jx = m.jx; t.xj = m.xj; }
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        int cnt = 0, nch = 0, fail = 0;
+        double p = 0.0, hs = 0.0, mx = -1.0, xj = 0.0;
+        long long jx = LLONG_MAX;
+        if (lane < c) {
+            const Msg& m = msg[hb * c + lane];
+            cnt = m.cnt;
+            nch = m.nch;
+            fail = m.fail;
+            p = m.p;
+            hs = m.hs;
+            if (m.jx != LLONG_MAX) { mx = m.mx; jx = m.jx; xj = m.xj; }
         }
-        *out = t;
+        cnt = __reduce_add_sync(FULL, cnt);
+        nch = __reduce_add_sync(FULL, nch);
+        fail = __reduce_or_sync(FULL, fail);
+        #pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            p += __shfl_xor_sync(FULL, p, o);
+            hs += __shfl_xor_sync(FULL, hs, o);
+            const double m2 = __shfl_xor_sync(FULL, mx, o);
+            const long long j2 = __shfl_xor_sync(FULL, jx, o);
+            const double x2 = __shfl_xor_sync(FULL, xj, o);
+            if (m2 > mx || (m2 == mx && j2 < jx)) { mx = m2; jx = j2; xj = x2; }
+        }
+        if (lane == 0) {
+            Tot t{cnt, nch, fail, 0, p, hs, mx, xj, jx};
+            *out = t;
+        }
     }
+}
+
+// Words of a message that carry information: the header and the integer dots, plus the
+// weighted dots in the weighted kernel.
+__device__ __forceinline__ int msg_words(bool weighted) {
+    return (int)((offsetof(Msg, ddotw) + (weighted ? sizeof(double) * MAX_PENDING : 0)) / 4);
 }
 
 // Trace of one half-step (test hook): this CTA's quarter of the vector, its trits, and
@@ -670,7 +696,7 @@ __device__ __noinline__ int half2(const Prob& P, Ctx& x, const KCfg& cfg, const 
             while (sp + 1 < c && soff[sp + 1] <= j) ++sp;
             cl.map_shared_rank(s.xin, sp)[((size_t)hb * (c + 1) + x.r) * wpm + (j - soff[sp])] = s.part[j];
         }
-        const int words = (int)(sizeof(Msg) / 4);
+        const int words = msg_words(WTD);
         for (int t = tid; t < words * c; t += NT) {
             const int peer = t / words, k = t - peer * words;
             reinterpret_cast<uint32_t*>(cl.map_shared_rank(s.msg + hb * c + x.r, peer))[k] =
@@ -908,7 +934,7 @@ __device__ __noinline__ int end_round(Ctx& x, const Smem2& s, int L) {
             cl.map_shared_rank(s.psgV, peer)[(wc0 + kv) * Ls + L] = s.sgV[kv];
         }
     }
-    const int words = (int)(sizeof(Msg) / 4);
+    const int words = (int)(offsetof(Msg, ddot) / 4);   // the header (count, u^T y, fallback)
     for (int t = tid; t < words * c; t += NT) {
         const int peer = t / words, k = t - peer * words;
         reinterpret_cast<uint32_t*>(cl.map_shared_rank(s.msg + hb * c + x.r, peer))[k] =

@@ -1255,7 +1255,7 @@ __device__ bool run_problem(const Prob& P, int q, const KCfg& cfg, const Smem& s
     const int64_t kk = (mode == MODE_FACTOR) ? P.k : 1;
     // §2.4 refinement sweeps: visits kk .. nvis-1 revisit components 0 .. kk-1 in order.
     // (Little of this is held in registers across the visit loop: the half-steps already
-    // use all 64 of a 1024-thread CTA's.)  s.scal[12] counts the visits that kept the
+    // use most of a thread's registers.)  s.scal[12] counts the visits that kept the
     // stored pair.
     const int64_t nvis = kk * (int64_t)(1 + ((SWP && mode == MODE_FACTOR) ? P.sweeps : 0));
     if constexpr (SWP) if (tid == 0) s.scal[12] = 0.0;

@@ -6,7 +6,9 @@
 //
 // Design (B200):
 //  * One persistent cooperative launch runs every component of a matrix.  A
-//    matrix is served by a group of G CTAs (one per SM, 1024 threads each).
+//    matrix is served by a group of G CTAs (one per SM, 512 threads each: at 1024
+//    threads the 64-register cap spilled the half-step loop to local memory, and 512
+//    measured faster at every size).
 //  * The residual R is kept twice in HBM, each copy cut into one private block
 //    per CTA so that both half-steps read only what they need and no CTA ever
 //    reads another CTA's residual:
@@ -53,7 +55,7 @@
 namespace externd {
 
 #ifndef EXTERND_NT
-#define EXTERND_NT 1024
+#define EXTERND_NT 512
 #endif
 constexpr int NT = EXTERND_NT;        // threads per CTA of the ALS kernel
 constexpr int NWARP = NT / 32;
