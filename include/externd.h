@@ -181,6 +181,24 @@ int externd_factor_batched_ex(int count, const float* const* A, const int64_t* m
                               double* const* energy_out, int* status_out, void* stream,
                               const externd_batch_options* opt);
 
+/* Batched block ALS with decorrelated targets ("ExTernD: Expanded-Rank Ternary Decomposition",
+ * §2.4 "Batched block ALS"): components in blocks of b,
+ *   V <- T_tau([(U^T U + eps I)^-1 U^T R]^T),  U <- T_tau(R V (V^T V + eps I)^-1)  column-wise,
+ * `iters` times from the start vectors of the block's components (those of externd_factor, so
+ * b = 1 is the sequential method), then the joint scales [(U^T U) o (V^T V)] d = diag(U^T R V)
+ * and R <- R - U diag(d) V^T; blocks follow each other sequentially.  The pages leave eps open:
+ * here eps = 1e-6 x the mean diagonal of the Gram matrix.  The residual is held in fp64.
+ *   b          block width; 0 = the pages' default, 256 capped at floor(min(m, n) / 8).
+ *   energy_out [out] nullable; k doubles: E after the block holding component i.
+ *   d64_out    [out] nullable; k fp64 scales.
+ * A and all outputs are DEVICE pointers (EXTERND_EINVAL otherwise).  Other arguments and the
+ * output formats are those of externd_factor.  EXTERND_ELIMIT if a block's joint scale system is
+ * not positive definite (a component repeated within a block) or the shape exceeds 32-bit
+ * element indices. */
+int externd_factor_block(const float* A, int64_t m, int64_t n, double mu, double tau, int iters,
+                         uint64_t seed, int b, uint8_t* B_out, float* D_out, uint8_t* C_out,
+                         double* energy_out, double* d64_out, void* stream);
+
 /* Ahat = B diag(D) C (§2.1) with fp64 accumulation, written as fp32 m x n
  * row-major.  B, C packed as produced by externd_factor. */
 int externd_reconstruct(const uint8_t* B, const float* D, const uint8_t* C, int64_t m, int64_t n,

@@ -19,6 +19,7 @@ EXPORTS = (
     "externd_factor_ex",
     "externd_factor_weighted",
     "externd_factor_noalloc",
+    "externd_factor_block",
     "externd_factor_batched",
     "externd_factor_batched_ex",
     "externd_reconstruct",
@@ -131,6 +132,8 @@ def load():
     L.externd_factor_weighted.restype = c_int
     L.externd_factor_noalloc.argtypes = [vp, i64, i64, dbl, dbl, c_int, u64, vp, vp, vp, vp, vp]
     L.externd_factor_noalloc.restype = c_int
+    L.externd_factor_block.argtypes = [vp, i64, i64, dbl, dbl, c_int, u64, c_int, vp, vp, vp, vp, vp, vp]
+    L.externd_factor_block.restype = c_int
     L.externd_factor_batched.argtypes = [c_int, vp, vp, vp, vp, vp, c_int, vp, vp, vp, vp, vp, vp, vp]
     L.externd_factor_batched.restype = c_int
     L.externd_factor_batched_ex.argtypes = [c_int, vp, vp, vp, vp, vp, c_int, vp, vp, vp, vp, vp, vp, vp, vp]

@@ -274,6 +274,29 @@ def factor_noalloc(A: torch.Tensor, mu: float, tau: float, iters: int = 15, seed
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
+def factor_block(A: torch.Tensor, mu: float, tau: float, iters: int = 15, seed: int = 0, *, b: int = 0,
+                 want_d64: bool = False, stream=None) -> Factors:
+    """§2.4 batched block ALS with decorrelated targets (externd_factor_block); b = 0 takes the
+    pages' default width (256 capped at min(m, n) / 8).  A must be a float32 CUDA tensor."""
+    if not (isinstance(A, torch.Tensor) and A.is_cuda and A.dtype == torch.float32 and A.dim() == 2):
+        raise ValueError("A must be a 2-D float32 CUDA tensor")
+    A = A.contiguous()
+    m, n = A.shape
+    k = rank(m, n, mu)
+    if k < 1:
+        raise ExterndError(STATUS["EINVAL"], "externd_rank")
+    B = torch.empty((k, trit_bytes(m)), dtype=torch.uint8, device=A.device)
+    C = torch.empty((k, trit_bytes(n)), dtype=torch.uint8, device=A.device)
+    D = torch.empty((k,), dtype=torch.float32, device=A.device)
+    E = torch.empty((k,), dtype=torch.float64, device=A.device)
+    d64 = torch.empty((k,), dtype=torch.float64, device=A.device) if want_d64 else None
+    with _on_device(A):
+        rc = _lib.load().externd_factor_block(_ptr(A), m, n, float(mu), float(tau), int(iters), int(seed), int(b),
+                                              _ptr(B), _ptr(D), _ptr(C), _ptr(E), _ptr(d64), _stream(stream, A.device))
+    _check(rc, "externd_factor_block")
+    return Factors(B=B, D=D, C=C, energy=E, m=m, n=n, k=k, mu=float(mu), tau=float(tau), d64=d64, stats=last_stats())
+
+
 def factor_batched(As: Sequence, mus: Sequence[float], taus: Sequence[float], iters: int = 15,
                    seeds: Optional[Sequence[int]] = None, *, hs: Optional[Sequence] = None,
                    lams: Optional[Sequence[float]] = None, sweeps: int = 0, grid: int = 0, cluster: int = 0,

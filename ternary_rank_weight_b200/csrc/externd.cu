@@ -1566,6 +1566,7 @@ __global__ void __launch_bounds__(NT, 1) als_kernel(const KCfg cfg) {
 }  // namespace externd
 
 #include "als_cluster.cuh"
+#include "block_als.cuh"
 
 namespace externd {
 
@@ -2416,6 +2417,118 @@ int validate_factor(const float* A, int64_t m, int64_t n, double mu, double tau,
 
 }  // namespace
 
+namespace {
+
+// §2.4 batched block ALS on the device: blocks of b components, each a sequence of kernels
+// (see block_als.cuh).  A and the outputs are device pointers.
+int run_block(const float* A, int64_t m, int64_t n, int64_t k, double tau, int iters, uint64_t seed, int b,
+              uint8_t* B, float* D, uint8_t* C, double* E, double* d64, cudaStream_t stream, externd_stats& st) {
+    int rc = EXTERND_OK;
+    const int64_t bb = std::min<int64_t>(b, k);
+    const size_t f8 = sizeof(double);
+    const int nparts = 296;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { const size_t at = off; off += round_up(bytes, 256); return at; };
+    const size_t oR = take(f8 * (size_t)(m * n)), oU = take(f8 * (size_t)(m * bb)), oV = take(f8 * (size_t)(n * bb)),
+                 oP = take(f8 * (size_t)(bb * n)), oQ = take(f8 * (size_t)(m * bb)), oS = take(f8 * (size_t)(m * bb)),
+                 oGu = take(f8 * (size_t)(bb * bb)), oGv = take(f8 * (size_t)(bb * bb)), oL = take(f8 * (size_t)(bb * bb)),
+                 oH = take(f8 * (size_t)(bb * bb)), orhs = take(f8 * (size_t)bb), opart = take(f8 * nparts),
+                 oscal = take(f8 * 4), oflag = take(sizeof(int) * 4);
+    unsigned char* w = nullptr;
+    cudaEvent_t e0 = nullptr, e1 = nullptr;
+    int hflag[4] = {0, 0, 0, 0};
+    double hn0 = 0.0;
+    int launches = 0;
+    float ms = 0.f;
+    CK(cudaEventCreate(&e0));
+    CK(cudaEventCreate(&e1));
+    CK(cudaMallocAsync((void**)&w, off, stream));
+    CK(cudaEventRecord(e0, stream));
+    {
+        double *R = (double*)(w + oR), *U = (double*)(w + oU), *V = (double*)(w + oV), *P = (double*)(w + oP),
+               *Q = (double*)(w + oQ), *S = (double*)(w + oS), *Gu = (double*)(w + oGu), *Gv = (double*)(w + oGv),
+               *Lm = (double*)(w + oL), *H = (double*)(w + oH), *rhs = (double*)(w + orhs), *part = (double*)(w + opart),
+               *scal = (double*)(w + oscal);
+        int* flag = (int*)(w + oflag);
+        CK(cudaMemsetAsync(flag, 0, sizeof(int) * 4, stream));
+        block_setup_kernel<<<592, 256, 0, stream>>>(A, m * n, R, reinterpret_cast<unsigned*>(flag));
+        sumsq_kernel<<<nparts, 1024, 0, stream>>>(R, m * n, part);
+        sum_partials_kernel<<<1, 1024, 0, stream>>>(part, nparts, scal + 0);   // ||A||^2
+        CK(cudaGetLastError());
+        launches += 3;
+        CK(cudaMemcpyAsync(hflag, flag, sizeof(int), cudaMemcpyDeviceToHost, stream));
+        CK(cudaMemcpyAsync(&hn0, scal, sizeof(double), cudaMemcpyDeviceToHost, stream));
+        CK(cudaStreamSynchronize(stream));
+        if (hflag[0]) { rc = EXTERND_ENONFINITE; goto done; }
+        if (!(hn0 > 0.0)) { rc = EXTERND_EZERO; goto done; }
+        auto gemm = [&](int M, int N, int K, const double* Am, int lda, bool ta, const double* Bm, int ldb, bool tb,
+                        double* Cm, int ldc, double alpha, double beta) {
+            dim3 grid((unsigned)((N + BT - 1) / BT), (unsigned)((M + BT - 1) / BT));
+            gemm64_kernel<<<grid, BTH, 0, stream>>>(M, N, K, Am, lda, ta, Bm, ldb, tb, Cm, ldc, alpha, beta);
+            ++launches;
+        };
+        for (int64_t s0 = 0; s0 < k; s0 += bb) {
+            const int nb = (int)std::min<int64_t>(bb, k - s0);
+            block_start_kernel<<<nb, 256, 0, stream>>>(seed, s0, m, tau, U, nb);
+            ++launches;
+            for (int it = 0; it < iters; ++it) {
+                // V <- T_tau([(U^T U + eps I)^-1 U^T R]^T)
+                gemm(nb, nb, (int)m, U, nb, true, U, nb, false, Gu, nb, 1.0, 0.0);
+                CK(cudaMemcpyAsync(Lm, Gu, f8 * nb * nb, cudaMemcpyDeviceToDevice, stream));
+                chol_kernel<<<1, 1024, 0, stream>>>(Lm, nb, BLOCK_EPS_REL, flag + 1);
+                gemm(nb, (int)n, (int)m, U, nb, true, R, (int)n, false, P, (int)n, 1.0, 0.0);
+                chol_solve_kernel<<<(unsigned)((n + 127) / 128), 128, 0, stream>>>(Lm, nb, P, n, (int)n, false);
+                ternarize_cols_kernel<<<nb, 256, 0, stream>>>(P, n, (int)n, true, tau, V, nb);
+                // U <- T_tau(R V (V^T V + eps I)^-1)
+                gemm(nb, nb, (int)n, V, nb, true, V, nb, false, Gv, nb, 1.0, 0.0);
+                CK(cudaMemcpyAsync(Lm, Gv, f8 * nb * nb, cudaMemcpyDeviceToDevice, stream));
+                chol_kernel<<<1, 1024, 0, stream>>>(Lm, nb, BLOCK_EPS_REL, flag + 1);
+                gemm((int)m, nb, (int)n, R, (int)n, false, V, nb, false, Q, nb, 1.0, 0.0);
+                CK(cudaMemcpyAsync(S, Q, f8 * (size_t)(m * nb), cudaMemcpyDeviceToDevice, stream));
+                chol_solve_kernel<<<(unsigned)((m + 127) / 128), 128, 0, stream>>>(Lm, nb, S, m, nb, true);
+                ternarize_cols_kernel<<<nb, 256, 0, stream>>>(S, m, nb, false, tau, U, nb);
+                launches += 6;
+                CK(cudaGetLastError());
+            }
+            // joint scales: [(U^T U) o (V^T V)] d = diag(U^T R V), with Q = R V of the final V
+            gemm(nb, nb, (int)m, U, nb, true, U, nb, false, Gu, nb, 1.0, 0.0);
+            block_scale_system_kernel<<<std::max(1, std::min(nb, 148)), 256, 0, stream>>>(Gu, Gv, nb, U, Q, m, H, rhs);
+            chol_kernel<<<1, 1024, 0, stream>>>(H, nb, 0.0, flag + 2);
+            chol_solve_kernel<<<1, 128, 0, stream>>>(H, nb, rhs, 1, 1, false);
+            // deflation R <- R - U diag(d) V^T, energy, outputs
+            scale_cols_kernel<<<148, 256, 0, stream>>>(U, m, nb, rhs, S);
+            gemm((int)m, (int)n, nb, S, nb, false, V, nb, true, R, (int)n, -1.0, 1.0);
+            sumsq_kernel<<<nparts, 1024, 0, stream>>>(R, m * n, part);
+            sum_partials_kernel<<<1, 1024, 0, stream>>>(part, nparts, scal + 1);
+            block_pack_kernel<<<nb, 128, 0, stream>>>(U, m, nb, nb, s0, B, (int64_t)trit_bytes(m));
+            block_pack_kernel<<<nb, 128, 0, stream>>>(V, n, nb, nb, s0, C, (int64_t)trit_bytes(n));
+            block_out_kernel<<<1, 256, 0, stream>>>(rhs, nb, s0, scal + 1, scal + 0, D, d64, E);
+            launches += 10;
+            CK(cudaGetLastError());
+        }
+        CK(cudaEventRecord(e1, stream));
+        CK(cudaMemcpyAsync(hflag, flag, sizeof(int) * 4, cudaMemcpyDeviceToHost, stream));
+        CK(cudaStreamSynchronize(stream));
+        cudaEventElapsedTime(&ms, e0, e1);
+        // a scale system that is not positive definite (repeated components in a block)
+        if (hflag[2]) rc = EXTERND_ELIMIT;
+    }
+    st.total_ms = ms;
+    st.als_ms = ms;
+    st.launches = launches;
+    st.components = k;
+    st.group = (int)bb;   // block width
+    st.workspace_bytes = off;
+done:
+    if (w) { cudaFreeAsync(w, stream); cudaStreamSynchronize(stream); }
+    if (e0) cudaEventDestroy(e0);
+    if (e1) cudaEventDestroy(e1);
+    cudaGetLastError();
+    return rc;
+}
+
+}  // namespace
+
 // ---------------------------------------------------------------------------
 // Scratch memory of externd_factor_noalloc: one file-scope device array,
 // EXTERND_NOALLOC_SCRATCH_BYTES on every device that loads this library, kept
@@ -2539,6 +2652,28 @@ int externd_factor_noalloc(const float* A, int64_t m, int64_t n, double mu, doub
     fw.cap = EXTERND_NOALLOC_SCRATCH_BYTES;
     int st = 0;
     return run(&I, 1, ro, reinterpret_cast<cudaStream_t>(stream), &st, &fw);
+}
+
+int externd_factor_block(const float* A, int64_t m, int64_t n, double mu, double tau, int iters, uint64_t seed, int b,
+                         uint8_t* B_out, float* D_out, uint8_t* C_out, double* energy_out, double* d64_out,
+                         void* stream) {
+    int64_t k = 0;
+    int rc = validate_factor(A, m, n, mu, tau, iters, B_out, D_out, C_out, &k);
+    if (rc != EXTERND_OK) return rc;
+    if (b < 0) return EXTERND_EINVAL;
+    const void* ptrs[4] = {A, B_out, D_out, C_out};
+    for (const void* q : ptrs)
+        if (!is_device_ptr(q)) return EXTERND_EINVAL;
+    if ((energy_out && !is_device_ptr(energy_out)) || (d64_out && !is_device_ptr(d64_out))) return EXTERND_EINVAL;
+    // §2.4: b = 256 by default, capped at floor(min(m, n) / 8), at least 1
+    const int64_t cap = std::max<int64_t>(1, std::min(m, n) / 8);
+    const int bw = (int)std::min<int64_t>(b > 0 ? b : 256, b > 0 ? INT_MAX : cap);
+    if (m * n > (int64_t)INT_MAX || (int64_t)bw * std::max(m, n) > (int64_t)INT_MAX) return EXTERND_ELIMIT;
+    externd_stats st = {};
+    rc = run_block(A, m, n, k, tau, iters, seed, bw, B_out, D_out, C_out, energy_out, d64_out,
+                   reinterpret_cast<cudaStream_t>(stream), st);
+    g_last = st;
+    return rc;
 }
 
 int externd_factor_batched(int count, const float* const* A, const int64_t* m, const int64_t* n, const double* mu,

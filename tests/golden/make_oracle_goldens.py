@@ -17,6 +17,10 @@ For every workload matrix it stores
   of the int8 trits (u_i then v_i), which locate the first component where another
   implementation's trits differ.
 
+The job "block_mlp_2560x6912" runs the §2.4 batched block ALS (oracle block_als at the
+pages' default width) on the same matrix; its energy_index holds every 64th component,
+i.e. the energy after each block of 256 is sampled several times.
+
 Usage: python tests/golden/make_oracle_goldens.py [NAME ...]   (default: all)
 """
 from __future__ import annotations
@@ -42,6 +46,7 @@ EVERY = 64
 # (golden name, workload name, matrix index in the workload)
 JOBS = {
     "mlp_2560x6912": ("mlp_2560x6912_bf16_mu3_tau1.0", 0),
+    "block_mlp_2560x6912": ("mlp_2560x6912_bf16_mu3_tau1.0", 0),   # §2.4 block ALS at the default width
     "llm_4096x4096": ("llm_4096x4096_mu3.5_tau0.7", 0),
     "attn_1536_b0_tau0.7": ("attn_16x1536x1536_mu2.5_tau_cycle", 0),
     "attn_1536_b1_tau1.0": ("attn_16x1536x1536_mu2.5_tau_cycle", 1),
@@ -65,13 +70,17 @@ def make(name: str) -> dict:
     mu, tau, seed = w.mu[b], w.tau[b], w.seeds[b]
     k = ora.rank(m, n, mu)
     t0 = time.time()
-    ref = ora.greedy_als(A, k=k, tau=tau, iters=w.iters, seed=seed)
+    if name.startswith("block_"):
+        ref = ora.block_als(A, k=k, tau=tau, iters=w.iters, seed=seed)
+    else:
+        ref = ora.greedy_als(A, k=k, tau=tau, iters=w.iters, seed=seed)
     secs = time.time() - t0
     idx = sorted(set(range(0, k, EVERY)) | {k - 1})
     out = {
-        "_source": ("fp64 oracle (oracle/externd_oracle.py greedy_als) of ExTernD greedy sequential ALS, "
-                    "'ExTernD: Expanded-Rank Ternary Decomposition' §2.1-§2.3; written by "
-                    "tests/golden/make_oracle_goldens.py"),
+        "_source": ("fp64 oracle (oracle/externd_oracle.py " + ("block_als" if name.startswith("block_") else "greedy_als")
+                    + ") of 'ExTernD: Expanded-Rank Ternary Decomposition' " + ("§2.4 batched block ALS"
+                    if name.startswith("block_") else "§2.1-§2.3 greedy sequential ALS")
+                    + "; written by tests/golden/make_oracle_goldens.py"),
         "workload": wname, "matrix": b, "m": m, "n": n, "mu": mu, "tau": tau, "seed": seed, "iters": w.iters,
         "k": k,
         "energy_index": idx,
