@@ -49,9 +49,10 @@ def _peaks():
 
 
 def _kernel_source_hash() -> str:
-    """Hash of the device code: externd_kernels.cuh and externd.cu up to its host half (which
-    starts at `struct ProbIn`), line comments and blank lines removed, so editing a comment or
-    the host entry points does not invalidate the recorded ncu traffic."""
+    """Hash of the ALS kernel's device code: externd_kernels.cuh and externd.cu up to its host half
+    (which starts at `struct ProbIn`), line comments, blank lines and #include lines removed, so
+    editing a comment, the host entry points or another kernel's header does not invalidate the
+    recorded ncu traffic."""
     h = hashlib.sha256()
     for name in ("externd.cu", "externd_kernels.cuh"):
         with open(os.path.join(ROOT, "ternary_rank_weight_b200", "csrc", name), encoding="utf-8") as f:
@@ -59,7 +60,7 @@ def _kernel_source_hash() -> str:
                 if line.startswith("struct ProbIn"):
                     break
                 code = line.split("//", 1)[0].rstrip()
-                if code:
+                if code and not code.startswith("#include"):
                     h.update(code.encode() + b"\n")
     return h.hexdigest()
 
@@ -462,6 +463,90 @@ def run_matvec(args):
     return 0
 
 
+# ---------------------------------------------------------------------------
+# Batched block ALS (§2.4) on the workload's matrix 0
+# ---------------------------------------------------------------------------
+
+FP64_NOMINAL_TFLOPS = 37.0       # B200 fp64 (CUDA cores and DMMA), NVIDIA's published per-GPU figure
+BF16_NOMINAL_TFLOPS = 2250.0     # dense bf16, the recipe's nominal figure
+
+
+def _fp64_peak():
+    """fp64 roofline denominator: the measured bf16 GEMM peak times the nominal fp64 / bf16 ratio."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]) * FP64_NOMINAL_TFLOPS / BF16_NOMINAL_TFLOPS, "measured bf16 x nominal fp64/bf16"
+    except Exception:
+        return 1590.0 * FP64_NOMINAL_TFLOPS / BF16_NOMINAL_TFLOPS, "fallback bf16 x nominal fp64/bf16"
+
+
+def run_block(args):
+    """Time externd_factor_block (device-resident A) and, end to end, with A uploaded from pinned
+    host memory and the factors downloaded inside the timed region."""
+    import torch
+    import ternary_rank_weight_b200 as ext
+    from ternary_rank_weight_b200 import dist
+
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w, mats = _workload_arrays(args.workload, rank, args.mu)
+    A = torch.from_numpy(mats[0]).to(dev)
+    Ah = torch.from_numpy(mats[0]).pin_memory()
+    mu, tau, seed = w.mu[0], w.tau[0], w.seeds[0]
+    m, n = mats[0].shape
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        f = ext.factor_block(A, mu, tau, iters=w.iters, seed=seed)
+    dist.barrier(dev)
+    with ClockSampler(dev.index) as clk:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            f = ext.factor_block(A, mu, tau, iters=w.iters, seed=seed)
+        e1.record(stream)
+        dist.barrier(dev)
+    t_ms = dist.max_over_ranks(e0.elapsed_time(e1), dev) / args.steps
+    k, b = f.k, f.stats["group"]
+    # end to end: upload, factor, download
+    h2d = Ah.numel() * 4
+    d2h = f.B.numel() + f.C.numel() + f.D.numel() * 4 + f.energy.numel() * 8
+    e0.record(stream)
+    for _ in range(args.steps):
+        g = ext.factor_block(Ah.to(dev, non_blocking=True), mu, tau, iters=w.iters, seed=seed)
+        for t in (g.B, g.C, g.D, g.energy):
+            t.cpu()
+    e1.record(stream)
+    dist.barrier(dev)
+    e2e_ms = dist.max_over_ranks(e0.elapsed_time(e1), dev) / args.steps
+    # fp64 GEMM flops per call: per block and iteration U^T U, R^T U, V^T V, R V; per block the
+    # final U^T U and the deflation
+    flops = 0.0
+    for s0 in range(0, k, b):
+        nb = min(b, k - s0)
+        flops += w.iters * 2.0 * nb * (nb * m + n * m + nb * n + m * n) + 2.0 * nb * (nb * m + m * n)
+    peak, peak_kind = _fp64_peak()
+    achieved = flops / (t_ms / 1000.0) / 1e12
+    out = {"op": "block", "metric": "ternary components fitted/s, batched block ALS (§2.4)",
+           "value": dist.sum_over_ranks(k, dev) / (t_ms / 1000.0), "unit": "components/s", "n_gpus": ws,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": _config(w, {"k": k, "block": b, "l2": "inputs larger than L2 (A and the fp64 residual); no flush"}),
+           "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                        "frac": achieved / peak, "traffic": None, "kernel": "fp64 GEMMs (cuBLAS DGEMM)",
+                        "peak_kind": peak_kind, "gemm_flops_per_call": flops,
+                        "note": "achieved = the GEMMs' flops / the whole call's time (a lower bound for the GEMMs)"},
+           "e2e": {"value": dist.sum_over_ranks(k, dev) / (e2e_ms / 1000.0), "unit": "components/s",
+                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+           "gpu_launches": f.stats["launches"],
+           "clocks": clk.summary(),
+           "energy": float(f.energy[-1].item())}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    return 0
+
+
 def main():
     from ternary_rank_weight_b200.workloads import HEADLINE, WORKLOADS
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
@@ -480,8 +565,9 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of oracle work per sample")
     ap.add_argument("--mu", type=float, default=None, help="override mu (short runs for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=("factor", "matvec"), default="factor",
-                    help="factor: the factorization (default); matvec: inference with the factors")
+    ap.add_argument("--op", choices=("factor", "matvec", "block"), default="factor",
+                    help="factor: the factorization (default); matvec: inference with the factors; "
+                         "block: the batched block ALS of §2.4")
     ap.add_argument("--batch", type=int, default=1, help="input vectors per matvec call (--op matvec)")
     args = ap.parse_args()
     args.ref_budget = min(args.ref_budget, 150.0 / max(args.steps, 1))
@@ -489,6 +575,8 @@ def main():
         return run_reference(args)
     if args.op == "matvec":
         return run_matvec(args)
+    if args.op == "block":
+        return run_block(args)
     if args.all:
         for name in WORKLOADS:
             args.workload = name

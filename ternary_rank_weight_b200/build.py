@@ -12,13 +12,16 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SOURCES = [os.path.join(HERE, "csrc", "externd.cu"), os.path.join(HERE, "csrc", "infer.cu")]
-DEPS = SOURCES + [os.path.join(HERE, "csrc", "externd_kernels.cuh"), os.path.join(ROOT, "include", "externd.h")]
+DEPS = SOURCES + [os.path.join(HERE, "csrc", name) for name in ("externd_kernels.cuh", "als_cluster.cuh", "block_als.cuh")] \
+    + [os.path.join(ROOT, "include", "externd.h")]
 OUT = os.path.join(HERE, "libexternd.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",
     "-Xcompiler", "-fPIC", "-shared",
+    # the block ALS (§2.4) hands its plain fp64 GEMMs and Cholesky solves to the vendor libraries
+    "-lcublas", "-lcusolver", "-Xlinker", "-rpath=/usr/local/cuda/lib64",
 ]
 
 

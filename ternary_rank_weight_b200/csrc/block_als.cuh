@@ -7,75 +7,16 @@
 // the Gram matrix it regularizes.
 //
 // B200 design: the block method is dense linear algebra on the fp64 residual (m x n, kept
-// in fp64 so that its deflation by whole blocks does not round), so each block is a short
-// sequence of kernels: a tiled fp64 GEMM (U^T R, R V, the Gram matrices, the deflation),
-// a one-CTA Cholesky factorization of each b x b system with column-parallel triangular
-// solves, and a column-wise T_tau.  U and V are held as fp64 +-1/0 matrices.
+// in fp64 so that its deflation by whole blocks does not round).  Each block is a short
+// sequence of launches on one stream: the plain fp64 GEMMs (U^T U, R^T U, V^T V, R V and the
+// deflation) and the Cholesky factorizations and solves of the b x b systems go to the
+// vendor libraries (cuBLAS DGEMM, cuSOLVER POTRF/POTRS); the method's own steps run in the
+// kernels below: start trits, the ridge, the column-wise T_tau, the joint scale system, the
+// energy, and the packing of the trits.  U and V are held as fp64 +-1/0 matrices.
 
 namespace externd {
 
 constexpr double BLOCK_EPS_REL = 1e-6;   // the ridge: eps = this x the Gram matrix's mean diagonal
-constexpr int BT = 64;     // GEMM tile (rows x columns of the output)
-constexpr int BK = 16;     // GEMM depth step
-constexpr int BTH = 256;   // GEMM threads: 16 x 16, each 4 x 4 outputs
-
-// C (M x N, row stride ldc) = alpha * op(A) op(B) + beta * C, fp64; op(A) is M x K, op(B) K x N.
-// ta: A is stored K x M (row stride lda) and transposed; tb: B is stored N x K and transposed.
-__global__ void __launch_bounds__(BTH) gemm64_kernel(int M, int N, int K, const double* __restrict__ A, int lda,
-                                                    bool ta, const double* __restrict__ B, int ldb, bool tb,
-                                                    double* __restrict__ C, int ldc, double alpha, double beta) {
-    __shared__ double As[BK][BT + 1];
-    __shared__ double Bs[BK][BT + 1];
-    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-    const int row0 = blockIdx.y * BT, col0 = blockIdx.x * BT;
-    double acc[4][4];
-    #pragma unroll
-    for (int i = 0; i < 4; ++i)
-        #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
-    for (int k0 = 0; k0 < K; k0 += BK) {
-        for (int t = threadIdx.x; t < BK * BT; t += BTH) {
-            const int kk = t / BT, ii = t % BT;
-            const int r = row0 + ii, k = k0 + kk;
-            double a = 0.0;
-            if (r < M && k < K) a = ta ? A[(int64_t)k * lda + r] : A[(int64_t)r * lda + k];
-            As[kk][ii] = a;
-            const int c = col0 + ii;
-            double bv = 0.0;
-            if (c < N && k < K) bv = tb ? B[(int64_t)c * ldb + k] : B[(int64_t)k * ldb + c];
-            Bs[kk][ii] = bv;
-        }
-        __syncthreads();
-        #pragma unroll
-        for (int kk = 0; kk < BK; ++kk) {
-            double a[4], bv[4];
-            #pragma unroll
-            for (int i = 0; i < 4; ++i) a[i] = As[kk][ty + 16 * i];
-            #pragma unroll
-            for (int j = 0; j < 4; ++j) bv[j] = Bs[kk][tx + 16 * j];
-            #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                #pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fma(a[i], bv[j], acc[i][j]);
-        }
-        __syncthreads();
-    }
-    #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int r = row0 + ty + 16 * i;
-        if (r >= M) continue;
-        #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int c = col0 + tx + 16 * j;
-            if (c < N) {
-                double* p = C + (int64_t)r * ldc + c;
-                *p = alpha * acc[i][j] + (beta != 0.0 ? beta * *p : 0.0);
-            }
-        }
-    }
-}
-
-// R (m x n fp64) <- A (fp32); counts non-finite entries.
 __global__ void block_setup_kernel(const float* __restrict__ A, int64_t total, double* __restrict__ R,
                                    unsigned* nonfinite) {
     for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < total; t += (int64_t)gridDim.x * blockDim.x) {
@@ -168,59 +109,32 @@ __global__ void __launch_bounds__(256) ternarize_cols_kernel(const double* __res
     }
 }
 
-// In-place Cholesky factorization L L^T = G + eps I of a b x b matrix (one CTA), eps =
-// eps_rel x mean diagonal (eps_rel = 0: no ridge).  status: 0, or 1 if a pivot is not positive.
-__global__ void __launch_bounds__(1024) chol_kernel(double* G, int b, double eps_rel, int* status) {
-    __shared__ double eps;
-    __shared__ int bad;
+// Lm = G + eps I, eps = eps_rel x mean diagonal of G (b x b, one CTA).
+__global__ void __launch_bounds__(1024) ridge_kernel(const double* __restrict__ G, int b, double eps_rel,
+                                                     double* __restrict__ Lm) {
+    __shared__ double part[32];
+    double tr = 0.0;
+    for (int i = threadIdx.x; i < b; i += blockDim.x) tr += G[(int64_t)i * b + i];
+    #pragma unroll
+    for (int o = 16; o; o >>= 1) tr += __shfl_xor_sync(FULL, tr, o);
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = tr;
+    __syncthreads();
     if (threadIdx.x == 0) {
-        double tr = 0.0;
-        for (int i = 0; i < b; ++i) tr += G[(int64_t)i * b + i];
-        eps = eps_rel * tr / (double)b;
-        bad = 0;
+        double t = 0.0;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += part[w];   // fixed order
+        part[0] = eps_rel * t / (double)b;
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < b; i += 1024) G[(int64_t)i * b + i] += eps;
-    __syncthreads();
-    for (int k = 0; k < b; ++k) {
-        if (threadIdx.x == 0) {
-            const double dkk = G[(int64_t)k * b + k];
-            if (!(dkk > 0.0)) bad = 1;
-            G[(int64_t)k * b + k] = dkk > 0.0 ? sqrt(dkk) : 1.0;
-        }
-        __syncthreads();
-        const double lkk = G[(int64_t)k * b + k];
-        for (int i = k + 1 + threadIdx.x; i < b; i += 1024) G[(int64_t)i * b + k] /= lkk;
-        __syncthreads();
-        // trailing update of the lower triangle
-        const int rest = b - k - 1;
-        for (int t = threadIdx.x; t < rest * rest; t += 1024) {
-            const int i = k + 1 + t / rest, jj = k + 1 + t % rest;
-            if (jj <= i) G[(int64_t)i * b + jj] -= G[(int64_t)i * b + k] * G[(int64_t)jj * b + k];
-        }
-        __syncthreads();
-    }
-    if (threadIdx.x == 0 && bad) *status = 1;
+    const double eps = part[0];
+    for (int64_t t = threadIdx.x; t < (int64_t)b * b; t += blockDim.x)
+        Lm[t] = G[t] + ((t / b == t % b) ? eps : 0.0);
 }
 
-// Solve (L L^T) y = x for `cols` right-hand sides: x_c is column c of X (b x ldx, col-major
-// use: element i of right-hand side c at X[i * ldx + c]) when !rows, or row c (X[c * ldx + i])
-// when rows.  One thread per right-hand side, in place.
-__global__ void __launch_bounds__(128) chol_solve_kernel(const double* __restrict__ L, int b, double* X, int64_t cols,
-                                                        int ldx, bool rows) {
-    const int64_t c = (int64_t)blockIdx.x * 128 + threadIdx.x;
-    if (c >= cols) return;
-    auto at = [&](int i) -> double& { return rows ? X[c * ldx + i] : X[(int64_t)i * ldx + c]; };
-    for (int i = 0; i < b; ++i) {          // forward: L z = x
-        double s = at(i);
-        for (int k = 0; k < i; ++k) s -= L[(int64_t)i * b + k] * at(k);
-        at(i) = s / L[(int64_t)i * b + i];
-    }
-    for (int i = b - 1; i >= 0; --i) {     // backward: L^T y = z
-        double s = at(i);
-        for (int k = i + 1; k < b; ++k) s -= L[(int64_t)k * b + i] * at(k);
-        at(i) = s / L[(int64_t)i * b + i];
-    }
+// Any nonzero status among n (the factorization info words) -> *flag = 1.
+__global__ void info_any_kernel(const int* __restrict__ info, int n, int* flag) {
+    int bad = 0;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) bad |= (info[i] != 0);
+    if (__syncthreads_or(bad) && threadIdx.x == 0) *flag = 1;
 }
 
 // Start vectors of components s0 .. s0 + nb - 1 as fp64 columns of U (m x ldu): T_tau of the

@@ -5,7 +5,9 @@
 // The data layout and the synchronisation scheme are described at the top of
 // externd_kernels.cuh.
 #include <cooperative_groups.h>
+#include <cublas_v2.h>
 #include <cuda_runtime.h>
+#include <cusolverDn.h>
 
 #include <climits>
 #include <cmath>
@@ -2419,38 +2421,72 @@ int validate_factor(const float* A, int64_t m, int64_t n, double mu, double tau,
 
 namespace {
 
-// §2.4 batched block ALS on the device: blocks of b components, each a sequence of kernels
-// (see block_als.cuh).  A and the outputs are device pointers.
+// §2.4 batched block ALS on the device: blocks of b components, each a sequence of launches on
+// `stream` (kernels in block_als.cuh; the plain GEMMs, Cholesky factorizations and solves in
+// cuBLAS / cuSOLVER).  A and the outputs are device pointers.
+struct Linalg {
+    cublasHandle_t blas = nullptr;
+    cusolverDnHandle_t sol = nullptr;
+};
+std::mutex g_linalg_mu;          // one block factorization at a time per process (the handles' stream)
+Linalg g_linalg[64];
+
+bool linalg_for(int dev, Linalg*& out) {
+    if (dev < 0 || dev >= 64) return false;
+    Linalg& h = g_linalg[dev];
+    if (!h.blas && cublasCreate(&h.blas) != CUBLAS_STATUS_SUCCESS) { h.blas = nullptr; return false; }
+    if (!h.sol && cusolverDnCreate(&h.sol) != CUSOLVER_STATUS_SUCCESS) { h.sol = nullptr; return false; }
+    out = &h;
+    return true;
+}
+
 int run_block(const float* A, int64_t m, int64_t n, int64_t k, double tau, int iters, uint64_t seed, int b,
               uint8_t* B, float* D, uint8_t* C, double* E, double* d64, cudaStream_t stream, externd_stats& st) {
     int rc = EXTERND_OK;
     const int64_t bb = std::min<int64_t>(b, k);
+    const int64_t nblocks = (k + bb - 1) / bb;
+    const int ninfo = (int)(nblocks * (2 * (int64_t)iters + 1));   // one word per factorization
     const size_t f8 = sizeof(double);
     const int nparts = 296;
+    std::lock_guard<std::mutex> lock(g_linalg_mu);
+    int dev = 0;
+    Linalg* la = nullptr;
+    if (cudaGetDevice(&dev) != cudaSuccess || !linalg_for(dev, la)) { cudaGetLastError(); return EXTERND_ECUDA; }
+    if (cublasSetStream(la->blas, stream) != CUBLAS_STATUS_SUCCESS ||
+        cusolverDnSetStream(la->sol, stream) != CUSOLVER_STATUS_SUCCESS)
+        return EXTERND_ECUDA;
+    int lwork = 0;
+    if (cusolverDnDpotrf_bufferSize(la->sol, CUBLAS_FILL_MODE_LOWER, (int)bb, nullptr, (int)bb, &lwork) !=
+        CUSOLVER_STATUS_SUCCESS)
+        return EXTERND_ECUDA;
     size_t off = 0;
     auto take = [&](size_t bytes) { const size_t at = off; off += round_up(bytes, 256); return at; };
     const size_t oR = take(f8 * (size_t)(m * n)), oU = take(f8 * (size_t)(m * bb)), oV = take(f8 * (size_t)(n * bb)),
                  oP = take(f8 * (size_t)(bb * n)), oQ = take(f8 * (size_t)(m * bb)), oS = take(f8 * (size_t)(m * bb)),
                  oGu = take(f8 * (size_t)(bb * bb)), oGv = take(f8 * (size_t)(bb * bb)), oL = take(f8 * (size_t)(bb * bb)),
                  oH = take(f8 * (size_t)(bb * bb)), orhs = take(f8 * (size_t)bb), opart = take(f8 * nparts),
-                 oscal = take(f8 * 4), oflag = take(sizeof(int) * 4);
+                 oscal = take(f8 * 4), owork = take(f8 * (size_t)std::max(lwork, 1)),
+                 oinfo = take(sizeof(int) * (size_t)(ninfo + 1)), oflag = take(sizeof(int) * 4);
     unsigned char* w = nullptr;
     cudaEvent_t e0 = nullptr, e1 = nullptr;
     int hflag[4] = {0, 0, 0, 0};
     double hn0 = 0.0;
     int launches = 0;
     float ms = 0.f;
+    bool la_ok = true;
     CK(cudaEventCreate(&e0));
     CK(cudaEventCreate(&e1));
     CK(cudaMallocAsync((void**)&w, off, stream));
     CK(cudaEventRecord(e0, stream));
     {
-        double *R = (double*)(w + oR), *U = (double*)(w + oU), *V = (double*)(w + oV), *P = (double*)(w + oP),
+        double *R = (double*)(w + oR), *U = (double*)(w + oU), *V = (double*)(w + oV), *PT = (double*)(w + oP),
                *Q = (double*)(w + oQ), *S = (double*)(w + oS), *Gu = (double*)(w + oGu), *Gv = (double*)(w + oGv),
                *Lm = (double*)(w + oL), *H = (double*)(w + oH), *rhs = (double*)(w + orhs), *part = (double*)(w + opart),
-               *scal = (double*)(w + oscal);
+               *scal = (double*)(w + oscal), *work = (double*)(w + owork);
+        int* info = (int*)(w + oinfo);
         int* flag = (int*)(w + oflag);
         CK(cudaMemsetAsync(flag, 0, sizeof(int) * 4, stream));
+        CK(cudaMemsetAsync(info, 0, sizeof(int) * (size_t)(ninfo + 1), stream));
         block_setup_kernel<<<592, 256, 0, stream>>>(A, m * n, R, reinterpret_cast<unsigned*>(flag));
         sumsq_kernel<<<nparts, 1024, 0, stream>>>(R, m * n, part);
         sum_partials_kernel<<<1, 1024, 0, stream>>>(part, nparts, scal + 0);   // ||A||^2
@@ -2461,40 +2497,51 @@ int run_block(const float* A, int64_t m, int64_t n, int64_t k, double tau, int i
         CK(cudaStreamSynchronize(stream));
         if (hflag[0]) { rc = EXTERND_ENONFINITE; goto done; }
         if (!(hn0 > 0.0)) { rc = EXTERND_EZERO; goto done; }
+        // row-major C (M x N) = alpha op(A) op(B) + beta C: the column-major product C^T = op(B)^T op(A)^T
         auto gemm = [&](int M, int N, int K, const double* Am, int lda, bool ta, const double* Bm, int ldb, bool tb,
                         double* Cm, int ldc, double alpha, double beta) {
-            dim3 grid((unsigned)((N + BT - 1) / BT), (unsigned)((M + BT - 1) / BT));
-            gemm64_kernel<<<grid, BTH, 0, stream>>>(M, N, K, Am, lda, ta, Bm, ldb, tb, Cm, ldc, alpha, beta);
-            ++launches;
+            la_ok = la_ok && cublasDgemm(la->blas, tb ? CUBLAS_OP_T : CUBLAS_OP_N, ta ? CUBLAS_OP_T : CUBLAS_OP_N, N, M, K,
+                                         &alpha, Bm, ldb, Am, lda, &beta, Cm, ldc) == CUBLAS_STATUS_SUCCESS;
         };
+        // Cholesky of the b x b matrix in Lm, then solve (L L^T) X = Y for nrhs right-hand sides
+        // stored as rows of a row-major nrhs x b matrix (= columns of a column-major b x nrhs one)
+        auto factor = [&](int nb, double* Mat, int* inf) {
+            la_ok = la_ok && cusolverDnDpotrf(la->sol, CUBLAS_FILL_MODE_LOWER, nb, Mat, nb, work, lwork, inf) ==
+                                 CUSOLVER_STATUS_SUCCESS;
+        };
+        auto solve = [&](int nb, const double* Mat, double* Y, int nrhs, int* inf) {
+            la_ok = la_ok && cusolverDnDpotrs(la->sol, CUBLAS_FILL_MODE_LOWER, nb, nrhs, Mat, nb, Y, nb, inf) ==
+                                 CUSOLVER_STATUS_SUCCESS;
+        };
+        int slot = 0;
         for (int64_t s0 = 0; s0 < k; s0 += bb) {
             const int nb = (int)std::min<int64_t>(bb, k - s0);
             block_start_kernel<<<nb, 256, 0, stream>>>(seed, s0, m, tau, U, nb);
             ++launches;
             for (int it = 0; it < iters; ++it) {
-                // V <- T_tau([(U^T U + eps I)^-1 U^T R]^T)
+                // V <- T_tau([(U^T U + eps I)^-1 U^T R]^T): the rows of P^T = R^T U solved in place
                 gemm(nb, nb, (int)m, U, nb, true, U, nb, false, Gu, nb, 1.0, 0.0);
-                CK(cudaMemcpyAsync(Lm, Gu, f8 * nb * nb, cudaMemcpyDeviceToDevice, stream));
-                chol_kernel<<<1, 1024, 0, stream>>>(Lm, nb, BLOCK_EPS_REL, flag + 1);
-                gemm(nb, (int)n, (int)m, U, nb, true, R, (int)n, false, P, (int)n, 1.0, 0.0);
-                chol_solve_kernel<<<(unsigned)((n + 127) / 128), 128, 0, stream>>>(Lm, nb, P, n, (int)n, false);
-                ternarize_cols_kernel<<<nb, 256, 0, stream>>>(P, n, (int)n, true, tau, V, nb);
-                // U <- T_tau(R V (V^T V + eps I)^-1)
+                ridge_kernel<<<1, 1024, 0, stream>>>(Gu, nb, BLOCK_EPS_REL, Lm);
+                factor(nb, Lm, info + slot++);
+                gemm((int)n, nb, (int)m, R, (int)n, true, U, nb, false, PT, nb, 1.0, 0.0);
+                solve(nb, Lm, PT, (int)n, info + ninfo);
+                ternarize_cols_kernel<<<nb, 256, 0, stream>>>(PT, n, nb, false, tau, V, nb);
+                // U <- T_tau(R V (V^T V + eps I)^-1): the rows of Q = R V solved in place
                 gemm(nb, nb, (int)n, V, nb, true, V, nb, false, Gv, nb, 1.0, 0.0);
-                CK(cudaMemcpyAsync(Lm, Gv, f8 * nb * nb, cudaMemcpyDeviceToDevice, stream));
-                chol_kernel<<<1, 1024, 0, stream>>>(Lm, nb, BLOCK_EPS_REL, flag + 1);
+                ridge_kernel<<<1, 1024, 0, stream>>>(Gv, nb, BLOCK_EPS_REL, Lm);
+                factor(nb, Lm, info + slot++);
                 gemm((int)m, nb, (int)n, R, (int)n, false, V, nb, false, Q, nb, 1.0, 0.0);
-                CK(cudaMemcpyAsync(S, Q, f8 * (size_t)(m * nb), cudaMemcpyDeviceToDevice, stream));
-                chol_solve_kernel<<<(unsigned)((m + 127) / 128), 128, 0, stream>>>(Lm, nb, S, m, nb, true);
-                ternarize_cols_kernel<<<nb, 256, 0, stream>>>(S, m, nb, false, tau, U, nb);
-                launches += 6;
+                if (it == iters - 1) CK(cudaMemcpyAsync(S, Q, f8 * (size_t)(m * nb), cudaMemcpyDeviceToDevice, stream));
+                solve(nb, Lm, Q, (int)m, info + ninfo);
+                ternarize_cols_kernel<<<nb, 256, 0, stream>>>(Q, m, nb, false, tau, U, nb);
+                launches += 4;
                 CK(cudaGetLastError());
             }
-            // joint scales: [(U^T U) o (V^T V)] d = diag(U^T R V), with Q = R V of the final V
+            // joint scales: [(U^T U) o (V^T V)] d = diag(U^T R V), with S = R V of the final V
             gemm(nb, nb, (int)m, U, nb, true, U, nb, false, Gu, nb, 1.0, 0.0);
-            block_scale_system_kernel<<<std::max(1, std::min(nb, 148)), 256, 0, stream>>>(Gu, Gv, nb, U, Q, m, H, rhs);
-            chol_kernel<<<1, 1024, 0, stream>>>(H, nb, 0.0, flag + 2);
-            chol_solve_kernel<<<1, 128, 0, stream>>>(H, nb, rhs, 1, 1, false);
+            block_scale_system_kernel<<<std::max(1, std::min(nb, 148)), 256, 0, stream>>>(Gu, Gv, nb, U, S, m, H, rhs);
+            factor(nb, H, info + slot++);
+            solve(nb, H, rhs, 1, info + ninfo);
             // deflation R <- R - U diag(d) V^T, energy, outputs
             scale_cols_kernel<<<148, 256, 0, stream>>>(U, m, nb, rhs, S);
             gemm((int)m, (int)n, nb, S, nb, false, V, nb, true, R, (int)n, -1.0, 1.0);
@@ -2503,14 +2550,18 @@ int run_block(const float* A, int64_t m, int64_t n, int64_t k, double tau, int i
             block_pack_kernel<<<nb, 128, 0, stream>>>(U, m, nb, nb, s0, B, (int64_t)trit_bytes(m));
             block_pack_kernel<<<nb, 128, 0, stream>>>(V, n, nb, nb, s0, C, (int64_t)trit_bytes(n));
             block_out_kernel<<<1, 256, 0, stream>>>(rhs, nb, s0, scal + 1, scal + 0, D, d64, E);
-            launches += 10;
+            launches += 7;
             CK(cudaGetLastError());
+            if (!la_ok) { rc = EXTERND_ECUDA; goto done; }
         }
+        // a factorization that failed: a ridge system (cannot happen for eps > 0 and finite input)
+        // or a scale system that is not positive definite (repeated components in a block)
+        info_any_kernel<<<1, 256, 0, stream>>>(info, ninfo + 1, flag + 2);
+        ++launches;
         CK(cudaEventRecord(e1, stream));
         CK(cudaMemcpyAsync(hflag, flag, sizeof(int) * 4, cudaMemcpyDeviceToHost, stream));
         CK(cudaStreamSynchronize(stream));
         cudaEventElapsedTime(&ms, e0, e1);
-        // a scale system that is not positive definite (repeated components in a block)
         if (hflag[2]) rc = EXTERND_ELIMIT;
     }
     st.total_ms = ms;

@@ -11,11 +11,10 @@
 // dots of 2-bit trit rows with a dense fp32 vector:
 //     z_i = D_i * sum_j C[i, j] x_j        (k rows of n trits)
 //     y_r = sum_i B[r, i] z_i              (m rows of k trits)
-// One warp per row.  When the vectors fit in shared memory (NB * len * 4 bytes
-// up to ~200 KB) they are staged there and every trit is one fused multiply-add
-// with its code read as a signed 2-bit integer (rowdot_smem_kernel); otherwise each lane walks
-// the nonzero trits of its 16-byte chunks and reads the vector through L1
-// (rowdot_kernel).
+// When the vectors fit in shared memory (NB * len * 4 bytes up to 200 KB) they are
+// staged there once per CTA and every trit is decoded exactly in registers and applied
+// with f32x2 arithmetic (tdot_kernel); otherwise one warp per row walks the nonzero
+// trits of its 16-byte chunks and reads the vector through L1 (rowdot_kernel).
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -90,45 +89,151 @@ __global__ void __launch_bounds__(RD_THREADS) rowdot_kernel(const uint8_t* __res
     }
 }
 
-// Shared-memory variant: the NB vectors (NB * len fp32) are staged in shared
-// memory.  Each nibble of a trit row (two trits) indexes a 16-entry table of
-// coefficient pairs in {-1, 0, 1} (a 2-bit code read as a signed 2-bit integer is
-// the trit); the table is exactly 128 bytes, so lanes that read the same entry
-// share one access and different entries sit in different banks.  Each trit is
-// then one fused multiply-add per vector, with no divergence.  A warp
-// takes R rows at once: lane l reads the 32-bit words l, l + 32, ... of each (16
-// trits per word, up to G words per row issued before any is used), and every
-// vector value it loads from shared memory serves the R rows.  The staged vector
-// is swizzled: the four 16-byte groups of word w are rotated by (w / 2) % 4, so
-// the eight lanes of a quarter-warp (eight consecutive words) read distinct banks.
-constexpr int RS_THREADS = 128;   // shared-memory row-dot block: 4 warps; several blocks per SM
+// Shared-memory variant with exact in-register trit decoding (sm_100a f32x2 arithmetic).
+//
+// A trit's 2-bit code q (bit 0: nonzero, bit 1: negative) is the trit read as a signed
+// 2-bit integer, t = q0 - 2 q1.  With its high bit flipped it becomes the field
+// v = t + 2 in {1, 2, 3}.  Placed at bit 2p (p <= 10) of the mantissa of 2.0 by one
+// three-input logic operation, it gives F = 2 + v 2^(2p-22) exactly, and
+// F - (2 + 2^(2p-21)) = t 2^(2p-22) is exact as well (both operands lie in [2, 4)).
+// The staged vector entry is pre-scaled by 2^(22-2p), so the product of the two is
+// exactly t x, and each row dot is a plain fp32 sum of exact terms in a fixed order.
+// Trits 0..10 of a 32-bit word sit at p = 0..10 of the word itself, trits 11..15 at
+// p = 0..4 of the word shifted right by 22.  Pairs of trits go through one f32x2
+// subtraction and one f32x2 fused multiply-add per vector: with the logic operations,
+// about two instructions per trit and row, and no table lookups.
+//
+// Layout: a warp takes R rows at once; lane l reads 32-bit words l, l + 32, ... of each row
+// (G words per lane issued ahead of their use: the next chunk's words are loaded while the
+// current chunk is decoded), and each float4 of the staged vector serves the R rows.  The staged
+// vector keeps the 16 entries of word w at floats 20 w .. 20 w + 15 (4 floats of padding per
+// word), so the eight lanes of a quarter-warp, reading eight consecutive words, hit distinct banks
+// and each quad's offset within its word is a constant.  The grid is at most one CTA per SM; each
+// CTA stages the vectors once and its warps take row groups interleaved across CTAs.  Vectors
+// whose largest magnitude reaches 2^104 are staged with an extra power-of-two scale (undone on
+// the outputs), so the pre-scaling cannot overflow.
+//
+// The second product of a matvec (y = B z) is launched as a programmatic dependent of
+// the first: its CTAs may start while the first kernel runs, prefetch their trit rows into
+// L2, and wait (griddepcontrol.wait) before they read z.
+constexpr int TD_MAX_WARPS = 16;
 
-__device__ __forceinline__ int64_t swz(int64_t j) {    // position of vector entry j in shared memory
-    const int64_t w = j >> 4;
-    const int h = (int)((j >> 2) & 3);
-    return 16 * w + 4 * ((h + (int)(w >> 1)) & 3) + (j & 3);
+constexpr int SW = 20;   // floats per staged word of 16 entries (4 of padding: conflict-free float4 reads)
+
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ float2 upk2(uint64_t v) {
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+    return r;
+}
+__device__ __forceinline__ uint64_t sub_x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t fma_x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+// position p of trit j (0..15) of a word, and the word it is read from
+template <int J> struct TritPos { static constexpr int P = J <= 10 ? J : J - 11; static constexpr bool HI = J > 10; };
+
+// The words a trit is read from carry the exponent bits of 2.0 already (wa = flipped word | 2.0,
+// wb = flipped word >> 22 | 2.0), so F = 2 + (t + 2) 2^(2p-22) is one AND with the field mask plus bit 30.
+// the subtrahend 2 + 2 * 2^(2p-22) of each trit pair, as the packed pairs the loop uses
+// (pairs (0,1) (2,3) (4,5) (6,7) (8,9) (10,11) (12,13) (14,15) of a word)
+__host__ __device__ constexpr uint32_t trit_bias_bits(int j) {
+    return 0x40000000u | (2u << (2 * (j <= 10 ? j : j - 11)));
+}
+__constant__ uint64_t c_trit_bias[8] = {
+    (uint64_t)trit_bias_bits(0) | ((uint64_t)trit_bias_bits(1) << 32),
+    (uint64_t)trit_bias_bits(2) | ((uint64_t)trit_bias_bits(3) << 32),
+    (uint64_t)trit_bias_bits(4) | ((uint64_t)trit_bias_bits(5) << 32),
+    (uint64_t)trit_bias_bits(6) | ((uint64_t)trit_bias_bits(7) << 32),
+    (uint64_t)trit_bias_bits(8) | ((uint64_t)trit_bias_bits(9) << 32),
+    (uint64_t)trit_bias_bits(10) | ((uint64_t)trit_bias_bits(11) << 32),
+    (uint64_t)trit_bias_bits(12) | ((uint64_t)trit_bias_bits(13) << 32),
+    (uint64_t)trit_bias_bits(14) | ((uint64_t)trit_bias_bits(15) << 32)};
+// coefficient pair of trits J, J+1 (exact t 2^(2p-22) each); kb = c_trit_bias[J / 2].  The pair is
+// masked out of a 64-bit source that holds the words of both trits (wa:wa, wa:wb or wb:wb), so the two
+// halves land in the register pair the f32x2 subtraction reads.
+__host__ __device__ constexpr uint32_t trit_mask(int j) {
+    return (3u << (2 * (j <= 10 ? j : j - 11))) | 0x40000000u;
+}
+template <int J>
+__device__ __forceinline__ uint64_t trit_pair(uint64_t waa, uint64_t wab, uint64_t wbb, uint64_t kb) {
+    constexpr uint64_t M = (uint64_t)trit_mask(J) | ((uint64_t)trit_mask(J + 1) << 32);
+    const uint64_t src = (J + 1 <= 10) ? waa : (J >= 11 ? wbb : wab);
+    return sub_x2(src & M, kb);
+}
+
+__host__ __device__ __forceinline__ float pow2f(int e) {       // 2^e for -126 <= e <= 127
+    union { uint32_t u; float f; } c;
+    c.u = (uint32_t)(127 + e) << 23;
+    return c.f;
 }
 
 template <int NB, int R>
-__global__ void __launch_bounds__(RS_THREADS) rowdot_smem_kernel(const uint8_t* __restrict__ T, int64_t rows,
-                                                               int64_t len, int64_t tb, const float* __restrict__ V,
-                                                               int64_t vstride, const float* __restrict__ scale,
-                                                               float* __restrict__ out, int64_t ostride) {
-    extern __shared__ __align__(128) float smem_rd[];
-    float2* lut2 = reinterpret_cast<float2*>(smem_rd);     // 16 entries, 128 bytes: a nibble -> 2 trits
-    float* sv = smem_rd + 32;                               // NB x lenp, lenp = 16 * words, swizzled
+__global__ void __launch_bounds__(32 * TD_MAX_WARPS) tdot_kernel(const uint8_t* __restrict__ T, int64_t rows,
+                                                                  int64_t len, int64_t tb, const float* __restrict__ V,
+                                                                  int64_t vstride, const float* __restrict__ scale,
+                                                                  float* __restrict__ out, int64_t ostride,
+                                                                  int dependent) {
+    extern __shared__ __align__(16) float sv[];   // NB x spitch, pre-scaled, word w at SW * w
+    __shared__ uint32_t vmax[NB];
+    const int lane = threadIdx.x & 31;
+    const int nw = blockDim.x >> 5;
     const int64_t words = tb / 4;
     const int64_t lenp = words * 16;
-    if (threadIdx.x < 16) {
-        const int v = threadIdx.x;
-        lut2[v] = make_float2((float)((v << 30) >> 30), (float)(((v >> 2) << 30) >> 30));
+    const int64_t spitch = words * SW;
+    const int64_t groups = (rows + R - 1) / R;
+    const int64_t g0 = (int64_t)(threadIdx.x >> 5) * gridDim.x + blockIdx.x;
+    const int64_t gstride = (int64_t)nw * gridDim.x;
+    // the first chunk of this warp's first row group is loaded before anything else, so that its
+    // memory latency overlaps the staging (and, in a dependent launch, the producer's tail: the
+    // trits are not written by the producer)
+    constexpr int G = R >= 4 ? 4 : 8;                          // words per row and lane in flight
+    auto load_chunk = [&](uint32_t (&dst)[G][R], int64_t grp, int64_t w0) {
+        #pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const int64_t w = w0 + lane + 32 * g;
+            #pragma unroll
+            for (int rr = 0; rr < R; ++rr) {
+                const int64_t r = grp * R + rr;
+                dst[g][rr] = (r < rows && w < words) ? __ldg(reinterpret_cast<const uint32_t*>(T + r * tb) + w) : 0u;
+            }
+        }
+    };
+    uint32_t q[G][R], qn[G][R];
+    if (g0 < groups) load_chunk(q, g0, 0);
+    if (dependent) {
+        // this warp's trit rows into L2 while the producer of V runs, then wait for it
+        for (int64_t g = g0; g < groups; g += gstride) {
+            const int64_t r = g * R + lane;
+            if (lane < R && r < rows)
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(T + r * tb), "r"((uint32_t)tb) : "memory");
+        }
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+    } else {
+        asm volatile("griddepcontrol.launch_dependents;");
     }
+    if (threadIdx.x < NB) vmax[threadIdx.x] = 0u;
+    // stage the raw vectors: 16-byte asynchronous copies, all in flight at once, or plain loads
+    // when V is not 16-byte aligned.  Group g (entries 4 g .. 4 g + 3) goes to word g / 4, quad g % 4.
     const bool vec4 = ((len & 3) == 0) && ((vstride & 3) == 0) && ((reinterpret_cast<uintptr_t>(V) & 15) == 0);
+    const int64_t ngroups = lenp / 4;
+    auto slot = [&](int64_t g) { return SW * (g >> 2) + 4 * (g & 3); };
     for (int b = 0; b < NB; ++b) {
-        if (vec4) {   // 16-byte groups copied asynchronously (all in flight at once); the swizzle moves whole groups
+        if (vec4) {
             const float4* V4 = reinterpret_cast<const float4*>(V + b * vstride);
-            for (int64_t g = threadIdx.x; g < lenp / 4; g += RS_THREADS) {
-                float* dst = sv + b * lenp + swz(4 * g);
+            for (int64_t g = threadIdx.x; g < ngroups; g += blockDim.x) {
+                float* dst = sv + b * spitch + slot(g);
                 if (4 * g < len) {
                     const unsigned saddr = (unsigned)__cvta_generic_to_shared(dst);
                     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr), "l"(V4 + g) : "memory");
@@ -137,72 +242,125 @@ __global__ void __launch_bounds__(RS_THREADS) rowdot_smem_kernel(const uint8_t* 
                 }
             }
         } else {
-            for (int64_t j = threadIdx.x; j < lenp; j += RS_THREADS)
-                sv[b * lenp + swz(j)] = j < len ? __ldg(V + b * vstride + j) : 0.f;
+            for (int64_t g0s = threadIdx.x; g0s < ngroups; g0s += 2 * (int64_t)blockDim.x) {
+                float v[2][4];
+                #pragma unroll
+                for (int u = 0; u < 2; ++u)
+                    #pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int64_t j = 4 * (g0s + u * (int64_t)blockDim.x) + e;
+                        v[u][e] = j < len ? __ldg(V + b * vstride + j) : 0.f;
+                    }
+                #pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int64_t g = g0s + u * (int64_t)blockDim.x;
+                    if (g < ngroups)
+                        *reinterpret_cast<float4*>(sv + b * spitch + slot(g)) = make_float4(v[u][0], v[u][1], v[u][2], v[u][3]);
+                }
+            }
         }
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
-    const int lane = threadIdx.x & 31;
-    const int64_t groups = (rows + R - 1) / R;
-    const int64_t warps = (int64_t)gridDim.x * (RS_THREADS / 32);
-    constexpr int G = (R >= 4) ? 4 : 8;                     // words per row and lane issued together
-    for (int64_t grp = (int64_t)blockIdx.x * (RS_THREADS / 32) + (threadIdx.x >> 5); grp < groups; grp += warps) {
+    // largest magnitude of each vector (from shared memory), then the pre-scaling in place
+    for (int b = 0; b < NB; ++b) {
+        uint32_t mx = 0u;
+        for (int64_t g = threadIdx.x; g < ngroups; g += blockDim.x) {
+            const float4 t = *reinterpret_cast<const float4*>(sv + b * spitch + slot(g));
+            mx = max(mx, max(max(__float_as_uint(t.x) & 0x7fffffffu, __float_as_uint(t.y) & 0x7fffffffu),
+                             max(__float_as_uint(t.z) & 0x7fffffffu, __float_as_uint(t.w) & 0x7fffffffu)));
+        }
+        #pragma unroll
+        for (int o = 16; o; o >>= 1) mx = max(mx, __shfl_xor_sync(FULL, mx, o));
+        if (lane == 0) atomicMax(&vmax[b], mx);
+    }
+    __syncthreads();
+    int shift[NB];
+    #pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        const int e = (int)(vmax[b] >> 23) - 127;               // inf / NaN: 128, left unscaled
+        shift[b] = (e >= 104 && e < 128) ? e - 103 : 0;
+    }
+    for (int b = 0; b < NB; ++b) {
+        for (int64_t g = threadIdx.x; g < ngroups; g += blockDim.x) {
+            float4* p4 = reinterpret_cast<float4*>(sv + b * spitch + slot(g));
+            float4 t = *p4;
+            float* tv = &t.x;
+            #pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int q = 4 * (int)(g & 3) + u;               // trit position within the word
+                const int p = q <= 10 ? q : q - 11;
+                tv[u] *= pow2f(22 - 2 * p - shift[b]);
+            }
+            *p4 = t;
+        }
+    }
+    __syncthreads();
+    uint64_t kb[8];                                            // loop-invariant subtrahends, in registers
+    #pragma unroll
+    for (int i = 0; i < 8; ++i) kb[i] = c_trit_bias[i];
+    for (int64_t grp = g0; grp < groups; grp += gstride) {
         const int64_t r0 = grp * R;
-        float acc[R][NB];
+        uint64_t acc[R][NB], acc2[R][NB];   // for one or two vectors, two sums per row and vector: shorter chains
         #pragma unroll
         for (int rr = 0; rr < R; ++rr)
             #pragma unroll
-            for (int b = 0; b < NB; ++b) acc[rr][b] = 0.f;
+            for (int b = 0; b < NB; ++b) acc[rr][b] = acc2[rr][b] = 0ull;
+        // software pipeline: the words of the next chunk are loaded before the current chunk is used
+        if (grp != g0) load_chunk(q, grp, 0);
         for (int64_t w0 = 0; w0 < words; w0 += 32 * G) {
-            uint32_t q[R][G];
-            #pragma unroll
-            for (int rr = 0; rr < R; ++rr) {
-                const uint32_t* row = reinterpret_cast<const uint32_t*>(T + (r0 + rr) * tb);
-                #pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    const int64_t w = w0 + lane + 32 * g;
-                    q[rr][g] = (r0 + rr < rows && w < words) ? __ldg(row + w) : 0u;
-                }
-            }
+            load_chunk(qn, grp, w0 + 32 * G);
             #pragma unroll
             for (int g = 0; g < G; ++g) {
                 const int64_t w = w0 + lane + 32 * g;
                 if (w >= words) break;
-                const int rot = (int)(w >> 1);
+                const float* svw = sv + SW * w;
+                uint64_t waa[R], wab[R], wbb[R];
                 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    const int64_t at = 16 * w + 4 * ((h + rot) & 3);
-                    float x[NB][4];
-                    #pragma unroll
-                    for (int b = 0; b < NB; ++b) {
-                        const float4 t4 = *reinterpret_cast<const float4*>(sv + b * lenp + at);
-                        x[b][0] = t4.x; x[b][1] = t4.y; x[b][2] = t4.z; x[b][3] = t4.w;
-                    }
-                    #pragma unroll
-                    for (int rr = 0; rr < R; ++rr) {
-                        const uint32_t byte = (q[rr][g] >> (8 * h)) & 0xFFu;   // trits 4h .. 4h+3
-                        const float2 c01 = lut2[byte & 15u];
-                        const float2 c23 = lut2[byte >> 4];
-                        #pragma unroll
-                        for (int b = 0; b < NB; ++b) {
-                            acc[rr][b] = fmaf(c01.x, x[b][0], acc[rr][b]);
-                            acc[rr][b] = fmaf(c01.y, x[b][1], acc[rr][b]);
-                            acc[rr][b] = fmaf(c23.x, x[b][2], acc[rr][b]);
-                            acc[rr][b] = fmaf(c23.y, x[b][3], acc[rr][b]);
-                        }
-                    }
+                for (int rr = 0; rr < R; ++rr) {
+                    const uint32_t fl = q[g][rr] ^ 0xAAAAAAAAu;   // field v = t + 2 of every trit
+                    const uint32_t wa = fl | 0x40000000u;
+                    const uint32_t wb = (fl >> 22) | 0x40000000u;
+                    waa[rr] = ((uint64_t)wa << 32) | wa;
+                    wab[rr] = ((uint64_t)wb << 32) | wa;
+                    wbb[rr] = ((uint64_t)wb << 32) | wb;
                 }
+#define EXTERND_TDOT_QUAD(H, J0)                                                                                   \
+                {                                                                                                   \
+                    float4 x4[NB];                                                                                  \
+                    _Pragma("unroll") for (int b = 0; b < NB; ++b)                                                 \
+                        x4[b] = *reinterpret_cast<const float4*>(svw + b * spitch + 4 * H);                         \
+                    _Pragma("unroll") for (int rr = 0; rr < R; ++rr) {                                             \
+                        const uint64_t c01 = trit_pair<J0>(waa[rr], wab[rr], wbb[rr], kb[J0 / 2]);                  \
+                        const uint64_t c23 = trit_pair<J0 + 2>(waa[rr], wab[rr], wbb[rr], kb[J0 / 2 + 1]);          \
+                        _Pragma("unroll") for (int b = 0; b < NB; ++b) {                                           \
+                            acc[rr][b] = fma_x2(c01, pk2(x4[b].x, x4[b].y), acc[rr][b]);                            \
+                            if constexpr (NB <= 2) acc2[rr][b] = fma_x2(c23, pk2(x4[b].z, x4[b].w), acc2[rr][b]);   \
+                            else acc[rr][b] = fma_x2(c23, pk2(x4[b].z, x4[b].w), acc[rr][b]);                       \
+                        }                                                                                           \
+                    }                                                                                               \
+                }
+                EXTERND_TDOT_QUAD(0, 0)
+                EXTERND_TDOT_QUAD(1, 4)
+                EXTERND_TDOT_QUAD(2, 8)
+                EXTERND_TDOT_QUAD(3, 12)
+#undef EXTERND_TDOT_QUAD
             }
+            #pragma unroll
+            for (int g = 0; g < G; ++g)
+                #pragma unroll
+                for (int rr = 0; rr < R; ++rr) q[g][rr] = qn[g][rr];
         }
+        float res[R][NB];
         #pragma unroll
         for (int rr = 0; rr < R; ++rr)
             #pragma unroll
             for (int b = 0; b < NB; ++b) {
-                float a = acc[rr][b];
+                const float2 v2 = upk2(acc[rr][b]), w2 = upk2(acc2[rr][b]);
+                float a = (v2.x + v2.y) + (w2.x + w2.y);
                 #pragma unroll
                 for (int o = 16; o; o >>= 1) a += __shfl_xor_sync(FULL, a, o);
-                acc[rr][b] = a;
+                res[rr][b] = a;
             }
         if (lane == 0) {
             #pragma unroll
@@ -210,7 +368,7 @@ __global__ void __launch_bounds__(RS_THREADS) rowdot_smem_kernel(const uint8_t* 
                 if (r0 + rr >= rows) break;
                 const float sc = scale ? __ldg(scale + r0 + rr) : 1.f;
                 #pragma unroll
-                for (int b = 0; b < NB; ++b) out[b * ostride + r0 + rr] = sc * acc[rr][b];
+                for (int b = 0; b < NB; ++b) out[b * ostride + r0 + rr] = sc * (res[rr][b] * pow2f(shift[b]));
             }
         }
     }
@@ -339,52 +497,73 @@ int sms() {
     return v;
 }
 
-constexpr size_t SMEM_CAP = 200 * 1024;   // shared memory for the staged vectors + table
+constexpr size_t SMEM_CAP = 200 * 1024;   // shared memory for the staged vectors
 
-size_t rowdot_smem_bytes(int nb, int64_t tb) { return (32 + (size_t)nb * (size_t)(tb / 4) * 16) * sizeof(float); }
+size_t tdot_smem_bytes(int nb, int64_t tb) { return (size_t)nb * (size_t)(tb / 4) * SW * sizeof(float); }
 
 template <int NB, int R>
-bool launch_rowdot_smem(const uint8_t* T, int64_t rows, int64_t len, int64_t tb, const float* V, int64_t vstride,
-                        const float* scale, float* out, int64_t ostride, cudaStream_t s) {
-    const size_t smem = rowdot_smem_bytes(NB, tb);
-    if (smem > SMEM_CAP) return false;
+cudaError_t launch_tdot(const uint8_t* T, int64_t rows, int64_t len, int64_t tb, const float* V, int64_t vstride,
+                        const float* scale, float* out, int64_t ostride, bool dependent, cudaStream_t s) {
+    const size_t smem = tdot_smem_bytes(NB, tb);
     static bool attr = false;   // per process; the attribute applies to every device
     if (!attr) {
-        cudaFuncSetAttribute(rowdot_smem_kernel<NB, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_CAP);
+        cudaFuncSetAttribute(tdot_kernel<NB, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_CAP);
         attr = true;
     }
-    const int64_t want = ((rows + R - 1) / R + RS_THREADS / 32 - 1) / (RS_THREADS / 32);
-    const int64_t cap = 16 * (int64_t)sms();
-    const unsigned grid = (unsigned)(want < cap ? (want > 0 ? want : 1) : cap);
-    rowdot_smem_kernel<NB, R><<<grid, RS_THREADS, smem, s>>>(T, rows, len, tb, V, vstride, scale, out, ostride);
-    return true;
+    const int64_t nsm = sms();
+    const int64_t groups = (rows + R - 1) / R;
+    int64_t warps = (groups + nsm - 1) / nsm;
+    warps = warps < 1 ? 1 : (warps > TD_MAX_WARPS ? TD_MAX_WARPS : warps);
+    int64_t grid = (groups + warps - 1) / warps;
+    grid = grid < nsm ? grid : nsm;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)(32 * warps));
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = dependent ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, tdot_kernel<NB, R>, T, rows, len, tb, V, vstride, scale, out, ostride,
+                              dependent ? 1 : 0);
 }
 
 template <int NB>
-void launch_rowdot(const uint8_t* T, int64_t rows, int64_t len, int64_t tb, const float* V, int64_t vstride,
-                   const float* scale, float* out, int64_t ostride, cudaStream_t s) {
-    // rows per warp: share each staged vector load among R rows, but keep >= 16
-    // warps per SM busy (R = 1 for short matrices)
-    const int64_t nsm = sms();
-    bool done;
-    if (NB == 1 && rows >= 4 * 24 * nsm) done = launch_rowdot_smem<NB, NB == 1 ? 4 : 1>(T, rows, len, tb, V, vstride, scale, out, ostride, s);
-    else if (NB <= 2 && rows >= 2 * 16 * nsm) done = launch_rowdot_smem<NB, NB <= 2 ? 2 : 1>(T, rows, len, tb, V, vstride, scale, out, ostride, s);
-    else done = launch_rowdot_smem<NB, 1>(T, rows, len, tb, V, vstride, scale, out, ostride, s);
-    if (done) return;
+cudaError_t launch_rowdot(const uint8_t* T, int64_t rows, int64_t len, int64_t tb, const float* V, int64_t vstride,
+                          const float* scale, float* out, int64_t ostride, bool dependent, cudaStream_t s) {
+    if (tdot_smem_bytes(NB, tb) <= SMEM_CAP) {
+        // rows per warp: four when that still leaves >= 8 warps per SM, so each staged float4 serves several rows
+        const int64_t nsm = sms();
+        if constexpr (NB == 1) {
+            if (rows >= 4 * 8 * nsm) return launch_tdot<NB, 4>(T, rows, len, tb, V, vstride, scale, out, ostride, dependent, s);
+            return launch_tdot<NB, 2>(T, rows, len, tb, V, vstride, scale, out, ostride, dependent, s);
+        } else if constexpr (NB == 2) {
+            return launch_tdot<NB, 2>(T, rows, len, tb, V, vstride, scale, out, ostride, dependent, s);
+        } else {
+            return launch_tdot<NB, 1>(T, rows, len, tb, V, vstride, scale, out, ostride, dependent, s);
+        }
+    }
     const int64_t want = (rows + 7) / 8;
-    const int64_t cap = nsm * 8;
+    const int64_t cap = (int64_t)sms() * 8;
     const unsigned grid = (unsigned)(want < cap ? (want > 0 ? want : 1) : cap);
     rowdot_kernel<NB><<<grid, RD_THREADS, 0, s>>>(T, rows, len, tb, V, vstride, scale, out, ostride);
+    return cudaGetLastError();
 }
 
-void rowdot(int nb, const uint8_t* T, int64_t rows, int64_t len, int64_t tb, const float* V, int64_t vstride,
-            const float* scale, float* out, int64_t ostride, cudaStream_t s) {
-    switch (nb) {
-        case 1: launch_rowdot<1>(T, rows, len, tb, V, vstride, scale, out, ostride, s); break;
-        case 2: launch_rowdot<2>(T, rows, len, tb, V, vstride, scale, out, ostride, s); break;
-        case 3: launch_rowdot<3>(T, rows, len, tb, V, vstride, scale, out, ostride, s); break;
-        case 4: launch_rowdot<4>(T, rows, len, tb, V, vstride, scale, out, ostride, s); break;
-        default: launch_rowdot<MAXB>(T, rows, len, tb, V, vstride, scale, out, ostride, s); break;
+cudaError_t rowdot(int nb, const uint8_t* T, int64_t rows, int64_t len, int64_t tb, const float* V, int64_t vstride,
+                   const float* scale, float* out, int64_t ostride, bool dependent, cudaStream_t s) {
+    switch (nb) {   // one instantiation per vector count: a kernel touches exactly nb vectors
+        case 1: return launch_rowdot<1>(T, rows, len, tb, V, vstride, scale, out, ostride, dependent, s);
+        case 2: return launch_rowdot<2>(T, rows, len, tb, V, vstride, scale, out, ostride, dependent, s);
+        case 3: return launch_rowdot<3>(T, rows, len, tb, V, vstride, scale, out, ostride, dependent, s);
+        case 4: return launch_rowdot<4>(T, rows, len, tb, V, vstride, scale, out, ostride, dependent, s);
+        case 5: return launch_rowdot<5>(T, rows, len, tb, V, vstride, scale, out, ostride, dependent, s);
+        case 6: return launch_rowdot<6>(T, rows, len, tb, V, vstride, scale, out, ostride, dependent, s);
+        case 7: return launch_rowdot<7>(T, rows, len, tb, V, vstride, scale, out, ostride, dependent, s);
+        case 8: return launch_rowdot<8>(T, rows, len, tb, V, vstride, scale, out, ostride, dependent, s);
+        default: return cudaErrorInvalidValue;
     }
 }
 
@@ -413,17 +592,18 @@ int externd_matvec(const uint8_t* Bt, const float* D, const uint8_t* C, int64_t 
     if (!Bt || !D || !C || !X || !Y || !z_work || m < 1 || n < 1 || k < 1 || batch < 1) return EXTERND_EINVAL;
     if (!is_device(Bt) || !is_device(D) || !is_device(C) || !is_device(X) || !is_device(Y) || !is_device(z_work))
         return EXTERND_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(Bt) & 15) || (reinterpret_cast<uintptr_t>(C) & 15)) return EXTERND_EINVAL;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int64_t cb = (int64_t)trit_bytes(n), bb = (int64_t)trit_bytes(k);
     // vectors per pass: the most that still fit shared memory for both products
     int per = MAXB;
-    while (per > 1 && (rowdot_smem_bytes(per, cb) > SMEM_CAP || rowdot_smem_bytes(per, bb) > SMEM_CAP)) per /= 2;
+    while (per > 1 && (tdot_smem_bytes(per, cb) > SMEM_CAP || tdot_smem_bytes(per, bb) > SMEM_CAP)) --per;
     for (int64_t b0 = 0; b0 < batch; b0 += per) {
         const int nb = (int)(batch - b0 < per ? batch - b0 : per);
         // z = diag(D) (C x): k rows of n trits
-        rowdot(nb, C, k, n, cb, X + b0 * n, n, D, z_work, k, s);
-        // y = B z: m rows of k trits (B transposed)
-        rowdot(nb, Bt, m, k, bb, z_work, k, nullptr, Y + b0 * m, m, s);
+        if (rowdot(nb, C, k, n, cb, X + b0 * n, n, D, z_work, k, false, s) != cudaSuccess) { cudaGetLastError(); return EXTERND_ECUDA; }
+        // y = B z: m rows of k trits (B transposed), a programmatic dependent of the first product
+        if (rowdot(nb, Bt, m, k, bb, z_work, k, nullptr, Y + b0 * m, m, true, s) != cudaSuccess) { cudaGetLastError(); return EXTERND_ECUDA; }
     }
     if (cudaGetLastError() != cudaSuccess) return EXTERND_ECUDA;
     return EXTERND_OK;

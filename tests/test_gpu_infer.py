@@ -1,12 +1,16 @@
 """Parity of the inference path (§2.6: y = B diag(D) C x, mask+sign storage) with the oracle.
 
-Tolerance of the products (derived from the arithmetic): every row dot adds at
-most len fp32 terms, each lane of a warp summing its share sequentially and the
-32 lane sums combined by a butterfly, so the rounding error of z = D (C x) is at
-most ~(len/32 + 5) 2^-24 |D| (|C| |x|) and y = B z adds the same relative error
-on top of the error carried by z.  For len <= 16384 that is below
-3e-5 * (|B| |D| |C| |x|) elementwise, which the tests use (plus 1e-30 absolute).
-Transposes and the mask+sign storage are bit-exact.
+Tolerance of the products (derived from the arithmetic): every term t x of a row
+dot is formed exactly (the trit is decoded into an exact power-of-two multiple and
+the staged vector entry carries the inverse power of two), and the terms are summed
+in fp32: each lane keeps two running sums (even and odd trits of its words), adds
+them, and the 32 lane sums are combined by a butterfly.  The rounding error of
+z = D (C x) is therefore at most ~(len/64 + 7) 2^-24 |D| (|C| |x|), and y = B z adds
+the same relative error on top of the error carried by z.  For len <= 16384 that is
+below 3e-5 * (|B| |D| |C| |x|) elementwise, which the tests use (plus 1e-30
+absolute).  With small-integer inputs every partial sum is an exactly representable
+integer, so the result is exact.  Transposes and the mask+sign storage are
+bit-exact.
 """
 import numpy as np
 import pytest
@@ -55,7 +59,8 @@ def test_transpose_trits_is_exact(rows, length):
 
 
 @pytest.mark.parametrize("m,n,k,batch", [(1, 1, 1, 1), (7, 5, 9, 1), (33, 65, 40, 3), (130, 70, 300, 9),
-                                         (512, 384, 1024, 2)])
+                                         (512, 384, 1024, 2), (40, 90, 77, 5), (64, 33, 129, 6), (19, 200, 64, 7),
+                                         (5000, 700, 300, 1), (3000, 1000, 6000, 1)])
 def test_matvec_random_factors_match_oracle(m, n, k, batch):
     B, D, C = _random_factors(m, n, k, 0.45, seed=m + n + k)
     Bp, Dg, Cp = _device_factors(B, D, C)
@@ -131,3 +136,53 @@ def test_matvec_headline_factors_full_size():
         X = np.random.default_rng(batch).standard_normal((batch, f.n)).astype(np.float32)
         Y = ext.matvec(Bt, f.D, f.C, f.m, f.n, torch.from_numpy(X).cuda()).cpu().numpy()
         _check_matvec(Bg, Dh, Cg, X, Y)
+
+
+def test_matvec_small_integers_are_exact():
+    """Integer inputs with every partial sum below 2^24: each term t x is formed exactly and
+    each sum of integers is exact, so y equals the exact product bit for bit (a dropped or
+    sign-flipped trit anywhere would show)."""
+    m, n, k = 300, 500, 260
+    B, _, C = _random_factors(m, n, k, 0.6, seed=21)
+    D = np.ones(k, dtype=np.float32)
+    Bp, Dg, Cp = _device_factors(B, D, C)
+    Bt = ext.transpose_trits(Bp, k, m)
+    for batch in (1, 2, 3, 8):
+        X = np.random.default_rng(batch).integers(-8, 9, size=(batch, n)).astype(np.float32)
+        Y = ext.matvec(Bt, Dg, Cp, m, n, torch.from_numpy(X).cuda()).cpu().numpy()
+        want = (B.astype(np.int64) @ (C.astype(np.int64) @ X.T.astype(np.int64))).T
+        assert np.array_equal(Y.astype(np.int64), want), batch
+
+
+def test_matvec_huge_and_tiny_input_ranges():
+    """Inputs near the top of the fp32 range (|x| ~ 2^110: staged with an extra power-of-two
+    scale) and tiny ones (~2^-100), mixed in one batch, against the oracle."""
+    m, n, k = 96, 130, 200
+    B, D, C = _random_factors(m, n, k, 0.5, seed=33)
+    D = np.abs(D) * 1e-3 + 1e-4
+    D = D.astype(np.float32)
+    Bp, Dg, Cp = _device_factors(B, D, C)
+    Bt = ext.transpose_trits(Bp, k, m)
+    rng = np.random.default_rng(4)
+    X = rng.standard_normal((3, n)).astype(np.float32)
+    X[0] *= np.float32(2.0 ** 110)
+    X[2] *= np.float32(2.0 ** -100)
+    Y = ext.matvec(Bt, Dg, Cp, m, n, torch.from_numpy(X).cuda()).cpu().numpy()
+    assert np.all(np.isfinite(Y))
+    _check_matvec(B, D, C, X, Y)
+
+
+def test_matvec_rejects_unaligned_factors():
+    """The trit rows are read in 16-byte units: factor pointers off a 16-byte boundary are refused
+    before any launch."""
+    B, D, C = _random_factors(8, 64, 16, 0.5, seed=2)
+    Bp, Dg, Cp = _device_factors(B, D, C)
+    Bt = ext.transpose_trits(Bp, 16, 8)
+    buf = torch.zeros(Cp.numel() + 16, dtype=torch.uint8, device="cuda")
+    buf[4:4 + Cp.numel()] = Cp.reshape(-1)
+    X = torch.zeros((1, 64), device="cuda")
+    Y = torch.empty((1, 8), device="cuda")
+    Z = torch.empty((1, 16), device="cuda")
+    rc = ext._lib.load().externd_matvec(ext.api._ptr(Bt), ext.api._ptr(Dg), buf.data_ptr() + 4, 8, 64, 16,
+                                        ext.api._ptr(X), 1, ext.api._ptr(Y), ext.api._ptr(Z), None)
+    assert rc == ext.STATUS["EINVAL"]
