@@ -22,11 +22,16 @@
  *   Device buffers of B/C rows must be 16-byte aligned.
  * - `stream` is a cudaStream_t (NULL = legacy default stream) of the current
  *   device.  Every call is stream-ordered and SYNCHRONOUS: it returns after
- *   the work finished, because the return code carries the device status.
- * - The library keeps no pointer after return.  Workspace (the residual in
- *   two layouts, each entry an fp32 pair hi + lo; exchange buffers, start
- *   trits) is allocated stream-ordered inside the call and released before it
- *   returns.
+ *   the work finished, because the return code carries the device status --
+ *   except the factorizations given an async_status int (externd_options,
+ *   externd_batch_options), which return once their work is queued and deliver
+ *   the status through that int, and externd_matvec.
+ * - The library keeps no pointer after return (an asynchronous call's queued
+ *   work still uses the caller's buffers until the stream reaches its end).
+ *   Workspace (the residual in two layouts, each entry an fp32 pair hi + lo;
+ *   exchange buffers, start trits) is allocated stream-ordered inside the call
+ *   and released before it returns (asynchronous calls: released in stream
+ *   order).
  * - Ternary outputs are packed 2 bits per trit: 00 = 0, 01 = +1, 11 = -1
  *   (10 is never written).  Trit j of a row sits in byte j/4, bits 2*(j%4).
  *   A row of `len` trits occupies externd_trit_bytes(len) bytes (ceil(len/4)
@@ -122,9 +127,9 @@ int externd_factor_weighted(const float* A, int64_t m, int64_t n, double mu, dou
  *     the caller's device current), so the address stays right after a
  *     cudaDeviceReset.  The first call on a device may load the library's device
  *     code there: make that first call before any stream capture on the device.
- *   - Like every entry point of this library the call is synchronous: it waits
- *     for `stream` before returning, because the return code carries the device
- *     status (also when it fails after queueing work on the array).
+ *   - The call is synchronous: it waits for `stream` before returning, because
+ *     the return code carries the device status (also when it fails after
+ *     queueing work on the array).
  *   - All calls share the one array and it keeps the previous call's contents
  *     (each call clears what must start at zero).  Calls that overlap on the GPU
  *     (e.g. on two streams, or from two host threads) race and corrupt each
@@ -172,6 +177,8 @@ typedef struct {
     int grid;
     int cluster;
     int plan_only;
+    int* async_status;   /* as externd_options.async_status: one status for the whole batch
+                          * (the first matrix's failure, else EXTERND_OK) */
 } externd_batch_options;
 
 /* externd_factor_batched with per-matrix extensions (opt may be NULL: the plain call). */
@@ -339,6 +346,15 @@ typedef struct {
      * (EXTERND_ELAUNCH if they cannot all be resident, EXTERND_EINVAL for other values).
      * Results depend on the partition: the same grid and cluster size give the same bits. */
     int cluster;
+    /* Asynchronous call: non-NULL = a DEVICE int.  The call queues all its work on `stream` and
+     * returns EXTERND_OK without waiting; when the stream reaches the end of the work, the
+     * int receives the factorization's status (EXTERND_OK or a negative EXTERND_* code, e.g.
+     * EXTERND_ETIMEOUT).  A, the outputs and every optional buffer must be device memory
+     * (EXTERND_EINVAL otherwise: host buffers would need a synchronous copy).  The workspace
+     * is released in stream order.  A non-OK return means nothing was left queued (the call
+     * waited for what it had queued).  externd_last_stats records the plan only (timings,
+     * byte counts and safeguard counts are 0). */
+    int* async_status;
 } externd_options;
 
 /* externd_factor with options (opt may be NULL). */

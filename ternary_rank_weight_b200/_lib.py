@@ -55,6 +55,7 @@ class Options(ctypes.Structure):
         ("trace_thr_u", ctypes.c_void_p),
         ("trace_trit_u", ctypes.c_void_p),
         ("cluster", ctypes.c_int),
+        ("async_status", ctypes.c_void_p),
     ]
 
 
@@ -67,6 +68,7 @@ class BatchOptions(ctypes.Structure):
         ("grid", ctypes.c_int),
         ("cluster", ctypes.c_int),
         ("plan_only", ctypes.c_int),
+        ("async_status", ctypes.c_void_p),
     ]
 
 

@@ -155,7 +155,7 @@ class Trace:
 def factor(A, mu: float, tau: float, iters: int = 15, seed: int = 0, *, grid: int = 0, pending: int = 0,
            wait_limit_s: float = 0.0, fault_skip_cta: Optional[int] = None, want_d64: bool = False,
            want_energy: bool = True, sweeps: int = 0, h=None, lam: float = 0.0, trace=None, cluster: int = 0,
-           stream=None) -> Factors:
+           async_status=None, stream=None) -> Factors:
     """Factor one matrix (externd_factor_ex).  Outputs are allocated where A lives.
 
     sweeps: §2.4 refinement sweeps after extraction (``energy`` keeps the extraction
@@ -164,7 +164,10 @@ def factor(A, mu: float, tau: float, iters: int = 15, seed: int = 0, *, grid: in
     trace: (first, count) -- test hook, records the half-steps of those visits: visit
     i < k extracts component i, visit (s + 1) k + i is sweep s's refit of component i
     (``Factors.trace``; A must be on the GPU).  cluster: kernel choice (0 automatic, 1 one
-    CTA per residual stripe, 2/4/8/16 the clustered kernel with that cluster size)."""
+    CTA per residual stripe, 2/4/8/16 the clustered kernel with that cluster size).
+    async_status: a one-element int32 CUDA tensor: the call queues its work and returns at
+    once; the tensor receives the status (0 or a negative code) when the stream gets there
+    (A and every output on the GPU; ``stats`` then holds the launch plan only)."""
     A = _as_matrix(A)
     m, n = A.shape
     if h is not None:
@@ -190,6 +193,11 @@ def factor(A, mu: float, tau: float, iters: int = 15, seed: int = 0, *, grid: in
     opt.h = _ptr(h)
     opt.lambda_ = float(lam)
     opt.cluster = int(cluster)
+    if async_status is not None:
+        if not (isinstance(async_status, torch.Tensor) and async_status.is_cuda and async_status.dtype == torch.int32
+                and async_status.numel() >= 1 and A.is_cuda):
+            raise ValueError("async_status must be an int32 CUDA tensor and A must be on the GPU")
+        opt.async_status = _ptr(async_status)
     tr = None
     if trace is not None:
         if not A.is_cuda:
@@ -300,12 +308,14 @@ def factor_block(A: torch.Tensor, mu: float, tau: float, iters: int = 15, seed: 
 def factor_batched(As: Sequence, mus: Sequence[float], taus: Sequence[float], iters: int = 15,
                    seeds: Optional[Sequence[int]] = None, *, hs: Optional[Sequence] = None,
                    lams: Optional[Sequence[float]] = None, sweeps: int = 0, grid: int = 0, cluster: int = 0,
-                   plan_only: bool = False, stream=None):
+                   plan_only: bool = False, async_status=None, stream=None):
     """Factor independent matrices in one launch (externd_factor_batched_ex).
 
     hs: per-matrix importance weights (§2.5; every matrix or none), lams their lambdas;
     sweeps: refinement sweeps (§2.4) for every matrix; grid, cluster: the launch (0:
     automatic).  plan_only: return (None, stats of the plan) without device work.
+    async_status: a one-element int32 CUDA tensor: queue the work and return at once; the
+    tensor receives the batch's status when the stream gets there (every matrix on the GPU).
     Returns (list of Factors, list of per-matrix status codes)."""
     mats = [_as_matrix(a) for a in As]
     cnt = len(mats)
@@ -347,6 +357,11 @@ def factor_batched(As: Sequence, mus: Sequence[float], taus: Sequence[float], it
     opt.grid = int(grid)
     opt.cluster = int(cluster)
     opt.plan_only = 1 if plan_only else 0
+    if async_status is not None:
+        if not (isinstance(async_status, torch.Tensor) and async_status.is_cuda and async_status.dtype == torch.int32
+                and async_status.numel() >= 1 and all(a.is_cuda for a in mats)):
+            raise ValueError("async_status must be an int32 CUDA tensor and every matrix must be on the GPU")
+        opt.async_status = _ptr(async_status)
     if sweeps > 0:
         sarr = P(*[_ptr(x) for x in SEs])
         keep.append(sarr)

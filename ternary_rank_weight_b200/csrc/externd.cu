@@ -1793,7 +1793,20 @@ struct RunOpts {
     bool init_only = false;
     bool plan_only = false;   // fill the stats with the launch plan and return (no device work)
     int cluster = 0;          // 0: automatic; 1: the one-CTA-per-stripe kernel; 2, 4, 8, 16: clusters of that size
+    int* async_status = nullptr;   // device int: queue everything, write the status there, do not wait
 };
+
+// Status of an asynchronous call: the first matrix's failure (a group that stopped before a
+// matrix finished counts as a timeout), else EXTERND_OK.
+__global__ void async_status_kernel(const int* __restrict__ status, int np, int* out) {
+    if (threadIdx.x != 0) return;
+    int r = EXTERND_OK;
+    for (int b = 0; b < np && r == EXTERND_OK; ++b) {
+        const int s = status[b];
+        r = (s == ST_RUNNING) ? EXTERND_ETIMEOUT : s;
+    }
+    *out = r;
+}
 
 // Plan of the clustered kernel for one launch (see als_cluster.cuh).
 struct Plan2 {
@@ -2128,13 +2141,18 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
         }
     }
 
-    if (fixed) {
+    const bool async = opt.async_status != nullptr;
+    if (fixed || async) {
         for (int b = 0; b < np; ++b)
             if (off_A[b] != SIZE_MAX || off_B[b] != SIZE_MAX || off_C[b] != SIZE_MAX || off_D[b] != SIZE_MAX ||
                 off_E[b] != SIZE_MAX || off_d64[b] != SIZE_MAX || off_pre[b] != SIZE_MAX || off_thr[b] != SIZE_MAX ||
-                off_tro[b] != SIZE_MAX || off_SE[b] != SIZE_MAX)
-                return EXTERND_EINVAL;   // host buffers would need staging memory
-        if (ws > fixed->cap) return EXTERND_ELIMIT;
+                off_tro[b] != SIZE_MAX || off_SE[b] != SIZE_MAX || off_h[b] != SIZE_MAX)
+                return EXTERND_EINVAL;   // host buffers would need staging memory (and a synchronous copy)
+        if (fixed && ws > fixed->cap) return EXTERND_ELIMIT;
+        if (async && (fixed || opt.init_only || !is_device_ptr(opt.async_status))) return EXTERND_EINVAL;
+        if (async)
+            for (int b = 0; b < np; ++b)
+                if (in[b].mode != MODE_FACTOR) return EXTERND_EINVAL;
     }
     unsigned char* dws = nullptr;
     cudaEvent_t ev[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
@@ -2147,7 +2165,8 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
     if (fixed) {
         dws = fixed->base;
     } else {
-        for (int i = 0; i < 5; ++i) CK(cudaEventCreate(&ev[i]));
+        if (!async)
+            for (int i = 0; i < 5; ++i) CK(cudaEventCreate(&ev[i]));
         CK(cudaMallocAsync((void**)&dws, ws, stream));
     }
     if (ev[0]) CK(cudaEventRecord(ev[0], stream));
@@ -2325,6 +2344,26 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
             if (off_tro[b] != SIZE_MAX) CK(cudaMemcpyAsync(I.trit_out, P.trit_out, trit_bytes(lout), cudaMemcpyDeviceToHost, stream));
         }
     }
+    if (async) {
+        // the batch's status into the caller's int when the stream gets here; the workspace is
+        // released in stream order below and the call returns without waiting
+        async_status_kernel<<<1, 32, 0, stream>>>(reinterpret_cast<const int*>(dws + off_status), np, opt.async_status);
+        CK(cudaGetLastError());
+        ++launches;
+        st.launches = launches;
+        st.grid = NG * Gg;
+        st.group = Gg;
+        st.block = NT;
+        st.vec_v = probs[0].pv.vec;
+        st.vec_u = probs[0].pu.vec;
+        st.pending = Lcap;
+        st.cluster = clustered ? pl.c : 1;
+        st.smem_bytes = smem;
+        st.workspace_bytes = ws;
+        for (int b = 0; b < np; ++b) statuses[b] = EXTERND_OK;
+        rc = EXTERND_OK;
+        goto done;
+    }
     CK(cudaMemcpyAsync(hstatus.data(), dws + off_status, sizeof(int) * np, cudaMemcpyDeviceToHost, stream));
     CK(cudaMemcpyAsync(hstats.data(), dws + off_stats, sizeof(DevStats) * np, cudaMemcpyDeviceToHost, stream));
     if (ev[4]) CK(cudaEventRecord(ev[4], stream));
@@ -2377,7 +2416,12 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
         if (statuses[b] != ST_OK) { rc = statuses[b]; break; }
 
 done:
-    if (dws && !fixed) { cudaFreeAsync(dws, stream); cudaStreamSynchronize(stream); }
+    // an asynchronous call that queued everything frees its workspace in stream order and returns;
+    // every other exit waits for the work it queued
+    if (dws && !fixed) {
+        cudaFreeAsync(dws, stream);
+        if (!(async && rc == EXTERND_OK)) cudaStreamSynchronize(stream);
+    }
     // fixed scratch: work already queued on the shared array must end before the
     // call returns, also when a later queueing step failed
     if (fixed && rc != EXTERND_OK) cudaStreamSynchronize(stream);
@@ -2519,12 +2563,14 @@ int run_block(const float* A, int64_t m, int64_t n, int64_t k, double tau, int i
             block_start_kernel<<<nb, 256, 0, stream>>>(seed, s0, m, tau, U, nb);
             ++launches;
             for (int it = 0; it < iters; ++it) {
-                // V <- T_tau([(U^T U + eps I)^-1 U^T R]^T): the rows of P^T = R^T U solved in place
+                // V <- T_tau([(U^T U + eps I)^-1 U^T R]^T) = T_tau(R^T [U (U^T U + eps I)^-1]): the m rows
+                // of U are solved (fewer right-hand sides than the n rows of R^T U), then one GEMM
                 gemm(nb, nb, (int)m, U, nb, true, U, nb, false, Gu, nb, 1.0, 0.0);
                 ridge_kernel<<<1, 1024, 0, stream>>>(Gu, nb, BLOCK_EPS_REL, Lm);
                 factor(nb, Lm, info + slot++);
-                gemm((int)n, nb, (int)m, R, (int)n, true, U, nb, false, PT, nb, 1.0, 0.0);
-                solve(nb, Lm, PT, (int)n, info + ninfo);
+                CK(cudaMemcpyAsync(S, U, f8 * (size_t)(m * nb), cudaMemcpyDeviceToDevice, stream));
+                solve(nb, Lm, S, (int)m, info + ninfo);
+                gemm((int)n, nb, (int)m, R, (int)n, true, S, nb, false, PT, nb, 1.0, 0.0);
                 ternarize_cols_kernel<<<nb, 256, 0, stream>>>(PT, n, nb, false, tau, V, nb);
                 // U <- T_tau(R V (V^T V + eps I)^-1): the rows of Q = R V solved in place
                 gemm(nb, nb, (int)n, V, nb, true, V, nb, false, Gv, nb, 1.0, 0.0);
@@ -2643,6 +2689,7 @@ int externd_factor_ex(const float* A, int64_t m, int64_t n, double mu, double ta
         if (opt->cluster < 0 || opt->cluster > 16 || (opt->cluster > 1 && (opt->cluster & (opt->cluster - 1))))
             return EXTERND_EINVAL;
         ro.cluster = opt->cluster;
+        ro.async_status = opt->async_status;
         I.d64 = opt->d64_out;
         if (opt->sweeps < 0 || opt->sweeps > 1000) return EXTERND_EINVAL;
         I.sweeps = opt->sweeps;
@@ -2788,6 +2835,7 @@ int externd_factor_batched_ex(int count, const float* const* A, const int64_t* m
         ro.grid = opt->grid;
         ro.cluster = opt->cluster;
         ro.plan_only = opt->plan_only != 0;
+        ro.async_status = opt->async_status;
     }
     return run(ins.data(), count, ro, reinterpret_cast<cudaStream_t>(stream), status_out);
 }
