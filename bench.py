@@ -542,6 +542,22 @@ def run_block(args):
            "gpu_launches": f.stats["launches"],
            "clocks": clk.summary(),
            "energy": float(f.energy[-1].item())}
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        # the oracle's block_als on the first blocks of the same matrix (per-block cost is constant)
+        from oracle import externd_oracle as ora
+        t0 = time.perf_counter()
+        nblk = 0
+        while True:
+            nblk += 1
+            ora.block_als(mats[0], k=min(k, nblk * b), tau=tau, iters=w.iters, seed=seed)
+            dt = time.perf_counter() - t0
+            if dt > args.ref_budget / 2 or nblk * b >= k:
+                break
+            t0 = time.perf_counter()
+        out["cpu_baseline"] = {"value": min(k, nblk * b) / dt, "unit": "components/s", "cores": _oracle_threads(),
+                               "kind": "oracle",
+                               "sample": f"first {min(k, nblk * b)} of {k} components ({nblk} block(s) of {b}) of "
+                                         f"the {m}x{n} matrix, {dt:.1f} s, numpy fp64"}
     if rank == 0:
         print(json.dumps(out), flush=True)
     return 0

@@ -534,7 +534,8 @@ template <int NB>
 cudaError_t launch_rowdot(const uint8_t* T, int64_t rows, int64_t len, int64_t tb, const float* V, int64_t vstride,
                           const float* scale, float* out, int64_t ostride, bool dependent, cudaStream_t s) {
     if (tdot_smem_bytes(NB, tb) <= SMEM_CAP) {
-        // rows per warp: four when that still leaves >= 8 warps per SM, so each staged float4 serves several rows
+        // rows per warp: four when that still leaves >= 8 warps per SM, else two, so each staged float4
+        // serves several rows (one row per warp makes the staged-vector reads the limit for batches)
         const int64_t nsm = sms();
         if constexpr (NB == 1) {
             if (rows >= 4 * 8 * nsm) return launch_tdot<NB, 4>(T, rows, len, tb, V, vstride, scale, out, ostride, dependent, s);
@@ -542,7 +543,7 @@ cudaError_t launch_rowdot(const uint8_t* T, int64_t rows, int64_t len, int64_t t
         } else if constexpr (NB == 2) {
             return launch_tdot<NB, 2>(T, rows, len, tb, V, vstride, scale, out, ostride, dependent, s);
         } else {
-            return launch_tdot<NB, 1>(T, rows, len, tb, V, vstride, scale, out, ostride, dependent, s);
+            return launch_tdot<NB, 2>(T, rows, len, tb, V, vstride, scale, out, ostride, dependent, s);
         }
     }
     const int64_t want = (rows + 7) / 8;
