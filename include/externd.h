@@ -236,6 +236,8 @@ int externd_transpose_trits(const uint8_t* T, int64_t rows, int64_t len, uint8_t
  *   X       [in]  batch x n fp32, row-major (one input vector per row).
  *   Y       [out] batch x m fp32, row-major.
  *   z_work  [tmp] k x min(batch, 8) fp32 scratch owned by the caller (C x per vector).
+ * Bt and C must be 16-byte aligned (EXTERND_EINVAL otherwise); the padding trits of their rows
+ * (past k and n) are ignored.
  * fp32 arithmetic; stream-ordered and asynchronous (no allocation, no host sync). */
 int externd_matvec(const uint8_t* Bt, const float* D, const uint8_t* C, int64_t m, int64_t n, int64_t k,
                    const float* X, int64_t batch, float* Y, float* z_work, void* stream);

@@ -59,11 +59,11 @@ __global__ void __launch_bounds__(1024) sum_partials_kernel(const double* partia
     }
 }
 
-// T_tau of one column of a matrix (CTA j: column j of an len x ld matrix X, or row j when
-// by_rows), written as +-1 / 0 into column j of O (len x ldo, fp64).  §2.2 with the all-zero
-// fallback (lowest index among the largest magnitudes).
+// T_tau of one column of a matrix (CTA j: column j of an len x ld row-major matrix X), written
+// as +-1 / 0 into column j of O (len x ldo, fp64).  §2.2 with the all-zero fallback (lowest
+// index among the largest magnitudes).
 __global__ void __launch_bounds__(256) ternarize_cols_kernel(const double* __restrict__ X, int64_t len, int ld,
-                                                            bool by_rows, double tau, double* __restrict__ O, int ldo) {
+                                                            double tau, double* __restrict__ O, int ldo) {
     __shared__ double shs[9], shm[9];
     __shared__ long long shj[9];
     const int j = blockIdx.x;
@@ -71,7 +71,7 @@ __global__ void __launch_bounds__(256) ternarize_cols_kernel(const double* __res
     double s = 0.0, mx = -1.0;
     long long jx = LLONG_MAX;
     for (int64_t i = threadIdx.x; i < len; i += 256) {
-        const double v = by_rows ? X[(int64_t)j * ld + i] : X[i * ld + j];
+        const double v = X[i * ld + j];
         const double a = fabs(v);
         s += a;
         if (a > mx) { mx = a; jx = i; }
@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(256) ternarize_cols_kernel(const double* __res
     const double thr = tau * shs[8] / (double)len;
     int any = 0;
     for (int64_t i = threadIdx.x; i < len; i += 256) {
-        const double v = by_rows ? X[(int64_t)j * ld + i] : X[i * ld + j];
+        const double v = X[i * ld + j];
         const double t = fabs(v) > thr ? (v < 0.0 ? -1.0 : 1.0) : 0.0;
         any |= (t != 0.0);
         O[i * ldo + j] = t;
@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(256) ternarize_cols_kernel(const double* __res
     any = __syncthreads_or(any);
     if (!any && threadIdx.x == 0) {
         const long long J = (shj[8] >= 0 && shj[8] < len) ? shj[8] : 0;
-        const double v = by_rows ? X[(int64_t)j * ld + J] : X[J * ld + j];
+        const double v = X[J * ld + j];
         O[J * ldo + j] = v < 0.0 ? -1.0 : 1.0;
     }
 }

@@ -2571,7 +2571,7 @@ int run_block(const float* A, int64_t m, int64_t n, int64_t k, double tau, int i
                 CK(cudaMemcpyAsync(S, U, f8 * (size_t)(m * nb), cudaMemcpyDeviceToDevice, stream));
                 solve(nb, Lm, S, (int)m, info + ninfo);
                 gemm((int)n, nb, (int)m, R, (int)n, true, S, nb, false, PT, nb, 1.0, 0.0);
-                ternarize_cols_kernel<<<nb, 256, 0, stream>>>(PT, n, nb, false, tau, V, nb);
+                ternarize_cols_kernel<<<nb, 256, 0, stream>>>(PT, n, nb, tau, V, nb);
                 // U <- T_tau(R V (V^T V + eps I)^-1): the rows of Q = R V solved in place
                 gemm(nb, nb, (int)n, V, nb, true, V, nb, false, Gv, nb, 1.0, 0.0);
                 ridge_kernel<<<1, 1024, 0, stream>>>(Gv, nb, BLOCK_EPS_REL, Lm);
@@ -2579,7 +2579,7 @@ int run_block(const float* A, int64_t m, int64_t n, int64_t k, double tau, int i
                 gemm((int)m, nb, (int)n, R, (int)n, false, V, nb, false, Q, nb, 1.0, 0.0);
                 if (it == iters - 1) CK(cudaMemcpyAsync(S, Q, f8 * (size_t)(m * nb), cudaMemcpyDeviceToDevice, stream));
                 solve(nb, Lm, Q, (int)m, info + ninfo);
-                ternarize_cols_kernel<<<nb, 256, 0, stream>>>(Q, m, nb, false, tau, U, nb);
+                ternarize_cols_kernel<<<nb, 256, 0, stream>>>(Q, m, nb, tau, U, nb);
                 launches += 4;
                 CK(cudaGetLastError());
             }

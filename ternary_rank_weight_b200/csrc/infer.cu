@@ -58,13 +58,14 @@ __global__ void __launch_bounds__(RD_THREADS) rowdot_kernel(const uint8_t* __res
             const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
             #pragma unroll
             for (int h = 0; h < 4; ++h) {
-                // positions j0 .. j0+15; padding trits beyond len are zero codes
+                // positions j0 .. j0+15; padding trits past len are skipped
                 const int64_t j0 = c * 64 + 16 * h;
                 uint32_t nz = even_bits(w4[h]);
                 const uint32_t ng = even_bits(w4[h] >> 1);
                 while (nz) {
                     const int t = __ffs(nz) - 1;
                     nz &= nz - 1u;
+                    if (j0 + t >= len) break;                 // padding trits past len are not read
                     const bool neg = (ng >> t) & 1u;
                     #pragma unroll
                     for (int b = 0; b < NB; ++b) {

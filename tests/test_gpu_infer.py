@@ -60,8 +60,11 @@ def test_transpose_trits_is_exact(rows, length):
 
 @pytest.mark.parametrize("m,n,k,batch", [(1, 1, 1, 1), (7, 5, 9, 1), (33, 65, 40, 3), (130, 70, 300, 9),
                                          (512, 384, 1024, 2), (40, 90, 77, 5), (64, 33, 129, 6), (19, 200, 64, 7),
-                                         (5000, 700, 300, 1), (3000, 1000, 6000, 1)])
+                                         (5000, 700, 300, 1), (3000, 1000, 6000, 1),
+                                         (16, 60000, 40, 2), (8, 16, 50000, 1)])
 def test_matvec_random_factors_match_oracle(m, n, k, batch):
+    """Random factors; the last two shapes have rows too long for the staged-vector kernel (n = 60000,
+    k = 50000 trits), so one of their two products runs the L1 kernel."""
     B, D, C = _random_factors(m, n, k, 0.45, seed=m + n + k)
     Bp, Dg, Cp = _device_factors(B, D, C)
     Bt = ext.transpose_trits(Bp, k, m)
