@@ -803,9 +803,17 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
         double S2 = lane < NWARP ? s.wS[lane] : 0.0;
         #pragma unroll
         for (int o = 16; o; o >>= 1) S2 += __shfl_xor_sync(FULL, S2, o);
-        if (lane == 0 && !skip) {
-            st_relaxed_u64(partials + q, tag_value(S2, tag));
-            red_relaxed_add(&gs->ctr[q % NCTR][0], 1u);
+        if (lane == 0) {
+            if (Gg > 1) {
+                if (!skip) {
+                    st_relaxed_u64(partials + q, tag_value(S2, tag));
+                    red_relaxed_add(&gs->ctr[q % NCTR][0], 1u);
+                }
+            } else {
+                // a group of one CTA: its own partial, rounded as a published word would be, is
+                // the total; there is nothing to wait for
+                s.gS[0] = untag(tag_value(S2, tag));
+            }
         }
     }
     ++arrivals;
@@ -813,7 +821,7 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
     // ---- wait for all arrivals (NCTR threads poll one counter each, bounded), then
     //      everyone's partials
     int ok = 1;
-    if ((int)threadIdx.x < NCTR && (int)threadIdx.x < Gg) {
+    if (Gg > 1 && (int)threadIdx.x < NCTR && (int)threadIdx.x < Gg) {
         const int c = threadIdx.x;
         const unsigned want = arrivals * (unsigned)((Gg - c + NCTR - 1) / NCTR);
         const unsigned* ctr = &gs->ctr[c][0];
@@ -848,14 +856,14 @@ __device__ int exchange_threshold(unsigned long long* partials, int q, int Gg, u
         const int64_t idx = ((int64_t)w << 5) + lane;
         wb[i] = (w < w1 && idx < len) ? ld_relaxed_u64(gvec + idx) : (unsigned long long)tag;
     }
-    if (warp * 32 < Gg) {   // the warps that hold partials
+    if (Gg > 1 && warp * 32 < Gg) {   // the warps that hold partials
         double Sq = 0.0;
         if ((int)threadIdx.x < Gg) Sq = untag(wait_tagged(partials + threadIdx.x, tag, gs, limit_ns, status, ok));
         #pragma unroll
         for (int o = 16; o; o >>= 1) Sq += __shfl_xor_sync(FULL, Sq, o);
         if (lane == 0) s.gS[warp] = Sq;
     }
-    ok = __syncthreads_and(ok);
+    if (Gg > 1) ok = __syncthreads_and(ok);   // (one CTA: gS[0] was written before the barrier above)
     phase_mark(s, 4);
     if (!ok) { ok_out = false; return 0; }
     double St = 0.0;   // the same fixed order in every thread
