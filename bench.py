@@ -140,6 +140,24 @@ def _dist():
     return r.world, r.rank, r.local
 
 
+def _init_nccl(ws: int, local: int):
+    """One process per GPU: bind the device and, for N > 1, join the NCCL group (barriers, max and
+    sums over ranks).  Returns the device."""
+    import torch
+    torch.cuda.set_device(local)
+    if ws > 1:
+        from datetime import timedelta
+        torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=120))
+    return torch.device("cuda", local)
+
+
+def _fini_nccl(ws: int):
+    import torch
+    if ws > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
 def _workload_arrays(name: str, rank: int, mu=None):
     """This rank's workload (weak scaling: same shapes and recipe, seeds offset by rank) and matrices."""
     import dataclasses
@@ -401,8 +419,7 @@ def run_matvec(args):
     from ternary_rank_weight_b200 import dist
 
     ws, rank, local = _dist()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
+    dev = _init_nccl(ws, local)
     w, mats = _workload_arrays(args.workload, rank, args.mu)
     f = ext.factor(torch.from_numpy(mats[0]).to(dev), w.mu[0], w.tau[0], iters=w.iters, seed=w.seeds[0])
     Bt = ext.inference_layout(f)
@@ -460,6 +477,7 @@ def run_matvec(args):
                                "sample": f"{reps} calls of numpy fp64 B (D (C X)) on dense int8 trits, batch {batch}"}
     if rank == 0:
         print(json.dumps(out), flush=True)
+    _fini_nccl(ws)
     return 0
 
 
@@ -489,8 +507,7 @@ def run_block(args):
     from ternary_rank_weight_b200 import dist
 
     ws, rank, local = _dist()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
+    dev = _init_nccl(ws, local)
     w, mats = _workload_arrays(args.workload, rank, args.mu)
     A = torch.from_numpy(mats[0]).to(dev)
     Ah = torch.from_numpy(mats[0]).pin_memory()
@@ -569,6 +586,7 @@ def run_block(args):
                                          f"the {m}x{n} matrix, {dt:.1f} s, numpy fp64"}
     if rank == 0:
         print(json.dumps(out), flush=True)
+    _fini_nccl(ws)
     return 0
 
 
