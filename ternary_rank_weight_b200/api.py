@@ -166,8 +166,12 @@ def factor(A, mu: float, tau: float, iters: int = 15, seed: int = 0, *, grid: in
     (``Factors.trace``; A must be on the GPU).  cluster: kernel choice (0 automatic, 1 one
     CTA per residual stripe, 2/4/8/16 the clustered kernel with that cluster size).
     async_status: a one-element int32 CUDA tensor: the call queues its work and returns at
-    once; the tensor receives the status (0 or a negative code) when the stream gets there
-    (A and every output on the GPU; ``stats`` then holds the launch plan only)."""
+    once; the tensor receives the status (0 or a negative code) when the stream gets there.
+    A (and h) must then be contiguous float32 CUDA tensors, which the queued work reads until
+    the stream reaches its end: keep them alive and unchanged until then (the outputs are the
+    returned tensors).  ``stats`` then holds the launch plan only."""
+    if async_status is not None:
+        _check_async_inputs([A], h, async_status)
     A = _as_matrix(A)
     m, n = A.shape
     if h is not None:
@@ -194,9 +198,6 @@ def factor(A, mu: float, tau: float, iters: int = 15, seed: int = 0, *, grid: in
     opt.lambda_ = float(lam)
     opt.cluster = int(cluster)
     if async_status is not None:
-        if not (isinstance(async_status, torch.Tensor) and async_status.is_cuda and async_status.dtype == torch.int32
-                and async_status.numel() >= 1 and A.is_cuda):
-            raise ValueError("async_status must be an int32 CUDA tensor and A must be on the GPU")
         opt.async_status = _ptr(async_status)
     tr = None
     if trace is not None:
@@ -213,6 +214,19 @@ def factor(A, mu: float, tau: float, iters: int = 15, seed: int = 0, *, grid: in
     _check(rc, "externd_factor")
     return Factors(B=B, D=D, C=C, energy=E, m=m, n=n, k=k, mu=float(mu), tau=float(tau), d64=d64,
                    stats=last_stats(), sweep_energy=SE, trace=tr)
+
+
+def _check_async_inputs(As, h, async_status, hs=None):
+    """An asynchronous call reads its inputs after it returns: they must be the caller's own
+    tensors (contiguous float32 on the GPU, so no temporary copy is made) and the status an
+    int32 CUDA tensor."""
+    if not (isinstance(async_status, torch.Tensor) and async_status.is_cuda and async_status.dtype == torch.int32
+            and async_status.numel() >= 1):
+        raise ValueError("async_status must be an int32 CUDA tensor")
+    ins = list(As) + ([h] if h is not None else []) + (list(hs) if hs is not None else [])
+    for t in ins:
+        if not (isinstance(t, torch.Tensor) and t.is_cuda and t.dtype == torch.float32 and t.is_contiguous()):
+            raise ValueError("an asynchronous call needs contiguous float32 CUDA tensors as inputs")
 
 
 def _weights(h, n: int) -> torch.Tensor:
@@ -315,8 +329,11 @@ def factor_batched(As: Sequence, mus: Sequence[float], taus: Sequence[float], it
     sweeps: refinement sweeps (§2.4) for every matrix; grid, cluster: the launch (0:
     automatic).  plan_only: return (None, stats of the plan) without device work.
     async_status: a one-element int32 CUDA tensor: queue the work and return at once; the
-    tensor receives the batch's status when the stream gets there (every matrix on the GPU).
+    tensor receives the batch's status when the stream gets there.  Every matrix (and weight
+    vector) must then be a contiguous float32 CUDA tensor, kept alive and unchanged until then.
     Returns (list of Factors, list of per-matrix status codes)."""
+    if async_status is not None:
+        _check_async_inputs(As, None, async_status, hs)
     mats = [_as_matrix(a) for a in As]
     cnt = len(mats)
     if seeds is None:
@@ -358,9 +375,6 @@ def factor_batched(As: Sequence, mus: Sequence[float], taus: Sequence[float], it
     opt.cluster = int(cluster)
     opt.plan_only = 1 if plan_only else 0
     if async_status is not None:
-        if not (isinstance(async_status, torch.Tensor) and async_status.is_cuda and async_status.dtype == torch.int32
-                and async_status.numel() >= 1 and all(a.is_cuda for a in mats)):
-            raise ValueError("async_status must be an int32 CUDA tensor and every matrix must be on the GPU")
         opt.async_status = _ptr(async_status)
     if sweeps > 0:
         sarr = P(*[_ptr(x) for x in SEs])
