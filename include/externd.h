@@ -204,8 +204,7 @@ int externd_factor_batched_ex(int count, const float* const* A, const int64_t* m
  * element indices.  Synchronous; allocates about 8 m n + 8 b (3 m + 2 n) bytes of stream-ordered
  * workspace.  The plain fp64 GEMMs and the b x b Cholesky factorizations and solves run in
  * cuBLAS / cuSOLVER (the V-step's solve is applied to U's m rows, R^T [U (U^T U + eps I)^-1],
- * which equals the pages' form); calls of this function are serialised within a process (the
- * library's handles are shared). */
+ * which equals the pages' form), through handles the call creates and destroys itself. */
 int externd_factor_block(const float* A, int64_t m, int64_t n, double mu, double tau, int iters,
                          uint64_t seed, int b, uint8_t* B_out, float* D_out, uint8_t* C_out,
                          double* energy_out, double* d64_out, void* stream);

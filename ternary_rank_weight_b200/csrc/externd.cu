@@ -2476,21 +2476,23 @@ namespace {
 // §2.4 batched block ALS on the device: blocks of b components, each a sequence of launches on
 // `stream` (kernels in block_als.cuh; the plain GEMMs, Cholesky factorizations and solves in
 // cuBLAS / cuSOLVER).  A and the outputs are device pointers.
+// The vendor-library handles of one call: created on the current device at the start and
+// destroyed at the end (a few milliseconds against a factorization of hundreds), so no handle
+// outlives its context and concurrent calls share nothing.
 struct Linalg {
     cublasHandle_t blas = nullptr;
     cusolverDnHandle_t sol = nullptr;
+    bool open(cudaStream_t stream) {
+        if (cublasCreate(&blas) != CUBLAS_STATUS_SUCCESS) { blas = nullptr; return false; }
+        if (cusolverDnCreate(&sol) != CUSOLVER_STATUS_SUCCESS) { sol = nullptr; return false; }
+        return cublasSetStream(blas, stream) == CUBLAS_STATUS_SUCCESS &&
+               cusolverDnSetStream(sol, stream) == CUSOLVER_STATUS_SUCCESS;
+    }
+    ~Linalg() {
+        if (sol) cusolverDnDestroy(sol);
+        if (blas) cublasDestroy(blas);
+    }
 };
-std::mutex g_linalg_mu;          // one block factorization at a time per process (the handles' stream)
-Linalg g_linalg[64];
-
-bool linalg_for(int dev, Linalg*& out) {
-    if (dev < 0 || dev >= 64) return false;
-    Linalg& h = g_linalg[dev];
-    if (!h.blas && cublasCreate(&h.blas) != CUBLAS_STATUS_SUCCESS) { h.blas = nullptr; return false; }
-    if (!h.sol && cusolverDnCreate(&h.sol) != CUSOLVER_STATUS_SUCCESS) { h.sol = nullptr; return false; }
-    out = &h;
-    return true;
-}
 
 int run_block(const float* A, int64_t m, int64_t n, int64_t k, double tau, int iters, uint64_t seed, int b,
               uint8_t* B, float* D, uint8_t* C, double* E, double* d64, cudaStream_t stream, externd_stats& st) {
@@ -2500,13 +2502,9 @@ int run_block(const float* A, int64_t m, int64_t n, int64_t k, double tau, int i
     const int ninfo = (int)(nblocks * (2 * (int64_t)iters + 1));   // one word per factorization
     const size_t f8 = sizeof(double);
     const int nparts = 296;
-    std::lock_guard<std::mutex> lock(g_linalg_mu);
-    int dev = 0;
-    Linalg* la = nullptr;
-    if (cudaGetDevice(&dev) != cudaSuccess || !linalg_for(dev, la)) { cudaGetLastError(); return EXTERND_ECUDA; }
-    if (cublasSetStream(la->blas, stream) != CUBLAS_STATUS_SUCCESS ||
-        cusolverDnSetStream(la->sol, stream) != CUSOLVER_STATUS_SUCCESS)
-        return EXTERND_ECUDA;
+    Linalg lh;
+    Linalg* la = &lh;
+    if (!lh.open(stream)) { cudaGetLastError(); return EXTERND_ECUDA; }
     int lwork = 0;
     if (cusolverDnDpotrf_bufferSize(la->sol, CUBLAS_FILL_MODE_LOWER, (int)bb, nullptr, (int)bb, &lwork) !=
         CUSOLVER_STATUS_SUCCESS)

@@ -506,10 +506,14 @@ template <int NB, int R>
 cudaError_t launch_tdot(const uint8_t* T, int64_t rows, int64_t len, int64_t tb, const float* V, int64_t vstride,
                         const float* scale, float* out, int64_t ostride, bool dependent, cudaStream_t s) {
     const size_t smem = tdot_smem_bytes(NB, tb);
-    static bool attr = false;   // per process; the attribute applies to every device
-    if (!attr) {
-        cudaFuncSetAttribute(tdot_kernel<NB, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_CAP);
-        attr = true;
+    static bool attr[64] = {};   // set once per device of the process
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaGetLastError();
+    if (dev < 0 || dev >= 64 || !attr[dev]) {
+        const cudaError_t e = cudaFuncSetAttribute(tdot_kernel<NB, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)SMEM_CAP);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr[dev] = true;
     }
     const int64_t nsm = sms();
     const int64_t groups = (rows + R - 1) / R;
