@@ -11,7 +11,7 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SOURCES = [os.path.join(HERE, "csrc", "externd.cu"), os.path.join(HERE, "csrc", "infer.cu")]
+SOURCES = [os.path.join(HERE, "csrc", name) for name in ("externd.cu", "externd_nt1024.cu", "infer.cu")]
 DEPS = SOURCES + [os.path.join(HERE, "csrc", name) for name in ("externd_kernels.cuh", "als_cluster.cuh", "block_als.cuh")] \
     + [os.path.join(ROOT, "include", "externd.h")]
 OUT = os.path.join(HERE, "libexternd.so")

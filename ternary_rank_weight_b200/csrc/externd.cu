@@ -21,6 +21,18 @@
 #include "externd.h"
 #include "externd_kernels.cuh"
 
+#ifndef EXTERND_SECONDARY
+// The ALS machinery of this file compiled a second time with 1024 threads per CTA
+// (externd_nt1024.cu): the factorization plan of groups of 2 to 12 CTAs, where each CTA's share of
+// the per-half-step vector work is large enough that twice the threads pay (the plan's group size
+// alone decides, so a matrix gets the same kernel, and the same bits, from a batched call and from
+// a single call with the same grid).
+constexpr int NT1024_MIN_GROUP = 2;
+constexpr int NT1024_MAX_GROUP = 12;
+int externd_run_nt1024(const void* in, int np, const void* opt, cudaStream_t stream, int* statuses,
+                       externd_stats* stats);
+#endif
+
 namespace externd {
 
 // ---------------------------------------------------------------------------
@@ -1576,7 +1588,9 @@ __global__ void __launch_bounds__(NT, 1) als_kernel(const KCfg cfg) {
 }  // namespace externd
 
 #include "als_cluster.cuh"
+#ifndef EXTERND_SECONDARY
 #include "block_als.cuh"
+#endif
 
 namespace externd {
 
@@ -1962,6 +1976,14 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
         if (Gg > in[b].n) Gg = (int)in[b].n;
     }
     if (Gg < 1) Gg = 1;
+#ifndef EXTERND_SECONDARY
+    if (!fixed && opt.cluster <= 1 && Gg >= NT1024_MIN_GROUP && Gg <= NT1024_MAX_GROUP) {
+        externd_stats st2 = {};
+        const int rc2 = externd_run_nt1024(in, np, &opt, stream, statuses, &st2);
+        g_last = st2;
+        return rc2;
+    }
+#endif
 
     // ---- lazy deflation depth from the shared-memory budget
     if (Gg > NT) Gg = NT;   // one thread per CTA of the group polls its stripe
@@ -2471,6 +2493,7 @@ int validate_factor(const float* A, int64_t m, int64_t n, double mu, double tau,
 
 }  // namespace
 
+#ifndef EXTERND_SECONDARY
 namespace {
 
 // §2.4 batched block ALS on the device: blocks of b components, each a sequence of launches on
@@ -2957,3 +2980,5 @@ int externd_last_stats(externd_stats* out) {
 }
 
 }  // extern "C"
+
+#endif  // EXTERND_SECONDARY
