@@ -20,7 +20,7 @@ import torch
 
 import ternary_rank_weight_b200 as ext
 from oracle import externd_oracle as ora
-from ternary_rank_weight_b200.workloads import WORKLOADS
+from ternary_rank_weight_b200.workloads import WORKLOADS, llm_matrix
 
 import _parity
 
@@ -114,3 +114,15 @@ def test_batch_slices_run_with_the_batch_plan_equal_the_whole_batch():
             for j, i in enumerate(idx):
                 assert torch.equal(part[j].B, res[i].B) and torch.equal(part[j].C, res[i].C), (world, rank, i)
                 assert torch.equal(part[j].D, res[i].D) and torch.equal(part[j].energy, res[i].energy)
+
+
+def test_block_size_follows_the_group_size():
+    """Plans of 2 to 12 CTAs per matrix run the 1024-thread build of the ALS kernel, all others the
+    512-thread build; the group size alone decides (a batch and a single call with the same grid
+    get the same kernel)."""
+    A = torch.from_numpy(llm_matrix(256, 512, seed=1)).cuda()
+    for grid, want in ((1, 512), (2, 1024), (9, 1024), (12, 1024), (13, 512), (16, 512), (148, 512)):
+        _, st = ext.factor_batched([A], [1.0], [0.7], grid=grid, plan_only=True)
+        assert (st["group"], st["block"]) == (grid, want)
+    _, st = ext.factor_batched([A, A], [1.0, 1.0], [0.7, 0.7], grid=9, plan_only=True)
+    assert (st["group"], st["block"]) == (9, 1024)
