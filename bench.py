@@ -259,7 +259,7 @@ def run_ours(args):
     from ternary_rank_weight_b200 import dist
 
     strong = args.scaling == "strong"
-    plan = {"grid": args.grid, "cluster": args.cluster}
+    plan = {"grid": args.grid, "cluster": args.cluster, "block": args.block}
     if strong:
         # one fixed batch split over the ranks: every rank takes a contiguous slice of the SAME
         # matrices and runs it with the plan of the whole batch on one GPU, so each matrix gets
@@ -270,8 +270,8 @@ def run_ours(args):
         _, pst = ext.factor_batched([torch.from_numpy(a) for a in mats_full], list(w_full.mu), list(w_full.tau),
                                     iters=w_full.iters, seeds=list(w_full.seeds), sweeps=w_full.sweeps,
                                     hs=[w_full.weights(b) for b in range(w_full.count)] if w_full.weighted else None,
-                                    grid=args.grid, cluster=args.cluster, plan_only=True)
-        plan = {"grid": pst["group"], "cluster": pst["cluster"]}
+                                    grid=args.grid, cluster=args.cluster, block=args.block, plan_only=True)
+        plan = {"grid": pst["group"], "cluster": pst["cluster"], "block": pst["block"]}
         w, idx = dist.slice_workload(w_full, ws, rank)
         mats = [mats_full[i] for i in idx]
     else:
@@ -290,7 +290,7 @@ def run_ours(args):
         if strong:
             res, st = ext.factor_batched(inputs, w.mu, w.tau, iters=w.iters, seeds=list(w.seeds), hs=hw,
                                          lams=[w.lam] * w.count if w.weighted else None, sweeps=w.sweeps,
-                                         grid=plan["grid"], cluster=plan["cluster"])
+                                         grid=plan["grid"], cluster=plan["cluster"], block=plan["block"])
             assert all(x == 0 for x in st), st
             return res, res[0].stats
         if w.weighted and not w.sweeps and w.count == 1:
@@ -299,11 +299,11 @@ def run_ours(args):
         if w.count == 1:
             f = ext.factor(inputs[0], w.mu[0], w.tau[0], iters=w.iters, seed=w.seeds[0],
                            grid=args.grid, pending=args.pending, sweeps=w.sweeps,
-                           h=hw[0] if w.weighted else None, lam=w.lam, cluster=args.cluster)
+                           h=hw[0] if w.weighted else None, lam=w.lam, cluster=args.cluster, block=args.block)
             return [f], f.stats
         res, st = ext.factor_batched(inputs, w.mu, w.tau, iters=w.iters, seeds=list(w.seeds), hs=hw,
                                      lams=[w.lam] * w.count if w.weighted else None, sweeps=w.sweeps,
-                                     grid=args.grid, cluster=args.cluster)
+                                     grid=args.grid, cluster=args.cluster, block=args.block)
         assert all(s == 0 for s in st), st
         return res, res[0].stats
 
@@ -600,6 +600,8 @@ def main():
     ap.add_argument("--workload", default=HEADLINE, choices=sorted(WORKLOADS))
     ap.add_argument("--all", action="store_true", help="one line per workload (reporting, not the driver's line)")
     ap.add_argument("--grid", type=int, default=0)
+    ap.add_argument("--block", type=int, default=0,
+                    help="threads per CTA of the one-CTA-per-stripe ALS kernel: 0 automatic, 256, 512 or 1024")
     ap.add_argument("--cluster", type=int, default=0,
                     help="ALS kernel: 0 automatic, 1 one CTA per stripe, 2/4/8/16 clustered with that cluster size")
     ap.add_argument("--scaling", choices=("weak", "strong"), default="weak",

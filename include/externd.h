@@ -162,13 +162,14 @@ int externd_factor_batched(int count, const float* const* A, const int64_t* m, c
  *             0 .. 1000.
  *   sweep_energy_out  NULL, or `count` pointers (entries may be NULL) to `sweeps` doubles each.
  *   grid      CTAs per matrix (0: automatic), as externd_options.grid.
- *   cluster   kernel choice, as externd_options.cluster.  A matrix gets the same bits from
- *             any launch with the same grid and cluster size -- e.g. one slice of a batch per
- *             GPU, run with the plan of the whole batch.
+ *   cluster   kernel choice, as externd_options.cluster.
+ *   block     threads per CTA, as externd_options.block.  A matrix gets the same bits from
+ *             any launch with the same grid, cluster size and block size -- e.g. one slice of a
+ *             batch per GPU, run with the plan of the whole batch.
  *   plan_only nonzero: validate the arguments, choose the launch (CTAs per matrix, cluster
- *             size, lazy-deflation depth) exactly as the call would, record it for
- *             externd_last_stats (grid, group, cluster, pending, smem_bytes) and return
- *             without device work. */
+ *             size, lazy-deflation depth, threads per CTA) exactly as the call would, record it
+ *             for externd_last_stats (grid, group, cluster, pending, block, smem_bytes) and
+ *             return without device work. */
 typedef struct {
     const float* const* h;
     const double* lambda;
@@ -179,6 +180,7 @@ typedef struct {
     int plan_only;
     int* async_status;   /* as externd_options.async_status: one status for the whole batch
                           * (the first matrix's failure, else EXTERND_OK) */
+    int block;
 } externd_batch_options;
 
 /* externd_factor_batched with per-matrix extensions (opt may be NULL: the plain call). */
@@ -349,7 +351,8 @@ typedef struct {
      * residual stripe (the kernel that also runs refinement sweeps); 2, 4, 8 or 16 = the
      * clustered kernel with clusters of that many CTAs, for factorizations without sweeps
      * (EXTERND_ELAUNCH if they cannot all be resident, EXTERND_EINVAL for other values).
-     * Results depend on the partition: the same grid and cluster size give the same bits. */
+     * Results depend on the partition: the same grid, cluster size and block size give the
+     * same bits. */
     int cluster;
     /* Asynchronous call: non-NULL = a DEVICE int.  The call queues all its work on `stream` and
      * returns EXTERND_OK without waiting; when the stream reaches the end of the work, the
@@ -360,6 +363,15 @@ typedef struct {
      * waited for what it had queued).  externd_last_stats records the plan only (timings,
      * byte counts and safeguard counts are 0). */
     int* async_status;
+    /* Threads per CTA of the one-CTA-per-stripe kernel: 0 = automatic, else 256, 512 or 1024
+     * (EXTERND_EINVAL otherwise; the clustered kernel runs at 512 only, so with cluster > 1
+     * only 0 and 512 are accepted).  The automatic choice follows the work one CTA does per
+     * half-step, W = m n / G + 8 (m + n) for G CTAs per matrix (the largest matrix of a batch):
+     * its share of the residual plus the two vectors it thresholds.  256 below W = 170000, 512
+     * up to 230000, 1024 above.  The block size sets how the fp64 sums inside a CTA are split
+     * across warps, so, as with the partition, only the same grid, cluster size and block
+     * size are guaranteed to give the same bits. */
+    int block;
 } externd_options;
 
 /* externd_factor with options (opt may be NULL). */

@@ -56,6 +56,7 @@ class Options(ctypes.Structure):
         ("trace_trit_u", ctypes.c_void_p),
         ("cluster", ctypes.c_int),
         ("async_status", ctypes.c_void_p),
+        ("block", ctypes.c_int),
     ]
 
 
@@ -69,6 +70,7 @@ class BatchOptions(ctypes.Structure):
         ("cluster", ctypes.c_int),
         ("plan_only", ctypes.c_int),
         ("async_status", ctypes.c_void_p),
+        ("block", ctypes.c_int),
     ]
 
 

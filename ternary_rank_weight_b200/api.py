@@ -155,7 +155,7 @@ class Trace:
 def factor(A, mu: float, tau: float, iters: int = 15, seed: int = 0, *, grid: int = 0, pending: int = 0,
            wait_limit_s: float = 0.0, fault_skip_cta: Optional[int] = None, want_d64: bool = False,
            want_energy: bool = True, sweeps: int = 0, h=None, lam: float = 0.0, trace=None, cluster: int = 0,
-           async_status=None, stream=None) -> Factors:
+           block: int = 0, async_status=None, stream=None) -> Factors:
     """Factor one matrix (externd_factor_ex).  Outputs are allocated where A lives.
 
     sweeps: §2.4 refinement sweeps after extraction (``energy`` keeps the extraction
@@ -165,6 +165,8 @@ def factor(A, mu: float, tau: float, iters: int = 15, seed: int = 0, *, grid: in
     i < k extracts component i, visit (s + 1) k + i is sweep s's refit of component i
     (``Factors.trace``; A must be on the GPU).  cluster: kernel choice (0 automatic, 1 one
     CTA per residual stripe, 2/4/8/16 the clustered kernel with that cluster size).
+    block: threads per CTA (0 automatic, 256, 512 or 1024); the same grid, cluster and block
+    give the same bits.
     async_status: a one-element int32 CUDA tensor: the call queues its work and returns at
     once; the tensor receives the status (0 or a negative code) when the stream gets there.
     A (and h) must then be contiguous float32 CUDA tensors, which the queued work reads until
@@ -197,6 +199,7 @@ def factor(A, mu: float, tau: float, iters: int = 15, seed: int = 0, *, grid: in
     opt.h = _ptr(h)
     opt.lambda_ = float(lam)
     opt.cluster = int(cluster)
+    opt.block = int(block)
     if async_status is not None:
         opt.async_status = _ptr(async_status)
     tr = None
@@ -322,12 +325,12 @@ def factor_block(A: torch.Tensor, mu: float, tau: float, iters: int = 15, seed: 
 def factor_batched(As: Sequence, mus: Sequence[float], taus: Sequence[float], iters: int = 15,
                    seeds: Optional[Sequence[int]] = None, *, hs: Optional[Sequence] = None,
                    lams: Optional[Sequence[float]] = None, sweeps: int = 0, grid: int = 0, cluster: int = 0,
-                   plan_only: bool = False, async_status=None, stream=None):
+                   block: int = 0, plan_only: bool = False, async_status=None, stream=None):
     """Factor independent matrices in one launch (externd_factor_batched_ex).
 
     hs: per-matrix importance weights (§2.5; every matrix or none), lams their lambdas;
-    sweeps: refinement sweeps (§2.4) for every matrix; grid, cluster: the launch (0:
-    automatic).  plan_only: return (None, stats of the plan) without device work.
+    sweeps: refinement sweeps (§2.4) for every matrix; grid, cluster, block: the launch (0:
+    automatic; a matrix gets the same bits from any launch with the same three).  plan_only: return (None, stats of the plan) without device work.
     async_status: a one-element int32 CUDA tensor: queue the work and return at once; the
     tensor receives the batch's status when the stream gets there.  Every matrix (and weight
     vector) must then be a contiguous float32 CUDA tensor, kept alive and unchanged until then.
@@ -373,6 +376,7 @@ def factor_batched(As: Sequence, mus: Sequence[float], taus: Sequence[float], it
     opt.sweeps = int(sweeps)
     opt.grid = int(grid)
     opt.cluster = int(cluster)
+    opt.block = int(block)
     opt.plan_only = 1 if plan_only else 0
     if async_status is not None:
         opt.async_status = _ptr(async_status)

@@ -22,15 +22,14 @@
 #include "externd_kernels.cuh"
 
 #ifndef EXTERND_SECONDARY
-// The ALS machinery of this file compiled a second time with 1024 threads per CTA
-// (externd_nt1024.cu): the factorization plan of groups of 2 to 12 CTAs, where each CTA's share of
-// the per-half-step vector work is large enough that twice the threads pay (the plan's group size
-// alone decides, so a matrix gets the same kernel, and the same bits, from a batched call and from
-// a single call with the same grid).
-constexpr int NT1024_MIN_GROUP = 2;
-constexpr int NT1024_MAX_GROUP = 12;
+// The ALS machinery of this file is compiled at three block sizes, each in its own namespace: 512
+// threads per CTA here, 256 in externd_nt256.cu and 1024 in externd_nt1024.cu.  Every C-ABI entry
+// point lives here; a plan whose block size is not 512 runs through the other build's run()
+// (arguments as validated here; fixed_base/fixed_cap: the caller-fixed workspace or null).
+int externd_run_nt256(const void* in, int np, const void* opt, cudaStream_t stream, int* statuses,
+                      externd_stats* stats, void* fixed_base, size_t fixed_cap);
 int externd_run_nt1024(const void* in, int np, const void* opt, cudaStream_t stream, int* statuses,
-                       externd_stats* stats);
+                       externd_stats* stats, void* fixed_base, size_t fixed_cap);
 #endif
 
 namespace externd {
@@ -1816,6 +1815,7 @@ struct RunOpts {
     bool plan_only = false;   // fill the stats with the launch plan and return (no device work)
     int cluster = 0;          // 0: automatic; 1: the one-CTA-per-stripe kernel; 2, 4, 8, 16: clusters of that size
     int* async_status = nullptr;   // device int: queue everything, write the status there, do not wait
+    int block = 0;            // threads per CTA: 0 automatic, else 256, 512 or 1024
 };
 
 // Status of an asynchronous call: the first matrix's failure (a group that stopped before a
@@ -1942,6 +1942,22 @@ struct FixedWs {
     size_t cap = 0;
 };
 
+#ifndef EXTERND_SECONDARY
+// Threads per CTA of the one-CTA-per-stripe kernel for a plan of G CTAs per matrix.  A CTA's
+// work per half-step grows with its share of the residual (the stripe its GEMV reads, m n / G
+// elements) and with the whole vector it thresholds (m or n entries: 8 (m + n) weighs them like
+// stripe elements).  Fewer threads shorten the barrier-bound chain of a half-step; more threads
+// pay once the share is large.  Measured on B200 (ALS time, 15 iterations): 256 threads are
+// fastest below W = 170k -- single matrices of 1024^2 to 2048^2 at 65k elements per CTA run
+// 7-20 % faster than at 512, 256^2 on one CTA 23 % -- 512 up to 230k (2560 x 6912 over 148 CTAs,
+// W = 196k: 4 % ahead of 256, 3 % of 1024), 1024 above (16 matrices of 1536^2 over 9 CTAs
+// each, W = 287k: 12 % ahead of 512; 2560 x 6912 over 74 CTAs, W = 315k: 8 %).
+int auto_block(double work_max, int64_t m_max, int64_t n_max, int G) {
+    const double W = work_max / G + 8.0 * (double)(m_max + n_max);
+    return W < 170000.0 ? 256 : (W < 230000.0 ? 512 : 1024);
+}
+#endif
+
 int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* statuses,
         const FixedWs* fixed = nullptr) {
     int rc = EXTERND_OK;
@@ -1977,11 +1993,16 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
     }
     if (Gg < 1) Gg = 1;
 #ifndef EXTERND_SECONDARY
-    if (!fixed && opt.cluster <= 1 && Gg >= NT1024_MIN_GROUP && Gg <= NT1024_MAX_GROUP) {
-        externd_stats st2 = {};
-        const int rc2 = externd_run_nt1024(in, np, &opt, stream, statuses, &st2);
-        g_last = st2;
-        return rc2;
+    // ---- block size: the caller's, else by the work of one CTA (the clustered kernel: 512)
+    if (opt.cluster <= 1) {
+        const int nt = opt.block > 0 ? opt.block : auto_block(work_max, m_max, n_max, Gg);
+        if (nt != NT) {
+            externd_stats st2 = {};
+            const int rc2 = (nt == 256 ? externd_run_nt256 : externd_run_nt1024)(
+                in, np, &opt, stream, statuses, &st2, fixed ? fixed->base : nullptr, fixed ? fixed->cap : 0);
+            if (!fixed) g_last = st2;   // the allocation-free call leaves the stats alone
+            return rc2;
+        }
     }
 #endif
 
@@ -2474,6 +2495,28 @@ int check_trace(int64_t first, int64_t count, int64_t k, const double* pv, const
     return EXTERND_OK;
 }
 
+#ifdef EXTERND_SECONDARY
+// Entry of a secondary build (another block size): the primary build validated the arguments and
+// chose the block size; this build plans and runs the call, in the caller-fixed workspace if any.
+int run_secondary(const void* in, int np, const void* opt, cudaStream_t stream, int* statuses, externd_stats* stats,
+                  void* fixed_base, size_t fixed_cap) {
+    FixedWs fw;
+    fw.base = static_cast<unsigned char*>(fixed_base);
+    fw.cap = fixed_cap;
+    const int rc = run(static_cast<const ProbIn*>(in), np, *static_cast<const RunOpts*>(opt), stream, statuses,
+                       fixed_base ? &fw : nullptr);
+    *stats = g_last;
+    return rc;
+}
+#endif
+
+// Threads per CTA asked of the one-CTA-per-stripe kernel: 0 (automatic), 256, 512 or 1024; the
+// clustered kernel (cluster > 1) runs at 512 only.
+bool block_ok(int block, int cluster) {
+    if (block != 0 && block != 256 && block != 512 && block != 1024) return false;
+    return cluster <= 1 || block == 0 || block == 512;
+}
+
 int check_rows_aligned(const void* p) {
     return (reinterpret_cast<uintptr_t>(p) & 15u) == 0 ? EXTERND_OK : EXTERND_EINVAL;
 }
@@ -2718,6 +2761,8 @@ int externd_factor_ex(const float* A, int64_t m, int64_t n, double mu, double ta
         if (opt->cluster < 0 || opt->cluster > 16 || (opt->cluster > 1 && (opt->cluster & (opt->cluster - 1))))
             return EXTERND_EINVAL;
         ro.cluster = opt->cluster;
+        if (!block_ok(opt->block, opt->cluster)) return EXTERND_EINVAL;
+        ro.block = opt->block;
         ro.async_status = opt->async_status;
         I.d64 = opt->d64_out;
         if (opt->sweeps < 0 || opt->sweeps > 1000) return EXTERND_EINVAL;
@@ -2857,12 +2902,14 @@ int externd_factor_batched_ex(int count, const float* const* A, const int64_t* m
     }
     RunOpts ro;
     if (opt) {
-        if (opt->grid < 0 || opt->cluster < 0 || opt->cluster > 16 || (opt->cluster > 1 && (opt->cluster & (opt->cluster - 1)))) {
+        if (opt->grid < 0 || opt->cluster < 0 || opt->cluster > 16 || (opt->cluster > 1 && (opt->cluster & (opt->cluster - 1))) ||
+            !block_ok(opt->block, opt->cluster)) {
             for (int c = 0; c < count; ++c) status_out[c] = EXTERND_EINVAL;
             return EXTERND_EINVAL;
         }
         ro.grid = opt->grid;
         ro.cluster = opt->cluster;
+        ro.block = opt->block;
         ro.plan_only = opt->plan_only != 0;
         ro.async_status = opt->async_status;
     }

@@ -68,11 +68,11 @@ def test_batched_attention_workload_full_size():
         e = r.energy.cpu().numpy()
         assert np.all(np.diff(e) >= -1e-12) and 0.5 < e[-1] < 1.0
     for b in (0, 7):
-        f = ext.factor(torch.from_numpy(mats[b]).cuda(), w.mu[b], w.tau[b], seed=w.seeds[b], grid=G, cluster=res[0].stats["cluster"])
+        f = ext.factor(torch.from_numpy(mats[b]).cuda(), w.mu[b], w.tau[b], seed=w.seeds[b], grid=G, cluster=res[0].stats["cluster"], block=res[0].stats["block"])
         assert torch.equal(f.B, res[b].B) and torch.equal(f.C, res[b].C) and torch.equal(f.D, res[b].D)
         assert torch.equal(f.energy, res[b].energy)
-    f0 = ext.factor(torch.from_numpy(mats[0]).cuda(), w.mu[0], w.tau[0], seed=w.seeds[0], grid=G, cluster=res[0].stats["cluster"], want_d64=True)
-    ndiv = _parity.teacher_forced(mats[0], f0, w.seeds[0], w.tau[0], (0, 1, 1919, 3839), "attn 1536 matrix 0", grid=G, cluster=res[0].stats["cluster"])
+    f0 = ext.factor(torch.from_numpy(mats[0]).cuda(), w.mu[0], w.tau[0], seed=w.seeds[0], grid=G, cluster=res[0].stats["cluster"], block=res[0].stats["block"], want_d64=True)
+    ndiv = _parity.teacher_forced(mats[0], f0, w.seeds[0], w.tau[0], (0, 1, 1919, 3839), "attn 1536 matrix 0", grid=G, cluster=res[0].stats["cluster"], block=res[0].stats["block"])
     assert ndiv <= 1
 
 
@@ -103,26 +103,46 @@ def test_batch_slices_run_with_the_batch_plan_equal_the_whole_batch():
     res, st = ext.factor_batched(mats, list(w.mu), list(w.tau), seeds=list(w.seeds))
     assert st == [0] * w.count
     _, plan = ext.factor_batched(mats, list(w.mu), list(w.tau), seeds=list(w.seeds), plan_only=True)
-    G, cl = res[0].stats["group"], res[0].stats["cluster"]
-    assert (plan["group"], plan["cluster"], plan["pending"]) == (G, cl, res[0].stats["pending"])
+    G, cl, nt = res[0].stats["group"], res[0].stats["cluster"], res[0].stats["block"]
+    assert (plan["group"], plan["cluster"], plan["pending"], plan["block"]) == (G, cl, res[0].stats["pending"], nt)
     for world in (2, 3):
         for rank in range(world):
             ws, idx = dist.slice_workload(w, world, rank)
             part, st2 = ext.factor_batched([mats[i] for i in idx], list(ws.mu), list(ws.tau), seeds=list(ws.seeds),
-                                           grid=G, cluster=cl)
+                                           grid=G, cluster=cl, block=nt)
             assert st2 == [0] * len(idx)
             for j, i in enumerate(idx):
                 assert torch.equal(part[j].B, res[i].B) and torch.equal(part[j].C, res[i].C), (world, rank, i)
                 assert torch.equal(part[j].D, res[i].D) and torch.equal(part[j].energy, res[i].energy)
 
 
-def test_block_size_follows_the_group_size():
-    """Plans of 2 to 12 CTAs per matrix run the 1024-thread build of the ALS kernel, all others the
-    512-thread build; the group size alone decides (a batch and a single call with the same grid
-    get the same kernel)."""
-    A = torch.from_numpy(llm_matrix(256, 512, seed=1)).cuda()
-    for grid, want in ((1, 512), (2, 1024), (9, 1024), (12, 1024), (13, 512), (16, 512), (148, 512)):
+def test_block_size_follows_the_work_per_cta():
+    """The ALS kernel runs at 256, 512 or 1024 threads per CTA.  The automatic choice follows the
+    work of one CTA per half-step, W = m n / G + 8 (m + n) for G CTAs per matrix: 256 below
+    170000, 512 below 230000, 1024 above; an explicit block size overrides it, and a batch and a
+    single call with the same grid choose alike."""
+    A = torch.zeros((1536, 1536), device="cuda")
+    want = {148: 256, 64: 256, 16: 512, 12: 512, 11: 1024, 9: 1024}   # W: 40k 61k 172k 221k 239k 287k
+    for grid, nt in want.items():
         _, st = ext.factor_batched([A], [1.0], [0.7], grid=grid, plan_only=True)
-        assert (st["group"], st["block"]) == (grid, want)
+        assert (st["group"], st["block"]) == (grid, nt), grid
     _, st = ext.factor_batched([A, A], [1.0, 1.0], [0.7, 0.7], grid=9, plan_only=True)
     assert (st["group"], st["block"]) == (9, 1024)
+    for nt in (256, 512, 1024):
+        _, st = ext.factor_batched([A], [1.0], [0.7], grid=148, block=nt, plan_only=True)
+        assert st["block"] == nt
+    # the workloads: 256^2 and 1024^2 on 256 threads, 2560 x 6912 on 512, the 1536^2 batch on 1024
+    for name, nt in (("iid_256x256_mu2_tau0.7", 256), ("llm_1024x1024_mu2_tau0.7", 256),
+                     ("mlp_2560x6912_bf16_mu3_tau1.0", 512), ("attn_16x1536x1536_mu2.5_tau_cycle", 1024)):
+        w = WORKLOADS[name]
+        mats = [torch.zeros(shape, device="cuda") for shape in w.shapes]
+        _, st = ext.factor_batched(mats, list(w.mu), list(w.tau), plan_only=True)
+        assert st["block"] == nt, name
+    # other sizes, and anything but 512 with the clustered kernel, are refused
+    for kw in (dict(block=300), dict(block=128), dict(block=256, cluster=2), dict(block=1024, cluster=4)):
+        with pytest.raises(ext.ExterndError) as e:
+            ext.factor_batched([A], [1.0], [0.7], plan_only=True, **kw)
+        assert e.value.status == ext.STATUS["EINVAL"], kw
+        with pytest.raises(ext.ExterndError) as e:
+            ext.factor(A[:64, :64].contiguous() + 1.0, 1.0, 0.7, **kw)
+        assert e.value.status == ext.STATUS["EINVAL"], kw

@@ -105,6 +105,6 @@ def test_attention_batch_matches_the_oracle_runs_for_every_tau():
         g = _golden(name)
         assert g["matrix"] == b and g["tau"] == w.tau[b]
         # the d64 scales of the batched run: a single call with the same group size repeats it bit for bit
-        f = ext.factor(torch.from_numpy(mats[b]).cuda(), w.mu[b], w.tau[b], seed=w.seeds[b], grid=G, cluster=res[0].stats["cluster"], want_d64=True)
+        f = ext.factor(torch.from_numpy(mats[b]).cuda(), w.mu[b], w.tau[b], seed=w.seeds[b], grid=G, cluster=res[0].stats["cluster"], block=res[0].stats["block"], want_d64=True)
         assert torch.equal(f.B, res[b].B) and torch.equal(f.C, res[b].C) and torch.equal(f.D, res[b].D)
-        _compare(g, mats[b], f, f"attn 1536 matrix {b} end to end", grid=G, cluster=res[0].stats["cluster"])
+        _compare(g, mats[b], f, f"attn 1536 matrix {b} end to end", grid=G, cluster=res[0].stats["cluster"], block=res[0].stats["block"])
