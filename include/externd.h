@@ -367,8 +367,8 @@ typedef struct {
      * (EXTERND_EINVAL otherwise; the clustered kernel runs at 512 only, so with cluster > 1
      * only 0 and 512 are accepted).  The automatic choice follows the work one CTA does per
      * half-step, W = m n / G + 8 (m + n) for G CTAs per matrix (the largest matrix of a batch):
-     * its share of the residual plus the two vectors it thresholds.  256 below W = 170000, 512
-     * up to 230000, 1024 above.  The block size sets how the fp64 sums inside a CTA are split
+     * its share of the residual plus the two vectors it thresholds.  256 below W = 170000 (512
+     * with refinement sweeps, whose refits are faster there), 512 up to 230000, 1024 above.  The block size sets how the fp64 sums inside a CTA are split
      * across warps, so, as with the partition, only the same grid, cluster size and block
      * size are guaranteed to give the same bits. */
     int block;

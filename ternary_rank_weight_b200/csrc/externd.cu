@@ -1951,10 +1951,14 @@ struct FixedWs {
 // fastest below W = 170k -- single matrices of 1024^2 to 2048^2 at 65k elements per CTA run
 // 7-20 % faster than at 512, 256^2 on one CTA 23 % -- 512 up to 230k (2560 x 6912 over 148 CTAs,
 // W = 196k: 4 % ahead of 256, 3 % of 1024), 1024 above (16 matrices of 1536^2 over 9 CTAs
-// each, W = 287k: 12 % ahead of 512; 2560 x 6912 over 74 CTAs, W = 315k: 8 %).
-int auto_block(double work_max, int64_t m_max, int64_t n_max, int G) {
+// each, W = 287k: 12 % ahead of 512; 2560 x 6912 over 74 CTAs, W = 315k: 8 %).  Refinement
+// sweeps are the exception below 170k: their refits of stored components ran 18 % slower at 256
+// threads than at 512 (1024^2 with ten sweeps: 9636 against 10669 fits/s), so plans with sweeps
+// take 512 there.
+int auto_block(double work_max, int64_t m_max, int64_t n_max, int G, bool sweeping) {
     const double W = work_max / G + 8.0 * (double)(m_max + n_max);
-    return W < 170000.0 ? 256 : (W < 230000.0 ? 512 : 1024);
+    if (W >= 230000.0) return 1024;
+    return (W < 170000.0 && !sweeping) ? 256 : 512;
 }
 #endif
 
@@ -1995,7 +1999,9 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
 #ifndef EXTERND_SECONDARY
     // ---- block size: the caller's, else by the work of one CTA (the clustered kernel: 512)
     if (opt.cluster <= 1) {
-        const int nt = opt.block > 0 ? opt.block : auto_block(work_max, m_max, n_max, Gg);
+        bool sweeps = false;
+        for (int b = 0; b < np; ++b) sweeps = sweeps || (in[b].mode == MODE_FACTOR && in[b].sweeps > 0);
+        const int nt = opt.block > 0 ? opt.block : auto_block(work_max, m_max, n_max, Gg, sweeps);
         if (nt != NT) {
             externd_stats st2 = {};
             const int rc2 = (nt == 256 ? externd_run_nt256 : externd_run_nt1024)(

@@ -119,8 +119,8 @@ def test_batch_slices_run_with_the_batch_plan_equal_the_whole_batch():
 def test_block_size_follows_the_work_per_cta():
     """The ALS kernel runs at 256, 512 or 1024 threads per CTA.  The automatic choice follows the
     work of one CTA per half-step, W = m n / G + 8 (m + n) for G CTAs per matrix: 256 below
-    170000, 512 below 230000, 1024 above; an explicit block size overrides it, and a batch and a
-    single call with the same grid choose alike."""
+    170000 (512 with refinement sweeps), 512 below 230000, 1024 above; an explicit block size
+    overrides it, and a batch and a single call with the same grid choose alike."""
     A = torch.zeros((1536, 1536), device="cuda")
     want = {148: 256, 64: 256, 16: 512, 12: 512, 11: 1024, 9: 1024}   # W: 40k 61k 172k 221k 239k 287k
     for grid, nt in want.items():
@@ -131,12 +131,18 @@ def test_block_size_follows_the_work_per_cta():
     for nt in (256, 512, 1024):
         _, st = ext.factor_batched([A], [1.0], [0.7], grid=148, block=nt, plan_only=True)
         assert st["block"] == nt
-    # the workloads: 256^2 and 1024^2 on 256 threads, 2560 x 6912 on 512, the 1536^2 batch on 1024
+    # refinement sweeps take 512 where the extraction alone would take 256
+    for grid, nt in ((148, 512), (16, 512), (9, 1024)):
+        _, st = ext.factor_batched([A], [1.0], [0.7], grid=grid, sweeps=1, plan_only=True)
+        assert st["block"] == nt, grid
+    # the workloads: 256^2 and 1024^2 on 256 threads (1024^2 with ten sweeps on 512), 2560 x 6912
+    # on 512, the 1536^2 batch on 1024
     for name, nt in (("iid_256x256_mu2_tau0.7", 256), ("llm_1024x1024_mu2_tau0.7", 256),
-                     ("mlp_2560x6912_bf16_mu3_tau1.0", 512), ("attn_16x1536x1536_mu2.5_tau_cycle", 1024)):
+                     ("llm_1024x1024_mu2_tau0.7_sweep10", 512), ("mlp_2560x6912_bf16_mu3_tau1.0", 512),
+                     ("attn_16x1536x1536_mu2.5_tau_cycle", 1024)):
         w = WORKLOADS[name]
         mats = [torch.zeros(shape, device="cuda") for shape in w.shapes]
-        _, st = ext.factor_batched(mats, list(w.mu), list(w.tau), plan_only=True)
+        _, st = ext.factor_batched(mats, list(w.mu), list(w.tau), sweeps=w.sweeps, plan_only=True)
         assert st["block"] == nt, name
     # other sizes, and anything but 512 with the clustered kernel, are refused
     for kw in (dict(block=300), dict(block=128), dict(block=256, cluster=2), dict(block=1024, cluster=4)):

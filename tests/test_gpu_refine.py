@@ -31,9 +31,12 @@ def _canonical(B, D, C):
 
 
 def _run(A, mu, tau, seed, sweeps, h=None):
+    """The factorization with sweeps (ref) and without (base).  Bits depend on the block size, and
+    the automatic choice gives plans with sweeps 512 threads where it gives extraction alone 256,
+    so base runs at ref's block size: its extraction is then ref's, bit for bit."""
     Ag = torch.from_numpy(A).cuda()
-    base = ext.factor(Ag, mu, tau, seed=seed, want_d64=True, h=h)
     ref = ext.factor(Ag, mu, tau, seed=seed, want_d64=True, sweeps=sweeps, h=h)
+    base = ext.factor(Ag, mu, tau, seed=seed, want_d64=True, h=h, block=ref.stats["block"])
     ref.run_seed = seed
     return base, ref
 
@@ -209,10 +212,10 @@ def test_batched_sweeps_equal_single_calls(weighted):
     res, st = ext.factor_batched([torch.from_numpy(a).cuda() for a in mats], mus, taus, seeds=seeds,
                                  hs=hs, lams=lams, sweeps=2)
     assert st == [0, 0, 0]
-    G = res[0].stats["group"]
+    G, nt = res[0].stats["group"], res[0].stats["block"]
     for i, (A, mu, tau, sd, r) in enumerate(zip(mats, mus, taus, seeds, res)):
         kw = {"h": hs[i], "lam": lams[i]} if weighted else {}
-        f = ext.factor(torch.from_numpy(A).cuda(), mu, tau, seed=sd, grid=G, sweeps=2, **kw)
+        f = ext.factor(torch.from_numpy(A).cuda(), mu, tau, seed=sd, grid=G, block=nt, sweeps=2, **kw)
         assert torch.equal(f.B, r.B) and torch.equal(f.C, r.C) and torch.equal(f.D, r.D)
         assert torch.equal(f.energy, r.energy) and torch.equal(f.sweep_energy, r.sweep_energy)
         assert r.sweep_energy[-1].item() >= r.energy[-1].item() - 1e-9
