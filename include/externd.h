@@ -368,7 +368,9 @@ typedef struct {
      * only 0 and 512 are accepted).  The automatic choice follows the work one CTA does per
      * half-step, W = m n / G + 8 (m + n) for G CTAs per matrix (the largest matrix of a batch):
      * its share of the residual plus the two vectors it thresholds.  256 below W = 170000 (512
-     * with refinement sweeps, whose refits are faster there), 512 up to 230000, 1024 above.  The block size sets how the fp64 sums inside a CTA are split
+     * with refinement sweeps, whose refits are faster there), 512 up to 230000, 1024 above --
+     * unless the 1024-thread plan, which keeps more shared state per CTA, would leave a
+     * lazy-deflation depth below 8 (the largest shapes), where 512 is kept.  The block size sets how the fp64 sums inside a CTA are split
      * across warps, so, as with the partition, only the same grid, cluster size and block
      * size are guaranteed to give the same bits. */
     int block;

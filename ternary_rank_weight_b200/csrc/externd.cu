@@ -1955,6 +1955,7 @@ struct FixedWs {
 // sweeps are the exception below 170k: their refits of stored components ran 18 % slower at 256
 // threads than at 512 (1024^2 with ten sweeps: 9636 against 10669 fits/s), so plans with sweeps
 // take 512 there.
+constexpr int AUTO_MIN_DEPTH = 8;   // a shorter pending list folds the residual every few components
 int auto_block(double work_max, int64_t m_max, int64_t n_max, int G, bool sweeping) {
     const double W = work_max / G + 8.0 * (double)(m_max + n_max);
     if (W >= 230000.0) return 1024;
@@ -2001,7 +2002,20 @@ int run(const ProbIn* in, int np, const RunOpts& opt, cudaStream_t stream, int* 
     if (opt.cluster <= 1) {
         bool sweeps = false;
         for (int b = 0; b < np; ++b) sweeps = sweeps || (in[b].mode == MODE_FACTOR && in[b].sweeps > 0);
-        const int nt = opt.block > 0 ? opt.block : auto_block(work_max, m_max, n_max, Gg, sweeps);
+        int nt = opt.block > 0 ? opt.block : auto_block(work_max, m_max, n_max, Gg, sweeps);
+        if (opt.block == 0 && nt == 1024) {
+            // the 1024-thread layout keeps more shared state per CTA, so on the largest shapes it
+            // leaves a shorter lazy-deflation depth, or none: below AUTO_MIN_DEPTH the 512-thread plan
+            // is kept (every shape the 512-thread build can plan stays plannable)
+            RunOpts probe = opt;
+            probe.plan_only = true;
+            probe.pending = 0;
+            externd_stats pst = {};
+            std::vector<int> pstat(np, 0);
+            if (externd_run_nt1024(in, np, &probe, stream, pstat.data(), &pst, nullptr, 0) != EXTERND_OK ||
+                pst.pending < AUTO_MIN_DEPTH)
+                nt = 512;
+        }
         if (nt != NT) {
             externd_stats st2 = {};
             const int rc2 = (nt == 256 ? externd_run_nt256 : externd_run_nt1024)(

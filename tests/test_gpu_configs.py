@@ -144,6 +144,19 @@ def test_block_size_follows_the_work_per_cta():
         mats = [torch.zeros(shape, device="cuda") for shape in w.shapes]
         _, st = ext.factor_batched(mats, list(w.mu), list(w.tau), sweeps=w.sweeps, plan_only=True)
         assert st["block"] == nt, name
+    # where the 1024-thread layout would leave a lazy-deflation depth below 8, 512 is kept: every
+    # shape the 512-thread build can plan stays plannable
+    big = torch.empty((12288, 12288), device="cuda")
+    _, st = ext.factor_batched([big], [3.0], [1.0], plan_only=True)
+    assert st["block"] == 1024 and st["pending"] >= 8
+    _, st = ext.factor_batched([big], [3.0], [1.0], hs=[torch.ones(12288, device="cuda")], plan_only=True)
+    assert st["block"] == 512 and st["pending"] >= 1
+    del big
+    big = torch.empty((20480, 20480), device="cuda")
+    _, st = ext.factor_batched([big], [3.0], [1.0], plan_only=True)
+    assert st["block"] == 512 and st["pending"] >= 1
+    del big
+    torch.cuda.empty_cache()
     # other sizes, and anything but 512 with the clustered kernel, are refused
     for kw in (dict(block=300), dict(block=128), dict(block=256, cluster=2), dict(block=1024, cluster=4)):
         with pytest.raises(ext.ExterndError) as e:

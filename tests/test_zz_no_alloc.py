@@ -20,9 +20,13 @@ from ternary_rank_weight_b200.workloads import llm_matrix
 pytestmark = pytest.mark.gpu
 
 
-def test_noalloc_matches_the_allocating_entry_point_on_two_calls():
-    A = torch.from_numpy(llm_matrix(384, 512, seed=7)).cuda()
+@pytest.mark.parametrize("m,n,block", [(384, 512, 256), (64, 14000, 512), (80, 22000, 1024)])
+def test_noalloc_matches_the_allocating_entry_point_on_two_calls(m, n, block):
+    """One shape per build of the ALS machinery (256, 512 and 1024 threads per CTA, chosen by the
+    work of one CTA): the allocation-free call hands its static array to the build the plan picks."""
+    A = torch.from_numpy(llm_matrix(m, n, seed=7)).cuda()
     ref = ext.factor(A, 1.5, 0.7, iters=15, seed=3)
+    assert ref.stats["block"] == block
     for call in range(2):
         out = (torch.full_like(ref.B, 0xAA), torch.full_like(ref.D, float("nan")),
                torch.full_like(ref.C, 0x55), torch.full_like(ref.energy, float("nan")))
