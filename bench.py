@@ -367,7 +367,11 @@ def run_ours(args):
         e = res[0].energy.cpu()
         m0, n0 = w.shapes[0]
         energy_curve = {str(mu): float(e[ext.rank(m0, n0, mu) - 1].item()) for mu in w.mu_sweep}
-    kernel = "externd::als2_kernel (clusters of %d)" % st["cluster"] if st.get("cluster", 1) > 1 else "externd::als_kernel"
+    if st.get("cluster", 1) > 1:
+        kernel = "externd::als2_kernel (clusters of %d)" % st["cluster"]
+    else:   # the build of the ALS machinery the plan's block size selects
+        space = {256: "externd_nt256", 1024: "externd_nt1024"}.get(st["block"], "externd")
+        kernel = f"{space}::als_kernel ({st['block']} threads per CTA)"
     parallelism = (f"batch split over {ws} GPUs (contiguous slices, plan of the whole batch: {plan['grid']} CTAs per "
                    f"matrix, clusters of {plan['cluster']})" if strong
                    else f"replicas x{ws} (independent matrices per rank)")
