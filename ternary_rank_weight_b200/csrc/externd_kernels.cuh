@@ -6,9 +6,12 @@
 //
 // Design (B200):
 //  * One persistent cooperative launch runs every component of a matrix.  A
-//    matrix is served by a group of G CTAs (one per SM, 512 threads each: at 1024
-//    threads the 64-register cap spilled the half-step loop to local memory, and 512
-//    measured faster at every size).
+//    matrix is served by a group of G CTAs, one per SM, of NT threads each.  NT is a
+//    compile-time constant (EXTERND_NT: 256, 512 or 1024); the library compiles this
+//    code at all three and the host picks one per launch by the work of one CTA.
+//    Fewer threads shorten the barrier-bound half-step and leave more registers per
+//    thread (255 at 256 threads: no spills; 128 at 512 and 64 at 1024: the fp64 sums
+//    spill); more threads pay once a CTA's share of the residual is large.
 //  * The residual R is kept twice in HBM, each copy cut into one private block
 //    per CTA so that both half-steps read only what they need and no CTA ever
 //    reads another CTA's residual:
