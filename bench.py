@@ -373,7 +373,7 @@ def run_ours(args):
         space = {256: "externd_nt256", 1024: "externd_nt1024"}.get(st["block"], "externd")
         kernel = f"{space}::als_kernel ({st['block']} threads per CTA)"
     parallelism = (f"batch split over {ws} GPUs (contiguous slices, plan of the whole batch: {plan['grid']} CTAs per "
-                   f"matrix, clusters of {plan['cluster']})" if strong
+                   f"matrix, clusters of {plan['cluster']}, {plan['block'] or 'automatic'} threads per CTA)" if strong
                    else f"replicas x{ws} (independent matrices per rank)")
     out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": t_ms / args.steps, "higher_is_better": True,
